@@ -1,0 +1,194 @@
+"""Float64 CPU oracle for the PACK3D operator ("Geometry Matters in Packed 3D Attention").
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
+CPU-baseline leg may use this package; the product path never does.  The
+arithmetic lives in ``pack3d_oracle.c`` (plain C, float64, OpenMP over rows);
+this module compiles it with the host C compiler and marshals numpy arrays.
+It imports nothing from the CUDA package.
+
+Each wrapper names the passage of the pages it follows; the C file restates
+the equations and lists the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pack3d_oracle.c")
+_LIB = os.path.join(_HERE, "liborc.so")
+
+__all__ = ["build", "threads", "build_index", "rotate", "summaries", "local_attn",
+           "summary_attn", "gate_mix", "forward", "as_f64"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``pack3d_oracle.c`` into ``liborc.so`` next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".%d.tmp" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-Wall",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("Z", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("dh", ctypes.c_int32),
+                ("mz", ctypes.c_int32), ("my", ctypes.c_int32), ("mx", ctypes.c_int32),
+                ("base", ctypes.c_double),
+                ("bz", ctypes.c_int32), ("by", ctypes.c_int32), ("bx", ctypes.c_int32),
+                ("rz", ctypes.c_int32), ("ry", ctypes.c_int32), ("rx", ctypes.c_int32),
+                ("scale", ctypes.c_double)]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        lib.orc_build_index.argtypes = [P, P, P, P]
+        lib.orc_build_index.restype = ctypes.c_int
+        lib.orc_rotate.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_long]
+        lib.orc_summaries.argtypes = [P, P, P, P, P, P, P, P]
+        lib.orc_local_attn.argtypes = [P, P, P, P, P, P, P, ctypes.c_long, P]
+        lib.orc_summary_attn.argtypes = [P, P, P, P, ctypes.c_long, P, ctypes.c_long, P]
+        lib.orc_gate_mix.argtypes = [P, P, P, ctypes.c_long, P, P, P]
+        _lib = lib
+    return _lib
+
+
+def threads() -> int:
+    """OpenMP threads the oracle runs on (OMP_NUM_THREADS, else all cores)."""
+    env = os.environ.get("OMP_NUM_THREADS")
+    return int(env) if env else (os.cpu_count() or 1)
+
+
+def _cfg(s, scale: Optional[float] = None) -> _Cfg:
+    return _Cfg(s.Z, s.H, s.W, s.Hq, s.Hkv, s.d_h, s.m_z, s.m_y, s.m_x, float(s.rope_base),
+                s.bz, s.by, s.bx, s.rz, s.ry, s.rx,
+                float(s.softmax_scale if scale is None else scale))
+
+
+def as_f64(x) -> np.ndarray:
+    """Contiguous float64 numpy copy of a numpy array or torch tensor (bf16 widened exactly)."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _i32(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def build_index(s, coords):
+    """Bijection check, grid-to-packed map and block membership.
+
+    Key design 1 (coordinate-preserving packings) and Key design 2 (contiguous
+    blocks).  Returns ``(status, g2p [N], members [M, v])``; status 0 = ok,
+    1 = coordinate out of range, 2 = duplicate coordinate.
+    """
+    c = _i32(coords)
+    g2p = np.empty(s.N, np.int32)
+    mem = np.empty((s.M, s.v), np.int32)
+    cfg = _cfg(s)
+    st = _load().orc_build_index(ctypes.byref(cfg), _ptr(c), _ptr(g2p), _ptr(mem))
+    return st, g2p, mem
+
+
+def rotate(s, coords, x, heads: Optional[int] = None) -> np.ndarray:
+    """Axial grid RoPE ``R(c_i) x_i`` per head (Key design 1, equation R(c))."""
+    xa = as_f64(x)
+    n = xa.shape[0]
+    heads = heads if heads is not None else xa.shape[1]
+    c = _i32(coords)
+    y = np.empty_like(xa)
+    cfg = _cfg(s)
+    _load().orc_rotate(ctypes.byref(cfg), _ptr(c), _ptr(xa), _ptr(y), heads, n)
+    return y
+
+
+def summaries(s, coords, members, k_cmp, v_cmp, scores):
+    """Rotate-before-compress summaries (Key design 2, equations k~_j^R and v~_j)."""
+    c, m = _i32(coords), _i32(members)
+    kc, vc, sc = as_f64(k_cmp), as_f64(v_cmp), as_f64(scores)
+    ks = np.empty((s.M, s.Hkv, s.d_h))
+    vs = np.empty((s.M, s.Hkv, s.d_h))
+    cfg = _cfg(s)
+    _load().orc_summaries(ctypes.byref(cfg), _ptr(c), _ptr(m), _ptr(kc), _ptr(vc), _ptr(sc),
+                          _ptr(ks), _ptr(vs))
+    return ks, vs
+
+
+def _rows(s, rows):
+    if rows is None:
+        return np.arange(s.N, dtype=np.int64)
+    return np.ascontiguousarray(rows, dtype=np.int64)
+
+
+def local_attn(s, coords, g2p, q_rot, k_rot, v_loc, rows=None, scale=None) -> np.ndarray:
+    """Exact local attention over the clipped box window (Key design 3)."""
+    r = _rows(s, rows)
+    c, g = _i32(coords), _i32(g2p)
+    qa, ka, va = as_f64(q_rot), as_f64(k_rot), as_f64(v_loc)
+    o = np.empty((r.shape[0], s.Hq, s.d_h))
+    cfg = _cfg(s, scale)
+    _load().orc_local_attn(ctypes.byref(cfg), _ptr(c), _ptr(g), _ptr(qa), _ptr(ka), _ptr(va),
+                           _ptr(r), r.shape[0], _ptr(o))
+    return o
+
+
+def summary_attn(s, q_rot, k_sum, v_sum, rows=None, scale=None) -> np.ndarray:
+    """Every query against all M summaries with its own softmax (Key design 3)."""
+    r = _rows(s, rows)
+    qa, ka, va = as_f64(q_rot), as_f64(k_sum), as_f64(v_sum)
+    o = np.empty((r.shape[0], s.Hq, s.d_h))
+    cfg = _cfg(s, scale)
+    _load().orc_summary_attn(ctypes.byref(cfg), _ptr(qa), _ptr(ka), _ptr(va), ka.shape[0],
+                             _ptr(r), r.shape[0], _ptr(o))
+    return o
+
+
+def gate_mix(s, gate, o_loc, o_cmp, rows=None) -> np.ndarray:
+    """Tokenwise two-way softmax gate (overall framework, learned mixer)."""
+    r = _rows(s, rows)
+    ga, la, ca = as_f64(gate), as_f64(o_loc), as_f64(o_cmp)
+    out = np.empty_like(la)
+    cfg = _cfg(s)
+    _load().orc_gate_mix(ctypes.byref(cfg), _ptr(ga), _ptr(r), r.shape[0], _ptr(la), _ptr(ca),
+                         _ptr(out))
+    return out
+
+
+def forward(s, inputs: Dict, rows=None) -> Dict[str, np.ndarray]:
+    """The whole operator, stage by stage in the pages' order, for ``rows`` (default all).
+
+    ``inputs`` holds ``coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate`` in
+    packed order (numpy or torch; bf16 values are widened exactly).
+    """
+    st, g2p, mem = build_index(s, inputs["coords"])
+    if st != 0:
+        raise ValueError("coordinates are not a bijection onto the lattice (status %d)" % st)
+    coords = inputs["coords"]
+    qr = rotate(s, coords, inputs["q"])
+    klr = rotate(s, coords, inputs["k_loc"])
+    ks, vs = summaries(s, coords, mem, inputs["k_cmp"], inputs["v_cmp"], inputs["scores"])
+    r = _rows(s, rows)
+    ol = local_attn(s, coords, g2p, qr, klr, inputs["v_loc"], r)
+    oc = summary_attn(s, qr, ks, vs, r)
+    out = gate_mix(s, inputs["gate"], ol, oc, r)
+    return {"out": out, "o_loc": ol, "o_cmp": oc, "q_rot": qr, "k_rot": klr,
+            "k_sum": ks, "v_sum": vs, "g2p": g2p, "members": mem, "rows": r}

@@ -1,0 +1,288 @@
+/*
+ * PACK3D oracle: a plain, slow, float64 CPU statement of what the operator
+ * computes, written from "Geometry Matters in Packed 3D Attention".
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header or table with the CUDA
+ * library; it reads plain float64 arrays and writes plain float64 arrays.
+ *
+ * Every function follows one passage of the pages:
+ *   - lattice / index map ........ method "Key design 1" (coordinate-preserving
+ *                                  permutations) and "Key design 2" (blocks);
+ *                                  the summary's "Methodology in Plain English"
+ *                                  (a packing is a bijection onto the lattice).
+ *   - axial RoPE ................. "Key design 1", equation R(c).
+ *   - summaries .................. "Key design 2", equations k~_j^R and v~_j.
+ *   - local branch ............... "Key design 3" (neighbourhood N(i)); summary
+ *                                  "local attention stays exact".
+ *   - compressed branch .......... "Key design 3" / summary "every token attends
+ *                                  to all M summaries".
+ *   - gate ....................... "overall framework" (tokenwise learned gate).
+ *
+ * Readings where the pages are silent (all listed in the design notes):
+ *   omega_{a,r} = base^(-r/m_a); rotary pair p occupies dims (2p, 2p+1); pairs
+ *   are ordered z, then y, then x; dims past 2(m_z+m_y+m_x) are untouched;
+ *   the rotation maps (x0,x1) to (x0 cos t - x1 sin t, x0 sin t + x1 cos t);
+ *   the window is an axis-aligned box of radii (rz,ry,rx) clipped at the
+ *   volume boundary with the query itself included; block scores are one per
+ *   token and kv head; q head h reads kv head floor(h*Hkv/Hq); gate channel 0
+ *   weighs the local branch and channel 1 the compressed one; summaries are
+ *   numbered in raster order over the block grid and block members in raster
+ *   order inside a block.  The frequency values and pair layout are fixed by
+ *   that convention only (no identity on the pages distinguishes them).
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC -o liborc.so pack3d_oracle.c -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int32_t Z, H, W;
+    int32_t Hq, Hkv, dh;
+    int32_t mz, my, mx;
+    double base;
+    int32_t bz, by, bx;
+    int32_t rz, ry, rx;
+    double scale;
+} orc_cfg;
+
+/* ---- lattice and index map ------------------------------------------- */
+
+/* Checks that coords is a bijection onto [0,Z)x[0,H)x[0,W) and builds
+ * g2p[(z*H+y)*W+x] = packed index and members[j*v + t] = packed index of the
+ * t-th site (raster inside the block) of block j (raster over the block grid).
+ * Returns 0 on success, 1 if a coordinate is out of range, 2 on a duplicate. */
+int orc_build_index(const orc_cfg *c, const int32_t *coords, int32_t *g2p, int32_t *members)
+{
+    long N = (long)c->Z * c->H * c->W;
+    for (long s = 0; s < N; ++s) g2p[s] = -1;
+    for (long i = 0; i < N; ++i) {
+        int z = coords[3 * i], y = coords[3 * i + 1], x = coords[3 * i + 2];
+        if (z < 0 || z >= c->Z || y < 0 || y >= c->H || x < 0 || x >= c->W) return 1;
+        long s = ((long)z * c->H + y) * c->W + x;
+        if (g2p[s] != -1) return 2;
+        g2p[s] = (int32_t)i;
+    }
+    /* N distinct in-range sites for N tokens: every site is filled. */
+    int nby = c->H / c->by, nbx = c->W / c->bx;
+    int v = c->bz * c->by * c->bx;
+    for (int z = 0; z < c->Z; ++z)
+        for (int y = 0; y < c->H; ++y)
+            for (int x = 0; x < c->W; ++x) {
+                long j = ((long)(z / c->bz) * nby + y / c->by) * nbx + x / c->bx;
+                int t = ((z % c->bz) * c->by + y % c->by) * c->bx + x % c->bx;
+                members[j * v + t] = g2p[((long)z * c->H + y) * c->W + x];
+            }
+    return 0;
+}
+
+/* ---- axial grid RoPE, equation R(c) ------------------------------------ */
+
+/* Angle of rotary pair p for coordinate (z,y,x); returns 0 for untouched dims
+ * through *active = 0. */
+static double pair_angle(const orc_cfg *c, int p, int z, int y, int x, int *active)
+{
+    int axis_pairs[3] = {c->mz, c->my, c->mx};
+    int coord[3] = {z, y, x};
+    int first = 0;
+    for (int a = 0; a < 3; ++a) {
+        if (p < first + axis_pairs[a]) {
+            int r = p - first;
+            double omega = pow(c->base, -(double)r / (double)axis_pairs[a]);
+            *active = 1;
+            return omega * (double)coord[a];
+        }
+        first += axis_pairs[a];
+    }
+    *active = 0;
+    return 0.0;
+}
+
+/* y = R(c) x for one head vector of d_h values at coordinate (cz,cy,cx). */
+static void rotate_row(const orc_cfg *c, int cz, int cy, int cx, const double *xi, double *yi)
+{
+    for (int p = 0; p < c->dh / 2; ++p) {
+        int active;
+        double t = pair_angle(c, p, cz, cy, cx, &active);
+        double x0 = xi[2 * p], x1 = xi[2 * p + 1];
+        if (active) {
+            yi[2 * p] = x0 * cos(t) - x1 * sin(t);
+            yi[2 * p + 1] = x0 * sin(t) + x1 * cos(t);
+        } else {
+            yi[2 * p] = x0;
+            yi[2 * p + 1] = x1;
+        }
+    }
+}
+
+/* y[i,h,:] = R(c_i) x[i,h,:] for n tokens with `heads` heads each. */
+void orc_rotate(const orc_cfg *c, const int32_t *coords, const double *x, double *y,
+                int heads, long n)
+{
+    int d = c->dh;
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; ++i)
+        for (int h = 0; h < heads; ++h)
+            rotate_row(c, coords[3 * i], coords[3 * i + 1], coords[3 * i + 2],
+                       x + ((long)i * heads + h) * d, y + ((long)i * heads + h) * d);
+}
+
+/* ---- rotate-before-compress block summaries, equations k~_j^R, v~_j ---- */
+
+/* For every block j and kv head g:
+ *   a_{j,u} = exp(s_{u,g}) / sum_{u' in B_j} exp(s_{u',g})
+ *   ksum[j,g] = sum_u a_{j,u} R(c_u) kcmp[u,g]
+ *   vsum[j,g] = sum_u a_{j,u} vcmp[u,g]
+ * The softmax is evaluated with its maximum subtracted (same value). */
+void orc_summaries(const orc_cfg *c, const int32_t *coords, const int32_t *members,
+                   const double *kcmp, const double *vcmp, const double *scores,
+                   double *ksum, double *vsum)
+{
+    long N = (long)c->Z * c->H * c->W;
+    int v = c->bz * c->by * c->bx;
+    long M = N / v;
+    int d = c->dh, Hkv = c->Hkv;
+#pragma omp parallel for schedule(static)
+    for (long j = 0; j < M; ++j) {
+        double *a = (double *)malloc(sizeof(double) * v);
+        double *kr = (double *)malloc(sizeof(double) * d);
+        for (int g = 0; g < Hkv; ++g) {
+            double smax = -INFINITY, den = 0.0;
+            for (int t = 0; t < v; ++t) {
+                double s = scores[(long)members[j * v + t] * Hkv + g];
+                if (s > smax) smax = s;
+            }
+            for (int t = 0; t < v; ++t) {
+                a[t] = exp(scores[(long)members[j * v + t] * Hkv + g] - smax);
+                den += a[t];
+            }
+            for (int t = 0; t < v; ++t) a[t] /= den;
+            double *ks = ksum + (j * Hkv + g) * d;
+            double *vs = vsum + (j * Hkv + g) * d;
+            for (int e = 0; e < d; ++e) { ks[e] = 0.0; vs[e] = 0.0; }
+            for (int t = 0; t < v; ++t) {
+                long u = members[j * v + t];
+                rotate_row(c, coords[3 * u], coords[3 * u + 1], coords[3 * u + 2],
+                           kcmp + (u * Hkv + g) * d, kr);
+                for (int e = 0; e < d; ++e) {
+                    ks[e] += a[t] * kr[e];
+                    vs[e] += a[t] * vcmp[(u * Hkv + g) * d + e];
+                }
+            }
+        }
+        free(a);
+        free(kr);
+    }
+}
+
+/* ---- exact local branch ------------------------------------------------ */
+
+/* For each sampled packed row i (rows[r]) and q head h, with g = kv head of h:
+ *   N(i) = tokens at lattice sites within the clipped box of radii (rz,ry,rx)
+ *   l_j  = scale * <qr[i,h], klr[j,g]>,  o = sum_j softmax(l)_j vloc[j,g]. */
+void orc_local_attn(const orc_cfg *c, const int32_t *coords, const int32_t *g2p,
+                    const double *qr, const double *klr, const double *vloc,
+                    const int64_t *rows, long nrows, double *oloc)
+{
+    int d = c->dh, Hq = c->Hq, Hkv = c->Hkv;
+    long wmax = (long)(2 * c->rz + 1) * (2 * c->ry + 1) * (2 * c->rx + 1);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long r = 0; r < nrows; ++r) {
+        long i = rows[r];
+        int zi = coords[3 * i], yi = coords[3 * i + 1], xi = coords[3 * i + 2];
+        long *nb = (long *)malloc(sizeof(long) * wmax);
+        double *l = (double *)malloc(sizeof(double) * wmax);
+        long cnt = 0;
+        for (int z = zi - c->rz; z <= zi + c->rz; ++z)
+            for (int y = yi - c->ry; y <= yi + c->ry; ++y)
+                for (int x = xi - c->rx; x <= xi + c->rx; ++x) {
+                    if (z < 0 || z >= c->Z || y < 0 || y >= c->H || x < 0 || x >= c->W) continue;
+                    nb[cnt++] = g2p[((long)z * c->H + y) * c->W + x];
+                }
+        for (int h = 0; h < Hq; ++h) {
+            int g = (int)(((long)h * Hkv) / Hq);
+            const double *q = qr + (i * Hq + h) * d;
+            double lmax = -INFINITY, den = 0.0;
+            for (long k = 0; k < cnt; ++k) {
+                const double *kk = klr + (nb[k] * Hkv + g) * d;
+                double s = 0.0;
+                for (int e = 0; e < d; ++e) s += q[e] * kk[e];
+                l[k] = c->scale * s;
+                if (l[k] > lmax) lmax = l[k];
+            }
+            double *o = oloc + (r * Hq + h) * d;
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            for (long k = 0; k < cnt; ++k) {
+                double p = exp(l[k] - lmax);
+                den += p;
+                const double *vv = vloc + (nb[k] * Hkv + g) * d;
+                for (int e = 0; e < d; ++e) o[e] += p * vv[e];
+            }
+            for (int e = 0; e < d; ++e) o[e] /= den;
+        }
+        free(nb);
+        free(l);
+    }
+}
+
+/* ---- compressed branch: every query against all M summaries ------------ */
+
+void orc_summary_attn(const orc_cfg *c, const double *qr, const double *ksum,
+                      const double *vsum, long M, const int64_t *rows, long nrows,
+                      double *ocmp)
+{
+    int d = c->dh, Hq = c->Hq, Hkv = c->Hkv;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long r = 0; r < nrows; ++r) {
+        long i = rows[r];
+        double *l = (double *)malloc(sizeof(double) * M);
+        for (int h = 0; h < Hq; ++h) {
+            int g = (int)(((long)h * Hkv) / Hq);
+            const double *q = qr + (i * Hq + h) * d;
+            double lmax = -INFINITY, den = 0.0;
+            for (long j = 0; j < M; ++j) {
+                const double *kk = ksum + (j * Hkv + g) * d;
+                double s = 0.0;
+                for (int e = 0; e < d; ++e) s += q[e] * kk[e];
+                l[j] = c->scale * s;
+                if (l[j] > lmax) lmax = l[j];
+            }
+            double *o = ocmp + (r * Hq + h) * d;
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            for (long j = 0; j < M; ++j) {
+                double p = exp(l[j] - lmax);
+                den += p;
+                const double *vv = vsum + (j * Hkv + g) * d;
+                for (int e = 0; e < d; ++e) o[e] += p * vv[e];
+            }
+            for (int e = 0; e < d; ++e) o[e] /= den;
+        }
+        free(l);
+    }
+}
+
+/* ---- tokenwise softmax gate ------------------------------------------- */
+
+/* (gamma0, gamma1) = softmax(gate[i,h,0], gate[i,h,1]);
+ * out = gamma0 * oloc + gamma1 * ocmp, for the sampled rows. */
+void orc_gate_mix(const orc_cfg *c, const double *gate, const int64_t *rows, long nrows,
+                  const double *oloc, const double *ocmp, double *out)
+{
+    int d = c->dh, Hq = c->Hq;
+    for (long r = 0; r < nrows; ++r) {
+        long i = rows[r];
+        for (int h = 0; h < Hq; ++h) {
+            double g0 = gate[(i * Hq + h) * 2], g1 = gate[(i * Hq + h) * 2 + 1];
+            double gm = g0 > g1 ? g0 : g1;
+            double e0 = exp(g0 - gm), e1 = exp(g1 - gm);
+            double w0 = e0 / (e0 + e1), w1 = e1 / (e0 + e1);
+            for (int e = 0; e < d; ++e) {
+                long k = (r * Hq + h) * d + e;
+                out[k] = w0 * oloc[k] + w1 * ocmp[k];
+            }
+        }
+    }
+}
