@@ -1,0 +1,403 @@
+"""Benchmark of the PACK3D forward pass on B200: tokens/s, per-stage roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 65k|262k|1m|tiny]
+                    [--impl ours|reference]
+
+One step = one pass of the whole hot path over one synthetic volume: index
+map, axial RoPE on Q and K_loc, block summaries, local attention, query x
+summary attention with the gate.  The timed step calls the C ABI stage entry
+points in the order pack3d_forward runs them, with CUDA events between stages
+on the launching stream, so each kernel's live duration is known.  L2 is
+flushed (a 256 MiB write) between steps, outside the timed events.  ``e2e``
+times pack3d_forward end to end from pinned host buffers (inputs copied in,
+output copied out, inside the timed region).
+
+Under torchrun (N > 1) every rank runs an independent replica of the volume
+(the operator is single-GPU; ranks exchange nothing on the data path), the
+time is the max over ranks and ``value`` counts every rank's tokens.
+
+``--impl reference`` times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "PACK3D fwd tokens/s at 65k/262k/1M tokens, 1 B200; % of tensor/HBM roofline"
+WORKLOAD_TEXT = {
+    "tiny": "4x8x8 lattice (256 tokens), raster packing, fp32, Hq=2, Hkv=1, d_h=64, blocks 1x4x4 (M=16), window 3x3x3",
+    "65k": "16x64x64 lattice (65,536 tokens), Morton packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=4,096), window 3x7x7",
+    "262k": "16x128x128 lattice (262,144 tokens), block-contiguous packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=16,384), window 3x7x7",
+    "1m": "64x128x128 lattice (1,048,576 tokens), random packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=65,536), window 3x7x7",
+}
+STAGES = ("index", "rope", "summaries", "local", "summary_attn")
+KERNELS_PER_STEP = 8   # 2 fills + index, rope Q, rope K, summaries, local, summary attention
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def mean_window(s) -> float:
+    """Mean clipped window size: product over axes of the mean clipped count."""
+    def axis(n, r):
+        return float(np.mean([min(n - 1, i + r) - max(0, i - r) + 1 for i in range(n)]))
+    return axis(s.Z, s.rz) * axis(s.H, s.ry) * axis(s.W, s.rx)
+
+
+def algorithmic_work(s):
+    """Per-launch algorithmic bytes / flops of each stage (the design doc derives them)."""
+    eb = 2 if s.dtype == "bf16" else 4
+    d = s.d_h
+    N, M = s.N, s.M
+    wbar = mean_window(s)
+    return {
+        "index": {"bytes": N * (12 + 4 + 4)},
+        "rope": {"bytes": N * ((s.Hq + s.Hkv) * d * eb * 2 + 12)},
+        "summaries": {"bytes": N * (s.Hkv * d * eb * 2 + s.Hkv * 4 + 4) + M * s.Hkv * d * eb * 2},
+        "local": {"bytes": N * (s.Hq * d * eb + 2 * s.Hkv * d * eb + s.Hq * d * 4 + 4),
+                  "flops": 4.0 * d * s.Hq * N * wbar},
+        "summary_attn": {"flops": 4.0 * d * s.Hq * N * M,
+                         "bytes": N * (s.Hq * d * eb * 2 + s.Hq * d * 4 + s.Hq * 8) + 2 * M * s.Hkv * d * eb},
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples taken during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    import torch
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def cpu_oracle_sample(s, inp, target_s: float = 12.0):
+    """Times the oracle on this workload: the whole-volume stages (index map, K_loc
+    rotation, summaries) once, the per-query stages on a sample of rows sized to
+    about ``target_s`` seconds, extrapolated to all N rows.  Returns a dict."""
+    import torch
+
+    import oracle
+    t0 = time.perf_counter()
+    st, g2p, mem = oracle.build_index(s, inp["coords"])
+    coords = inp["coords"].numpy()
+    klr = oracle.rotate(s, coords, inp["k_loc"])
+    ks, vs = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"])
+    t_shared = time.perf_counter() - t0
+
+    def per_rows(count, seed):
+        rows = synth.sample_rows(s.N, count, seed)
+        t = time.perf_counter()
+        qr = oracle.rotate(s, coords[rows], inp["q"][torch.from_numpy(rows)])
+        ol = oracle.local_attn(s, coords, g2p, qr, klr, inp["v_loc"], rows)
+        oc = oracle.summary_attn(s, qr, ks, vs)
+        oracle.gate_mix(s, inp["gate"], ol, oc, rows)
+        return len(rows), time.perf_counter() - t
+
+    n0, t0r = per_rows(min(64, s.N), 11)
+    n1 = int(min(s.N, max(64, n0 * max(0.0, target_s - t_shared) / max(t0r, 1e-6))))
+    n1, t1 = per_rows(n1, 12)
+    total = t_shared + t1 * s.N / n1
+    return {"value": s.N / total, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": (f"float64 C oracle, OpenMP: whole-volume index map, K_loc RoPE and summaries "
+                       f"({t_shared:.2f} s) + RoPE/local/summary attention/gate for {n1} of {s.N} query "
+                       f"rows ({t1:.2f} s), per-row time extrapolated to all rows"),
+            "seconds": t_shared + t1}
+
+
+def run_reference(args, s):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = synth.make_inputs(s, s.packing, seed=0)
+    vals = []
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; warm-up steps are not run
+    base = None
+    for _ in range(args.steps):
+        base = cpu_oracle_sample(s, inp, target_s=max(2.0, 60.0 / max(1, args.steps)))
+        vals.append(base["value"])
+    value = statistics.mean(vals)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": s.N / value * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT[args.config], "tokens": s.N},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": base["cores"], "kind": "oracle",
+                             "sample": base["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, s):
+    import torch
+
+    import geometry_aware_local_b200 as p3
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = p3.config_from_shape(s)
+    inp_host = synth.make_inputs(s, s.packing, seed=rank)
+    names = ("coords", "q", "k_loc", "v_loc", "k_cmp", "v_cmp", "scores", "gate")
+    d = {k: inp_host[k].to(dev) for k in names}
+    dt = d["q"].dtype
+    err = torch.zeros(4, dtype=torch.int32, device=dev)
+    g2p = torch.empty(s.N, dtype=torch.int32, device=dev)
+    mem = torch.empty(s.M, s.v, dtype=torch.int32, device=dev)
+    qr, kr = torch.empty_like(d["q"]), torch.empty_like(d["k_loc"])
+    ks = torch.empty(s.M, s.Hkv, s.d_h, dtype=dt, device=dev)
+    vs = torch.empty_like(ks)
+    ol = torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device=dev)
+    out = torch.empty_like(d["q"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    lib = p3.lib
+    import ctypes
+    cfgp = ctypes.byref(cfg)
+    sh = stream.cuda_stream
+    P = lambda t: t.data_ptr()  # noqa: E731
+
+    def step(ev):
+        # The same launches pack3d_forward makes, one entry point per stage.
+        ev[0].record(stream)
+        st = lib.pack3d_build_index(cfgp, P(d["coords"]), P(g2p), P(mem), P(err), sh)
+        ev[1].record(stream)
+        st |= lib.pack3d_rope(cfgp, P(d["coords"]), P(d["q"]), P(qr), s.Hq, sh)
+        st |= lib.pack3d_rope(cfgp, P(d["coords"]), P(d["k_loc"]), P(kr), s.Hkv, sh)
+        ev[2].record(stream)
+        st |= lib.pack3d_build_summaries(cfgp, P(mem), P(d["k_cmp"]), P(d["v_cmp"]), P(d["scores"]), P(ks),
+                                         P(vs), sh)
+        ev[3].record(stream)
+        st |= lib.pack3d_local_attn(cfgp, P(g2p), P(qr), P(kr), P(d["v_loc"]), P(ol), sh)
+        ev[4].record(stream)
+        st |= lib.pack3d_summary_attn(cfgp, P(qr), P(ks), P(vs), P(ol), P(d["gate"]), P(out), P(err), sh)
+        ev[5].record(stream)
+        if st:
+            raise RuntimeError("a PACK3D entry point failed")
+
+    def events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    for _ in range(args.warmup):
+        step(events())
+    if p3.check_status(err) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [events() for _ in range(args.steps)]
+    barrier(world)
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            step(evs[k])
+        barrier(world)
+    st_ms = {name: 0.0 for name in STAGES}
+    step_ms = []
+    for ev in evs:
+        for i, name in enumerate(STAGES):
+            st_ms[name] += ev[i].elapsed_time(ev[i + 1])
+        step_ms.append(ev[0].elapsed_time(ev[5]))
+    if p3.check_status(err) != 0:
+        raise RuntimeError("device error during the timed steps")
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+    st_ms = {k: v / args.steps for k, v in st_ms.items()}
+    value = s.N * world / (ms * 1e-3)
+
+    # pack3d_forward from the device buffers (same kernels, one C-ABI call).
+    ws = torch.empty(p3.workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    fwd_ms = []
+    for k in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        p3.forward(cfg, d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
+                   d["gate"], out, ws, err)
+        e1.record(stream)
+        if k >= args.warmup:
+            fwd_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    fwd = statistics.mean(a.elapsed_time(b) for a, b in fwd_ms)
+
+    # End to end through the public API from pinned host buffers.
+    hin = {k: inp_host[k].pin_memory() for k in names}
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hin.values())
+    d2h = hout.numel() * hout.element_size()
+    e2e = []
+    for k in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for n in names:
+            d[n].copy_(hin[n], non_blocking=True)
+        p3.forward(cfg, d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
+                   d["gate"], out, ws, err)
+        hout.copy_(out, non_blocking=True)
+        e1.record(stream)
+        if k >= args.warmup:
+            e2e.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in e2e), world)
+    if p3.check_status(err) != 0:
+        raise RuntimeError("device error during the e2e steps")
+
+    peaks = load_peaks()
+    work = algorithmic_work(s)
+    stages = {}
+    for name in STAGES:
+        t = st_ms[name] * 1e-3
+        w = work[name]
+        e = {"ms": st_ms[name]}
+        if "bytes" in w:
+            e["hbm_gbs"] = w["bytes"] / t / 1e9
+            e["hbm_frac"] = e["hbm_gbs"] / peaks["hbm_gbs"]
+        if "flops" in w:
+            e["tflops"] = w["flops"] / t / 1e12
+            e["tensor_frac"] = e["tflops"] / peaks["bf16_tflops"]
+        stages[name] = e
+    sa = stages["summary_attn"]
+    roof = {"bound": "tensor", "achieved": sa["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": sa["tflops"] / peaks["bf16_tflops"], "traffic": None,
+            "kernel": "summary_attn_tc_kernel" if s.dtype == "bf16" else "summary_attn_simt_kernel",
+            "peak_source": peaks["source"] + " burst bf16 (MEASURED_PEAKS.json bf16_tflops)"}
+    if s.dtype != "bf16":
+        roof["bound"] = "alu"
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[args.config], "tokens": s.N, "summaries": s.M,
+                       "parallelism": "replicas only" if world > 1 else "single GPU",
+                       "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+            "e2e": {"value": s.N * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "roofline": roof, "stages": stages, "forward_call_ms": fwd,
+            "clocks": clk.summary()}
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_oracle_sample(s, inp_host, target_s=12.0)
+            cb.pop("seconds")
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="65k", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    s = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, s)
+    else:
+        run_ours(args, s)
+
+
+if __name__ == "__main__":
+    main()

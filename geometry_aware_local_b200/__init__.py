@@ -1,0 +1,217 @@
+"""Python binding of libpack3d.so: the PACK3D local-global attention forward pass on B200.
+
+Argument marshalling only: every stage runs in the CUDA kernels behind the C ABI
+declared in ``include/pack3d.h`` ("Geometry Matters in Packed 3D Attention",
+Key designs 1-3).  Tensors must be CUDA, contiguous and 16-byte aligned; calls
+are asynchronous on torch's current stream.  There is no CPU fallback: if the
+library was not built, importing the binding raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpack3d.so")
+
+F32, BF16 = 0, 1
+FLAG_SIMT_SUMMARY = 0x1
+DEVERR_COORD_RANGE, DEVERR_DUPLICATE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: "NOT_PERMUTATION",
+          6: "WORKSPACE", 7: "CUDA", 8: "TIMEOUT"}
+
+ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
+                "pack3d_build_index", "pack3d_rope", "pack3d_build_summaries", "pack3d_local_attn",
+                "pack3d_summary_attn", "pack3d_forward", "pack3d_check_status",
+                "pack3d_status_string", "pack3d_backend_info")
+
+
+class Pack3DError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_string(status)})")
+
+
+class Config(ctypes.Structure):
+    """Mirror of ``pack3d_config``."""
+    _fields_ = [("Z", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d_h", ctypes.c_int32),
+                ("m_z", ctypes.c_int32), ("m_y", ctypes.c_int32), ("m_x", ctypes.c_int32),
+                ("reserved0", ctypes.c_int32), ("rope_base", ctypes.c_double),
+                ("bz", ctypes.c_int32), ("by", ctypes.c_int32), ("bx", ctypes.c_int32),
+                ("rz", ctypes.c_int32), ("ry", ctypes.c_int32), ("rx", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("flags", ctypes.c_int32), ("reserved1", ctypes.c_int32)]
+
+    @property
+    def N(self) -> int:
+        return self.Z * self.H * self.W
+
+    @property
+    def M(self) -> int:
+        return self.N // (self.bz * self.by * self.bx)
+
+    @property
+    def v(self) -> int:
+        return self.bz * self.by * self.bx
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python geometry_aware_local_b200/build.py` "
+                          "(there is no fallback implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, C = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(Config)
+    sig = {
+        "pack3d_default_config": (None, [C, I32, I32, I32]),
+        "pack3d_validate_config": (ctypes.c_int, [C]),
+        "pack3d_workspace_bytes": (ctypes.c_size_t, [C]),
+        "pack3d_build_index": (ctypes.c_int, [C, P, P, P, P, P]),
+        "pack3d_rope": (ctypes.c_int, [C, P, P, P, I32, P]),
+        "pack3d_build_summaries": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
+        "pack3d_local_attn": (ctypes.c_int, [C, P, P, P, P, P, P]),
+        "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
+        "pack3d_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
+        "pack3d_check_status": (ctypes.c_int, [P, P]),
+        "pack3d_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "pack3d_backend_info": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _status_string(st: int) -> str:
+    return lib.pack3d_status_string(st).decode()
+
+
+def backend_info() -> str:
+    return lib.pack3d_backend_info().decode()
+
+
+def make_config(Z: int, H: int, W: int, *, Hq: int = 8, Hkv: int = 2, d_h: int = 64,
+                m: Sequence[int] = (11, 11, 10), rope_base: float = 10000.0,
+                block: Sequence[int] = (1, 4, 4), radius: Sequence[int] = (1, 3, 3),
+                softmax_scale: Optional[float] = None, dtype: str = "bf16", flags: int = 0) -> Config:
+    c = Config()
+    c.Z, c.H, c.W = Z, H, W
+    c.Hq, c.Hkv, c.d_h = Hq, Hkv, d_h
+    c.m_z, c.m_y, c.m_x = m
+    c.rope_base = rope_base
+    c.bz, c.by, c.bx = block
+    c.rz, c.ry, c.rx = radius
+    c.softmax_scale = 1.0 / math.sqrt(d_h) if softmax_scale is None else softmax_scale
+    c.dtype = BF16 if dtype in ("bf16", BF16) else F32
+    c.flags = flags
+    return c
+
+
+def config_from_shape(s, flags: int = 0) -> Config:
+    """Config from any object with the fields of ``synth.Pack3DShape``."""
+    return make_config(s.Z, s.H, s.W, Hq=s.Hq, Hkv=s.Hkv, d_h=s.d_h, m=(s.m_z, s.m_y, s.m_x),
+                       rope_base=s.rope_base, block=(s.bz, s.by, s.bx), radius=(s.rz, s.ry, s.rx),
+                       softmax_scale=s.softmax_scale, dtype=s.dtype, flags=flags)
+
+
+def validate(cfg: Config) -> int:
+    return lib.pack3d_validate_config(ctypes.byref(cfg))
+
+
+def workspace_bytes(cfg: Config) -> int:
+    return lib.pack3d_workspace_bytes(ctypes.byref(cfg))
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("PACK3D kernels take CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("PACK3D kernels take contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise Pack3DError(st, what)
+
+
+def build_index(cfg, coords, g2p, members, err, stream=None):
+    _check(lib.pack3d_build_index(ctypes.byref(cfg), _ptr(coords), _ptr(g2p), _ptr(members), _ptr(err),
+                                  _stream(stream)), "pack3d_build_index")
+
+
+def rope(cfg, coords, x, y, heads: int, stream=None):
+    _check(lib.pack3d_rope(ctypes.byref(cfg), _ptr(coords), _ptr(x), _ptr(y), heads, _stream(stream)),
+           "pack3d_rope")
+
+
+def build_summaries(cfg, members, k_cmp, v_cmp, scores, k_sum, v_sum, stream=None):
+    _check(lib.pack3d_build_summaries(ctypes.byref(cfg), _ptr(members), _ptr(k_cmp), _ptr(v_cmp),
+                                      _ptr(scores), _ptr(k_sum), _ptr(v_sum), _stream(stream)),
+           "pack3d_build_summaries")
+
+
+def local_attn(cfg, g2p, q_rot, k_rot, v_loc, o_loc, stream=None):
+    _check(lib.pack3d_local_attn(ctypes.byref(cfg), _ptr(g2p), _ptr(q_rot), _ptr(k_rot), _ptr(v_loc),
+                                 _ptr(o_loc), _stream(stream)), "pack3d_local_attn")
+
+
+def summary_attn(cfg, q_rot, k_sum, v_sum, o_loc, gate, out, err=None, stream=None):
+    _check(lib.pack3d_summary_attn(ctypes.byref(cfg), _ptr(q_rot), _ptr(k_sum), _ptr(v_sum), _ptr(o_loc),
+                                   _ptr(gate), _ptr(out), _ptr(err), _stream(stream)), "pack3d_summary_attn")
+
+
+def forward(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, workspace, err, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pack3d_forward(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc), _ptr(k_cmp),
+                              _ptr(v_cmp), _ptr(scores), _ptr(gate), _ptr(out), _ptr(workspace), ws_bytes,
+                              _ptr(err), _stream(stream)), "pack3d_forward")
+
+
+def check_status(err, stream=None) -> int:
+    """Synchronises the stream, reads and clears the device error word; returns the status code."""
+    return lib.pack3d_check_status(_ptr(err), _stream(stream))
+
+
+class Pack3D:
+    """Owns the workspace and error word of one configuration on one device."""
+
+    def __init__(self, cfg: Config, device="cuda"):
+        import torch
+        st = validate(cfg)
+        if st != 0:
+            raise Pack3DError(st, "pack3d_validate_config")
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.workspace = torch.empty(workspace_bytes(cfg), dtype=torch.uint8, device=self.device)
+        self.err = torch.zeros(4, dtype=torch.int32, device=self.device)
+
+    def __call__(self, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        forward(self.cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, self.workspace, self.err)
+        return out
+
+    def check(self):
+        st = check_status(self.err)
+        if st != 0:
+            raise Pack3DError(st, "pack3d_forward")

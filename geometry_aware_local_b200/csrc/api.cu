@@ -1,0 +1,261 @@
+// C ABI of the PACK3D forward pass (see pack3d.h): host-side validation,
+// workspace carving and stream-ordered launches.  No entry point allocates,
+// frees or synchronises except pack3d_check_status.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "pack3d.h"
+
+namespace pack3d {
+
+Shape make_shape(const pack3d_config& c) {
+  Shape s;
+  memset(&s, 0, sizeof(s));
+  s.Z = c.Z; s.H = c.H; s.W = c.W;
+  s.N = c.Z * c.H * c.W;
+  s.Hq = c.Hq; s.Hkv = c.Hkv; s.G = c.Hq / c.Hkv;
+  s.bz = c.bz; s.by = c.by; s.bx = c.bx;
+  s.v = c.bz * c.by * c.bx;
+  s.M = s.N / s.v;
+  s.nbz = c.Z / c.bz; s.nby = c.H / c.by; s.nbx = c.W / c.bx;
+  s.rz = c.rz; s.ry = c.ry; s.rx = c.rx;
+  s.mz = c.m_z; s.my = c.m_y; s.mx = c.m_x;
+  s.tab_entries = c.Z * c.m_z + c.H * c.m_y + c.W * c.m_x;
+  s.scale = c.softmax_scale;
+  s.scale_log2 = (float)((double)c.softmax_scale * 1.4426950408889634);
+  const int m[3] = {c.m_z, c.m_y, c.m_x};
+  int p = 0;
+  for (int a = 0; a < 3; ++a)
+    for (int r = 0; r < m[a]; ++r) s.omega[p++] = pow(c.rope_base, -(double)r / (double)m[a]);
+  return s;
+}
+
+}  // namespace pack3d
+
+using namespace pack3d;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int elem_bytes(int dtype) { return dtype == PACK3D_BF16 ? 2 : 4; }
+
+pack3d_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return PACK3D_OK;
+  cudaGetLastError();  // clear a sticky launch-configuration error
+  return PACK3D_ERR_CUDA;
+}
+
+struct Workspace {
+  int32_t* g2p;
+  int32_t* members;
+  void* q_rot;
+  void* k_rot;
+  void* k_sum;
+  void* v_sum;
+  float* o_loc;
+  size_t bytes;
+};
+
+Workspace carve(const pack3d_config& c, uintptr_t base) {
+  const size_t N = (size_t)c.Z * c.H * c.W;
+  const size_t v = (size_t)c.bz * c.by * c.bx;
+  const size_t M = N / v;
+  const size_t eb = elem_bytes(c.dtype);
+  const size_t A = 1024;
+  Workspace w;
+  size_t off = 0;
+  w.g2p = reinterpret_cast<int32_t*>(base + off);      off = round_up(off + N * 4, A);
+  w.members = reinterpret_cast<int32_t*>(base + off);  off = round_up(off + M * v * 4, A);
+  w.q_rot = reinterpret_cast<void*>(base + off);                off = round_up(off + N * c.Hq * c.d_h * eb, A);
+  w.k_rot = reinterpret_cast<void*>(base + off);                off = round_up(off + N * c.Hkv * c.d_h * eb, A);
+  w.k_sum = reinterpret_cast<void*>(base + off);                off = round_up(off + M * c.Hkv * c.d_h * eb, A);
+  w.v_sum = reinterpret_cast<void*>(base + off);                off = round_up(off + M * c.Hkv * c.d_h * eb, A);
+  w.o_loc = reinterpret_cast<float*>(base + off);      off = round_up(off + N * c.Hq * c.d_h * 4, A);
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+void pack3d_default_config(pack3d_config* cfg, int32_t Z, int32_t H, int32_t W) {
+  if (!cfg) return;
+  memset(cfg, 0, sizeof(*cfg));
+  cfg->Z = Z; cfg->H = H; cfg->W = W;
+  cfg->Hq = 8; cfg->Hkv = 2; cfg->d_h = 64;
+  cfg->m_z = 11; cfg->m_y = 11; cfg->m_x = 10;
+  cfg->rope_base = 10000.0;
+  cfg->bz = 1; cfg->by = 4; cfg->bx = 4;
+  cfg->rz = 1; cfg->ry = 3; cfg->rx = 3;
+  cfg->softmax_scale = 0.125f;
+  cfg->dtype = PACK3D_BF16;
+}
+
+pack3d_status pack3d_validate_config(const pack3d_config* c) {
+  if (!c) return PACK3D_ERR_INVALID_ARG;
+  if (c->reserved0 != 0 || c->reserved1 != 0) return PACK3D_ERR_INVALID_ARG;
+  if (c->dtype != PACK3D_F32 && c->dtype != PACK3D_BF16) return PACK3D_ERR_DTYPE;
+  if (c->Z <= 0 || c->H <= 0 || c->W <= 0) return PACK3D_ERR_SHAPE;
+  const long long N = (long long)c->Z * c->H * c->W;
+  if (N >= (1LL << 31) / 128) return PACK3D_ERR_SHAPE;  // keeps every element index in 32 bits
+  if (c->d_h != kDh) return PACK3D_ERR_SHAPE;
+  if (c->Hq <= 0 || c->Hkv <= 0 || c->Hq % c->Hkv != 0) return PACK3D_ERR_SHAPE;
+  const int G = c->Hq / c->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PACK3D_ERR_SHAPE;
+  if (c->m_z < 0 || c->m_y < 0 || c->m_x < 0 || 2 * (c->m_z + c->m_y + c->m_x) > c->d_h)
+    return PACK3D_ERR_SHAPE;
+  if (!(c->rope_base > 0.0) || !isfinite(c->rope_base)) return PACK3D_ERR_INVALID_ARG;
+  if (c->bz <= 0 || c->by <= 0 || c->bx <= 0) return PACK3D_ERR_SHAPE;
+  if (c->Z % c->bz || c->H % c->by || c->W % c->bx) return PACK3D_ERR_SHAPE;
+  if (c->bz * c->by * c->bx > 64) return PACK3D_ERR_SHAPE;
+  if (c->rz < 0 || c->ry < 0 || c->rx < 0) return PACK3D_ERR_SHAPE;
+  if (!(c->softmax_scale > 0.f) || !isfinite(c->softmax_scale)) return PACK3D_ERR_INVALID_ARG;
+  const long long tab = (long long)c->Z * c->m_z + (long long)c->H * c->m_y + (long long)c->W * c->m_x;
+  if (tab * 8 > kMaxTableBytes) return PACK3D_ERR_SHAPE;
+  if (c->flags & ~PACK3D_FLAG_SIMT_SUMMARY) return PACK3D_ERR_INVALID_ARG;
+  return PACK3D_OK;
+}
+
+size_t pack3d_workspace_bytes(const pack3d_config* cfg) {
+  if (pack3d_validate_config(cfg) != PACK3D_OK) return 0;
+  return carve(*cfg, 0).bytes;
+}
+
+pack3d_status pack3d_build_index(const pack3d_config* cfg, const int32_t* coords, int32_t* g2p,
+                                 int32_t* members, int32_t* err_word, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!coords || !g2p || !members || !err_word) return PACK3D_ERR_INVALID_ARG;
+  if (!aligned16(coords) || !aligned16(g2p) || !aligned16(members)) return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  return cuda_status(launch_build_index(s, coords, g2p, members, err_word, (cudaStream_t)stream));
+}
+
+pack3d_status pack3d_rope(const pack3d_config* cfg, const int32_t* coords, const void* x, void* y,
+                          int32_t heads, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!coords || !x || !y || heads <= 0) return PACK3D_ERR_INVALID_ARG;
+  if ((long long)cfg->Z * cfg->H * cfg->W * heads >= (1LL << 31) / 16) return PACK3D_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(y)) return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  return cuda_status(launch_rope(s, cfg->dtype, coords, x, y, heads, nullptr, nullptr, 0,
+                                 (cudaStream_t)stream));
+}
+
+pack3d_status pack3d_build_summaries(const pack3d_config* cfg, const int32_t* members, const void* k_cmp,
+                                     const void* v_cmp, const float* scores, void* k_sum, void* v_sum,
+                                     void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!members || !k_cmp || !v_cmp || !scores || !k_sum || !v_sum) return PACK3D_ERR_INVALID_ARG;
+  if (!aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(k_sum) || !aligned16(v_sum))
+    return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  return cuda_status(
+      launch_summaries(s, cfg->dtype, members, k_cmp, v_cmp, scores, k_sum, v_sum, (cudaStream_t)stream));
+}
+
+pack3d_status pack3d_local_attn(const pack3d_config* cfg, const int32_t* g2p, const void* q_rot,
+                                const void* k_rot, const void* v_loc, float* o_loc, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!g2p || !q_rot || !k_rot || !v_loc || !o_loc) return PACK3D_ERR_INVALID_ARG;
+  if (!aligned16(q_rot) || !aligned16(k_rot) || !aligned16(v_loc) || !aligned16(o_loc))
+    return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  return cuda_status(launch_local_attn(s, cfg->dtype, g2p, q_rot, k_rot, v_loc, o_loc, (cudaStream_t)stream));
+}
+
+pack3d_status pack3d_summary_attn(const pack3d_config* cfg, const void* q_rot, const void* k_sum,
+                                  const void* v_sum, const float* o_loc, const float* gate, void* out,
+                                  int32_t* err_word, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!q_rot || !k_sum || !v_sum || !out || (gate && !o_loc)) return PACK3D_ERR_INVALID_ARG;
+  if (!aligned16(q_rot) || !aligned16(k_sum) || !aligned16(v_sum) || !aligned16(out) ||
+      (o_loc && !aligned16(o_loc)))
+    return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  cudaError_t e;
+  if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
+    e = launch_summary_attn_tc(s, q_rot, k_sum, v_sum, o_loc, gate, out, err_word, (cudaStream_t)stream);
+  else
+    e = launch_summary_attn_simt(s, cfg->dtype, q_rot, k_sum, v_sum, o_loc, gate, out, (cudaStream_t)stream);
+  return cuda_status(e);
+}
+
+pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, const void* q, const void* k_loc,
+                             const void* v_loc, const void* k_cmp, const void* v_cmp, const float* scores,
+                             const float* gate, void* out, void* workspace, size_t workspace_bytes,
+                             int32_t* err_word, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !out || !err_word)
+    return PACK3D_ERR_INVALID_ARG;
+  if (!workspace || ((uintptr_t)workspace & 255u)) return PACK3D_ERR_WORKSPACE;
+  Workspace w = carve(*cfg, (uintptr_t)workspace);
+  if (workspace_bytes < w.bytes) return PACK3D_ERR_WORKSPACE;
+  if (!aligned16(coords) || !aligned16(q) || !aligned16(k_loc) || !aligned16(v_loc) || !aligned16(k_cmp) ||
+      !aligned16(v_cmp) || !aligned16(out))
+    return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  const cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = launch_build_index(s, coords, w.g2p, w.members, err_word, cs);
+  if (e == cudaSuccess)
+    e = launch_rope(s, cfg->dtype, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, cs);
+  if (e == cudaSuccess)
+    e = launch_summaries(s, cfg->dtype, w.members, k_cmp, v_cmp, scores, w.k_sum, w.v_sum, cs);
+  if (e == cudaSuccess) e = launch_local_attn(s, cfg->dtype, w.g2p, w.q_rot, w.k_rot, v_loc, w.o_loc, cs);
+  if (e == cudaSuccess) {
+    if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
+      e = launch_summary_attn_tc(s, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, err_word, cs);
+    else
+      e = launch_summary_attn_simt(s, cfg->dtype, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, cs);
+  }
+  return cuda_status(e);
+}
+
+pack3d_status pack3d_check_status(int32_t* err_word, void* stream) {
+  if (!err_word) return PACK3D_ERR_INVALID_ARG;
+  int32_t h = 0;
+  const cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(&h, err_word, sizeof(h), cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(err_word, 0, sizeof(int32_t), cs);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (h & PACK3D_DEVERR_TIMEOUT) return PACK3D_ERR_TIMEOUT;
+  if (h & (PACK3D_DEVERR_COORD_RANGE | PACK3D_DEVERR_DUPLICATE)) return PACK3D_ERR_NOT_PERMUTATION;
+  return PACK3D_OK;
+}
+
+const char* pack3d_status_string(pack3d_status s) {
+  switch (s) {
+    case PACK3D_OK: return "ok";
+    case PACK3D_ERR_INVALID_ARG: return "invalid argument";
+    case PACK3D_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case PACK3D_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case PACK3D_ERR_DTYPE: return "unsupported dtype";
+    case PACK3D_ERR_NOT_PERMUTATION: return "coordinates are not a bijection onto the lattice";
+    case PACK3D_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case PACK3D_ERR_CUDA: return "CUDA runtime error";
+    case PACK3D_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* pack3d_backend_info(void) {
+  return "pack3d sm_100a: index map + axial RoPE + summaries (CUDA cores, 16-byte streams, shared-memory "
+         "cos/sin tables); local attention (CUDA cores, lattice bricks, float accumulation); query x summary "
+         "(bf16: tcgen05 MMA, TMEM accumulators, TMA 4-stage ring, two ping-pong softmax warpgroups; float: "
+         "CUDA cores)";
+}
+
+}  // extern "C"

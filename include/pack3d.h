@@ -1,0 +1,194 @@
+/*
+ * pack3d.h - C ABI of the B200 (sm_100a) implementation of the PACK3D
+ * local-global attention forward pass, from "Geometry Matters in Packed 3D
+ * Attention" (method section, Key designs 1-3).
+ *
+ * The operator maps packed 3D tokens and their lattice coordinates to packed
+ * outputs, A(X, c), in five stages:
+ *   1. axial grid RoPE R(c_i) on Q and K, driven by true (z,y,x) coordinates
+ *      (Key design 1, equation R(c));
+ *   2. exact local attention over each token's clipped lattice box, found
+ *      through a grid-to-packed index map (Key design 3);
+ *   3. rotate-before-compress block summaries over contiguous blocks
+ *      (Key design 2, equations k~_j^R and v~_j);
+ *   4. every query against all M = N / |B| summaries with its own softmax
+ *      (Key design 3);
+ *   5. a per-token, per-head two-way softmax gate mixing both branches
+ *      (overall framework).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named in the signatures are DEVICE pointers unless stated, owned
+ *   by the caller.  The library never allocates, frees or keeps a pointer
+ *   after a call returns.  Buffers must be contiguous and 16-byte aligned.
+ * - Layouts (packed order = the caller's token order):
+ *     coords   int32 [N,3]        (z, y, x), lattice indices from 0
+ *     q        T     [N,Hq,d_h]   T = float or bf16 (config.dtype)
+ *     k_loc, v_loc, k_cmp, v_cmp  T [N,Hkv,d_h]
+ *     scores   float [N,Hkv]      per-token block scores (one per kv head)
+ *     gate     float [N,Hq,2]     channel 0 weighs local, 1 compressed
+ *     out      T     [N,Hq,d_h]
+ *     g2p      int32 [Z*H*W]      g2p[(z*H+y)*W+x] = packed index of site
+ *     members  int32 [M,|B|]      packed index of the t-th site (raster inside
+ *                                 the block) of block j (raster over blocks)
+ *     k_sum, v_sum T [M,Hkv,d_h]  block summaries
+ *     o_loc    float [N,Hq,d_h]   local-branch output
+ *   q head h reads kv head floor(h*Hkv/Hq).
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream).  Errors that the host can see (bad config, null or
+ *   misaligned pointer, too-small workspace) are returned before anything is
+ *   launched.  Errors only the device can see (a coordinate out of range or
+ *   repeated, a bounded wait that ran out) are OR-ed into the caller's
+ *   device word `err_word` as PACK3D_DEVERR_* bits; pack3d_check_status()
+ *   reads them back.  Kernels never trap.
+ * - No entry point holds global mutable state; calls on different streams
+ *   may run concurrently as long as their buffers do not overlap.
+ * - Supported shapes: d_h == 64; Hq a multiple of Hkv with Hq/Hkv a power of
+ *   two <= 8; 2*(m_z+m_y+m_x) <= 64; block dims dividing the lattice, block
+ *   volume <= 64; lattice extents small enough that the per-axis cos/sin
+ *   tables (Z*m_z + H*m_y + W*m_x entries) fit 96 KiB of shared memory;
+ *   N < 2^31.
+ */
+#ifndef PACK3D_H
+#define PACK3D_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PACK3D_OK = 0,
+    PACK3D_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, bad enum   */
+    PACK3D_ERR_SHAPE = 2,           /* unsupported or inconsistent shape           */
+    PACK3D_ERR_ALIGNMENT = 3,       /* pointer not 16-byte aligned                 */
+    PACK3D_ERR_DTYPE = 4,           /* dtype not supported by this entry point     */
+    PACK3D_ERR_NOT_PERMUTATION = 5, /* coords are not a bijection onto the lattice */
+    PACK3D_ERR_WORKSPACE = 6,       /* workspace missing or too small              */
+    PACK3D_ERR_CUDA = 7,            /* a CUDA runtime call failed                  */
+    PACK3D_ERR_TIMEOUT = 8          /* a bounded device-side wait ran out          */
+} pack3d_status;
+
+typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
+
+/* Bits OR-ed into the caller's device error word. */
+#define PACK3D_DEVERR_COORD_RANGE 0x1  /* a coordinate outside the lattice */
+#define PACK3D_DEVERR_DUPLICATE   0x2  /* two tokens share one site        */
+#define PACK3D_DEVERR_TIMEOUT     0x4  /* a pipeline wait gave up          */
+
+/* config.flags */
+#define PACK3D_FLAG_SIMT_SUMMARY  0x1  /* bf16: use the CUDA-core query x summary
+                                          kernel instead of the tcgen05 one   */
+
+typedef struct {
+    int32_t Z, H, W;          /* lattice extents; N = Z*H*W tokens               */
+    int32_t Hq, Hkv, d_h;     /* query heads, key/value heads, head dim (64)     */
+    int32_t m_z, m_y, m_x;    /* rotary planes per axis (11, 11, 10 for d_h=64)  */
+    int32_t reserved0;        /* must be 0                                       */
+    double  rope_base;        /* omega_{a,r} = rope_base^(-r/m_a) (10000)        */
+    int32_t bz, by, bx;       /* summary block dims (1, 4, 4); divide Z, H, W    */
+    int32_t rz, ry, rx;       /* local window radii (1, 3, 3) = 3x7x7 box       */
+    float   softmax_scale;    /* logit scale in both branches (1/sqrt(d_h))      */
+    int32_t dtype;            /* pack3d_dtype of q, k, v, summaries, out         */
+    int32_t flags;            /* PACK3D_FLAG_* bits                              */
+    int32_t reserved1;        /* must be 0                                       */
+} pack3d_config;
+
+/* Fills cfg with the pages' defaults for a Z x H x W lattice: Hq=8, Hkv=2,
+ * d_h=64, m=(11,11,10), base 1e4, blocks 1x4x4, window 3x7x7, scale 1/8,
+ * bf16. */
+void pack3d_default_config(pack3d_config *cfg, int32_t Z, int32_t H, int32_t W);
+
+/* Checks a config without touching the device.  Returns PACK3D_OK or the
+ * reason it cannot be run. */
+pack3d_status pack3d_validate_config(const pack3d_config *cfg);
+
+/* Bytes of device workspace pack3d_forward needs (0 on an invalid config):
+ * g2p, members, rotated Q and K_loc, the summaries and the float o_loc, each
+ * region at a 1 KiB offset. */
+size_t pack3d_workspace_bytes(const pack3d_config *cfg);
+
+/* Stage 0 - grid-to-packed index map and block membership.
+ * Cites: Key design 1 (coordinate-preserving packings are bijections onto the
+ * lattice) and Key design 2 (contiguous blocks B_j).
+ * In: coords [N,3].  Out: g2p [Z*H*W], members [M,|B|].  A coordinate outside
+ * the lattice sets PACK3D_DEVERR_COORD_RANGE, two tokens on one site set
+ * PACK3D_DEVERR_DUPLICATE (err_word required); g2p/members are then
+ * unspecified. */
+pack3d_status pack3d_build_index(const pack3d_config *cfg, const int32_t *coords,
+                                 int32_t *g2p, int32_t *members, int32_t *err_word,
+                                 void *stream);
+
+/* Stage 1 - axial grid RoPE: y[i,h,:] = R(c_i) x[i,h,:] for `heads` heads per
+ * token.  Cites: Key design 1, equation R(c): planes (2p, 2p+1), z planes
+ * first, then y, then x, angle omega_{a,r} * c_a; dims past 2(m_z+m_y+m_x)
+ * copied.  x, y: T [N,heads,d_h]; y may equal x (in place). */
+pack3d_status pack3d_rope(const pack3d_config *cfg, const int32_t *coords, const void *x,
+                          void *y, int32_t heads, void *stream);
+
+/* Stage 3 - rotate-before-compress summaries.  For block j and kv head g:
+ *   a_{j,u} = softmax over u in B_j of scores[u,g]
+ *   k_sum[j,g] = sum_u a_{j,u} R(c_u) k_cmp[u,g],  v_sum[j,g] = sum_u a_{j,u} v_cmp[u,g]
+ * Cites: Key design 2, equations k~_j^R and v~_j.  k_cmp is NOT rotated by the
+ * caller: the rotation is applied here, before pooling.  members must come
+ * from pack3d_build_index on a valid coordinate set (member t of block j sits
+ * at the t-th raster site of the block). */
+pack3d_status pack3d_build_summaries(const pack3d_config *cfg, const int32_t *members,
+                                     const void *k_cmp, const void *v_cmp,
+                                     const float *scores, void *k_sum, void *v_sum,
+                                     void *stream);
+
+/* Stage 2 - exact local attention.  For token i at (z,y,x) and q head h:
+ *   o_loc[i,h] = sum_{j in N(i)} softmax_j(scale <q_rot[i,h], k_rot[j,g]>) v_loc[j,g]
+ * with N(i) the tokens whose sites lie in the box |dz|<=rz, |dy|<=ry,
+ * |dx|<=rx clipped at the volume (self included).  Cites: Key design 3 and
+ * the summary's "local attention stays exact" contract.  q_rot, k_rot are
+ * RoPE'd (stage 1); neighbours are reached through g2p, so any packing gives
+ * the same result and no gathered neighbour tensor is formed. */
+pack3d_status pack3d_local_attn(const pack3d_config *cfg, const int32_t *g2p,
+                                const void *q_rot, const void *k_rot, const void *v_loc,
+                                float *o_loc, void *stream);
+
+/* Stages 4+5 - every query against all M summaries, then the gate.
+ *   o_cmp[i,h] = sum_j softmax_j(scale <q_rot[i,h], k_sum[j,g]>) v_sum[j,g]
+ * streamed with an online softmax (no [N,M] tensor).  If gate is NULL, out =
+ * o_cmp.  Otherwise (gamma0,gamma1) = softmax(gate[i,h,0], gate[i,h,1]) and
+ * out = gamma0 o_loc + gamma1 o_cmp (o_loc required).  Cites: Key design 3
+ * (query-summary branch) and the overall framework's tokenwise gate.
+ * bf16 runs on tcgen05 tensor cores with float accumulation; float runs on
+ * CUDA cores in float.  err_word (nullable) receives PACK3D_DEVERR_TIMEOUT if
+ * a pipeline wait gives up. */
+pack3d_status pack3d_summary_attn(const pack3d_config *cfg, const void *q_rot,
+                                  const void *k_sum, const void *v_sum, const float *o_loc,
+                                  const float *gate, void *out, int32_t *err_word,
+                                  void *stream);
+
+/* The whole forward pass: index map, RoPE on Q and K_loc, summaries, local
+ * branch, query-summary branch with the gate, all stream-ordered on `stream`.
+ * workspace: device buffer of at least pack3d_workspace_bytes(cfg) bytes,
+ * 256-byte aligned; its contents on entry do not matter.  err_word: device int32
+ * the caller zeroed before its first use (required). */
+pack3d_status pack3d_forward(const pack3d_config *cfg, const int32_t *coords, const void *q,
+                             const void *k_loc, const void *v_loc, const void *k_cmp,
+                             const void *v_cmp, const float *scores, const float *gate,
+                             void *out, void *workspace, size_t workspace_bytes,
+                             int32_t *err_word, void *stream);
+
+/* Synchronises `stream`, reads the device error word, resets it to 0 and maps
+ * it: COORD_RANGE/DUPLICATE -> PACK3D_ERR_NOT_PERMUTATION, TIMEOUT ->
+ * PACK3D_ERR_TIMEOUT, none -> PACK3D_OK.  A failed CUDA call -> PACK3D_ERR_CUDA. */
+pack3d_status pack3d_check_status(int32_t *err_word, void *stream);
+
+/* Static text for a status code. */
+const char *pack3d_status_string(pack3d_status s);
+
+/* Static text naming the compiled architecture and kernel paths. */
+const char *pack3d_backend_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PACK3D_H */

@@ -59,7 +59,7 @@ def _load():
         lib.orc_rotate.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_long]
         lib.orc_summaries.argtypes = [P, P, P, P, P, P, P, P]
         lib.orc_local_attn.argtypes = [P, P, P, P, P, P, P, ctypes.c_long, P]
-        lib.orc_summary_attn.argtypes = [P, P, P, P, ctypes.c_long, P, ctypes.c_long, P]
+        lib.orc_summary_attn.argtypes = [P, P, P, P, ctypes.c_long, ctypes.c_long, P]
         lib.orc_gate_mix.argtypes = [P, P, P, ctypes.c_long, P, P, P]
         _lib = lib
     return _lib
@@ -140,10 +140,16 @@ def _rows(s, rows):
 
 
 def local_attn(s, coords, g2p, q_rot, k_rot, v_loc, rows=None, scale=None) -> np.ndarray:
-    """Exact local attention over the clipped box window (Key design 3)."""
+    """Exact local attention over the clipped box window (Key design 3).
+
+    ``q_rot`` holds the rotated queries of ``rows`` (all rows if None), in that
+    order; ``k_rot`` and ``v_loc`` hold every token.
+    """
     r = _rows(s, rows)
     c, g = _i32(coords), _i32(g2p)
     qa, ka, va = as_f64(q_rot), as_f64(k_rot), as_f64(v_loc)
+    if qa.shape[0] != r.shape[0]:
+        raise ValueError("q_rot must hold exactly the sampled rows")
     o = np.empty((r.shape[0], s.Hq, s.d_h))
     cfg = _cfg(s, scale)
     _load().orc_local_attn(ctypes.byref(cfg), _ptr(c), _ptr(g), _ptr(qa), _ptr(ka), _ptr(va),
@@ -151,14 +157,13 @@ def local_attn(s, coords, g2p, q_rot, k_rot, v_loc, rows=None, scale=None) -> np
     return o
 
 
-def summary_attn(s, q_rot, k_sum, v_sum, rows=None, scale=None) -> np.ndarray:
-    """Every query against all M summaries with its own softmax (Key design 3)."""
-    r = _rows(s, rows)
+def summary_attn(s, q_rot, k_sum, v_sum, scale=None) -> np.ndarray:
+    """Each row of ``q_rot`` against all M summaries with its own softmax (Key design 3)."""
     qa, ka, va = as_f64(q_rot), as_f64(k_sum), as_f64(v_sum)
-    o = np.empty((r.shape[0], s.Hq, s.d_h))
+    o = np.empty((qa.shape[0], s.Hq, s.d_h))
     cfg = _cfg(s, scale)
     _load().orc_summary_attn(ctypes.byref(cfg), _ptr(qa), _ptr(ka), _ptr(va), ka.shape[0],
-                             _ptr(r), r.shape[0], _ptr(o))
+                             qa.shape[0], _ptr(o))
     return o
 
 
@@ -177,18 +182,29 @@ def forward(s, inputs: Dict, rows=None) -> Dict[str, np.ndarray]:
     """The whole operator, stage by stage in the pages' order, for ``rows`` (default all).
 
     ``inputs`` holds ``coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate`` in
-    packed order (numpy or torch; bf16 values are widened exactly).
+    packed order (numpy or torch; bf16 values are widened exactly).  Only the
+    sampled rows' queries are rotated and attended; keys, values and summaries
+    are built for every token.
     """
     st, g2p, mem = build_index(s, inputs["coords"])
     if st != 0:
         raise ValueError("coordinates are not a bijection onto the lattice (status %d)" % st)
-    coords = inputs["coords"]
-    qr = rotate(s, coords, inputs["q"])
+    coords = _i32(inputs["coords"])
+    r = _rows(s, rows)
+    q = inputs["q"]
+    if rows is not None:
+        q = q[_torch_index(r)] if hasattr(q, "detach") else np.asarray(q)[r]
+    qr = rotate(s, coords[r], q)
     klr = rotate(s, coords, inputs["k_loc"])
     ks, vs = summaries(s, coords, mem, inputs["k_cmp"], inputs["v_cmp"], inputs["scores"])
-    r = _rows(s, rows)
     ol = local_attn(s, coords, g2p, qr, klr, inputs["v_loc"], r)
-    oc = summary_attn(s, qr, ks, vs, r)
-    out = gate_mix(s, inputs["gate"], ol, oc, r)
+    oc = summary_attn(s, qr, ks, vs)
+    gate = inputs["gate"]
+    out = gate_mix(s, gate, ol, oc, r)
     return {"out": out, "o_loc": ol, "o_cmp": oc, "q_rot": qr, "k_rot": klr,
             "k_sum": ks, "v_sum": vs, "g2p": g2p, "members": mem, "rows": r}
+
+
+def _torch_index(r):
+    import torch
+    return torch.from_numpy(r)

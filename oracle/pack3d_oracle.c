@@ -180,9 +180,10 @@ void orc_summaries(const orc_cfg *c, const int32_t *coords, const int32_t *membe
 
 /* ---- exact local branch ------------------------------------------------ */
 
-/* For each sampled packed row i (rows[r]) and q head h, with g = kv head of h:
+/* For each sampled packed row i = rows[r] and q head h, with g = kv head of h:
  *   N(i) = tokens at lattice sites within the clipped box of radii (rz,ry,rx)
- *   l_j  = scale * <qr[i,h], klr[j,g]>,  o = sum_j softmax(l)_j vloc[j,g]. */
+ *   l_j  = scale * <qr[r,h], klr[j,g]>,  o[r,h] = sum_j softmax(l)_j vloc[j,g].
+ * qr holds the rotated queries of the sampled rows only, in sample order. */
 void orc_local_attn(const orc_cfg *c, const int32_t *coords, const int32_t *g2p,
                     const double *qr, const double *klr, const double *vloc,
                     const int64_t *rows, long nrows, double *oloc)
@@ -204,7 +205,7 @@ void orc_local_attn(const orc_cfg *c, const int32_t *coords, const int32_t *g2p,
                 }
         for (int h = 0; h < Hq; ++h) {
             int g = (int)(((long)h * Hkv) / Hq);
-            const double *q = qr + (i * Hq + h) * d;
+            const double *q = qr + (r * Hq + h) * d;
             double lmax = -INFINITY, den = 0.0;
             for (long k = 0; k < cnt; ++k) {
                 const double *kk = klr + (nb[k] * Hkv + g) * d;
@@ -230,18 +231,19 @@ void orc_local_attn(const orc_cfg *c, const int32_t *coords, const int32_t *g2p,
 
 /* ---- compressed branch: every query against all M summaries ------------ */
 
+/* o[r,h] = sum_j softmax_j(scale <qr[r,h], ksum[j,g]>) vsum[j,g] over all M
+ * summaries; qr holds the sampled rows' rotated queries in sample order. */
+
 void orc_summary_attn(const orc_cfg *c, const double *qr, const double *ksum,
-                      const double *vsum, long M, const int64_t *rows, long nrows,
-                      double *ocmp)
+                      const double *vsum, long M, long nrows, double *ocmp)
 {
     int d = c->dh, Hq = c->Hq, Hkv = c->Hkv;
 #pragma omp parallel for schedule(dynamic, 4)
     for (long r = 0; r < nrows; ++r) {
-        long i = rows[r];
         double *l = (double *)malloc(sizeof(double) * M);
         for (int h = 0; h < Hq; ++h) {
             int g = (int)(((long)h * Hkv) / Hq);
-            const double *q = qr + (i * Hq + h) * d;
+            const double *q = qr + (r * Hq + h) * d;
             double lmax = -INFINITY, den = 0.0;
             for (long j = 0; j < M; ++j) {
                 const double *kk = ksum + (j * Hkv + g) * d;

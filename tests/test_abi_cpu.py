@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point its header declares, validates configs and rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def p3():
+    import geometry_aware_local_b200 as p3
+    return p3
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(pack3d_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(p3):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(p3.lib, n), n
+    assert set(p3.ENTRY_POINTS) <= set(names)
+
+
+def test_default_config_matches_pages(p3):
+    c = p3.Config()
+    p3.lib.pack3d_default_config(ctypes.byref(c), 16, 128, 128)
+    assert (c.Hq, c.Hkv, c.d_h, c.m_z, c.m_y, c.m_x) == (8, 2, 64, 11, 11, 10)
+    assert (c.bz, c.by, c.bx, c.rz, c.ry, c.rx) == (1, 4, 4, 1, 3, 3)
+    assert c.rope_base == 10000.0 and abs(c.softmax_scale - 0.125) < 1e-9
+    assert p3.validate(c) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d_h", 128, 2), ("Hq", 6, 2), ("Hkv", 3, 2), ("W", 63, 2), ("bx", 0, 2), ("rz", -1, 2),
+    ("m_z", 20, 2), ("dtype", 7, 4), ("softmax_scale", 0.0, 1), ("flags", 0x100, 1), ("reserved0", 1, 1),
+    ("rope_base", -1.0, 1), ("Z", 0, 2),
+])
+def test_validate_rejects(p3, field, value, status):
+    c = p3.make_config(16, 64, 64)
+    setattr(c, field, value)
+    assert p3.validate(c) == status
+
+
+def test_table_limit_and_sizes(p3):
+    assert p3.validate(p3.make_config(16, 2048, 2048)) == 2   # rope tables too large for shared memory
+    for name in ("tiny", "65k", "262k", "1m"):
+        s = synth.CONFIGS[name]
+        c = p3.config_from_shape(s)
+        assert p3.validate(c) == 0
+        eb = 2 if s.dtype == "bf16" else 4
+        need = s.N * 4 + s.N * 4 + s.N * (s.Hq + s.Hkv) * 64 * eb + 2 * s.M * s.Hkv * 64 * eb + s.N * s.Hq * 64 * 4
+        ws = p3.workspace_bytes(c)
+        assert need <= ws <= need + 7 * 1024
+
+
+def test_host_errors_return_before_launch(p3):
+    c = p3.make_config(16, 64, 64)
+    lib = p3.lib
+    fake = 1 << 20          # never dereferenced: every call below fails validation first
+    bad = fake + 8
+    cfgp = ctypes.byref(c)
+    assert lib.pack3d_build_index(cfgp, None, fake, fake, fake, None) == 1
+    assert lib.pack3d_build_index(cfgp, bad, fake, fake, fake, None) == 3
+    assert lib.pack3d_rope(cfgp, fake, fake, fake, 0, None) == 1
+    assert lib.pack3d_rope(cfgp, fake, bad, fake, 8, None) == 3
+    assert lib.pack3d_summary_attn(cfgp, fake, fake, fake, None, fake, fake, None, None) == 1
+    ws = p3.workspace_bytes(c)
+    args = [fake] * 9
+    assert lib.pack3d_forward(cfgp, *args, fake, ws - 1, fake, None) == 6
+    assert lib.pack3d_forward(cfgp, *args, fake + 16, ws, fake, None) == 6
+    assert lib.pack3d_forward(cfgp, *args, fake, ws, None, None) == 1
+    assert lib.pack3d_check_status(None, None) == 1
+    for st in range(9):
+        assert lib.pack3d_status_string(st)
+    assert b"sm_100a" in lib.pack3d_backend_info()
+
+
+def test_binding_refuses_host_tensors(p3):
+    import torch
+    c = p3.make_config(4, 8, 8, Hq=2, Hkv=1, radius=(1, 1, 1), dtype="f32")
+    x = torch.zeros(256, 2, 64)
+    with pytest.raises(ValueError):
+        p3.rope(c, torch.zeros(256, 3, dtype=torch.int32), x, x, 2, stream=0)

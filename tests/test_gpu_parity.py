@@ -1,0 +1,192 @@
+"""GPU parity: every stage of the CUDA path against the float64 oracle.
+
+The CUDA path is called through the C ABI (ctypes binding); the oracle is the
+plain definition of each stage.  Both see the same seeded inputs (bf16 values
+widened exactly for the oracle).  Tolerances follow the operator's contract:
+max |gpu - oracle| <= 1e-4 * max |oracle| on float inputs and
+<= 2e-2 * max |oracle| on bf16 inputs with float accumulation; the index map and
+block membership are compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module")
+def p3(cuda_device):
+    import geometry_aware_local_b200 as p3
+    return p3
+
+
+def to_dev(inp):
+    return {k: (v.cuda() if k != "sites" else v) for k, v in inp.items()}
+
+
+def rel_err(gpu, ref):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return float(np.abs(gpu - ref).max() / max(np.abs(ref).max(), 1e-30))
+
+
+def run_stages(p3, s, d, flags=0):
+    """Every entry point in order; returns the intermediates as CPU tensors."""
+    cfg = p3.config_from_shape(s, flags)
+    dt = d["q"].dtype
+    dev = d["q"].device
+    err = torch.zeros(4, dtype=torch.int32, device=dev)
+    g2p = torch.empty(s.N, dtype=torch.int32, device=dev)
+    mem = torch.empty(s.M, s.v, dtype=torch.int32, device=dev)
+    p3.build_index(cfg, d["coords"], g2p, mem, err)
+    qr = torch.empty_like(d["q"])
+    kr = torch.empty_like(d["k_loc"])
+    p3.rope(cfg, d["coords"], d["q"], qr, s.Hq)
+    p3.rope(cfg, d["coords"], d["k_loc"], kr, s.Hkv)
+    ks = torch.empty(s.M, s.Hkv, s.d_h, dtype=dt, device=dev)
+    vs = torch.empty_like(ks)
+    p3.build_summaries(cfg, mem, d["k_cmp"], d["v_cmp"], d["scores"], ks, vs)
+    ol = torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device=dev)
+    p3.local_attn(cfg, g2p, qr, kr, d["v_loc"], ol)
+    oc = torch.empty_like(d["q"])
+    p3.summary_attn(cfg, qr, ks, vs, None, None, oc, err)
+    out = torch.empty_like(d["q"])
+    p3.summary_attn(cfg, qr, ks, vs, ol, d["gate"], out, err)
+    assert p3.check_status(err) == 0
+    return {k: v.cpu() for k, v in dict(g2p=g2p, members=mem, q_rot=qr, k_rot=kr, k_sum=ks, v_sum=vs,
+                                         o_loc=ol, o_cmp=oc, out=out).items()}
+
+
+def run_forward(p3, s, d, flags=0):
+    cfg = p3.config_from_shape(s, flags)
+    op = p3.Pack3D(cfg, d["q"].device)
+    out = op(d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"], d["gate"])
+    op.check()
+    return out.cpu()
+
+
+def small(**kw):
+    base = dict(Z=3, H=12, W=20, Hq=8, Hkv=2, rz=1, ry=3, rx=3, dtype="bf16", value_scale=0.125)
+    base.update(kw)
+    return synth.Pack3DShape(**base)
+
+
+# ------------------------------------------------------------ stage by stage -----
+
+STAGE_CASES = [
+    ("tiny", synth.CONFIGS["tiny"], "raster"),
+    ("tiny-f32-random", synth.CONFIGS["tiny"].replace(packing="random"), "random"),
+    ("ragged-bf16", small(), "random"),                      # W, H not multiples of the 8x8 brick
+    ("ragged-f32", small(dtype="f32", value_scale=1.0), "morton"),
+    ("g1", small(Hq=2, Hkv=2), "block"),
+    ("g2", small(Hq=4, Hkv=2, Z=2, H=8, W=8), "raster"),
+    ("g8", small(Hq=8, Hkv=1), "random"),
+    ("m-tail", small(Z=2, H=20, W=24), "morton"),              # M = 60: a partial summary tile
+    ("m-multi", small(Z=4, H=32, W=40), "random"),             # M = 320: several tiles + tail
+]
+
+
+@pytest.mark.parametrize("name,s,packing", STAGE_CASES, ids=[c[0] for c in STAGE_CASES])
+def test_stages_match_oracle(p3, name, s, packing):
+    inp = synth.make_inputs(s, packing, seed=3)
+    gpu = run_stages(p3, s, to_dev(inp))
+    ref = oracle.forward(s, inp)
+    tol = TOL[s.dtype]
+    assert np.array_equal(gpu["g2p"].numpy(), ref["g2p"])
+    assert np.array_equal(gpu["members"].numpy(), ref["members"])
+    for key in ("q_rot", "k_rot", "k_sum", "v_sum", "o_loc", "o_cmp", "out"):
+        e = rel_err(gpu[key].double().numpy(), ref[key])
+        assert e <= tol, f"{name}: {key} rel err {e:.3e} > {tol}"
+
+
+def test_simt_and_tensor_core_summary_paths_agree(p3):
+    s = small(Z=4, H=32, W=40)
+    d = to_dev(synth.make_inputs(s, "random", seed=4))
+    a = run_stages(p3, s, d)
+    b = run_stages(p3, s, d, flags=p3.FLAG_SIMT_SUMMARY)
+    assert rel_err(a["out"].double(), b["out"].double()) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------ index map ---------
+
+@pytest.mark.parametrize("packing", synth.PACKINGS)
+def test_index_map_bit_exact_65k(p3, packing):
+    s = synth.CONFIGS["65k"]
+    coords = torch.from_numpy(synth.coords_for(s, packing))
+    cfg = p3.config_from_shape(s)
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    g2p = torch.empty(s.N, dtype=torch.int32, device="cuda")
+    mem = torch.empty(s.M, s.v, dtype=torch.int32, device="cuda")
+    p3.build_index(cfg, coords.cuda(), g2p, mem, err)
+    assert p3.check_status(err) == 0
+    st, rg, rm = oracle.build_index(s, coords)
+    assert st == 0
+    assert np.array_equal(g2p.cpu().numpy(), rg) and np.array_equal(mem.cpu().numpy(), rm)
+
+
+def test_bad_coordinates_are_reported(p3):
+    s = small()
+    cfg = p3.config_from_shape(s)
+    coords = torch.from_numpy(synth.coords_for(s, "random")).clone()
+    coords[7] = coords[11]
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    g2p = torch.empty(s.N, dtype=torch.int32, device="cuda")
+    mem = torch.empty(s.M, s.v, dtype=torch.int32, device="cuda")
+    p3.build_index(cfg, coords.cuda(), g2p, mem, err)
+    assert p3.check_status(err) == 5
+    coords = torch.from_numpy(synth.coords_for(s, "raster")).clone()
+    coords[3, 2] = s.W
+    p3.build_index(cfg, coords.cuda(), g2p, mem, err)
+    assert p3.check_status(err) == 5
+    assert p3.check_status(err) == 0   # the word was cleared
+
+
+# ------------------------------------------------------------ whole forward -----
+
+def test_forward_tiny_full(p3):
+    s = synth.CONFIGS["tiny"]
+    inp = synth.make_inputs(s, s.packing, seed=0)
+    out = run_forward(p3, s, to_dev(inp))
+    ref = oracle.forward(s, inp)["out"]
+    assert rel_err(out.double().numpy(), ref) <= TOL["f32"]
+
+
+def test_forward_65k_sampled_rows(p3):
+    s = synth.CONFIGS["65k"]
+    inp = synth.make_inputs(s, s.packing, seed=0)
+    out = run_forward(p3, s, to_dev(inp))
+    rows = synth.sample_rows(s.N, 1024, seed=1)
+    ref = oracle.forward(s, inp, rows)["out"]
+    assert rel_err(out[rows].double().numpy(), ref) <= TOL["bf16"]
+
+
+def test_stress_packing_equivariance_65k(p3):
+    # Proposition 1: out under packing P equals P applied to the raster output.
+    s = synth.CONFIGS["stress"]
+    sv = synth.draw_site_values(s, 5)
+    base = synth.make_inputs(s, "raster", 5, sv)
+    ref = run_forward(p3, s, to_dev(base)).double()
+    rows = synth.sample_rows(s.N, 256, seed=2)
+    oref = oracle.forward(s, base, rows)["out"]
+    assert rel_err(ref[rows].numpy(), oref) <= TOL["bf16"]
+    for packing in ("morton", "block", "random"):
+        inp = synth.make_inputs(s, packing, 5, sv)
+        out = run_forward(p3, s, to_dev(inp)).double()
+        sites = inp["sites"]
+        assert rel_err(out.numpy(), ref[sites].numpy()) <= TOL["bf16"], packing
+
+
+@pytest.mark.parametrize("name", ["262k", "1m"])
+def test_forward_large_sampled_rows(p3, name):
+    s = synth.CONFIGS[name]
+    inp = synth.make_inputs(s, s.packing, seed=0)
+    out = run_forward(p3, s, to_dev(inp))
+    rows = synth.sample_rows(s.N, 128, seed=3)
+    ref = oracle.forward(s, inp, rows)["out"]
+    assert rel_err(out[rows].double().numpy(), ref) <= TOL["bf16"]
+    assert torch.isfinite(out.float()).all()
