@@ -25,7 +25,7 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: 
 
 ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
                 "pack3d_build_index", "pack3d_rope", "pack3d_build_summaries", "pack3d_local_attn",
-                "pack3d_summary_attn", "pack3d_forward", "pack3d_check_status",
+                "pack3d_summary_attn", "pack3d_forward", "pack3d_forward_noalloc", "pack3d_check_status",
                 "pack3d_status_string", "pack3d_backend_info")
 
 
@@ -75,6 +75,7 @@ def _load():
         "pack3d_local_attn": (ctypes.c_int, [C, P, P, P, P, P, P]),
         "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "pack3d_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
+        "pack3d_forward_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
         "pack3d_check_status": (ctypes.c_int, [P, P]),
         "pack3d_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "pack3d_backend_info": (ctypes.c_char_p, []),
@@ -184,6 +185,14 @@ def forward(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, works
     _check(lib.pack3d_forward(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc), _ptr(k_cmp),
                               _ptr(v_cmp), _ptr(scores), _ptr(gate), _ptr(out), _ptr(workspace), ws_bytes,
                               _ptr(err), _stream(stream)), "pack3d_forward")
+
+
+def forward_noalloc(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err=None, stream=None):
+    """pack3d_forward with the library's built-in scratch array instead of a workspace (for
+    callers that cannot allocate device memory); see include/pack3d.h for its limit and rules."""
+    _check(lib.pack3d_forward_noalloc(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc),
+                                      _ptr(k_cmp), _ptr(v_cmp), _ptr(scores), _ptr(gate), _ptr(out), _ptr(err),
+                                      _stream(stream)), "pack3d_forward_noalloc")
 
 
 def check_status(err, stream=None) -> int:

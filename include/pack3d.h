@@ -176,6 +176,36 @@ pack3d_status pack3d_forward(const pack3d_config *cfg, const int32_t *coords, co
                              void *out, void *workspace, size_t workspace_bytes,
                              int32_t *err_word, void *stream);
 
+/* Size of the scratch array compiled into the library for
+ * pack3d_forward_noalloc (32 MiB; held on every GPU that loads the library
+ * until the process exits). */
+#define PACK3D_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* pack3d_forward without a workspace, for callers that cannot allocate device
+ * memory: a plugin whose host application owns every allocation and passes in
+ * only input and output buffers, or a path where cudaMalloc is not allowed
+ * because it may synchronise the device.  The paper has no counterpart; this
+ * is a deployment convenience.  Same arguments, results and error behaviour as
+ * pack3d_forward, except:
+ *   - the scratch comes from a fixed array inside the library of
+ *     PACK3D_NOALLOC_SCRATCH_BYTES bytes; a config whose workspace
+ *     (pack3d_workspace_bytes) exceeds it is rejected with
+ *     PACK3D_ERR_WORKSPACE before anything is launched (about 9,900 bf16
+ *     tokens at Hq=8, Hkv=2);
+ *   - err_word may be NULL, in which case device-detected errors are not
+ *     reported;
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it: make
+ *     that first call before any stream capture;
+ *   - every call shares the one array, so calls whose work overlaps on the
+ *     GPU (e.g. on two streams) race; the caller must serialise them.
+ * Nothing is allocated or freed. */
+pack3d_status pack3d_forward_noalloc(const pack3d_config *cfg, const int32_t *coords,
+                                     const void *q, const void *k_loc, const void *v_loc,
+                                     const void *k_cmp, const void *v_cmp, const float *scores,
+                                     const float *gate, void *out, int32_t *err_word,
+                                     void *stream);
+
 /* Synchronises `stream`, reads the device error word, resets it to 0 and maps
  * it: COORD_RANGE/DUPLICATE -> PACK3D_ERR_NOT_PERMUTATION, TIMEOUT ->
  * PACK3D_ERR_TIMEOUT, none -> PACK3D_OK.  A failed CUDA call -> PACK3D_ERR_CUDA. */
