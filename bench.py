@@ -265,7 +265,7 @@ def run_ours(args, s):
         st |= lib.pack3d_build_summaries(cfgp, P(mem), P(d["k_cmp"]), P(d["v_cmp"]), P(d["scores"]), P(ks),
                                          P(vs), sh)
         ev[3].record(stream)
-        st |= lib.pack3d_local_attn(cfgp, P(g2p), P(qr), P(kr), P(d["v_loc"]), P(ol), sh)
+        st |= lib.pack3d_local_attn(cfgp, P(g2p), P(qr), P(kr), P(d["v_loc"]), P(ol), P(err), sh)
         ev[4].record(stream)
         st |= lib.pack3d_summary_attn(cfgp, P(qr), P(ks), P(vs), P(ol), P(d["gate"]), P(out), P(err), sh)
         ev[5].record(stream)

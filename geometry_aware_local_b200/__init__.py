@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libpack3d.so")
 
 F32, BF16 = 0, 1
 FLAG_SIMT_SUMMARY = 0x1
+FLAG_SIMT_LOCAL = 0x2
 DEVERR_COORD_RANGE, DEVERR_DUPLICATE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: "NOT_PERMUTATION",
@@ -72,7 +73,7 @@ def _load():
         "pack3d_build_index": (ctypes.c_int, [C, P, P, P, P, P]),
         "pack3d_rope": (ctypes.c_int, [C, P, P, P, I32, P]),
         "pack3d_build_summaries": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
-        "pack3d_local_attn": (ctypes.c_int, [C, P, P, P, P, P, P]),
+        "pack3d_local_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
         "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "pack3d_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
         "pack3d_forward_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
@@ -170,9 +171,9 @@ def build_summaries(cfg, members, k_cmp, v_cmp, scores, k_sum, v_sum, stream=Non
            "pack3d_build_summaries")
 
 
-def local_attn(cfg, g2p, q_rot, k_rot, v_loc, o_loc, stream=None):
+def local_attn(cfg, g2p, q_rot, k_rot, v_loc, o_loc, err=None, stream=None):
     _check(lib.pack3d_local_attn(ctypes.byref(cfg), _ptr(g2p), _ptr(q_rot), _ptr(k_rot), _ptr(v_loc),
-                                 _ptr(o_loc), _stream(stream)), "pack3d_local_attn")
+                                 _ptr(o_loc), _ptr(err), _stream(stream)), "pack3d_local_attn")
 
 
 def summary_attn(cfg, q_rot, k_sum, v_sum, o_loc, gate, out, err=None, stream=None):

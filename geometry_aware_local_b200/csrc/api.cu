@@ -119,7 +119,7 @@ pack3d_status pack3d_validate_config(const pack3d_config* c) {
   if (!(c->softmax_scale > 0.f) || !isfinite(c->softmax_scale)) return PACK3D_ERR_INVALID_ARG;
   const long long tab = (long long)c->Z * c->m_z + (long long)c->H * c->m_y + (long long)c->W * c->m_x;
   if (tab * 8 > kMaxTableBytes) return PACK3D_ERR_SHAPE;
-  if (c->flags & ~PACK3D_FLAG_SIMT_SUMMARY) return PACK3D_ERR_INVALID_ARG;
+  if (c->flags & ~(PACK3D_FLAG_SIMT_SUMMARY | PACK3D_FLAG_SIMT_LOCAL)) return PACK3D_ERR_INVALID_ARG;
   return PACK3D_OK;
 }
 
@@ -164,14 +164,16 @@ pack3d_status pack3d_build_summaries(const pack3d_config* cfg, const int32_t* me
 }
 
 pack3d_status pack3d_local_attn(const pack3d_config* cfg, const int32_t* g2p, const void* q_rot,
-                                const void* k_rot, const void* v_loc, float* o_loc, void* stream) {
+                                const void* k_rot, const void* v_loc, float* o_loc, int32_t* err_word,
+                                void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
   if (!g2p || !q_rot || !k_rot || !v_loc || !o_loc) return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(q_rot) || !aligned16(k_rot) || !aligned16(v_loc) || !aligned16(o_loc))
     return PACK3D_ERR_ALIGNMENT;
   const Shape s = make_shape(*cfg);
-  return cuda_status(launch_local_attn(s, cfg->dtype, g2p, q_rot, k_rot, v_loc, o_loc, (cudaStream_t)stream));
+  return cuda_status(
+      launch_local(s, cfg->dtype, cfg->flags, g2p, q_rot, k_rot, v_loc, o_loc, err_word, (cudaStream_t)stream));
 }
 
 pack3d_status pack3d_summary_attn(const pack3d_config* cfg, const void* q_rot, const void* k_sum,
@@ -213,7 +215,8 @@ pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, co
     e = launch_rope(s, cfg->dtype, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, cs);
   if (e == cudaSuccess)
     e = launch_summaries(s, cfg->dtype, w.members, k_cmp, v_cmp, scores, w.k_sum, w.v_sum, cs);
-  if (e == cudaSuccess) e = launch_local_attn(s, cfg->dtype, w.g2p, w.q_rot, w.k_rot, v_loc, w.o_loc, cs);
+  if (e == cudaSuccess)
+    e = launch_local(s, cfg->dtype, cfg->flags, w.g2p, w.q_rot, w.k_rot, v_loc, w.o_loc, err_word, cs);
   if (e == cudaSuccess) {
     if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
       e = launch_summary_attn_tc(s, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, err_word, cs);

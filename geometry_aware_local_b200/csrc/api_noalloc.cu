@@ -117,7 +117,7 @@ extern "C" pack3d_status pack3d_forward_noalloc(const pack3d_config* cfg, const 
   cudaError_t e = launch_build_index(s, coords, g2p, members, err_word, cs);
   if (e == cudaSuccess) e = launch_rope(s, cfg->dtype, coords, q, q_rot, s.Hq, k_loc, k_rot, s.Hkv, cs);
   if (e == cudaSuccess) e = launch_summaries(s, cfg->dtype, members, k_cmp, v_cmp, scores, k_sum, v_sum, cs);
-  if (e == cudaSuccess) e = launch_local_attn(s, cfg->dtype, g2p, q_rot, k_rot, v_loc, o_loc, cs);
+  if (e == cudaSuccess) e = launch_local(s, cfg->dtype, cfg->flags, g2p, q_rot, k_rot, v_loc, o_loc, err_word, cs);
   if (e == cudaSuccess) {
     if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
       e = launch_summary_attn_tc(s, q_rot, k_sum, v_sum, o_loc, gate, out, err_word, cs);

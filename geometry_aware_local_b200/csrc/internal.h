@@ -23,6 +23,16 @@ cudaError_t launch_summaries(const Shape& s, int dtype, const int32_t* members, 
 cudaError_t launch_local_attn(const Shape& s, int dtype, const int32_t* g2p, const void* qr,
                               const void* kr, const void* vl, float* oloc, cudaStream_t st);
 
+// Local attention on the best kernel for the shape: tcgen05 when supported
+// and not disabled by PACK3D_FLAG_SIMT_LOCAL, else CUDA cores.
+cudaError_t launch_local(const Shape& s, int dtype, int flags, const int32_t* g2p, const void* qr,
+                         const void* kr, const void* vl, float* oloc, int32_t* err, cudaStream_t st);
+
+// tcgen05 local attention (bf16, G = 4, rz = 1, ry <= 3, rx <= 3).
+bool local_attn_tc_supported(const Shape& s, int dtype);
+cudaError_t launch_local_attn_tc(const Shape& s, const int32_t* g2p, const void* qr, const void* kr,
+                                 const void* vl, float* oloc, int32_t* err, cudaStream_t st);
+
 // CUDA-core query x summary kernel (float, or bf16 on request).
 cudaError_t launch_summary_attn_simt(const Shape& s, int dtype, const void* qr, const void* ks,
                                      const void* vs, const float* oloc, const float* gate,

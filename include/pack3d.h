@@ -81,6 +81,8 @@ typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
 /* config.flags */
 #define PACK3D_FLAG_SIMT_SUMMARY  0x1  /* bf16: use the CUDA-core query x summary
                                           kernel instead of the tcgen05 one   */
+#define PACK3D_FLAG_SIMT_LOCAL    0x2  /* bf16: use the CUDA-core local-attention
+                                          kernel instead of the tcgen05 one   */
 
 typedef struct {
     int32_t Z, H, W;          /* lattice extents; N = Z*H*W tokens               */
@@ -146,10 +148,13 @@ pack3d_status pack3d_build_summaries(const pack3d_config *cfg, const int32_t *me
  * |dx|<=rx clipped at the volume (self included).  Cites: Key design 3 and
  * the summary's "local attention stays exact" contract.  q_rot, k_rot are
  * RoPE'd (stage 1); neighbours are reached through g2p, so any packing gives
- * the same result and no gathered neighbour tensor is formed. */
+ * the same result and no gathered neighbour tensor is formed.  bf16 with
+ * Hq/Hkv = 4, rz = 1, ry <= 3, rx <= 3 runs on tcgen05 tensor cores (float
+ * accumulation); every other shape on CUDA cores in float.  err_word
+ * (nullable) receives PACK3D_DEVERR_TIMEOUT if a pipeline wait gives up. */
 pack3d_status pack3d_local_attn(const pack3d_config *cfg, const int32_t *g2p,
                                 const void *q_rot, const void *k_rot, const void *v_loc,
-                                float *o_loc, void *stream);
+                                float *o_loc, int32_t *err_word, void *stream);
 
 /* Stages 4+5 - every query against all M summaries, then the gate.
  *   o_cmp[i,h] = sum_j softmax_j(scale <q_rot[i,h], k_sum[j,g]>) v_sum[j,g]

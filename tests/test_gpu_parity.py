@@ -52,7 +52,7 @@ def run_stages(p3, s, d, flags=0):
     vs = torch.empty_like(ks)
     p3.build_summaries(cfg, mem, d["k_cmp"], d["v_cmp"], d["scores"], ks, vs)
     ol = torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device=dev)
-    p3.local_attn(cfg, g2p, qr, kr, d["v_loc"], ol)
+    p3.local_attn(cfg, g2p, qr, kr, d["v_loc"], ol, err)
     oc = torch.empty_like(d["q"])
     p3.summary_attn(cfg, qr, ks, vs, None, None, oc, err)
     out = torch.empty_like(d["q"])
@@ -88,6 +88,9 @@ STAGE_CASES = [
     ("g8", small(Hq=8, Hkv=1), "random"),
     ("m-tail", small(Z=2, H=20, W=24), "morton"),              # M = 60: a partial summary tile
     ("m-multi", small(Z=4, H=32, W=40), "random"),             # M = 320: several tiles + tail
+    ("ragged-brick", small(Z=3, H=10, W=14, by=2, bx=2), "random"),  # 2x4x4 bricks cut in z, y and x
+    ("window-2x1", small(Z=5, H=12, W=12, ry=2, rx=1), "morton"),     # 8x6 halo planes (48 keys)
+    ("window-1x1x1", small(Z=4, H=8, W=8, ry=1, rx=1, rz=1), "block"),
 ]
 
 
@@ -110,6 +113,14 @@ def test_simt_and_tensor_core_summary_paths_agree(p3):
     a = run_stages(p3, s, d)
     b = run_stages(p3, s, d, flags=p3.FLAG_SIMT_SUMMARY)
     assert rel_err(a["out"].double(), b["out"].double()) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("shape", [small(Z=4, H=32, W=40), small(Z=3, H=10, W=14, by=2, bx=2)])
+def test_simt_and_tensor_core_local_paths_agree(p3, shape):
+    d = to_dev(synth.make_inputs(shape, "random", seed=6))
+    a = run_stages(p3, shape, d)
+    b = run_stages(p3, shape, d, flags=p3.FLAG_SIMT_LOCAL)
+    assert rel_err(a["o_loc"].double(), b["o_loc"].double()) <= TOL["bf16"]
 
 
 # ------------------------------------------------------------ index map ---------
