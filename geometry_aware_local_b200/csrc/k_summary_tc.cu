@@ -5,23 +5,25 @@
 // softmax so that no [N, M] score tensor exists; the overall framework's
 // tokenwise two-way softmax gate mixes the result with the local branch.
 //
-// Design (one CTA = two 128-row query tiles of one kv head, sharing every
-// summary tile):
-//   * rows are (token, q head) pairs of one kv group, G = Hq/Hkv heads per
-//     token, so a 128-row tile is 128/G tokens x G heads and one k~/v~ tile
-//     serves all of them;
-//   * warp 9 streams k~ and v~ tiles (128 summaries x 64 dims, bf16, 128-byte
-//     swizzle) through a 4-stage TMA ring; Q tiles are loaded once;
-//   * warp 8 issues tcgen05.mma: S = Q k~^T into tensor memory (128 x 128
-//     float) and O += P v~ with P read back from tensor memory (bf16);
-//   * warps 0-3 and 4-7 are two softmax warpgroups, one per query tile; each
-//     thread owns one row (one TMEM lane).  While one group turns S into P,
-//     the tensor core works on the other group's tiles (ping-pong).
-//   * O is rescaled lazily: the running maximum used for P only moves when a
-//     row's new maximum exceeds it by more than 2^8, so most tiles skip the
-//     rescale.  P values stay below 256, well inside bf16 range.
-// Tensor memory (512 columns): group w owns columns [256w, 256w+256): S at +0
-// (128 cols), P at +128 (64 cols of packed bf16 pairs), O at +192 (64 cols).
+// One CTA = two 128-row query tiles of one kv head sharing every summary tile
+// (rows are (token, q head) pairs of the kv group: 128/G tokens x G heads).
+//   * warp 9 streams k~ / v~ tiles (128 summaries x 64 dims, bf16, 128-byte
+//     swizzle) through a 4-stage TMA ring; the Q tiles are loaded once.
+//   * warp 8 issues tcgen05.mma: S = Q k~^T (M=128, N=128, K=64) into tensor
+//     memory and O += P v~ (M=128, N=64, K=128) with P read from tensor memory.
+//     It is event driven: S for tile j+1 is issued as soon as a group has read
+//     S_j into registers (not after PV_j), and PV_j as soon as P_j is written,
+//     whichever group gets there first.
+//   * warps 0-3 / 4-7 are two softmax warpgroups, one per query tile, thread =
+//     row = TMEM lane.  A group only waits for the tensor core when it writes
+//     P_{j+1} over P_j (PV_j must have finished reading it).
+// At d_h = 64 each exponential pairs with only 256 MMA flops, so the softmax
+// sets the pace: it uses packed f32x2 FMA/add, a three-input max and MUFU.ex2
+// (an FMA-pipe cubic for 2^x is kept for a share of the columns, off by
+// default: it costs more issue slots than it frees while the kernel is
+// latency bound).  O is rescaled lazily (only when a row maximum grows by more
+// than 2^8).  Tensor memory (512 columns), group w at 256w: S at +0 (128
+// columns), P (packed bf16) at +128 (64), O at +192 (64).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -31,20 +33,28 @@
 namespace pack3d {
 namespace {
 
-constexpr int kBM = 128;          // rows per query tile
-constexpr int kBN = 128;          // summaries per tile
+constexpr int kBM = 128;                      // rows per query tile
+constexpr int kBN = 128;                      // summaries per tile
 constexpr int kStages = 4;
-constexpr int kThreads = 320;     // 8 softmax warps + MMA warp + TMA warp
-constexpr int kTileBytes = kBM * kDh * 2;  // 16 KiB bf16 tile
-constexpr int kQOff = 0;                   // two Q tiles
-constexpr int kKVOff = 2 * kTileBytes;     // stage s: k~ at +0, v~ at +16 KiB
-constexpr int kBarOff = kKVOff + kStages * 2 * kTileBytes;
-constexpr int kNumBars = 2 * kStages + 1 + 2 + 2 + 2 + 2;
-constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + slack for 1 KiB alignment
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kThreads = 320;                 // 8 softmax warps + MMA warp + TMA warp
+constexpr int kQBytes = kBM * kDh * 2;        // 16 KiB
+constexpr int kKVBytes = kBN * kDh * 2;       // 16 KiB
+constexpr int kQOff = 0;
+constexpr int kStageOff = 2 * kQBytes;        // stage s: k~ at +0, v~ at +kKVBytes
+constexpr int kStageBytes = 2 * kKVBytes;
+constexpr int kBarOff = kStageOff + kStages * kStageBytes;
+// barriers: full[S], empty[S], qfull, then per group: s_full, s_free, p_full, p_free, o_final
+constexpr int kGroupBars = 5;
+constexpr int kNumBars = 2 * kStages + 1 + 2 * kGroupBars;
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
-constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kBM, kBN, false);
-constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kDh, true);
+constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kBM, kBN, false);      // S: N = kBN summaries
+constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kDh, true);     // O: N = 64 dims, v~ MN-major
+
+// Pair k of the 64 column pairs of a tile uses the FMA-pipe exponential when
+// this holds; the others use MUFU.ex2.
+__host__ __device__ constexpr bool poly_pair(int) { return false; }
 
 struct TcArgs {
   int M;             // summaries
@@ -57,6 +67,32 @@ struct TcArgs {
   __nv_bfloat16* out;
   int32_t* err;
 };
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe: x = n + f with n = rint(x) (added to the
+// exponent field) and f in [-1/2, 1/2], 2^f from a cubic fitted here by a
+// Remez exchange on the relative error (max 7.5e-5, well under bf16's 3.9e-3).
+// Inputs are clamped at -125 so the result stays a normal float (~1e-38 in
+// place of 0 for masked columns).
+__device__ __forceinline__ float2 exp2_poly(float2 x) {
+  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
+  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -73,10 +109,12 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   auto full = [&](int s) { return bar0 + 8 * s; };
   auto empty = [&](int s) { return bar0 + 8 * (kStages + s); };
   const uint32_t qfull = bar0 + 8 * (2 * kStages);
-  auto s_full = [&](int w) { return bar0 + 8 * (2 * kStages + 1 + w); };
-  auto s_free = [&](int w) { return bar0 + 8 * (2 * kStages + 3 + w); };
-  auto p_full = [&](int w) { return bar0 + 8 * (2 * kStages + 5 + w); };
-  auto o_final = [&](int w) { return bar0 + 8 * (2 * kStages + 7 + w); };
+  auto gbar = [&](int w, int i) { return bar0 + 8 * (2 * kStages + 1 + w * kGroupBars + i); };
+  auto s_full = [&](int w) { return gbar(w, 0); };
+  auto s_free = [&](int w) { return gbar(w, 1); };
+  auto p_full = [&](int w) { return gbar(w, 2); };
+  auto p_free = [&](int w) { return gbar(w, 3); };
+  auto o_final = [&](int w) { return gbar(w, 4); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -90,6 +128,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ptx::mbar_init(s_full(w), 1);
       ptx::mbar_init(s_free(w), kBM);
       ptx::mbar_init(p_full(w), kBM);
+      ptx::mbar_init(p_free(w), 1);
       ptx::mbar_init(o_final(w), 1);
     }
     *abort_flag = 0;
@@ -111,17 +150,17 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ptx::tma_prefetch(&tmK);
       ptx::tma_prefetch(&tmV);
       const int tok_per_tile = kBM / a.G;
-      ptx::mbar_expect_tx(qfull, 2 * kTileBytes);
+      ptx::mbar_expect_tx(qfull, 2 * kQBytes);
       ptx::tma_load_4d(sbase + kQOff, &tmQ, 0, 0, g, tile0 * tok_per_tile, qfull);
-      ptx::tma_load_4d(sbase + kQOff + kTileBytes, &tmQ, 0, 0, g, (tile0 + 1) * tok_per_tile, qfull);
+      ptx::tma_load_4d(sbase + kQOff + kQBytes, &tmQ, 0, 0, g, (tile0 + 1) * tok_per_tile, qfull);
       int issued = 0;
       for (int j = 0; j < T; ++j) {
         const int st = j % kStages;
         if (j >= kStages && !ptx::mbar_wait(empty(st), ((j / kStages) - 1) & 1, abort_flag)) break;
-        const uint32_t kdst = sbase + kKVOff + st * 2 * kTileBytes;
-        ptx::mbar_expect_tx(full(st), 2 * kTileBytes);
-        ptx::tma_load_3d(kdst, &tmK, 0, g, j * kBN, full(st));
-        ptx::tma_load_3d(kdst + kTileBytes, &tmV, 0, g, j * kBN, full(st));
+        const uint32_t dst = sbase + kStageOff + st * kStageBytes;
+        ptx::mbar_expect_tx(full(st), kStageBytes);
+        ptx::tma_load_3d(dst, &tmK, 0, g, j * kBN, full(st));
+        ptx::tma_load_3d(dst + kKVBytes, &tmV, 0, g, j * kBN, full(st));
         issued = j + 1;
       }
       if (*abort_flag) {
@@ -134,46 +173,70 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t qaddr[2] = {sbase + kQOff, sbase + kQOff + kTileBytes};
-      auto issue_s = [&](int w, int st) {
-        const uint32_t kaddr = sbase + kKVOff + st * 2 * kTileBytes;
+      auto issue_s = [&](int w, int j) {
+        const uint32_t kaddr = sbase + kStageOff + (j % kStages) * kStageBytes;
+        const uint32_t qaddr = sbase + kQOff + w * kQBytes;
 #pragma unroll
-        for (int kk = 0; kk < kDh / 16; ++kk) {
-          const uint64_t ad = ptx::smem_desc_sw128(qaddr[w] + kk * 32, 16, 1024);
-          const uint64_t bd = ptx::smem_desc_sw128(kaddr + kk * 32, 16, 1024);
-          ptx::mma_ss(tmem + w * 256, ad, bd, kIdescS, kk > 0);
-        }
+        for (int kk = 0; kk < kDh / 16; ++kk)
+          ptx::mma_ss(tmem + w * 256, ptx::smem_desc_sw128(qaddr + kk * 32, 16, 1024),
+                      ptx::smem_desc_sw128(kaddr + kk * 32, 16, 1024), kIdesc, kk > 0);
         ptx::tc_commit(s_full(w));
       };
-      auto issue_pv = [&](int w, int st, bool first) {
-        const uint32_t vaddr = sbase + kKVOff + st * 2 * kTileBytes + kTileBytes;
+      auto issue_pv = [&](int w, int j) {
+        const uint32_t vaddr = sbase + kStageOff + (j % kStages) * kStageBytes + kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024);
-          ptx::mma_ts(tmem + w * 256 + 192, tmem + w * 256 + 128 + kk * 8, bd, kIdescPV,
-                      (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          ptx::mma_ts(tmem + w * 256 + 192, tmem + w * 256 + 128 + kk * 8,
+                      ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        ptx::tc_commit(p_free(w));
+        if (j == T - 1) ptx::tc_commit(o_final(w));
       };
+      // Event loop.  Parities: s_free(w) completes once per tile a group has
+      // read, p_full(w) once per P tile written, full(s) once per load of
+      // stage s; none can run ahead of the issue it waits for, so a parity
+      // test never aliases an older phase.
       bool ok = ptx::mbar_wait(qfull, 0, abort_flag) && ptx::mbar_wait(full(0), 0, abort_flag);
+      int next_s[2] = {1, 1}, next_pv[2] = {0, 0}, released = 0;
       if (ok) {
         ptx::tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
       }
-      for (int j = 0; ok && j < T; ++j) {
-        const int st = j % kStages;
-        for (int w = 0; w < 2 && ok; ++w) {
-          if (!(ok = ptx::mbar_wait(p_full(w), j & 1, abort_flag))) break;
-          ptx::tc_fence_after();
-          issue_pv(w, st, j == 0);
-          if (j == T - 1) ptx::tc_commit(o_final(w));
-          if (w == 1) ptx::tc_commit(empty(st));
-          if (j + 1 < T) {
-            const int st1 = (j + 1) % kStages;
-            if (!(ok = ptx::mbar_wait(full(st1), ((j + 1) / kStages) & 1, abort_flag))) break;
-            if (!(ok = ptx::mbar_wait(s_free(w), j & 1, abort_flag))) break;
+      uint64_t t0 = ptx::globaltimer_ns();
+      uint32_t idle = 0;
+      while (ok && (next_pv[0] < T || next_pv[1] < T)) {
+        bool progressed = false;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int jp = next_pv[w];
+          if (jp < T && jp < next_s[w] && ptx::mbar_try_wait(p_full(w), jp & 1)) {
             ptx::tc_fence_after();
-            issue_s(w, st1);
+            issue_pv(w, jp);
+            next_pv[w] = jp + 1;
+            progressed = true;
+          }
+          const int js = next_s[w];
+          if (js < T && ptx::mbar_try_wait(s_free(w), (js - 1) & 1) &&
+              ptx::mbar_try_wait(full(js % kStages), (js / kStages) & 1)) {
+            ptx::tc_fence_after();
+            issue_s(w, js);
+            next_s[w] = js + 1;
+            progressed = true;
+          }
+        }
+        // A stage is free once both groups' PV of its tile were issued.
+        while (released < min(next_pv[0], next_pv[1])) {
+          ptx::tc_commit(empty(released % kStages));
+          ++released;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if ((++idle & 255) == 0) {
+          if (*abort_flag) ok = false;
+          else if (idle == 256) t0 = ptx::globaltimer_ns();
+          else if (ptx::globaltimer_ns() - t0 > 2000000000ull) {
+            *abort_flag = 1;
+            ok = false;
           }
         }
       }
@@ -189,7 +252,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const int w = warp >> 2;
     const int lane_base = (warp & 3) * 32;
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16) + w * 256;
-    const uint32_t tS = trow, tP = trow + 128, tO = trow + 192;
+    const uint32_t tO = trow + 192;
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -198,7 +261,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ptx::tc_fence_after();
       uint32_t sv[kBN];
 #pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) ptx::tmem_ld32(tS + 32 * q, sv + 32 * q);
+      for (int q = 0; q < kBN / 32; ++q) ptx::tmem_ld32(trow + 32 * q, sv + 32 * q);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       ptx::mbar_arrive(s_free(w));
@@ -208,10 +271,17 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         for (int k = 0; k < kBN; ++k)
           if (k >= lim) sv[k] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(sv[0]);
+      float m4[4];
 #pragma unroll
-      for (int k = 1; k < kBN; ++k) mx = fmaxf(mx, __uint_as_float(sv[k]));
-      const float mxs = mx * c;
+      for (int q = 0; q < 4; ++q) m4[q] = __uint_as_float(sv[q]);
+#pragma unroll
+      for (int k = 4; k < kBN - 4; k += 8)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          m4[q] = max3(m4[q], __uint_as_float(sv[k + 2 * q]), __uint_as_float(sv[k + 2 * q + 1]));
+      m4[0] = max3(m4[0], __uint_as_float(sv[kBN - 4]), __uint_as_float(sv[kBN - 3]));
+      m4[1] = max3(m4[1], __uint_as_float(sv[kBN - 2]), __uint_as_float(sv[kBN - 1]));
+      const float mxs = max3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
       // Lazy rescale: the maximum used for P moves only when this tile's row
       // maximum exceeds it by more than the threshold.
       float f = 1.f;
@@ -221,24 +291,27 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         f = ptx::ex2(m_used - mxs);
         m_used = mxs;
       }
-      const float nm = -m_used;
-      float rs = 0.f;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_used, -m_used);
+      float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[32 * q + 2 * k]), c, nm));
-          const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[32 * q + 2 * k + 1]), c, nm));
-          rs += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
+      for (int pair = 0; pair < kBN / 2; ++pair) {
+        const float2 x =
+            __ffma2_rn(make_float2(__uint_as_float(sv[2 * pair]), __uint_as_float(sv[2 * pair + 1])), c2, nm2);
+        float2 p;
+        if (poly_pair(pair)) {
+          p = exp2_poly(x);
+        } else {
+          p.x = ptx::ex2(x.x);
+          p.y = ptx::ex2(x.y);
         }
-        ptx::tmem_st16(tP + 16 * q, pk);
+        rs[pair & 1] = __fadd2_rn(rs[pair & 1], p);
+        pk[pair] = pack_bf16x2(p.x, p.y);
       }
+      // P_j overwrites P_{j-1}: PV_{j-1} must be done (that also makes O stable).
+      if (j > 0 && !(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(w), (j - 1) & 1, abort_flag)))) break;
+      ptx::tc_fence_after();
       if (__any_sync(0xffffffffu, f != 1.f)) {
-        // O holds P_0..P_{j-1} v~ relative to the old maximum.  PV_{j-1}
-        // completed before S_j was committed, and PV_j waits for p_full, so O
-        // is stable here.
         uint32_t r[32];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -249,32 +322,28 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           ptx::tmem_st32(tO + 32 * q, r);
         }
       }
-      l = l * f + rs;
+#pragma unroll
+      for (int q = 0; q < kBN / 32; ++q) ptx::tmem_st16(trow + 128 + 16 * q, pk + 16 * q);
+      l = l * f + (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(p_full(w));
     }
     if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final(w), 0, abort_flag))) {
       ptx::tc_fence_after();
-      float o[kDh];
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          ptx::tmem_ld32(tO + 32 * q, r);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[32 * q + k] = __uint_as_float(r[k]);
-        }
-      }
+      uint32_t r[2][32];
+      ptx::tmem_ld32(tO, r[0]);
+      ptx::tmem_ld32(tO + 32, r[1]);
+      ptx::tmem_wait_ld();
       const long grow = (long)(tile0 + w) * kBM + lane_base + lane;
       if (grow < a.rows) {
         const long tok = grow / a.G;
         const int h = g * a.G + (int)(grow % a.G);
         const size_t orow = (size_t)tok * a.Hq + h;
         const float inv = 1.f / l;
+        float o[kDh];
 #pragma unroll
-        for (int e = 0; e < kDh; ++e) o[e] *= inv;
+        for (int e = 0; e < kDh; ++e) o[e] = __uint_as_float(r[e >> 5][e & 31]) * inv;
         if (a.gate != nullptr) {
           const float g0 = __ldg(a.gate + 2 * orow), g1 = __ldg(a.gate + 2 * orow + 1);
           const float gm = fmaxf(g0, g1);
