@@ -5,25 +5,25 @@
 // softmax so that no [N, M] score tensor exists; the overall framework's
 // tokenwise two-way softmax gate mixes the result with the local branch.
 //
-// One CTA = two 128-row query tiles of one kv head sharing every summary tile
-// (rows are (token, q head) pairs of the kv group: 128/G tokens x G heads).
-//   * warp 9 streams k~ / v~ tiles (128 summaries x 64 dims, bf16, 128-byte
-//     swizzle) through a 4-stage TMA ring; the Q tiles are loaded once.
-//   * warp 8 issues tcgen05.mma: S = Q k~^T (M=128, N=128, K=64) into tensor
-//     memory and O += P v~ (M=128, N=64, K=128) with P read from tensor memory.
-//     It is event driven: S for tile j+1 is issued as soon as a group has read
-//     S_j into registers (not after PV_j), and PV_j as soon as P_j is written,
-//     whichever group gets there first.
-//   * warps 0-3 / 4-7 are two softmax warpgroups, one per query tile, thread =
-//     row = TMEM lane.  A group only waits for the tensor core when it writes
-//     P_{j+1} over P_j (PV_j must have finished reading it).
+// One CTA = kGroups 128-row query tiles of one kv head sharing every summary
+// tile (rows are (token, q head) pairs of the kv group: 128/G tokens x G
+// heads); the default is two tiles and 128-summary tiles.
+//   * the last warp streams k~ / v~ tiles (kBN summaries x 64 dims, bf16,
+//     128-byte swizzle) through a TMA ring; the Q tiles are loaded once.
+//   * the warp before it issues tcgen05.mma: S = Q k~^T (M=128, N=kBN, K=64)
+//     into tensor memory and O += P v~ (M=128, N=64, K=kBN) with P read from
+//     tensor memory.  It is event driven, probing its barriers without
+//     blocking: S for tile j+1 of a group is issued as soon as that group has
+//     read S_j into registers, PV_j as soon as P_j is written, whichever group
+//     gets there first.
+//   * warps 0 .. 4*kGroups-1 are the softmax warpgroups, one per query tile,
+//     thread = row = TMEM lane.
 // At d_h = 64 each exponential pairs with only 256 MMA flops, so the softmax
-// sets the pace: it uses packed f32x2 FMA/add, a three-input max and MUFU.ex2
-// (an FMA-pipe cubic for 2^x is kept for a share of the columns, off by
-// default: it costs more issue slots than it frees while the kernel is
-// latency bound).  O is rescaled lazily (only when a row maximum grows by more
-// than 2^8).  Tensor memory (512 columns), group w at 256w: S at +0 (128
-// columns), P (packed bf16) at +128 (64), O at +192 (64).
+// sets the pace: packed f32x2 FMA/add, a three-input max and MUFU.ex2, with a
+// fixed share of the exponentials optionally evaluated by a cubic on the FMA
+// pipe.  O is rescaled lazily (only when a row maximum grows by more than
+// 2^8).  Tensor memory (512 columns), group w at w*kGroupCols: S, P (packed
+// bf16), O.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -33,26 +33,41 @@
 namespace pack3d {
 namespace {
 
+// Compile-time shape of the pipeline: query tiles (softmax warpgroups) per
+// CTA and summaries per tile.  Tensor memory per group: S (kBN columns), P
+// (kBN/2), O (64), i.e. 256 columns for (2, 128) and 160 for (3, 64).
+#ifndef PACK3D_SA_GROUPS
+#define PACK3D_SA_GROUPS 2
+#endif
+#ifndef PACK3D_SA_BN
+#define PACK3D_SA_BN 128
+#endif
 constexpr int kBM = 128;                      // rows per query tile
-constexpr int kBN = 128;                      // summaries per tile
-constexpr int kStages = 4;
-constexpr int kThreads = 320;                 // 8 softmax warps + MMA warp + TMA warp
+constexpr int kBN = PACK3D_SA_BN;             // summaries per tile
+constexpr int kGroups = PACK3D_SA_GROUPS;     // query tiles (softmax warpgroups) per CTA
+constexpr int kMmaWarp = 4 * kGroups, kTmaWarp = kMmaWarp + 1;
+constexpr int kThreads = 32 * (kTmaWarp + 1);
+constexpr int kColS = 0, kColP = kBN, kColO = kBN + kBN / 2;
+constexpr int kGroupCols = kColO + kDh;       // tensor-memory columns per group
 constexpr int kQBytes = kBM * kDh * 2;        // 16 KiB
-constexpr int kKVBytes = kBN * kDh * 2;       // 16 KiB
+constexpr int kKVBytes = kBN * kDh * 2;
+constexpr int kStages = ((192 * 1024 - kGroups * kQBytes) / (2 * kKVBytes)) < 8
+                            ? ((192 * 1024 - kGroups * kQBytes) / (2 * kKVBytes)) : 8;
 constexpr int kQOff = 0;
-constexpr int kStageOff = 2 * kQBytes;        // stage s: k~ at +0, v~ at +kKVBytes
+constexpr int kStageOff = kGroups * kQBytes;  // stage s: k~ at +0, v~ at +kKVBytes
 constexpr int kStageBytes = 2 * kKVBytes;
 constexpr int kBarOff = kStageOff + kStages * kStageBytes;
 // barriers: full[S], empty[S], qfull, then per group: s_full, s_free, p_full, p_free, o_final
 constexpr int kGroupBars = 5;
-constexpr int kNumBars = 2 * kStages + 1 + 2 * kGroupBars;
+constexpr int kNumBars = 2 * kStages + 1 + kGroups * kGroupBars;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+static_assert(kGroups * kGroupCols <= 512, "tensor memory plan");
 
 constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kBM, kBN, false);      // S: N = kBN summaries
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kDh, true);     // O: N = 64 dims, v~ MN-major
 
-// Pair k of the 64 column pairs of a tile uses the FMA-pipe exponential when
+// Pair k of the 32 column pairs of a tile uses the FMA-pipe exponential when
 // this holds; the others use MUFU.ex2.
 __host__ __device__ constexpr bool poly_pair(int) { return false; }
 
@@ -101,7 +116,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
-  const int tile0 = blockIdx.x * 2;
+  const int tile0 = blockIdx.x * kGroups;
   const int T = (a.M + kBN - 1) / kBN;
 
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -124,7 +139,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ptx::mbar_init(empty(s), 1);
     }
     ptx::mbar_init(qfull, 1);
-    for (int w = 0; w < 2; ++w) {
+    for (int w = 0; w < kGroups; ++w) {
       ptx::mbar_init(s_full(w), 1);
       ptx::mbar_init(s_free(w), kBM);
       ptx::mbar_init(p_full(w), kBM);
@@ -134,7 +149,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 512);
     ptx::tmem_relinquish();
   }
@@ -143,16 +158,16 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 9) {
+  if (warp == kTmaWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       ptx::tma_prefetch(&tmQ);
       ptx::tma_prefetch(&tmK);
       ptx::tma_prefetch(&tmV);
       const int tok_per_tile = kBM / a.G;
-      ptx::mbar_expect_tx(qfull, 2 * kQBytes);
-      ptx::tma_load_4d(sbase + kQOff, &tmQ, 0, 0, g, tile0 * tok_per_tile, qfull);
-      ptx::tma_load_4d(sbase + kQOff + kQBytes, &tmQ, 0, 0, g, (tile0 + 1) * tok_per_tile, qfull);
+      ptx::mbar_expect_tx(qfull, kGroups * kQBytes);
+      for (int w = 0; w < kGroups; ++w)
+        ptx::tma_load_4d(sbase + kQOff + w * kQBytes, &tmQ, 0, 0, g, (tile0 + w) * tok_per_tile, qfull);
       int issued = 0;
       for (int j = 0; j < T; ++j) {
         const int st = j % kStages;
@@ -170,7 +185,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       }
     }
     __syncwarp();
-  } else if (warp == 8) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       auto issue_s = [&](int w, int j) {
@@ -178,7 +193,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const uint32_t qaddr = sbase + kQOff + w * kQBytes;
 #pragma unroll
         for (int kk = 0; kk < kDh / 16; ++kk)
-          ptx::mma_ss(tmem + w * 256, ptx::smem_desc_sw128(qaddr + kk * 32, 16, 1024),
+          ptx::mma_ss(tmem + w * kGroupCols + kColS, ptx::smem_desc_sw128(qaddr + kk * 32, 16, 1024),
                       ptx::smem_desc_sw128(kaddr + kk * 32, 16, 1024), kIdesc, kk > 0);
         ptx::tc_commit(s_full(w));
       };
@@ -186,7 +201,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const uint32_t vaddr = sbase + kStageOff + (j % kStages) * kStageBytes + kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          ptx::mma_ts(tmem + w * 256 + 192, tmem + w * 256 + 128 + kk * 8,
+          ptx::mma_ts(tmem + w * kGroupCols + kColO, tmem + w * kGroupCols + kColP + kk * 8,
                       ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
         ptx::tc_commit(p_free(w));
         if (j == T - 1) ptx::tc_commit(o_final(w));
@@ -196,36 +211,43 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       // stage s; none can run ahead of the issue it waits for, so a parity
       // test never aliases an older phase.
       bool ok = ptx::mbar_wait(qfull, 0, abort_flag) && ptx::mbar_wait(full(0), 0, abort_flag);
-      int next_s[2] = {1, 1}, next_pv[2] = {0, 0}, released = 0;
+      int next_s[kGroups], next_pv[kGroups], released = 0;
+      for (int w = 0; w < kGroups; ++w) {
+        next_s[w] = 1;
+        next_pv[w] = 0;
+      }
       if (ok) {
         ptx::tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
+        for (int w = 0; w < kGroups; ++w) issue_s(w, 0);
       }
       uint64_t t0 = ptx::globaltimer_ns();
       uint32_t idle = 0;
-      while (ok && (next_pv[0] < T || next_pv[1] < T)) {
+      int min_pv = 0;
+      while (ok && min_pv < T) {
         bool progressed = false;
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
+        for (int w = 0; w < kGroups; ++w) {
           const int jp = next_pv[w];
-          if (jp < T && jp < next_s[w] && ptx::mbar_try_wait(p_full(w), jp & 1)) {
+          if (jp < T && jp < next_s[w] && ptx::mbar_test_wait(p_full(w), jp & 1)) {
             ptx::tc_fence_after();
             issue_pv(w, jp);
             next_pv[w] = jp + 1;
             progressed = true;
           }
           const int js = next_s[w];
-          if (js < T && ptx::mbar_try_wait(s_free(w), (js - 1) & 1) &&
-              ptx::mbar_try_wait(full(js % kStages), (js / kStages) & 1)) {
+          if (js < T && ptx::mbar_test_wait(s_free(w), (js - 1) & 1) &&
+              ptx::mbar_test_wait(full(js % kStages), (js / kStages) & 1)) {
             ptx::tc_fence_after();
             issue_s(w, js);
             next_s[w] = js + 1;
             progressed = true;
           }
         }
-        // A stage is free once both groups' PV of its tile were issued.
-        while (released < min(next_pv[0], next_pv[1])) {
+        // A stage is free once every group's PV of its tile was issued.
+        min_pv = next_pv[0];
+#pragma unroll
+        for (int w = 1; w < kGroups; ++w) min_pv = min(min_pv, next_pv[w]);
+        while (released < min_pv) {
           ptx::tc_commit(empty(released % kStages));
           ++released;
         }
@@ -251,8 +273,8 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     // ---------------- softmax warpgroups ----------------
     const int w = warp >> 2;
     const int lane_base = (warp & 3) * 32;
-    const uint32_t trow = tmem + ((uint32_t)lane_base << 16) + w * 256;
-    const uint32_t tO = trow + 192;
+    const uint32_t trow = tmem + ((uint32_t)lane_base << 16) + w * kGroupCols;
+    const uint32_t tP = trow + kColP, tO = trow + kColO;
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -323,7 +345,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
       }
 #pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) ptx::tmem_st16(trow + 128 + 16 * q, pk + 16 * q);
+      for (int q = 0; q < kBN / 32; ++q) ptx::tmem_st16(tP + 16 * q, pk + 16 * q);
       l = l * f + (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -370,7 +392,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
@@ -434,7 +456,7 @@ cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* k
   a.out = (__nv_bfloat16*)out;
   a.err = err;
   const long tiles = (a.rows + kBM - 1) / kBM;
-  dim3 grid((unsigned)((tiles + 1) / 2), s.Hkv);
+  dim3 grid((unsigned)((tiles + kGroups - 1) / kGroups), s.Hkv);
   summary_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
