@@ -27,9 +27,18 @@ Shape make_shape(const pack3d_config& c) {
   s.scale = c.softmax_scale;
   s.scale_log2 = (float)((double)c.softmax_scale * 1.4426950408889634);
   const int m[3] = {c.m_z, c.m_y, c.m_x};
-  int p = 0;
+  const int ext[3] = {c.Z, c.H, c.W};
+  int p = 0, off = 0;
   for (int a = 0; a < 3; ++a)
-    for (int r = 0; r < m[a]; ++r) s.omega[p++] = pow(c.rope_base, -(double)r / (double)m[a]);
+    for (int r = 0; r < m[a]; ++r) {
+      s.omega[p] = pow(c.rope_base, -(double)r / (double)m[a]);
+      s.pair_axis[p] = a;
+      s.pair_off[p] = off;
+      off += ext[a];
+      ++p;
+    }
+  s.npairs = p;
+  for (; p < kMaxPairs; ++p) s.pair_axis[p] = 3;
   return s;
 }
 

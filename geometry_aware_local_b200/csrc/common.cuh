@@ -25,9 +25,12 @@ struct Shape {
   int rz, ry, rx;                 // window radii
   int mz, my, mx;                 // rotary planes per axis
   int tab_entries;                // Z*mz + H*my + W*mx
+  int npairs;                     // mz + my + mx rotated planes
   float scale;                    // softmax scale
   float scale_log2;               // scale * log2(e)
   double omega[kMaxPairs];        // per rotary plane p: base^(-r/m_axis), 0 if unused
+  int pair_axis[kMaxPairs];       // 0 = z, 1 = y, 2 = x, 3 = untouched
+  int pair_off[kMaxPairs];        // first table entry of plane p
 };
 
 Shape make_shape(const pack3d_config& c);
@@ -74,10 +77,11 @@ __device__ __forceinline__ void stg16(void* p, const uint4& v) {
 }
 
 // ---- axial RoPE tables -----------------------------------------------------
-// Table layout (float2 = cos, sin): [z*mz + r] for the z planes, then
-// [Z*mz + y*my + r] for y, then [Z*mz + H*my + x*mx + r] for x.  The angle
-// omega * c is formed in double and reduced modulo 2*pi in double (a two-part
-// 2*pi, Cody-Waite style), so the float sincos sees an argument in [-pi, pi].
+// Table layout (float2 = cos, sin): plane p owns the contiguous entries
+// [pair_off[p], pair_off[p] + extent of its axis), one per coordinate value.
+// The angle omega * c is formed in double and reduced modulo 2*pi in double
+// (a two-part 2*pi, Cody-Waite style), so the float sincos sees an argument in
+// [-pi, pi].
 
 __device__ __forceinline__ float2 rope_cos_sin(double angle) {
   const double kTwoPiHi = 6.283185307179586;       // nearest double to 2*pi
@@ -90,44 +94,49 @@ __device__ __forceinline__ float2 rope_cos_sin(double angle) {
   return make_float2(c, s);
 }
 
+__device__ __forceinline__ int axis_extent(const Shape& s, int axis) {
+  return axis == 0 ? s.Z : (axis == 1 ? s.H : s.W);
+}
+
+// All threads fill the table together: entry e belongs to the last plane whose
+// first entry is <= e (a binary search over the increasing pair_off).
 __device__ __forceinline__ void build_rope_table(float2* tab, const Shape& s) {
   for (int e = threadIdx.x; e < s.tab_entries; e += blockDim.x) {
-    int coord, p;
-    if (e < s.Z * s.mz) {
-      coord = e / s.mz; p = e % s.mz;
-    } else if (e < s.Z * s.mz + s.H * s.my) {
-      int f = e - s.Z * s.mz;
-      coord = f / s.my; p = s.mz + f % s.my;
-    } else {
-      int f = e - s.Z * s.mz - s.H * s.my;
-      coord = f / s.mx; p = s.mz + s.my + f % s.mx;
-    }
-    tab[e] = rope_cos_sin(s.omega[p] * (double)coord);
-  }
-}
-
-// cos/sin of rotary plane p at coordinate (z, y, x); identity past the planes.
-__device__ __forceinline__ float2 rope_lookup(const float2* tab, const Shape& s, int p, int z,
-                                              int y, int x) {
-  if (p < s.mz) return tab[z * s.mz + p];
-  if (p < s.mz + s.my) return tab[s.Z * s.mz + y * s.my + (p - s.mz)];
-  if (p < s.mz + s.my + s.mx) return tab[s.Z * s.mz + s.H * s.my + x * s.mx + (p - s.mz - s.my)];
-  return make_float2(1.f, 0.f);
-}
-
-// Rotates the planes held by one chunk: elements f[0..n) are dims
-// [first_dim, first_dim + n), n even.
-template <int NE>
-__device__ __forceinline__ void rotate_chunk(float* f, int first_dim, const float2* tab,
-                                             const Shape& s, int z, int y, int x) {
+    int p = 0;
 #pragma unroll
-  for (int k = 0; k < NE; k += 2) {
-    float2 cs = rope_lookup(tab, s, (first_dim + k) >> 1, z, y, x);
-    float x0 = f[k], x1 = f[k + 1];
-    f[k] = x0 * cs.x - x1 * cs.y;
-    f[k + 1] = x0 * cs.y + x1 * cs.x;
+    for (int step = kMaxPairs / 2; step > 0; step >>= 1)
+      if (p + step < s.npairs && s.pair_off[p + step] <= e) p += step;
+    tab[e] = rope_cos_sin(s.omega[p] * (double)(e - s.pair_off[p]));
   }
 }
+
+// Per-thread lookup constants for the NP planes starting at plane p0 (the
+// planes one 16-byte chunk covers): axis and first table entry.
+template <int NP>
+struct PlaneLut {
+  int axis[NP];
+  int off[NP];
+  __device__ __forceinline__ void init(const Shape& s, int p0) {
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+      const int p = p0 + k;
+      axis[k] = p < s.npairs ? s.pair_axis[p] : 3;
+      off[k] = p < s.npairs ? s.pair_off[p] : 0;
+    }
+  }
+  // Rotates the 2*NP values f (planes p0 .. p0+NP-1) at coordinate (z, y, x).
+  __device__ __forceinline__ void rotate(float* f, const float2* tab, int z, int y, int x) const {
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+      if (axis[k] == 3) continue;
+      const int cval = axis[k] == 0 ? z : (axis[k] == 1 ? y : x);
+      const float2 cs = tab[off[k] + cval];
+      const float x0 = f[2 * k], x1 = f[2 * k + 1];
+      f[2 * k] = x0 * cs.x - x1 * cs.y;
+      f[2 * k + 1] = x0 * cs.y + x1 * cs.x;
+    }
+  }
+};
 
 __device__ __forceinline__ void set_err(int32_t* err, int bits) {
   if (err) atomicOr(err, bits);

@@ -198,8 +198,7 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
       uint32_t sv[kMaxKeys];
 #pragma unroll
       for (int q = 0; q < kMaxKeys / 16; ++q)
-        if (q * 16 < a.NP) ptx::tmem_ld16(tS + 16 * q, sv + 16 * q);
-      ptx::tmem_wait_ld();
+        if (q * 16 < a.NP) ptx::tmem_ld16_sync(tS + 16 * q, sv + 16 * q);
       float mx = -INFINITY;
 #pragma unroll
       for (int k = 0; k < kMaxKeys; ++k) {
@@ -237,8 +236,7 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
         uint32_t r[32];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          ptx::tmem_ld32(tO + 32 * q, r);
-          ptx::tmem_wait_ld();
+          ptx::tmem_ld32_sync(tO + 32 * q, r);
 #pragma unroll
           for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
           ptx::tmem_st32(tO + 32 * q, r);
@@ -272,9 +270,7 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
 
   if (ok) {
     uint32_t r[2][32];
-    ptx::tmem_ld32(tO, r[0]);
-    ptx::tmem_ld32(tO + 32, r[1]);
-    ptx::tmem_wait_ld();
+    ptx::tmem_ld64_sync(tO, &r[0][0]);
     if (qi >= 0) {
       const float inv = 1.f / l;
       float4* o = reinterpret_cast<float4*>(a.oloc + ((size_t)qi * a.Hq + h) * kDh);

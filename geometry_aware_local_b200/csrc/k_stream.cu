@@ -52,7 +52,67 @@ cudaError_t launch_build_index(const Shape& s, const int32_t* coords, int32_t* g
 constexpr int kRopeThreads = 256;
 constexpr int kRopeUnroll = 4;
 
-// Rotates up to two tensors (e.g. Q and K_loc) in one launch; y may alias x.
+// One tensor of the RoPE launch.  Each thread keeps one 16-byte chunk position
+// ct of a token row (so the planes it rotates, and their table entries, are
+// fixed) and walks the tokens; the threads of a block cover whole contiguous
+// token rows, so every load and store is fully coalesced.
+template <typename T>
+__device__ __forceinline__ void rope_tensor(const Shape& s, const float2* tab, const int32_t* __restrict__ coords,
+                                            const T* x, T* y, int heads) {
+  constexpr int NE = Elem<T>::kPerChunk;
+  constexpr int CPR = kDh / NE;  // chunks per head row
+  constexpr int NP = NE / 2;     // rotary planes per chunk
+  const int CPT = heads * CPR;   // chunks per token
+  if (CPT <= (int)blockDim.x) {
+    const int tpb = blockDim.x / CPT;
+    const int tl = threadIdx.x / CPT, ct = threadIdx.x % CPT;
+    if (tl >= tpb) return;
+    PlaneLut<NP> lut;
+    lut.init(s, (ct % CPR) * NP);
+    const int tstride = gridDim.x * tpb;
+    for (int t0 = blockIdx.x * tpb + tl; t0 < s.N; t0 += kRopeUnroll * tstride) {
+      uint4 u[kRopeUnroll];
+      int cz[kRopeUnroll], cy[kRopeUnroll], cx[kRopeUnroll];
+#pragma unroll
+      for (int k = 0; k < kRopeUnroll; ++k) {
+        const int t = t0 + k * tstride;
+        if (t < s.N) {
+          u[k] = *reinterpret_cast<const uint4*>(x + ((size_t)t * CPT + ct) * NE);
+          // Clamped so that a bad coordinate (reported by the index map) cannot
+          // index outside the tables.
+          cz[k] = min(max(__ldg(coords + 3 * t), 0), s.Z - 1);
+          cy[k] = min(max(__ldg(coords + 3 * t + 1), 0), s.H - 1);
+          cx[k] = min(max(__ldg(coords + 3 * t + 2), 0), s.W - 1);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kRopeUnroll; ++k) {
+        const int t = t0 + k * tstride;
+        if (t >= s.N) continue;
+        float f[NE];
+        chunk_to_float(u[k], f, T());
+        lut.rotate(f, tab, cz[k], cy[k], cx[k]);
+        stg16(y + ((size_t)t * CPT + ct) * NE, float_to_chunk(f, T()));
+      }
+    }
+  } else {
+    // Rows wider than a block: plain strided walk over all chunks.
+    const unsigned total = (unsigned)s.N * CPT;
+    for (unsigned c = blockIdx.x * blockDim.x + threadIdx.x; c < total; c += gridDim.x * blockDim.x) {
+      const unsigned t = c / CPT;
+      PlaneLut<NP> lut;
+      lut.init(s, (int)(c % CPR) * NP);
+      float f[NE];
+      chunk_to_float(*reinterpret_cast<const uint4*>(x + (size_t)c * NE), f, T());
+      lut.rotate(f, tab, min(max(__ldg(coords + 3 * t), 0), s.Z - 1), min(max(__ldg(coords + 3 * t + 1), 0), s.H - 1),
+                 min(max(__ldg(coords + 3 * t + 2), 0), s.W - 1));
+      stg16(y + (size_t)c * NE, float_to_chunk(f, T()));
+    }
+  }
+}
+
+// Rotates up to two tensors (e.g. Q and K_loc) in one launch; y may alias x
+// (each chunk is read and written by the same thread).
 template <typename T>
 __global__ void __launch_bounds__(kRopeThreads) rope_kernel(Shape s, const int32_t* __restrict__ coords,
                                                             const T* x0, T* y0, int h0,
@@ -60,48 +120,14 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(Shape s, const int32
   extern __shared__ float2 tab[];
   build_rope_table(tab, s);
   __syncthreads();
-  constexpr int NE = Elem<T>::kPerChunk;
-  constexpr int CPR = kDh / NE;  // chunks per head row
-  const unsigned stride = gridDim.x * blockDim.x;
-  for (int t = 0; t < 2; ++t) {
-    const T* x = t ? x1 : x0;
-    T* y = t ? y1 : y0;
-    const int heads = t ? h1 : h0;
-    if (x == nullptr) continue;
-    const unsigned per_tok = (unsigned)heads * CPR;
-    const unsigned total = (unsigned)s.N * per_tok;
-    for (unsigned base = blockIdx.x * blockDim.x + threadIdx.x; base < total;
-         base += kRopeUnroll * stride) {
-      uint4 u[kRopeUnroll];
-#pragma unroll
-      for (int k = 0; k < kRopeUnroll; ++k) {
-        const unsigned c = base + k * stride;
-        if (c < total) u[k] = *reinterpret_cast<const uint4*>(x + (size_t)c * NE);
-      }
-#pragma unroll
-      for (int k = 0; k < kRopeUnroll; ++k) {
-        const unsigned c = base + k * stride;
-        if (c >= total) continue;
-        const unsigned tok = c / per_tok;
-        const int part = c % CPR;
-        // Clamped so that a bad coordinate (reported by the index map) cannot
-        // index outside the tables.
-        const int cz = min(max(__ldg(coords + 3 * tok), 0), s.Z - 1);
-        const int cy = min(max(__ldg(coords + 3 * tok + 1), 0), s.H - 1);
-        const int cx = min(max(__ldg(coords + 3 * tok + 2), 0), s.W - 1);
-        float f[NE];
-        chunk_to_float(u[k], f, T());
-        rotate_chunk<NE>(f, part * NE, tab, s, cz, cy, cx);
-        stg16(y + (size_t)c * NE, float_to_chunk(f, T()));
-      }
-    }
-  }
+  rope_tensor(s, tab, coords, x0, y0, h0);
+  if (x1 != nullptr) rope_tensor(s, tab, coords, x1, y1, h1);
 }
 
 static int rope_grid(const Shape& s, int heads, int chunk_elems) {
   long chunks = (long)s.N * heads * (kDh / chunk_elems);
   long want = (chunks + kRopeThreads * kRopeUnroll - 1) / (kRopeThreads * kRopeUnroll);
-  return (int)max(1L, min(want, 148L * 6));
+  return (int)max(1L, min(want, 148L * 4));
 }
 
 template <typename T>
@@ -127,11 +153,93 @@ cudaError_t launch_rope(const Shape& s, int dtype, const int32_t* coords, const 
 
 constexpr int kSumThreads = 256;
 
+// Fast path (block volume <= U): a unit of U = 2 * (kDh / NE) lanes owns one
+// (block j, kv head g).  Lane t first holds member t: it loads that member's
+// score once, and the unit's softmax weights come from shuffle reductions.
+// Then lane l accumulates one 16-byte chunk of k~ (lanes 0 .. U/2-1, rotating
+// each member row before pooling) or of v~ (the other half) over the members,
+// with every member row read as a whole 128-byte line by U/2 lanes and four
+// rows in flight per lane.  V > 0 fixes the block volume at compile time;
+// V = 0 reads it from the shape.
+template <typename T, int V>
+__global__ void __launch_bounds__(kSumThreads) summaries_kernel(
+    Shape s, const int32_t* __restrict__ members, const T* __restrict__ kc,
+    const T* __restrict__ vc, const float* __restrict__ scores, T* __restrict__ ks,
+    T* __restrict__ vs) {
+  extern __shared__ float2 tab[];
+  build_rope_table(tab, s);
+  __syncthreads();
+  constexpr int NE = Elem<T>::kPerChunk;
+  constexpr int LPT = kDh / NE;          // lanes per tensor row
+  constexpr int U = 2 * LPT;             // lanes per unit (16 bf16, 32 float)
+  constexpr int NP = NE / 2;
+  constexpr int VMAX = V > 0 ? V : U;
+  const int vol = V > 0 ? V : s.v;
+  const int lu = threadIdx.x % U;
+  const int is_v = lu >= LPT;
+  const int part = lu % LPT;
+  const unsigned umask = U == 32 ? 0xffffffffu : (0xffffu << (threadIdx.x & 16));
+  PlaneLut<NP> lut;
+  lut.init(s, part * NP);
+  const long units = (long)s.M * s.Hkv;
+  const long ustride = (long)gridDim.x * (kSumThreads / U);
+  const T* src = is_v ? vc : kc;
+  for (long u = (long)blockIdx.x * (kSumThreads / U) + threadIdx.x / U; u < units; u += ustride) {
+    const int g = (int)(u % s.Hkv);
+    const int j = (int)(u / s.Hkv);
+    // a_{j,t}: softmax over the block's members of their scores for kv head g.
+    const int m = lu < vol ? __ldg(members + (size_t)j * vol + lu) : -1;
+    const float sc = m >= 0 ? __ldg(scores + (size_t)m * s.Hkv + g) : -INFINITY;
+    float mx = sc;
+#pragma unroll
+    for (int o = U / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(umask, mx, o, U));
+    const float e = m >= 0 ? expf(sc - mx) : 0.f;
+    float den = e;
+#pragma unroll
+    for (int o = U / 2; o > 0; o >>= 1) den += __shfl_xor_sync(umask, den, o, U);
+    const float a = den > 0.f ? e / den : 0.f;
+    const int jx = j % s.nbx, jy = (j / s.nbx) % s.nby, jz = j / (s.nbx * s.nby);
+    float acc[NE];
+#pragma unroll
+    for (int k = 0; k < NE; ++k) acc[k] = 0.f;
+    // Members in batches of kBatch rows in flight per lane.
+    constexpr int kBatch = 4;
+#pragma unroll 1
+    for (int t0 = 0; t0 < VMAX; t0 += kBatch) {
+      uint4 rowc[kBatch];
+      int mts[kBatch];
+      float ats[kBatch];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int t = t0 + b;
+        mts[b] = __shfl_sync(umask, m, t & (U - 1), U);
+        ats[b] = __shfl_sync(umask, a, t & (U - 1), U);
+        if (t < vol && mts[b] >= 0) rowc[b] = ldg16(src + ((size_t)mts[b] * s.Hkv + g) * kDh + part * NE);
+      }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int t = t0 + b;
+        if (t >= vol || mts[b] < 0) continue;
+        float f[NE];
+        chunk_to_float(rowc[b], f, T());
+        if (!is_v) {
+          const int tz = t / (s.by * s.bx), ty = (t / s.bx) % s.by, tx = t % s.bx;
+          lut.rotate(f, tab, jz * s.bz + tz, jy * s.by + ty, jx * s.bx + tx);
+        }
+#pragma unroll
+        for (int k = 0; k < NE; ++k) acc[k] = fmaf(ats[b], f[k], acc[k]);
+      }
+    }
+    T* dst = is_v ? vs : ks;
+    stg16(dst + ((size_t)j * s.Hkv + g) * kDh + part * NE, float_to_chunk(acc, T()));
+  }
+}
+
 // A unit is (block j, kv head g, K or V); kDh/NE lanes share a unit, each lane
 // owning one 16-byte chunk of the 64 dims.  Member t of block j sits at the
 // t-th raster site of the block, so its coordinates follow from (j, t).
 template <typename T>
-__global__ void __launch_bounds__(kSumThreads) summaries_kernel(
+__global__ void __launch_bounds__(kSumThreads) summaries_generic_kernel(
     Shape s, const int32_t* __restrict__ members, const T* __restrict__ kc,
     const T* __restrict__ vc, const float* __restrict__ scores, T* __restrict__ ks,
     T* __restrict__ vs) {
@@ -180,7 +288,9 @@ __global__ void __launch_bounds__(kSumThreads) summaries_kernel(
       chunk_to_float(c, f, T());
       if (!is_v) {
         const int tz = t / (s.by * s.bx), ty = (t / s.bx) % s.by, tx = t % s.bx;
-        rotate_chunk<NE>(f, part * NE, tab, s, jz * s.bz + tz, jy * s.by + ty, jx * s.bx + tx);
+        PlaneLut<NE / 2> lut;
+        lut.init(s, part * (NE / 2));
+        lut.rotate(f, tab, jz * s.bz + tz, jy * s.by + ty, jx * s.bx + tx);
       }
 #pragma unroll
       for (int k = 0; k < NE; ++k) acc[k] = fmaf(a, f[k], acc[k]);
@@ -194,15 +304,26 @@ template <typename T>
 static cudaError_t summaries_t(const Shape& s, const int32_t* members, const void* kc, const void* vc,
                                const float* scores, void* ks, void* vs, cudaStream_t st) {
   const size_t smem = (size_t)s.tab_entries * sizeof(float2);
-  cudaError_t e = cudaFuncSetAttribute(summaries_kernel<T>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int U = 2 * (kDh / Elem<T>::kPerChunk);
+  if (s.v <= U) {
+    auto kern = s.v == 16 ? summaries_kernel<T, 16> : summaries_kernel<T, 0>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long units = (long)s.M * s.Hkv;
+    const long per_cta = kSumThreads / U;
+    const int grid = (int)max(1L, min((units + per_cta - 1) / per_cta, 148L * 8));
+    kern<<<grid, kSumThreads, smem, st>>>(s, members, (const T*)kc, (const T*)vc, scores, (T*)ks, (T*)vs);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaFuncSetAttribute(summaries_generic_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   const int lpu = kDh / Elem<T>::kPerChunk;
   const long units = (long)s.M * s.Hkv * 2;
   const long per_cta = kSumThreads / lpu;
   const int grid = (int)max(1L, min((units + per_cta - 1) / per_cta, 148L * 8));
-  summaries_kernel<T><<<grid, kSumThreads, smem, st>>>(s, members, (const T*)kc, (const T*)vc, scores,
-                                                        (T*)ks, (T*)vs);
+  summaries_generic_kernel<T><<<grid, kSumThreads, smem, st>>>(s, members, (const T*)kc, (const T*)vc, scores,
+                                                                (T*)ks, (T*)vs);
   return cudaGetLastError();
 }
 

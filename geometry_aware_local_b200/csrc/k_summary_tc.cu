@@ -10,12 +10,10 @@
 // heads); the default is two tiles and 128-summary tiles.
 //   * the last warp streams k~ / v~ tiles (kBN summaries x 64 dims, bf16,
 //     128-byte swizzle) through a TMA ring; the Q tiles are loaded once.
-//   * the warp before it issues tcgen05.mma: S = Q k~^T (M=128, N=kBN, K=64)
-//     into tensor memory and O += P v~ (M=128, N=64, K=kBN) with P read from
-//     tensor memory.  It is event driven, probing its barriers without
-//     blocking: S for tile j+1 of a group is issued as soon as that group has
-//     read S_j into registers, PV_j as soon as P_j is written, whichever group
-//     gets there first.
+//   * one warp per group issues that group's tcgen05.mma: S = Q k~^T (M=128,
+//     N=kBN, K=64) into tensor memory and O += P v~ (M=128, N=64, K=kBN) with P
+//     read from tensor memory (issuing is slower than the small MMAs run, so
+//     one issuing thread for all groups would starve the tensor core).
 //   * warps 0 .. 4*kGroups-1 are the softmax warpgroups, one per query tile,
 //     thread = row = TMEM lane.
 // At d_h = 64 each exponential pairs with only 256 MMA flops, so the softmax
@@ -45,7 +43,8 @@ namespace {
 constexpr int kBM = 128;                      // rows per query tile
 constexpr int kBN = PACK3D_SA_BN;             // summaries per tile
 constexpr int kGroups = PACK3D_SA_GROUPS;     // query tiles (softmax warpgroups) per CTA
-constexpr int kMmaWarp = 4 * kGroups, kTmaWarp = kMmaWarp + 1;
+constexpr int kMmaWarp = 4 * kGroups;          // first MMA warp; one per group
+constexpr int kTmaWarp = kMmaWarp + kGroups;
 constexpr int kThreads = 32 * (kTmaWarp + 1);
 constexpr int kColS = 0, kColP = kBN, kColO = kBN + kBN / 2;
 constexpr int kGroupCols = kColO + kDh;       // tensor-memory columns per group
@@ -69,7 +68,7 @@ constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kDh, true);     // O: N =
 
 // Pair k of the 32 column pairs of a tile uses the FMA-pipe exponential when
 // this holds; the others use MUFU.ex2.
-__host__ __device__ constexpr bool poly_pair(int) { return false; }
+__host__ __device__ constexpr bool poly_pair(int k) { return false; }
 
 struct TcArgs {
   int M;             // summaries
@@ -136,7 +135,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(full(s), 1);
-      ptx::mbar_init(empty(s), 1);
+      ptx::mbar_init(empty(s), kGroups);   // one commit per group's MMA warp
     }
     ptx::mbar_init(qfull, 1);
     for (int w = 0; w < kGroups; ++w) {
@@ -185,87 +184,57 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp >= kMmaWarp) {
+    // ---------------- MMA issuers: one warp per group ----------------
+    // A single issuing thread cannot keep up (each tcgen05.mma takes longer to
+    // issue than a 128 x 64 x 16 step takes to run), so every group has its own.
+    // A group's events are ordered (s_free(j) before p_full(j) before
+    // s_free(j+1)), so plain bounded waits in that order suffice.
+    const int w = warp - kMmaWarp;
     if (lane == 0) {
-      auto issue_s = [&](int w, int j) {
+      const uint32_t qaddr = sbase + kQOff + w * kQBytes;
+      const uint32_t tS = tmem + w * kGroupCols + kColS;
+      const uint32_t tP = tmem + w * kGroupCols + kColP;
+      const uint32_t tO = tmem + w * kGroupCols + kColO;
+      auto issue_s = [&](int j) {
         const uint32_t kaddr = sbase + kStageOff + (j % kStages) * kStageBytes;
-        const uint32_t qaddr = sbase + kQOff + w * kQBytes;
 #pragma unroll
         for (int kk = 0; kk < kDh / 16; ++kk)
-          ptx::mma_ss(tmem + w * kGroupCols + kColS, ptx::smem_desc_sw128(qaddr + kk * 32, 16, 1024),
+          ptx::mma_ss(tS, ptx::smem_desc_sw128(qaddr + kk * 32, 16, 1024),
                       ptx::smem_desc_sw128(kaddr + kk * 32, 16, 1024), kIdesc, kk > 0);
         ptx::tc_commit(s_full(w));
       };
-      auto issue_pv = [&](int w, int j) {
+      auto issue_pv = [&](int j) {
         const uint32_t vaddr = sbase + kStageOff + (j % kStages) * kStageBytes + kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          ptx::mma_ts(tmem + w * kGroupCols + kColO, tmem + w * kGroupCols + kColP + kk * 8,
-                      ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024), kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_ts(tO, tP + kk * 8, ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024), kIdescPV,
+                      (j > 0 || kk > 0) ? 1u : 0u);
         ptx::tc_commit(p_free(w));
+        ptx::tc_commit(empty(j % kStages));
         if (j == T - 1) ptx::tc_commit(o_final(w));
       };
-      // Event loop.  Parities: s_free(w) completes once per tile a group has
-      // read, p_full(w) once per P tile written, full(s) once per load of
-      // stage s; none can run ahead of the issue it waits for, so a parity
-      // test never aliases an older phase.
       bool ok = ptx::mbar_wait(qfull, 0, abort_flag) && ptx::mbar_wait(full(0), 0, abort_flag);
-      int next_s[kGroups], next_pv[kGroups], released = 0;
-      for (int w = 0; w < kGroups; ++w) {
-        next_s[w] = 1;
-        next_pv[w] = 0;
-      }
       if (ok) {
         ptx::tc_fence_after();
-        for (int w = 0; w < kGroups; ++w) issue_s(w, 0);
+        issue_s(0);
       }
-      uint64_t t0 = ptx::globaltimer_ns();
-      uint32_t idle = 0;
-      int min_pv = 0;
-      while (ok && min_pv < T) {
-        bool progressed = false;
-#pragma unroll
-        for (int w = 0; w < kGroups; ++w) {
-          const int jp = next_pv[w];
-          if (jp < T && jp < next_s[w] && ptx::mbar_test_wait(p_full(w), jp & 1)) {
-            ptx::tc_fence_after();
-            issue_pv(w, jp);
-            next_pv[w] = jp + 1;
-            progressed = true;
-          }
-          const int js = next_s[w];
-          if (js < T && ptx::mbar_test_wait(s_free(w), (js - 1) & 1) &&
-              ptx::mbar_test_wait(full(js % kStages), (js / kStages) & 1)) {
-            ptx::tc_fence_after();
-            issue_s(w, js);
-            next_s[w] = js + 1;
-            progressed = true;
-          }
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) {
+          if (!(ok = ptx::mbar_wait(s_free(w), j & 1, abort_flag) &&
+                     ptx::mbar_wait(full((j + 1) % kStages), ((j + 1) / kStages) & 1, abort_flag)))
+            break;
+          ptx::tc_fence_after();
+          issue_s(j + 1);
         }
-        // A stage is free once every group's PV of its tile was issued.
-        min_pv = next_pv[0];
-#pragma unroll
-        for (int w = 1; w < kGroups; ++w) min_pv = min(min_pv, next_pv[w]);
-        while (released < min_pv) {
-          ptx::tc_commit(empty(released % kStages));
-          ++released;
-        }
-        if (progressed) {
-          idle = 0;
-        } else if ((++idle & 255) == 0) {
-          if (*abort_flag) ok = false;
-          else if (idle == 256) t0 = ptx::globaltimer_ns();
-          else if (ptx::globaltimer_ns() - t0 > 2000000000ull) {
-            *abort_flag = 1;
-            ok = false;
-          }
-        }
+        if (!(ok = ptx::mbar_wait(p_full(w), j & 1, abort_flag))) break;
+        ptx::tc_fence_after();
+        issue_pv(j);
       }
       if (!ok) {
-        // Drain whatever was issued before tensor memory is released.
-        ptx::tc_commit(o_final(0));
-        ptx::mbar_wait(o_final(0), 0, abort_flag);
+        // Drain whatever this warp issued before tensor memory is released.
+        ptx::tc_commit(o_final(w));
+        ptx::mbar_wait(o_final(w), 0, abort_flag);
       }
     }
     __syncwarp();
@@ -278,75 +247,92 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full(w), j & 1, abort_flag)))) break;
-      ptx::tc_fence_after();
-      uint32_t sv[kBN];
+    // Online softmax with a lazily moved maximum: m_used (log2 units) only
+    // moves when a tile's row maximum exceeds it by more than 8, so P stays
+    // below 2^8 and O is rescaled in tensor memory on few tiles.  S is read
+    // into registers and released at once, so S for the next tile runs on the
+    // tensor core while this tile's exponentials are computed.
+    auto load_s = [&](uint32_t* sv, int j) {
 #pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) ptx::tmem_ld32(trow + 32 * q, sv + 32 * q);
-      ptx::tmem_wait_ld();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(s_free(w));
+      for (int q = 0; q < kBN / 64; ++q) ptx::tmem_ld64_sync(trow + kColS + 64 * q, sv + 64 * q);
       if ((j + 1) * kBN > a.M) {
         const int lim = a.M - j * kBN;
 #pragma unroll
         for (int k = 0; k < kBN; ++k)
           if (k >= lim) sv[k] = __float_as_uint(-INFINITY);
       }
-      float m4[4];
+    };
+    // Row maximum over the kBN columns: 8 independent max3 chains, each chain
+    // covering one column pair of every 16-column group.
+    auto row_max = [&](const uint32_t* sv) {
+      static_assert(kBN % 16 == 0, "row_max walks 16-column groups");
+      float m8[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) m4[q] = __uint_as_float(sv[q]);
+      for (int q = 0; q < 8; ++q) m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
 #pragma unroll
-      for (int k = 4; k < kBN - 4; k += 8)
+      for (int k = 16; k < kBN; k += 16)
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          m4[q] = max3(m4[q], __uint_as_float(sv[k + 2 * q]), __uint_as_float(sv[k + 2 * q + 1]));
-      m4[0] = max3(m4[0], __uint_as_float(sv[kBN - 4]), __uint_as_float(sv[kBN - 3]));
-      m4[1] = max3(m4[1], __uint_as_float(sv[kBN - 2]), __uint_as_float(sv[kBN - 1]));
-      const float mxs = max3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
-      // Lazy rescale: the maximum used for P moves only when this tile's row
-      // maximum exceeds it by more than the threshold.
-      float f = 1.f;
-      if (j == 0) {
-        m_used = mxs;
-      } else if (mxs > m_used + kRescaleThreshold) {
-        f = ptx::ex2(m_used - mxs);
-        m_used = mxs;
-      }
+        for (int q = 0; q < 8; ++q)
+          m8[q] = max3(m8[q], __uint_as_float(sv[k + 2 * q]), __uint_as_float(sv[k + 2 * q + 1]));
+      return max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+    };
+    // Exponentials of one S row, written to the P buffer 32 columns at a time;
+    // returns the row sum of the (unrounded) P values.
+    auto exps_store = [&](const uint32_t* sv) {
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_used, -m_used);
       float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int pair = 0; pair < kBN / 2; ++pair) {
-        const float2 x =
-            __ffma2_rn(make_float2(__uint_as_float(sv[2 * pair]), __uint_as_float(sv[2 * pair + 1])), c2, nm2);
-        float2 p;
-        if (poly_pair(pair)) {
-          p = exp2_poly(x);
-        } else {
-          p.x = ptx::ex2(x.x);
-          p.y = ptx::ex2(x.y);
+      for (int q = 0; q < kBN / 32; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int pair = q * 16 + k;
+          const float2 x =
+              __ffma2_rn(make_float2(__uint_as_float(sv[2 * pair]), __uint_as_float(sv[2 * pair + 1])), c2, nm2);
+          float2 p;
+          if (poly_pair(pair)) {
+            p = exp2_poly(x);
+          } else {
+            p.x = ptx::ex2(x.x);
+            p.y = ptx::ex2(x.y);
+          }
+          rs[k & 1] = __fadd2_rn(rs[k & 1], p);
+          pk[k] = pack_bf16x2(p.x, p.y);
         }
-        rs[pair & 1] = __fadd2_rn(rs[pair & 1], p);
-        pk[pair] = pack_bf16x2(p.x, p.y);
+        ptx::tmem_st16(tP + 16 * q, pk);
       }
-      // P_j overwrites P_{j-1}: PV_{j-1} must be done (that also makes O stable).
-      if (j > 0 && !(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(w), (j - 1) & 1, abort_flag)))) break;
+      return (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
+    };
+    for (int j = 0; j < T; ++j) {
+      if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full(w), j & 1, abort_flag)))) break;
       ptx::tc_fence_after();
+      float f = 1.f, rs;
+      {
+        uint32_t sv[kBN];
+        load_s(sv, j);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(s_free(w));
+        const float mxs = row_max(sv) * c;
+        if (j == 0) m_used = mxs;
+        else if (mxs > m_used + kRescaleThreshold) {
+          f = ptx::ex2(m_used - mxs);
+          m_used = mxs;
+        }
+        if (j > 0 && !(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(w), (j - 1) & 1, abort_flag)))) break;
+        ptx::tc_fence_after();
+        rs = exps_store(sv);
+      }
       if (__any_sync(0xffffffffu, f != 1.f)) {
         uint32_t r[32];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          ptx::tmem_ld32(tO + 32 * q, r);
-          ptx::tmem_wait_ld();
+          ptx::tmem_ld32_sync(tO + 32 * q, r);
 #pragma unroll
           for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
           ptx::tmem_st32(tO + 32 * q, r);
         }
       }
-#pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) ptx::tmem_st16(tP + 16 * q, pk + 16 * q);
-      l = l * f + (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
+      l = l * f + rs;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(p_full(w));
@@ -354,9 +340,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final(w), 0, abort_flag))) {
       ptx::tc_fence_after();
       uint32_t r[2][32];
-      ptx::tmem_ld32(tO, r[0]);
-      ptx::tmem_ld32(tO + 32, r[1]);
-      ptx::tmem_wait_ld();
+      ptx::tmem_ld64_sync(tO, &r[0][0]);
       const long grow = (long)(tile0 + w) * kBM + lane_base + lane;
       if (grow < a.rows) {
         const long tok = grow / a.G;

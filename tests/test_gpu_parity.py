@@ -123,6 +123,31 @@ def test_simt_and_tensor_core_local_paths_agree(p3, shape):
     assert rel_err(a["o_loc"].double(), b["o_loc"].double()) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("order", ["rising", "falling"])
+def test_summary_attention_extreme_logit_ranges(p3, order):
+    # Logits that grow by far more than the float exponent range between
+    # summary tiles (rising) force the kernel's recompute-and-rescale path;
+    # falling logits underflow later tiles.  Both must still match the oracle.
+    s = small(Z=4, H=32, W=32)          # N = 4096, M = 256 -> two 128-summary tiles
+    gen = torch.Generator().manual_seed(11)
+    q = torch.randn(s.N, s.Hq, 64, generator=gen)
+    ks = torch.randn(s.M, s.Hkv, 64, generator=gen) * 0.05
+    vs = torch.randn(s.M, s.Hkv, 64, generator=gen)
+    big = slice(128, 256) if order == "rising" else slice(0, 128)
+    ks[big] = q[:128].reshape(128, s.Hq, 64)[:, ::4][:, :s.Hkv] * 8.0   # aligned with some queries
+    q, ks, vs = (t.bfloat16() for t in (q, ks, vs))
+    cfg = p3.config_from_shape(s)
+    out = torch.empty(s.N, s.Hq, 64, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    p3.summary_attn(cfg, q.cuda(), ks.cuda(), vs.cuda(), None, None, out, err)
+    assert p3.check_status(err) == 0
+    rows = synth.sample_rows(s.N, 300, seed=4)
+    ref = oracle.summary_attn(s, q[torch.from_numpy(rows)], ks, vs)
+    got = out.cpu()[torch.from_numpy(rows)].double().numpy()
+    assert np.isfinite(got).all()
+    assert rel_err(got, ref) <= TOL["bf16"]
+
+
 # ------------------------------------------------------------ index map ---------
 
 @pytest.mark.parametrize("packing", synth.PACKINGS)
