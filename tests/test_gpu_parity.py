@@ -148,6 +148,17 @@ def test_summary_attention_extreme_logit_ranges(p3, order):
     assert rel_err(got, ref) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("name", ["small", "65k"])
+def test_forward_is_deterministic(p3, name):
+    # Every kernel computes each output from a fixed sequence of operations, so
+    # repeated runs on the same inputs must agree bit for bit (a race or a read
+    # of uninitialised state shows up here first).
+    s = synth.CONFIGS["65k"] if name == "65k" else small(Z=4, H=16, W=24)
+    d = to_dev(synth.make_inputs(s, s.packing, seed=8))
+    outs = [run_forward(p3, s, d) for _ in range(3)]
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+
+
 # ------------------------------------------------------------ index map ---------
 
 @pytest.mark.parametrize("packing", synth.PACKINGS)
