@@ -45,6 +45,10 @@ WORKLOAD_TEXT = {
 }
 STAGES = ("index", "rope", "summaries", "local", "summary_attn")
 KERNELS_PER_STEP = 8   # 2 fills + index, rope Q, rope K, summaries, local, summary attention
+# DRAM bytes (read + write) of one summary_attn_tc_kernel launch, from an ncu
+# capture of this workload (profiles/summary_attn_tc_65k.md).  Set back to
+# None whenever that kernel changes until it is captured again.
+SUMMARY_ATTN_TRAFFIC = {"65k": 212.878592e6 + 47.812352e6}
 
 
 def load_peaks():
@@ -353,7 +357,7 @@ def run_ours(args, s):
         stages[name] = e
     sa = stages["summary_attn"]
     roof = {"bound": "tensor", "achieved": sa["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": sa["tflops"] / peaks["bf16_tflops"], "traffic": None,
+            "frac": sa["tflops"] / peaks["bf16_tflops"], "traffic": SUMMARY_ATTN_TRAFFIC.get(args.config),
             "kernel": "summary_attn_tc_kernel" if s.dtype == "bf16" else "summary_attn_simt_kernel",
             "peak_source": peaks["source"] + " burst bf16 (MEASURED_PEAKS.json bf16_tflops)"}
     if s.dtype != "bf16":
