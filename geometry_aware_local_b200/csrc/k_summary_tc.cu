@@ -12,8 +12,10 @@
 //     128-byte swizzle) through a TMA ring; the Q tiles are loaded once.
 //   * one warp per group issues that group's tcgen05.mma: S = Q k~^T (M=128,
 //     N=kBN, K=64) into tensor memory and O += P v~ (M=128, N=64, K=kBN) with P
-//     read from tensor memory (issuing is slower than the small MMAs run, so
-//     one issuing thread for all groups would starve the tensor core).
+//     read from tensor memory.  An SM accepts about one tcgen05.mma per 50
+//     clocks whichever warp issues it (so the N=64 steps of O += P v~ are
+//     issue bound); a warp per group lets each group's MMAs follow its own
+//     barriers instead of queueing behind the other group's waits.
 //   * warps 0 .. 4*kGroups-1 are the softmax warpgroups, one per query tile,
 //     thread = row = TMEM lane.
 // At d_h = 64 each exponential pairs with only 256 MMA flops, so the softmax
@@ -56,8 +58,21 @@ constexpr int kQOff = 0;
 constexpr int kStageOff = kGroups * kQBytes;  // stage s: k~ at +0, v~ at +kKVBytes
 constexpr int kStageBytes = 2 * kKVBytes;
 constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-// barriers: full[S], empty[S], qfull, then per group: s_full, s_free, p_full, p_free, o_final
-constexpr int kGroupBars = 5;
+// P can be handed between the softmax warps and the MMA warp in kPChunks
+// column chunks, so that O += P v~ for one chunk runs while the exponentials
+// of the next are computed.  Measured on B200 at 65k tokens: 1 chunk 0.81 ms,
+// 2 chunks 0.82 ms, 4 chunks 0.86 ms (the extra barriers cost more than the
+// overlap gains), so the default is a single hand-off per tile.
+#ifndef PACK3D_SA_PCHUNKS
+#define PACK3D_SA_PCHUNKS 1
+#endif
+constexpr int kPChunks = PACK3D_SA_PCHUNKS;
+constexpr int kPairsPerChunk = kBN / 2 / kPChunks;   // packed P columns per chunk
+constexpr int kMmasPerChunk = kBN / 16 / kPChunks;   // K = 16 steps of O += P v~ per chunk
+static_assert(kPairsPerChunk % 16 == 0, "P chunks are stored 16 columns at a time");
+// barriers: full[S], empty[S], qfull, then per group: s_full, s_free, o_final,
+// p_full[kPChunks], p_free[kPChunks]
+constexpr int kGroupBars = 3 + 2 * kPChunks;
 constexpr int kNumBars = 2 * kStages + 1 + kGroups * kGroupBars;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
@@ -68,7 +83,14 @@ constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kDh, true);     // O: N =
 
 // Pair k of the 32 column pairs of a tile uses the FMA-pipe exponential when
 // this holds; the others use MUFU.ex2.
-__host__ __device__ constexpr bool poly_pair(int k) { return false; }
+// PACK3D_SA_POLY of every 16 pairs (spread evenly) take the cubic; 0 by
+// default, since every share tried (2, 3, 4 and 6 of 16) was slower on B200.
+#ifndef PACK3D_SA_POLY
+#define PACK3D_SA_POLY 0
+#endif
+__host__ __device__ constexpr bool poly_pair(int k) {
+  return PACK3D_SA_POLY > 0 && ((k % 16) * PACK3D_SA_POLY) % 16 < PACK3D_SA_POLY;
+}
 
 struct TcArgs {
   int M;             // summaries
@@ -126,9 +148,9 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   auto gbar = [&](int w, int i) { return bar0 + 8 * (2 * kStages + 1 + w * kGroupBars + i); };
   auto s_full = [&](int w) { return gbar(w, 0); };
   auto s_free = [&](int w) { return gbar(w, 1); };
-  auto p_full = [&](int w) { return gbar(w, 2); };
-  auto p_free = [&](int w) { return gbar(w, 3); };
-  auto o_final = [&](int w) { return gbar(w, 4); };
+  auto o_final = [&](int w) { return gbar(w, 2); };
+  auto p_full = [&](int w, int c) { return gbar(w, 3 + c); };
+  auto p_free = [&](int w, int c) { return gbar(w, 3 + kPChunks + c); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -140,10 +162,12 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     ptx::mbar_init(qfull, 1);
     for (int w = 0; w < kGroups; ++w) {
       ptx::mbar_init(s_full(w), 1);
-      ptx::mbar_init(s_free(w), kBM);
-      ptx::mbar_init(p_full(w), kBM);
-      ptx::mbar_init(p_free(w), 1);
+      ptx::mbar_init(s_free(w), 4);       // one arrival per softmax warp
       ptx::mbar_init(o_final(w), 1);
+      for (int c = 0; c < kPChunks; ++c) {
+        ptx::mbar_init(p_full(w, c), 4);
+        ptx::mbar_init(p_free(w, c), 1);
+      }
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -188,8 +212,9 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     // ---------------- MMA issuers: one warp per group ----------------
     // A single issuing thread cannot keep up (each tcgen05.mma takes longer to
     // issue than a 128 x 64 x 16 step takes to run), so every group has its own.
-    // A group's events are ordered (s_free(j) before p_full(j) before
-    // s_free(j+1)), so plain bounded waits in that order suffice.
+    // A group's events are ordered (s_free(j), then the P chunks of tile j in
+    // column order, then s_free(j+1)), so plain bounded waits in that order
+    // suffice.
     const int w = warp - kMmaWarp;
     if (lane == 0) {
       const uint32_t qaddr = sbase + kQOff + w * kQBytes;
@@ -204,15 +229,19 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                       ptx::smem_desc_sw128(kaddr + kk * 32, 16, 1024), kIdesc, kk > 0);
         ptx::tc_commit(s_full(w));
       };
-      auto issue_pv = [&](int j) {
+      auto issue_pv = [&](int j, int c) {
         const uint32_t vaddr = sbase + kStageOff + (j % kStages) * kStageBytes + kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int i = 0; i < kMmasPerChunk; ++i) {
+          const int kk = c * kMmasPerChunk + i;
           ptx::mma_ts(tO, tP + kk * 8, ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024), kIdescPV,
                       (j > 0 || kk > 0) ? 1u : 0u);
-        ptx::tc_commit(p_free(w));
-        ptx::tc_commit(empty(j % kStages));
-        if (j == T - 1) ptx::tc_commit(o_final(w));
+        }
+        ptx::tc_commit(p_free(w, c));
+        if (c == kPChunks - 1) {
+          ptx::tc_commit(empty(j % kStages));
+          if (j == T - 1) ptx::tc_commit(o_final(w));
+        }
       };
       bool ok = ptx::mbar_wait(qfull, 0, abort_flag) && ptx::mbar_wait(full(0), 0, abort_flag);
       if (ok) {
@@ -227,9 +256,11 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           ptx::tc_fence_after();
           issue_s(j + 1);
         }
-        if (!(ok = ptx::mbar_wait(p_full(w), j & 1, abort_flag))) break;
-        ptx::tc_fence_after();
-        issue_pv(j);
+        for (int c = 0; ok && c < kPChunks; ++c) {
+          if (!(ok = ptx::mbar_wait(p_full(w, c), j & 1, abort_flag))) break;
+          ptx::tc_fence_after();
+          issue_pv(j, c);
+        }
       }
       if (!ok) {
         // Drain whatever this warp issued before tensor memory is released.
@@ -276,17 +307,16 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           m8[q] = max3(m8[q], __uint_as_float(sv[k + 2 * q]), __uint_as_float(sv[k + 2 * q + 1]));
       return max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
     };
-    // Exponentials of one S row, written to the P buffer 32 columns at a time;
-    // returns the row sum of the (unrounded) P values.
-    auto exps_store = [&](const uint32_t* sv) {
+    // Exponentials of chunk cc of one S row, written to the P buffer 16 packed
+    // columns at a time; the (unrounded) values are added to rs.
+    auto exps_chunk = [&](const uint32_t* sv, int cc, float2* rs) {
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_used, -m_used);
-      float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int q = 0; q < kBN / 32; ++q) {
+      for (int q = 0; q < kPairsPerChunk / 16; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const int pair = q * 16 + k;
+          const int pair = cc * kPairsPerChunk + q * 16 + k;
           const float2 x =
               __ffma2_rn(make_float2(__uint_as_float(sv[2 * pair]), __uint_as_float(sv[2 * pair + 1])), c2, nm2);
           float2 p;
@@ -299,43 +329,63 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           rs[k & 1] = __fadd2_rn(rs[k & 1], p);
           pk[k] = pack_bf16x2(p.x, p.y);
         }
-        ptx::tmem_st16(tP + 16 * q, pk);
+        ptx::tmem_st16(tP + cc * kPairsPerChunk + 16 * q, pk);
       }
-      return (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
+    };
+    // One arrival per warp: every lane's tensor-memory accesses are complete
+    // (waited and fenced) before the warp converges and lane 0 arrives (one
+    // arrival instead of 32 per warp took 0.92 -> 0.81 ms at 65k tokens).
+    auto warp_arrive = [&](uint32_t bar) {
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar);
     };
     for (int j = 0; j < T; ++j) {
       if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full(w), j & 1, abort_flag)))) break;
       ptx::tc_fence_after();
-      float f = 1.f, rs;
+      float f = 1.f;
+      float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       {
         uint32_t sv[kBN];
         load_s(sv, j);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(s_free(w));
+        warp_arrive(s_free(w));
         const float mxs = row_max(sv) * c;
         if (j == 0) m_used = mxs;
         else if (mxs > m_used + kRescaleThreshold) {
           f = ptx::ex2(m_used - mxs);
           m_used = mxs;
         }
-        if (j > 0 && !(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(w), (j - 1) & 1, abort_flag)))) break;
-        ptx::tc_fence_after();
-        rs = exps_store(sv);
-      }
-      if (__any_sync(0xffffffffu, f != 1.f)) {
-        uint32_t r[32];
+        const bool rescale = j > 0 && __any_sync(0xffffffffu, f != 1.f);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          ptx::tmem_ld32_sync(tO + 32 * q, r);
+        for (int cc = 0; cc < kPChunks; ++cc) {
+          if (j > 0) {
+            if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(w, cc), (j - 1) & 1, abort_flag)))) break;
+            ptx::tc_fence_after();
+          }
+          exps_chunk(sv, cc, rs);
+          if (cc == 0 && rescale) {
+            // O is rescaled before this tile's first O += P v~ is issued and
+            // after the previous tile's last one has completed (its commit
+            // covers all earlier MMAs of the group).
+            if (!(ok = __all_sync(0xffffffffu,
+                                  ptx::mbar_wait(p_free(w, kPChunks - 1), (j - 1) & 1, abort_flag))))
+              break;
+            ptx::tc_fence_after();
+            uint32_t r[16];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
-          ptx::tmem_st32(tO + 32 * q, r);
+            for (int q = 0; q < kDh / 16; ++q) {
+              ptx::tmem_ld16_sync(tO + 16 * q, r);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
+              ptx::tmem_st16(tO + 16 * q, r);
+            }
+          }
+          ptx::tmem_wait_st();
+          warp_arrive(p_full(w, cc));
         }
+        if (!ok) break;
       }
-      l = l * f + rs;
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(p_full(w));
+      l = l * f + ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y));
     }
     if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final(w), 0, abort_flag))) {
       ptx::tc_fence_after();
