@@ -300,13 +300,205 @@ __global__ void __launch_bounds__(kSumThreads) summaries_generic_kernel(
   }
 }
 
+// Warp-per-block path (block volume 16).  One warp owns block j for every kv
+// head and both tensors.  Lane l owns chunk slot c of a member's head rows
+// (head c / CPR, 16-byte part c % CPR) in BOTH K_cmp and V_cmp, so K and V
+// lanes never diverge; when a member has fewer than 32 slots the warp covers
+// MPI members per load and the lanes' partial sums are combined at the end.
+//
+// The rotation is split with R(c_base + d) = R(c_base) R(d) (each plane is a
+// 2-D rotation by omega * coordinate, so angles add): member t, at in-block
+// offset d_t of the block's first site c_base, is rotated by R(d_t) from a
+// small per-CTA table of the 16 offsets x 32 planes, and the pooled key is
+// rotated once by R(c_base):  k~_j = R(c_base) sum_t a_t R(d_t) k_t, the same
+// sum as sum_t a_t R(c_t) k_t.  Both are evaluated directly (angle reduced in
+// double, float sincos), so the kernel needs no whole-volume cos/sin table.
+constexpr int kSumWarpThreads = 256;
+
+template <typename T, int HKV>
+__global__ void __launch_bounds__(kSumWarpThreads) summaries_warp_kernel(
+    Shape s, const int32_t* __restrict__ members, const T* __restrict__ kc,
+    const T* __restrict__ vc, const float* __restrict__ scores, T* __restrict__ ks,
+    T* __restrict__ vs) {
+  constexpr int V = 16;
+  static_assert(kMaxPairs == 32, "one rotary plane per lane");
+  __shared__ float2 dtab[V][kMaxPairs];   // cos/sin of plane p at member t's in-block offset
+  const int lane = threadIdx.x & 31;
+  // Lane p holds rotary plane p's axis and frequency.
+  const int my_axis = lane < s.npairs ? s.pair_axis[lane] : 3;
+  const double my_omega = lane < s.npairs ? s.omega[lane] : 0.0;
+  for (int t = threadIdx.x >> 5; t < V; t += kSumWarpThreads / 32) {
+    const int d = my_axis == 0 ? t / (s.by * s.bx) : (my_axis == 1 ? (t / s.bx) % s.by : t % s.bx);
+    dtab[t][lane] = my_axis < 3 ? rope_cos_sin(my_omega * (double)d) : make_float2(1.f, 0.f);
+  }
+  __syncthreads();
+  constexpr int NE = Elem<T>::kPerChunk;
+  constexpr int NP = NE / 2;
+  constexpr int CPR = kDh / NE;                   // chunks per head row
+  constexpr int LPM = HKV * CPR;                  // chunk slots per member and tensor
+  constexpr int SPL = LPM >= 32 ? LPM / 32 : 1;   // slots per lane
+  constexpr int MPI = LPM >= 32 ? 1 : 32 / LPM;   // members per load instruction
+  constexpr int PPL = (V * HKV + 31) / 32;        // (member, head) score pairs per lane
+#ifndef PACK3D_SUM_LOADS
+#define PACK3D_SUM_LOADS 8
+#endif
+  // Members per batch: PACK3D_SUM_LOADS K and V chunk pairs in flight per lane.
+  constexpr int B = (PACK3D_SUM_LOADS * MPI / SPL) < V ? (PACK3D_SUM_LOADS * MPI / SPL) : V;
+  static_assert(V % B == 0 && B % MPI == 0, "member batches");
+  const int sub = MPI > 1 ? lane / LPM : 0;
+  int head[SPL], part[SPL];
+#pragma unroll
+  for (int i = 0; i < SPL; ++i) {
+    const int c = (lane % LPM) + 32 * i;
+    head[i] = c / CPR;
+    part[i] = c % CPR;
+  }
+  const int nwarps = gridDim.x * (kSumWarpThreads / 32);
+  int j = blockIdx.x * (kSumWarpThreads / 32) + (threadIdx.x >> 5);
+  // Block-grid position of block j, stepped by nwarps blocks per iteration.
+  int jx = j % s.nbx, jy = (j / s.nbx) % s.nby, jz = j / (s.nbx * s.nby);
+  const int sx = nwarps % s.nbx, sy = (nwarps / s.nbx) % s.nby, sz = nwarps / (s.nbx * s.nby);
+  // Member t of block j is held by lanes t and t + 16; the next block's
+  // indices are requested while this block is pooled.
+  int m_next = j < s.M ? __ldg(members + (size_t)j * V + (lane & 15)) : -1;
+  for (; j < s.M; j += nwarps) {
+    const int m_l = m_next;
+    if (j + nwarps < s.M) m_next = __ldg(members + (size_t)(j + nwarps) * V + (lane & 15));
+    // Scores: pair p = lane + 32 i is (member p % 16, head p / 16).
+    float sc[PPL];
+#pragma unroll
+    for (int i = 0; i < PPL; ++i) {
+      const int p = lane + 32 * i, h = p >> 4;
+      const int mt = __shfl_sync(0xffffffffu, m_l, p & 15);
+      sc[i] = (h < HKV && mt >= 0) ? __ldg(scores + (size_t)mt * HKV + h) : -INFINITY;
+    }
+    float ak[SPL][NE], av[SPL][NE];
+#pragma unroll
+    for (int i = 0; i < SPL; ++i)
+#pragma unroll
+      for (int k = 0; k < NE; ++k) ak[i][k] = av[i][k] = 0.f;
+    float wa[PPL];
+#pragma unroll 1
+    for (int t0 = 0; t0 < V; t0 += B) {
+      uint4 rk[B / MPI][SPL], rv[B / MPI][SPL];
+      int mts[B / MPI];
+#pragma unroll
+      for (int b = 0; b < B / MPI; ++b) {
+        mts[b] = __shfl_sync(0xffffffffu, m_l, t0 + b * MPI + sub);
+#pragma unroll
+        for (int i = 0; i < SPL; ++i)
+          if (mts[b] >= 0) {
+            const size_t off = ((size_t)mts[b] * HKV + head[i]) * kDh + part[i] * NE;
+            rk[b][i] = ldg16(kc + off);
+            rv[b][i] = ldg16(vc + off);
+          }
+      }
+      if (t0 == 0) {
+        // a_{j,t} = softmax over the block's members of their scores (per
+        // head): the 16 pairs of one head sit in one half-warp of a register.
+#pragma unroll
+        for (int i = 0; i < PPL; ++i) {
+          float mx = sc[i];
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float e = sc[i] == -INFINITY ? 0.f : expf(sc[i] - mx);
+          float den = e;
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+          wa[i] = den > 0.f ? e / den : 0.f;
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < B / MPI; ++b) {
+        const int t = t0 + b * MPI + sub;
+#pragma unroll
+        for (int i = 0; i < SPL; ++i) {
+          // Weight of (member t, head[i]): register head/2, lane (head%2)*16 + t.
+          float w = 0.f;
+#pragma unroll
+          for (int r = 0; r < PPL; ++r) {
+            const float x = __shfl_sync(0xffffffffu, wa[r], ((head[i] & 1) << 4) + t);
+            if (r == head[i] >> 1) w = x;
+          }
+          if (mts[b] < 0) continue;
+          float fk[NE], fv[NE];
+          chunk_to_float(rk[b][i], fk, T());
+          chunk_to_float(rv[b][i], fv, T());
+#pragma unroll
+          for (int k = 0; k < NP; ++k) {
+            const float2 cs = dtab[t][part[i] * NP + k];
+            const float x0 = fk[2 * k], x1 = fk[2 * k + 1];
+            ak[i][2 * k] = fmaf(w, x0 * cs.x - x1 * cs.y, ak[i][2 * k]);
+            ak[i][2 * k + 1] = fmaf(w, x0 * cs.y + x1 * cs.x, ak[i][2 * k + 1]);
+          }
+#pragma unroll
+          for (int k = 0; k < NE; ++k) av[i][k] = fmaf(w, fv[k], av[i][k]);
+        }
+      }
+    }
+    // Lanes that covered different members of the same slot combine.
+#pragma unroll
+    for (int o = LPM; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < SPL; ++i)
+#pragma unroll
+        for (int k = 0; k < NE; ++k) {
+          ak[i][k] += __shfl_xor_sync(0xffffffffu, ak[i][k], o);
+          av[i][k] += __shfl_xor_sync(0xffffffffu, av[i][k], o);
+        }
+    // R(c_base): lane p evaluates plane p at the block's first site, and every
+    // lane takes the pairs of its own planes by shuffle.
+    const float2 cb = my_axis < 3 ? rope_cos_sin(my_omega * (double)(my_axis == 0 ? jz * s.bz
+                                                                     : (my_axis == 1 ? jy * s.by : jx * s.bx)))
+                                  : make_float2(1.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < SPL; ++i)
+#pragma unroll
+      for (int k = 0; k < NP; ++k) {
+        const float c = __shfl_sync(0xffffffffu, cb.x, part[i] * NP + k);
+        const float sn = __shfl_sync(0xffffffffu, cb.y, part[i] * NP + k);
+        const float x0 = ak[i][2 * k], x1 = ak[i][2 * k + 1];
+        ak[i][2 * k] = x0 * c - x1 * sn;
+        ak[i][2 * k + 1] = x0 * sn + x1 * c;
+      }
+    if (sub == 0) {
+#pragma unroll
+      for (int i = 0; i < SPL; ++i) {
+        const size_t off = ((size_t)j * HKV + head[i]) * kDh + part[i] * NE;
+        stg16(ks + off, float_to_chunk(ak[i], T()));
+        stg16(vs + off, float_to_chunk(av[i], T()));
+      }
+    }
+    jx += sx;
+    if (jx >= s.nbx) { jx -= s.nbx; ++jy; }
+    jy += sy;
+    if (jy >= s.nby) { jy -= s.nby; ++jz; }
+    jz += sz;
+  }
+}
+
 template <typename T>
 static cudaError_t summaries_t(const Shape& s, const int32_t* members, const void* kc, const void* vc,
                                const float* scores, void* ks, void* vs, cudaStream_t st) {
   const size_t smem = (size_t)s.tab_entries * sizeof(float2);
   const int U = 2 * (kDh / Elem<T>::kPerChunk);
+  if (s.v == 16 && (s.Hkv == 1 || s.Hkv == 2 || s.Hkv == 4 || s.Hkv == 8)) {
+    auto kern = s.Hkv == 1   ? summaries_warp_kernel<T, 1>
+                : s.Hkv == 2 ? summaries_warp_kernel<T, 2>
+                : s.Hkv == 4 ? summaries_warp_kernel<T, 4>
+                             : summaries_warp_kernel<T, 8>;
+    // One persistent wave: every SM holds as many CTAs as fit, each warp walks blocks.
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSumWarpThreads, 0);
+    if (e != cudaSuccess) return e;
+    const long per_cta = kSumWarpThreads / 32;
+    const int grid = (int)max(1L, min((s.M + per_cta - 1) / per_cta, (long)sms * max(per_sm, 1)));
+    kern<<<grid, kSumWarpThreads, 0, st>>>(s, members, (const T*)kc, (const T*)vc, scores, (T*)ks, (T*)vs);
+    return cudaGetLastError();
+  }
   if (s.v <= U) {
-    auto kern = s.v == 16 ? summaries_kernel<T, 16> : summaries_kernel<T, 0>;
+    auto kern = summaries_kernel<T, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long units = (long)s.M * s.Hkv;
