@@ -386,12 +386,13 @@ __global__ void __launch_bounds__(kSumWarpThreads) summaries_warp_kernel(
       for (int b = 0; b < B / MPI; ++b) {
         mts[b] = __shfl_sync(0xffffffffu, m_l, t0 + b * MPI + sub);
 #pragma unroll
-        for (int i = 0; i < SPL; ++i)
-          if (mts[b] >= 0) {
-            const size_t off = ((size_t)mts[b] * HKV + head[i]) * kDh + part[i] * NE;
-            rk[b][i] = ldg16(kc + off);
-            rv[b][i] = ldg16(vc + off);
-          }
+        for (int i = 0; i < SPL; ++i) {
+          // A member slot left at -1 (coordinates that are not a bijection,
+          // reported by the index map) contributes zero rows with zero weight.
+          const size_t off = ((size_t)max(mts[b], 0) * HKV + head[i]) * kDh + part[i] * NE;
+          rk[b][i] = mts[b] >= 0 ? ldg16(kc + off) : make_uint4(0u, 0u, 0u, 0u);
+          rv[b][i] = mts[b] >= 0 ? ldg16(vc + off) : make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       if (t0 == 0) {
         // a_{j,t} = softmax over the block's members of their scores (per
@@ -408,19 +409,28 @@ __global__ void __launch_bounds__(kSumWarpThreads) summaries_warp_kernel(
           wa[i] = den > 0.f ? e / den : 0.f;
         }
       }
+      // Weights of (member t, head[i]) for the whole batch first (register
+      // head/2, lane (head%2)*16 + t), so the pooling below has no shuffle or
+      // branch between members.
+      float wt[B / MPI][SPL];
+#pragma unroll
+      for (int b = 0; b < B / MPI; ++b)
+#pragma unroll
+        for (int i = 0; i < SPL; ++i) {
+          float w = 0.f;
+#pragma unroll
+          for (int r = 0; r < PPL; ++r) {
+            const float x = __shfl_sync(0xffffffffu, wa[r], ((head[i] & 1) << 4) + t0 + b * MPI + sub);
+            if (r == head[i] >> 1) w = x;
+          }
+          wt[b][i] = w;
+        }
 #pragma unroll
       for (int b = 0; b < B / MPI; ++b) {
         const int t = t0 + b * MPI + sub;
 #pragma unroll
         for (int i = 0; i < SPL; ++i) {
-          // Weight of (member t, head[i]): register head/2, lane (head%2)*16 + t.
-          float w = 0.f;
-#pragma unroll
-          for (int r = 0; r < PPL; ++r) {
-            const float x = __shfl_sync(0xffffffffu, wa[r], ((head[i] & 1) << 4) + t);
-            if (r == head[i] >> 1) w = x;
-          }
-          if (mts[b] < 0) continue;
+          const float w = wt[b][i];
           float fk[NE], fv[NE];
           chunk_to_float(rk[b][i], fk, T());
           chunk_to_float(rv[b][i], fv, T());
