@@ -44,7 +44,7 @@ WORKLOAD_TEXT = {
     "1m": "64x128x128 lattice (1,048,576 tokens), random packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=65,536), window 3x7x7",
 }
 STAGES = ("index", "rope", "summaries", "local", "summary_attn")
-KERNELS_PER_STEP = 8   # 2 fills + index, rope Q, rope K, summaries, local, summary attention
+KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summary attention
 # DRAM bytes (read + write) of one summary_attn_tc_kernel launch, from an ncu
 # capture of this workload (profiles/summary_attn_tc_65k.md).  Set back to
 # None whenever that kernel changes until it is captured again.
@@ -263,8 +263,7 @@ def run_ours(args, s):
         ev[0].record(stream)
         st = lib.pack3d_build_index(cfgp, P(d["coords"]), P(g2p), P(mem), P(err), sh)
         ev[1].record(stream)
-        st |= lib.pack3d_rope(cfgp, P(d["coords"]), P(d["q"]), P(qr), s.Hq, sh)
-        st |= lib.pack3d_rope(cfgp, P(d["coords"]), P(d["k_loc"]), P(kr), s.Hkv, sh)
+        st |= lib.pack3d_rope_qk(cfgp, P(d["coords"]), P(d["q"]), P(qr), P(d["k_loc"]), P(kr), sh)
         ev[2].record(stream)
         st |= lib.pack3d_build_summaries(cfgp, P(mem), P(d["k_cmp"]), P(d["v_cmp"]), P(d["scores"]), P(ks),
                                          P(vs), sh)

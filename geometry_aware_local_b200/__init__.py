@@ -25,7 +25,7 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: 
           6: "WORKSPACE", 7: "CUDA", 8: "TIMEOUT"}
 
 ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
-                "pack3d_build_index", "pack3d_rope", "pack3d_build_summaries", "pack3d_local_attn",
+                "pack3d_build_index", "pack3d_rope", "pack3d_rope_qk", "pack3d_build_summaries", "pack3d_local_attn",
                 "pack3d_summary_attn", "pack3d_forward", "pack3d_forward_noalloc", "pack3d_check_status",
                 "pack3d_status_string", "pack3d_backend_info")
 
@@ -72,6 +72,7 @@ def _load():
         "pack3d_workspace_bytes": (ctypes.c_size_t, [C]),
         "pack3d_build_index": (ctypes.c_int, [C, P, P, P, P, P]),
         "pack3d_rope": (ctypes.c_int, [C, P, P, P, I32, P]),
+        "pack3d_rope_qk": (ctypes.c_int, [C, P, P, P, P, P, P]),
         "pack3d_build_summaries": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
         "pack3d_local_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
         "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
@@ -163,6 +164,11 @@ def build_index(cfg, coords, g2p, members, err, stream=None):
 def rope(cfg, coords, x, y, heads: int, stream=None):
     _check(lib.pack3d_rope(ctypes.byref(cfg), _ptr(coords), _ptr(x), _ptr(y), heads, _stream(stream)),
            "pack3d_rope")
+
+
+def rope_qk(cfg, coords, q, q_rot, k, k_rot, stream=None):
+    _check(lib.pack3d_rope_qk(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(q_rot), _ptr(k), _ptr(k_rot),
+                              _stream(stream)), "pack3d_rope_qk")
 
 
 def build_summaries(cfg, members, k_cmp, v_cmp, scores, k_sum, v_sum, stream=None):

@@ -159,6 +159,16 @@ pack3d_status pack3d_rope(const pack3d_config* cfg, const int32_t* coords, const
                                  (cudaStream_t)stream));
 }
 
+pack3d_status pack3d_rope_qk(const pack3d_config* cfg, const int32_t* coords, const void* q, void* q_rot,
+                             const void* k, void* k_rot, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!coords || !q || !q_rot || !k || !k_rot) return PACK3D_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(q_rot) || !aligned16(k) || !aligned16(k_rot)) return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  return cuda_status(launch_rope(s, cfg->dtype, coords, q, q_rot, s.Hq, k, k_rot, s.Hkv, (cudaStream_t)stream));
+}
+
 pack3d_status pack3d_build_summaries(const pack3d_config* cfg, const int32_t* members, const void* k_cmp,
                                      const void* v_cmp, const float* scores, void* k_sum, void* v_sum,
                                      void* stream) {

@@ -130,6 +130,14 @@ pack3d_status pack3d_build_index(const pack3d_config *cfg, const int32_t *coords
 pack3d_status pack3d_rope(const pack3d_config *cfg, const int32_t *coords, const void *x,
                           void *y, int32_t heads, void *stream);
 
+/* Stage 1 for both rotated tensors in one launch (the form pack3d_forward
+ * uses): q_rot = R(c) q with Hq heads and k_rot = R(c) k_loc with Hkv heads,
+ * each exactly as pack3d_rope would compute it.  q, q_rot: T [N,Hq,d_h];
+ * k, k_rot: T [N,Hkv,d_h]; each output may equal its input.  Device pointers,
+ * 16-byte aligned, owned by the caller; errors as pack3d_rope. */
+pack3d_status pack3d_rope_qk(const pack3d_config *cfg, const int32_t *coords, const void *q,
+                             void *q_rot, const void *k, void *k_rot, void *stream);
+
 /* Stage 3 - rotate-before-compress summaries.  For block j and kv head g:
  *   a_{j,u} = softmax over u in B_j of scores[u,g]
  *   k_sum[j,g] = sum_u a_{j,u} R(c_u) k_cmp[u,g],  v_sum[j,g] = sum_u a_{j,u} v_cmp[u,g]

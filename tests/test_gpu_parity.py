@@ -91,6 +91,10 @@ STAGE_CASES = [
     ("ragged-brick", small(Z=3, H=10, W=14, by=2, bx=2), "random"),  # 2x4x4 bricks cut in z, y and x
     ("window-2x1", small(Z=5, H=12, W=12, ry=2, rx=1), "morton"),     # 8x6 halo planes (48 keys)
     ("window-1x1x1", small(Z=4, H=8, W=8, ry=1, rx=1, rz=1), "block"),
+    # summaries at Hkv = 4 and 8: two and four chunk slots per lane (bf16 / float)
+    ("hkv4", small(Hq=8, Hkv=4), "random"),
+    ("hkv8-f32", small(Hq=8, Hkv=8, dtype="f32", value_scale=1.0), "block"),
+    ("hkv4-f32", small(Hq=8, Hkv=4, dtype="f32", value_scale=1.0), "morton"),
 ]
 
 
@@ -146,6 +150,21 @@ def test_summary_attention_extreme_logit_ranges(p3, order):
     got = out.cpu()[torch.from_numpy(rows)].double().numpy()
     assert np.isfinite(got).all()
     assert rel_err(got, ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_rope_qk_equals_two_rope_calls(p3, dtype):
+    """The fused Q/K launch computes exactly what the single-tensor entry point does."""
+    s = small(Z=4, H=16, W=24, dtype=dtype)
+    d = to_dev(synth.make_inputs(s, "random", seed=11))
+    cfg = p3.config_from_shape(s)
+    qa, ka = torch.empty_like(d["q"]), torch.empty_like(d["k_loc"])
+    p3.rope(cfg, d["coords"], d["q"], qa, s.Hq)
+    p3.rope(cfg, d["coords"], d["k_loc"], ka, s.Hkv)
+    qb, kb = torch.empty_like(qa), torch.empty_like(ka)
+    p3.rope_qk(cfg, d["coords"], d["q"], qb, d["k_loc"], kb)
+    torch.cuda.synchronize()
+    assert torch.equal(qa, qb) and torch.equal(ka, kb)
 
 
 @pytest.mark.parametrize("name", ["small", "65k"])
