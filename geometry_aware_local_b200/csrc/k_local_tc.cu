@@ -10,7 +10,7 @@
 // processed one lattice z-plane at a time: a plane of (4 + 2ry) x (4 + 2rx) <=
 // 10 x 10 sites, padded to NP <= 112 rows, is gathered through the index map
 // with cp.async (keys outside the volume are zero-filled) into a 128-byte-
-// swizzled K tile and V tile, double-buffered.  Per plane:
+// swizzled K tile and V tile.  Per plane:
 //   S = Q K^T  (M=128, N=NP, K=64; A, B from shared memory)
 //   softmax on the rows whose z window contains the plane (the other layer's
 //   warps write P = 0): the lattice-box mask is a per-row bit mask, the
@@ -18,10 +18,15 @@
 //   tensor memory when it does;
 //   O += P V   (M=128, N=64, K=NP; A = P from tensor memory, B = V from
 //   shared memory, MN-major).
-// Two CTAs share an SM (256 tensor-memory columns each: S 0-111, P 128-183,
-// O 192-255), so one CTA's softmax overlaps the other's gathers and MMAs.
+// Pipelining inside the CTA: every index-map lookup of the CTA (its query row
+// and its gather row of each plane) is issued at the start; three plane
+// buffers hold planes 0-2 from the start and plane 3 once plane 0's MMAs are
+// done; S of plane p+1 is issued as soon as every warp has read S of plane p
+// into registers, so it runs under plane p's exponentials.  Two CTAs share an
+// SM (256 tensor-memory columns each: S 0-111, P 128-183, O 192-255).
 // Supported: bf16, G = 4, rz = 1, ry <= 3, rx <= 3 (the SIMT kernel covers the
-// rest).  Every mbarrier wait is bounded.
+// rest).  Every mbarrier wait is bounded, and the CTA leaves the plane loop
+// only all together (barrier votes).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -34,15 +39,15 @@ namespace {
 constexpr int kRows = 128;
 constexpr int kThreads = 128;
 constexpr int kMaxKeys = 112;                     // padded keys per plane
+constexpr int kMaxPlanes = 4;                     // 2 brick layers + r_z = 1 on each side
 constexpr int kTileBytes = kMaxKeys * kDh * 2;    // 14 KiB, a multiple of 1 KiB
 constexpr int kQOff = 0;                          // 16 KiB query tile
 constexpr int kKV0 = kRows * kDh * 2;             // plane buffers: K at +0, V at +kTileBytes
+constexpr int kBufs = 3;
 constexpr int kBufBytes = 2 * kTileBytes;
-constexpr int kBarOff = kKV0 + 2 * kBufBytes;
-// Requesting more than a third of the SM's shared memory keeps at most two
-// CTAs per SM, matching the 2 x 256 tensor-memory columns.
-constexpr int kSmemBytes = 80 * 1024;
-static_assert(kBarOff + 64 + 1024 <= kSmemBytes, "shared memory plan");
+constexpr int kBarOff = kKV0 + kBufs * kBufBytes;
+constexpr int kSmemBytes = kBarOff + 64 + 1024;   // + barriers, + alignment slack
+static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
 constexpr float kRescaleThreshold = 8.0f;
 
 struct LocalArgs {
@@ -70,35 +75,32 @@ __device__ __forceinline__ void gather_row(uint32_t tile, int r, const __nv_bflo
   }
 }
 
-__device__ __forceinline__ void gather_plane(const LocalArgs& a, uint32_t kt, uint32_t vt, int g, int zp, int y0,
-                                             int x0) {
-  // 128 threads x NP rows x 2 tensors; each thread takes rows tid, tid+128, ...
-  // (NP <= 112 < 128: one row per thread, threads >= NP write nothing).
+// Packed index of this thread's gather row (row r = threadIdx.x of the padded
+// plane) in lattice plane zp, or -1 (padding or outside the volume).
+__device__ __forceinline__ int plane_row_index(const LocalArgs& a, int zp, int y0, int x0) {
+  const int r = threadIdx.x;
+  if (r >= a.PH * a.PW) return -1;
+  const int y = y0 - a.ry + r / a.PW, x = x0 - a.rx + r % a.PW;
+  if (y < 0 || y >= a.H || x < 0 || x >= a.W) return -1;
+  return __ldg(a.g2p + ((size_t)zp * a.H + y) * a.W + x);
+}
+
+// K and V rows of this thread's gather row into plane buffer (kt, vt).
+__device__ __forceinline__ void gather_plane(const LocalArgs& a, uint32_t kt, uint32_t vt, int g, int j) {
   const int r = threadIdx.x;
   if (r >= a.NP) return;
-  const __nv_bfloat16* ks = nullptr;
-  const __nv_bfloat16* vs = nullptr;
-  if (r < a.PH * a.PW) {
-    const int y = y0 - a.ry + r / a.PW, x = x0 - a.rx + r % a.PW;
-    if (y >= 0 && y < a.H && x >= 0 && x < a.W) {
-      const int j = __ldg(a.g2p + ((size_t)zp * a.H + y) * a.W + x);
-      if (j >= 0) {
-        ks = a.k + ((size_t)j * a.Hkv + g) * kDh;
-        vs = a.v + ((size_t)j * a.Hkv + g) * kDh;
-      }
-    }
-  }
-  gather_row(kt, r, ks, a.k);
-  gather_row(vt, r, vs, a.v);
+  gather_row(kt, r, j >= 0 ? a.k + ((size_t)j * a.Hkv + g) * kDh : nullptr, a.k);
+  gather_row(vt, r, j >= 0 ? a.v + ((size_t)j * a.Hkv + g) * kDh : nullptr, a.v);
 }
 
 __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
-  const uint32_t bar = sbase + kBarOff;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + 12);
+  const uint32_t s_full = sbase + kBarOff;        // S of the current plane is in tensor memory
+  const uint32_t pv_done = sbase + kBarOff + 8;   // O += P V of the last issued plane has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + 20);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int g = blockIdx.y;
 
@@ -115,7 +117,8 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
   const int h = g * 4 + hh;
 
   if (tid == 0) {
-    ptx::mbar_init(bar, 1);
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(pv_done, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -124,19 +127,24 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
     ptx::tmem_relinquish();
   }
 
-  // Query row gather (own row).
-  int qi = -1;
-  if (qvalid) qi = __ldg(a.g2p + ((size_t)qz * a.H + qy) * a.W + qx);
-  gather_row(sbase + kQOff, tid, qi >= 0 ? a.q + ((size_t)qi * a.Hq + h) * kDh : nullptr, a.q);
-
-  // Planes z0-1 .. z0+2 inside the volume.  cp.async groups: {Q, plane 0},
-  // {plane 1}, then one group per loop iteration (plane p + 2, possibly empty),
-  // so waiting until at most one group is pending always lands plane p.
+  // Every index-map lookup of the CTA at once: the query row and this
+  // thread's gather row of each plane z0-1 .. z0+2 inside the volume.
   const int zlo = max(0, z0 - 1), zhi = min(a.Z - 1, z0 + 2);
   const int nplanes = zhi - zlo + 1;
-  gather_plane(a, sbase + kKV0, sbase + kKV0 + kTileBytes, g, zlo, y0, x0);
+  const int qi = qvalid ? __ldg(a.g2p + ((size_t)qz * a.H + qy) * a.W + qx) : -1;
+  int gi[kMaxPlanes];
+#pragma unroll
+  for (int p = 0; p < kMaxPlanes; ++p) gi[p] = p < nplanes ? plane_row_index(a, zlo + p, y0, x0) : -1;
+
+  // cp.async groups: {Q, plane 0}, {plane 1}, {plane 2} (possibly empty), and
+  // later {plane 3} into plane 0's buffer.
+  auto kt_of = [&](int p) { return sbase + kKV0 + (p % kBufs) * kBufBytes; };
+  gather_row(sbase + kQOff, tid, qi >= 0 ? a.q + ((size_t)qi * a.Hq + h) * kDh : nullptr, a.q);
+  gather_plane(a, kt_of(0), kt_of(0) + kTileBytes, g, gi[0]);
   ptx::cp_async_commit();
-  if (nplanes > 1) gather_plane(a, sbase + kKV0 + kBufBytes, sbase + kKV0 + kBufBytes + kTileBytes, g, zlo + 1, y0, x0);
+  if (nplanes > 1) gather_plane(a, kt_of(1), kt_of(1) + kTileBytes, g, gi[1]);
+  ptx::cp_async_commit();
+  if (nplanes > 2) gather_plane(a, kt_of(2), kt_of(2) + kTileBytes, g, gi[2]);
   ptx::cp_async_commit();
 
   // Lattice-box mask of this row over the padded plane (bit k = key k
@@ -171,68 +179,102 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
   const uint32_t idescPV = ptx::idesc_bf16_f32(kRows, kDh, true);
   const float c = a.scale_log2;
 
-  float m_used = -INFINITY, l = 0.f;
-  uint32_t phase = 0;
-  bool ok = true;
-  for (int p = 0; p < nplanes && ok; ++p) {
-    const int zp = zlo + p;
-    const uint32_t kt = sbase + kKV0 + (p & 1) * kBufBytes, vt = kt + kTileBytes;
-    ptx::cp_async_wait_one();
-    ptx::fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      ptx::tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kDh / 16; ++kk)
-        ptx::mma_ss(tS, ptx::smem_desc_sw128(sbase + kQOff + kk * 32, 16, 1024),
-                    ptx::smem_desc_sw128(kt + kk * 32, 16, 1024), idescS, kk > 0);
-      ptx::tc_commit(bar);
-    }
-    __syncwarp();
-    if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar, phase, abort_flag)))) break;
-    phase ^= 1;
+  auto issue_s = [&](int p) {
     ptx::tc_fence_after();
+    const uint32_t kt = kt_of(p);
+#pragma unroll
+    for (int kk = 0; kk < kDh / 16; ++kk)
+      ptx::mma_ss(tmem, ptx::smem_desc_sw128(sbase + kQOff + kk * 32, 16, 1024),
+                  ptx::smem_desc_sw128(kt + kk * 32, 16, 1024), idescS, kk > 0);
+    ptx::tc_commit(s_full);
+  };
 
+  // S of plane 0 once Q and plane 0 are in shared memory (group 0 of 3).
+  ptx::cp_async_wait_two();
+  ptx::fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) issue_s(0);
+
+  float m_used = -INFINITY, l = 0.f;
+  bool ok = true;
+  int issued_pv = 0;
+  for (int p = 0; p < nplanes; ++p) {
+    const int zp = zlo + p;
     const bool uses = zp >= z0 + lz - 1 && zp <= z0 + lz + 1;  // warp-uniform (layer = warp / 2)
-    if (uses) {
-      uint32_t sv[kMaxKeys];
-#pragma unroll
-      for (int q = 0; q < kMaxKeys / 16; ++q)
-        if (q * 16 < a.NP) ptx::tmem_ld16_sync(tS + 16 * q, sv + 16 * q);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < kMaxKeys; ++k) {
-        const float sk = (mask[k >> 5] >> (k & 31)) & 1u ? __uint_as_float(sv[k]) : -INFINITY;
-        sv[k] = __float_as_uint(sk);
-        mx = fmaxf(mx, sk);
+    // S of plane p; each using warp keeps its rows in registers.
+    bool w_ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, p & 1, abort_flag));
+    uint32_t sv[kMaxKeys];
+    if (w_ok) {
+      ptx::tc_fence_after();
+      if (uses) {
+        ptx::tmem_ld64_sync(tS, sv);
+        ptx::tmem_ld48_sync(tS + 64, sv + 64);
       }
+    }
+    // Plane p+1 landed (groups: after plane 0 one more may be pending, later none).
+    if (p == 0) ptx::cp_async_wait_one(); else ptx::cp_async_wait_all();
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    if (!(ok = __syncthreads_and(w_ok))) break;
+    // Every warp has read S(p): S(p+1) may overwrite it and run under this
+    // plane's exponentials.
+    if (tid == 0 && p + 1 < nplanes) issue_s(p + 1);
+
+    float f = 1.f, rs = 0.f;
+    if (uses) {
+      // Masked row maximum: 8 independent max3 chains.
+      float m8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kMaxKeys; k += 2) {
+        const float s0 = (mask[k >> 5] >> (k & 31)) & 1u ? __uint_as_float(sv[k]) : -INFINITY;
+        const float s1 = (mask[(k + 1) >> 5] >> ((k + 1) & 31)) & 1u ? __uint_as_float(sv[k + 1]) : -INFINITY;
+        sv[k] = __float_as_uint(s0);
+        sv[k + 1] = __float_as_uint(s1);
+        float& mq = m8[(k >> 1) & 7];
+        asm("max.f32 %0, %0, %1, %2;" : "+f"(mq) : "f"(s0), "f"(s1));
+      }
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float mxs = mx * c;
-      float f = 1.f;
       if (m_used == -INFINITY) {
         m_used = mxs;            // first plane this row sees: its O row is still zero
       } else if (mxs > m_used + kRescaleThreshold) {
         f = ptx::ex2(m_used - mxs);
         m_used = mxs;
       }
+    }
+    // P and O are free again once O += P V of plane p-1 has completed.
+    if (p > 0) {
+      w_ok = __all_sync(0xffffffffu, ptx::mbar_wait(pv_done, (p - 1) & 1, abort_flag));
+      if (w_ok) ptx::tc_fence_after();
+    }
+    if (p == 1 && nplanes > 3 && w_ok) {
+      // Plane 0's buffer (read by S(0) and O += P V of plane 0, both done) takes plane 3.
+      gather_plane(a, kt_of(3), kt_of(3) + kTileBytes, g, gi[3]);
+    }
+    if (p == 1) ptx::cp_async_commit();
+    if (uses && w_ok) {
       // A row with no allowed key yet (only rows of sites outside the volume)
       // keeps P = 0 instead of exp2(-inf + inf).
       const float nm = m_used == -INFINITY ? 0.f : -m_used;
-      float rs = 0.f;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(nm, nm);
+      float2 r2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int q = 0; q < kMaxKeys / 16; ++q) {
         uint32_t pk[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[16 * q + 2 * k]), c, nm));
-          const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[16 * q + 2 * k + 1]), c, nm));
-          rs += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
+          const int i = 16 * q + 2 * k;
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, nm2);
+          const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+          r2[k & 1] = __fadd2_rn(r2[k & 1], pe);
+          pk[k] = pack_bf16x2(pe.x, pe.y);
         }
-        if (q * 16 < a.NP) ptx::tmem_st8(tP + 8 * q, pk);
+        ptx::tmem_st8(tP + 8 * q, pk);
       }
+      rs = (r2[0].x + r2[0].y) + (r2[1].x + r2[1].y);
       if (__any_sync(0xffffffffu, f != 1.f)) {
-        // PV of the previous plane completed before this plane's gather was
-        // waited on, so O is stable.
         uint32_t r[32];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -243,32 +285,28 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
         }
       }
       l = l * f + rs;
-    } else {
+    } else if (w_ok) {
       uint32_t zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-      for (int q = 0; q < kMaxKeys / 16; ++q)
-        if (q * 16 < a.NP) ptx::tmem_st8(tP + 8 * q, zero);
+      for (int q = 0; q < kMaxKeys / 16; ++q) ptx::tmem_st8(tP + 8 * q, zero);
     }
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
-    __syncthreads();
+    if (!(ok = __syncthreads_and(w_ok))) break;
     if (tid == 0) {
       ptx::tc_fence_after();
+      const uint32_t vt = kt_of(p) + kTileBytes;
       for (int kk = 0; kk < a.NP / 16; ++kk)
         ptx::mma_ts(tO, tmem + 128 + kk * 8, ptx::smem_desc_sw128(vt + kk * 2048, 8192, 1024), idescPV,
                     (p > 0 || kk > 0) ? 1u : 0u);
-      ptx::tc_commit(bar);
+      ptx::tc_commit(pv_done);
     }
-    __syncwarp();
-    if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar, phase, abort_flag)))) break;
-    phase ^= 1;
-    ptx::tc_fence_after();
-    // The buffer this plane used is free again: prefetch plane p + 2 into it.
-    if (p + 2 < nplanes) gather_plane(a, kt, vt, g, zlo + p + 2, y0, x0);
-    ptx::cp_async_commit();
+    issued_pv = p + 1;
   }
 
+  if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(pv_done, (nplanes - 1) & 1, abort_flag));
   if (ok) {
+    ptx::tc_fence_after();
     uint32_t r[2][32];
     ptx::tmem_ld64_sync(tO, &r[0][0]);
     if (qi >= 0) {
@@ -281,6 +319,10 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
                            __uint_as_float(r[q / 8][(4 * q + 2) % 32]) * inv,
                            __uint_as_float(r[q / 8][(4 * q + 3) % 32]) * inv);
     }
+  } else if (tid == 0) {
+    // Let whatever was issued drain before tensor memory is released.
+    ptx::tc_commit(pv_done);
+    ptx::mbar_wait(pv_done, issued_pv & 1, abort_flag);
   }
   ptx::cp_async_wait_all();
   ptx::tc_fence_before();

@@ -196,6 +196,20 @@ __device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t* r) {
       : "r"(taddr)
       : "memory");
 }
+// Columns taddr .. taddr+47: a 32-column and a 16-column load in flight, then the wait.
+__device__ __forceinline__ void tmem_ld48_sync(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "{ .reg .b32 ta;\n\t"
+      "add.u32 ta, %48, 32;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%48];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47}, "
+      "[ta];\n\t"
+      "tcgen05.wait::ld.sync.aligned; }"
+      : P3_R16(0), P3_R16(16), P3_R16(32)
+      : "r"(taddr)
+      : "memory");
+}
 #undef P3_R16
 #undef P3_R8
 #undef P3_W8
@@ -208,6 +222,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_two() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 // Makes this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core reads through descriptors).
 __device__ __forceinline__ void fence_proxy_async_smem() {
