@@ -26,7 +26,8 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: 
 
 ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
                 "pack3d_build_index", "pack3d_rope", "pack3d_rope_qk", "pack3d_build_summaries", "pack3d_local_attn",
-                "pack3d_summary_attn", "pack3d_forward", "pack3d_forward_noalloc", "pack3d_check_status",
+                "pack3d_summary_attn", "pack3d_forward", "pack3d_forward_noalloc", "pack3d_pipeline_create",
+                "pack3d_pipeline_destroy", "pack3d_host_workspace_bytes", "pack3d_forward_host", "pack3d_check_status",
                 "pack3d_status_string", "pack3d_backend_info")
 
 
@@ -78,6 +79,10 @@ def _load():
         "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "pack3d_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
         "pack3d_forward_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
+        "pack3d_pipeline_create": (ctypes.c_int, [ctypes.POINTER(P)]),
+        "pack3d_pipeline_destroy": (None, [P]),
+        "pack3d_host_workspace_bytes": (ctypes.c_size_t, [C]),
+        "pack3d_forward_host": (ctypes.c_int, [P, C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
         "pack3d_check_status": (ctypes.c_int, [P, P]),
         "pack3d_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "pack3d_backend_info": (ctypes.c_char_p, []),
@@ -200,6 +205,46 @@ def forward_noalloc(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, ou
     _check(lib.pack3d_forward_noalloc(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc),
                                       _ptr(k_cmp), _ptr(v_cmp), _ptr(scores), _ptr(gate), _ptr(out), _ptr(err),
                                       _stream(stream)), "pack3d_forward_noalloc")
+
+
+def _host_ptr(t) -> int:
+    if t.is_cuda:
+        raise ValueError("pack3d_forward_host takes host tensors (page-locked for asynchronous copies)")
+    if not t.is_contiguous():
+        raise ValueError("PACK3D takes contiguous tensors")
+    return t.data_ptr()
+
+
+def host_workspace_bytes(cfg: Config) -> int:
+    return int(lib.pack3d_host_workspace_bytes(ctypes.byref(cfg)))
+
+
+class Pipeline:
+    """The copy streams and events of pack3d_forward_host, bound to the current device."""
+
+    def __init__(self):
+        h = ctypes.c_void_p()
+        _check(lib.pack3d_pipeline_create(ctypes.byref(h)), "pack3d_pipeline_create")
+        self.handle = h
+
+    def close(self):
+        if self.handle:
+            lib.pack3d_pipeline_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        self.close()
+
+
+def forward_host(pipeline, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, workspace, err,
+                 stream=None):
+    """pack3d_forward from host tensors (inputs and `out`), copies overlapped with the stages; the result
+    is in `out` once the stream is synchronised."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pack3d_forward_host(pipeline.handle, ctypes.byref(cfg), _host_ptr(coords), _host_ptr(q),
+                                   _host_ptr(k_loc), _host_ptr(v_loc), _host_ptr(k_cmp), _host_ptr(v_cmp),
+                                   _host_ptr(scores), _host_ptr(gate), _host_ptr(out), _ptr(workspace), ws_bytes,
+                                   _ptr(err), _stream(stream)), "pack3d_forward_host")
 
 
 def check_status(err, stream=None) -> int:

@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <new>
+
 #include "common.cuh"
 #include "internal.h"
 #include "pack3d.h"
@@ -245,6 +247,182 @@ pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, co
   return cuda_status(e);
 }
 
+// ---- forward pass from host buffers -------------------------------------------
+
+}  // extern "C"
+
+// Streams and events of pack3d_forward_host, owned by the caller through the
+// opaque handle (the library itself keeps no state between calls).
+struct pack3d_pipeline {
+  int device;
+  cudaStream_t in, out;
+  cudaEvent_t start, coords, cmp, qk, vloc, gate, done;
+  cudaEvent_t chunk[PACK3D_HOST_MAX_CHUNKS];
+};
+
+namespace {
+
+// Device staging copies of the inputs and the output, after the regions of
+// the pack3d_forward workspace.
+struct Staging {
+  uintptr_t coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out;
+  size_t bytes;
+};
+
+Staging plan_staging(const pack3d_config& c, size_t base_off) {
+  const size_t N = (size_t)c.Z * c.H * c.W;
+  const size_t eb = elem_bytes(c.dtype);
+  const size_t A = 1024;
+  Staging g;
+  size_t off = round_up(base_off, A);
+  g.coords = off; off = round_up(off + N * 12, A);
+  g.q = off;      off = round_up(off + N * c.Hq * c.d_h * eb, A);
+  g.k_loc = off;  off = round_up(off + N * c.Hkv * c.d_h * eb, A);
+  g.v_loc = off;  off = round_up(off + N * c.Hkv * c.d_h * eb, A);
+  g.k_cmp = off;  off = round_up(off + N * c.Hkv * c.d_h * eb, A);
+  g.v_cmp = off;  off = round_up(off + N * c.Hkv * c.d_h * eb, A);
+  g.scores = off; off = round_up(off + N * c.Hkv * 4, A);
+  g.gate = off;   off = round_up(off + N * c.Hq * 8, A);
+  g.out = off;    off = round_up(off + N * c.Hq * c.d_h * eb, A);
+  g.bytes = off;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+pack3d_status pack3d_pipeline_create(pack3d_pipeline** out) {
+  if (!out) return PACK3D_ERR_INVALID_ARG;
+  *out = nullptr;
+  pack3d_pipeline* p = new (std::nothrow) pack3d_pipeline();
+  if (!p) return PACK3D_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->out, cudaStreamNonBlocking);
+  cudaEvent_t* evs[] = {&p->start, &p->coords, &p->cmp, &p->qk, &p->vloc, &p->gate, &p->done};
+  for (cudaEvent_t* ev : evs)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  for (int c = 0; c < PACK3D_HOST_MAX_CHUNKS && e == cudaSuccess; ++c)
+    e = cudaEventCreateWithFlags(&p->chunk[c], cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    pack3d_pipeline_destroy(p);
+    return PACK3D_ERR_CUDA;
+  }
+  *out = p;
+  return PACK3D_OK;
+}
+
+void pack3d_pipeline_destroy(pack3d_pipeline* p) {
+  if (!p) return;
+  cudaEvent_t evs[] = {p->start, p->coords, p->cmp, p->qk, p->vloc, p->gate, p->done};
+  for (cudaEvent_t ev : evs)
+    if (ev) cudaEventDestroy(ev);
+  for (int c = 0; c < PACK3D_HOST_MAX_CHUNKS; ++c)
+    if (p->chunk[c]) cudaEventDestroy(p->chunk[c]);
+  if (p->in) cudaStreamDestroy(p->in);
+  if (p->out) cudaStreamDestroy(p->out);
+  delete p;
+}
+
+size_t pack3d_host_workspace_bytes(const pack3d_config* cfg) {
+  if (pack3d_validate_config(cfg) != PACK3D_OK) return 0;
+  return plan_staging(*cfg, carve(*cfg, 0).bytes).bytes;
+}
+
+pack3d_status pack3d_forward_host(pack3d_pipeline* pl, const pack3d_config* cfg, const int32_t* coords,
+                                  const void* q, const void* k_loc, const void* v_loc, const void* k_cmp,
+                                  const void* v_cmp, const float* scores, const float* gate, void* out,
+                                  void* workspace, size_t workspace_bytes, int32_t* err_word, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (!pl || !coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !out || !err_word)
+    return PACK3D_ERR_INVALID_ARG;
+  if (!workspace || ((uintptr_t)workspace & 255u)) return PACK3D_ERR_WORKSPACE;
+  const Workspace w = carve(*cfg, (uintptr_t)workspace);
+  const Staging g = plan_staging(*cfg, w.bytes);
+  if (workspace_bytes < g.bytes) return PACK3D_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != pl->device) {
+    cudaGetLastError();
+    return PACK3D_ERR_INVALID_ARG;   // the pipeline belongs to another device
+  }
+  const Shape s = make_shape(*cfg);
+  const size_t N = (size_t)s.N, eb = elem_bytes(cfg->dtype);
+  const uintptr_t base = (uintptr_t)workspace;
+  auto dptr = [&](uintptr_t off) { return reinterpret_cast<void*>(base + off); };
+  const cudaStream_t cs = (cudaStream_t)stream, in = pl->in, outs = pl->out;
+  const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
+  const size_t qb = N * s.Hq * kDh * eb, kvb = N * s.Hkv * kDh * eb;
+
+  // The staging area may still be read by earlier work on `stream`.
+  cudaError_t e = cudaEventRecord(pl->start, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(in, pl->start, 0);
+  // Inputs in the order the stages need them, each group marked by an event.
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.coords), coords, N * 12, h2d, in);
+  if (e == cudaSuccess) e = cudaEventRecord(pl->coords, in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.k_cmp), k_cmp, kvb, h2d, in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.v_cmp), v_cmp, kvb, h2d, in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.scores), scores, N * s.Hkv * 4, h2d, in);
+  if (e == cudaSuccess) e = cudaEventRecord(pl->cmp, in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.k_loc), k_loc, kvb, h2d, in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.q), q, qb, h2d, in);
+  if (e == cudaSuccess) e = cudaEventRecord(pl->qk, in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.v_loc), v_loc, kvb, h2d, in);
+  if (e == cudaSuccess) e = cudaEventRecord(pl->vloc, in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dptr(g.gate), gate, N * s.Hq * 8, h2d, in);
+  if (e == cudaSuccess) e = cudaEventRecord(pl->gate, in);
+
+  // Each stage waits only for the copies it reads.
+  const int32_t* dcoords = (const int32_t*)dptr(g.coords);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, pl->coords, 0);
+  if (e == cudaSuccess) e = launch_build_index(s, dcoords, w.g2p, w.members, err_word, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, pl->cmp, 0);
+  if (e == cudaSuccess)
+    e = launch_summaries(s, cfg->dtype, w.members, dptr(g.k_cmp), dptr(g.v_cmp), (const float*)dptr(g.scores),
+                         w.k_sum, w.v_sum, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, pl->qk, 0);
+  if (e == cudaSuccess)
+    e = launch_rope(s, cfg->dtype, dcoords, dptr(g.q), w.q_rot, s.Hq, dptr(g.k_loc), w.k_rot, s.Hkv, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, pl->vloc, 0);
+  if (e == cudaSuccess)
+    e = launch_local(s, cfg->dtype, cfg->flags, w.g2p, w.q_rot, w.k_rot, dptr(g.v_loc), w.o_loc, err_word, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, pl->gate, 0);
+
+  // The query x summary stage in token chunks; each chunk's rows go back to
+  // the host on the second copy stream while the next chunk computes.
+  const float* dgate = (const float*)dptr(g.gate);
+  void* dout = dptr(g.out);
+  const size_t row_bytes = (size_t)s.Hq * kDh * eb;   // one token's output
+  const bool tc = cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY);
+  int chunks = 1;
+  long quantum = (long)N;
+  if (tc) {
+    quantum = summary_attn_tc_token_quantum(s);
+    // About 8 MiB of output per chunk, at most PACK3D_HOST_MAX_CHUNKS chunks.
+    chunks = (int)min((long)PACK3D_HOST_MAX_CHUNKS, max(1L, (long)(N * row_bytes / (8u << 20))));
+  }
+  const long per_chunk = ((long)N / chunks + quantum - 1) / quantum * quantum;
+  for (int c = 0; c < chunks && e == cudaSuccess; ++c) {
+    const long t0 = c * per_chunk, t1 = min((long)N, t0 + per_chunk);
+    if (t0 >= t1) break;
+    if (tc)
+      e = launch_summary_attn_tc(s, w.q_rot, w.k_sum, w.v_sum, w.o_loc, dgate, dout, err_word, cs, t0, t1);
+    else
+      e = launch_summary_attn_simt(s, cfg->dtype, w.q_rot, w.k_sum, w.v_sum, w.o_loc, dgate, dout, cs);
+    if (e == cudaSuccess) e = cudaEventRecord(pl->chunk[c], cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(outs, pl->chunk[c], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync((uint8_t*)out + t0 * row_bytes, (const uint8_t*)dout + t0 * row_bytes,
+                          (t1 - t0) * row_bytes, cudaMemcpyDeviceToHost, outs);
+  }
+  // Everything joins `stream`: synchronising it covers every copy.
+  if (e == cudaSuccess) e = cudaEventRecord(pl->done, outs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, pl->done, 0);
+  return cuda_status(e);
+}
+
 pack3d_status pack3d_check_status(int32_t* err_word, void* stream) {
   if (!err_word) return PACK3D_ERR_INVALID_ARG;
   int32_t h = 0;
@@ -274,10 +452,11 @@ const char* pack3d_status_string(pack3d_status s) {
 }
 
 const char* pack3d_backend_info(void) {
-  return "pack3d sm_100a: index map + axial RoPE + summaries (CUDA cores, 16-byte streams, shared-memory "
-         "cos/sin tables); local attention (CUDA cores, lattice bricks, float accumulation); query x summary "
-         "(bf16: tcgen05 MMA, TMEM accumulators, TMA 4-stage ring, two ping-pong softmax warpgroups; float: "
-         "CUDA cores)";
+  return "pack3d sm_100a: index map; axial RoPE (CUDA cores, 16-byte streams, shared-memory cos/sin tables); "
+         "summaries (warp per block, rotation split R(c_base) R(d)); local attention (bf16 G=4: tcgen05 MMA on "
+         "2x4x4 query bricks with gathered halo planes; else CUDA cores); query x summary (bf16: tcgen05 MMA, "
+         "TMEM accumulators, TMA 5-stage ring, two softmax warpgroups with one MMA warp each; float: CUDA "
+         "cores); host-buffer pipeline with copies overlapped on two copy streams";
 }
 
 }  // extern "C"

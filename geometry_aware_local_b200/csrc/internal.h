@@ -38,9 +38,12 @@ cudaError_t launch_summary_attn_simt(const Shape& s, int dtype, const void* qr, 
                                      const void* vs, const float* oloc, const float* gate,
                                      void* out, cudaStream_t st);
 
-// tcgen05 query x summary kernel (bf16 only).
+// tcgen05 query x summary kernel (bf16 only), for the tokens [tok_begin,
+// tok_end) (tok_end < 0: to the end); tok_begin must be a multiple of
+// summary_attn_tc_token_quantum(s), the tokens one CTA covers.
 cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
                                    const float* oloc, const float* gate, void* out, int32_t* err,
-                                   cudaStream_t st);
+                                   cudaStream_t st, long tok_begin = 0, long tok_end = -1);
+long summary_attn_tc_token_quantum(const Shape& s);
 
 }  // namespace pack3d

@@ -96,7 +96,8 @@ struct TcArgs {
   int M;             // summaries
   int G;             // q heads per kv head
   int Hq;
-  long rows;         // N * G rows per kv head
+  long rows;         // rows of this launch end here (token end * G)
+  int tile_base;     // first 128-row tile of this launch
   float scale_log2;  // softmax scale * log2(e)
   const float* oloc;
   const float* gate;
@@ -137,7 +138,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
-  const int tile0 = blockIdx.x * kGroups;
+  const int tile0 = a.tile_base + blockIdx.x * kGroups;
   const int T = (a.M + kBN - 1) / kBN;
 
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -463,9 +464,14 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
 
 }  // namespace
 
+long summary_attn_tc_token_quantum(const Shape& s) { return (long)kGroups * kBM / s.G; }
+
 cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
                                    const float* oloc, const float* gate, void* out, int32_t* err,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, long tok_begin, long tok_end) {
+  if (tok_end < 0) tok_end = s.N;
+  if (tok_begin < 0 || tok_begin >= tok_end || tok_end > s.N || tok_begin % summary_attn_tc_token_quantum(s))
+    return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   // Q viewed as [N][Hkv][G][64]: a box of 128/G tokens x G heads x 64 dims is one 128-row tile.
   const cuuint64_t qd[4] = {(cuuint64_t)kDh, (cuuint64_t)s.G, (cuuint64_t)s.Hkv, (cuuint64_t)s.N};
@@ -483,13 +489,14 @@ cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* k
   a.M = s.M;
   a.G = s.G;
   a.Hq = s.Hq;
-  a.rows = (long)s.N * s.G;
+  a.rows = tok_end * s.G;
+  a.tile_base = (int)(tok_begin * s.G / kBM);
   a.scale_log2 = s.scale_log2;
   a.oloc = oloc;
   a.gate = gate;
   a.out = (__nv_bfloat16*)out;
   a.err = err;
-  const long tiles = (a.rows + kBM - 1) / kBM;
+  const long tiles = (a.rows - tok_begin * s.G + kBM - 1) / kBM;
   dim3 grid((unsigned)((tiles + kGroups - 1) / kGroups), s.Hkv);
   summary_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
   return cudaGetLastError();

@@ -219,6 +219,48 @@ pack3d_status pack3d_forward_noalloc(const pack3d_config *cfg, const int32_t *co
                                      const float *gate, void *out, int32_t *err_word,
                                      void *stream);
 
+/* ---- forward pass from host buffers ------------------------------------------
+ * Not part of the paper's method: a deployment entry point that copies the
+ * inputs in, runs the forward pass and copies the output back, with the
+ * copies overlapped with the stages that do not read them. */
+
+/* Largest number of row chunks pack3d_forward_host splits the query x summary
+ * stage into (each chunk's output goes back while the next one computes). */
+#define PACK3D_HOST_MAX_CHUNKS 8
+
+/* Opaque: the two copy streams and the events of pack3d_forward_host, bound to
+ * the device current at creation.  Created and destroyed by the caller; one
+ * pipeline must not be used by two calls at the same time. */
+typedef struct pack3d_pipeline pack3d_pipeline;
+pack3d_status pack3d_pipeline_create(pack3d_pipeline **pipeline);
+void pack3d_pipeline_destroy(pack3d_pipeline *pipeline);
+
+/* Bytes of device workspace pack3d_forward_host needs: the pack3d_forward
+ * workspace plus device copies of every input and of the output (0 on an
+ * invalid config). */
+size_t pack3d_host_workspace_bytes(const pack3d_config *cfg);
+
+/* pack3d_forward from HOST buffers: coords, q, k_loc, v_loc, k_cmp, v_cmp,
+ * scores, gate and out are host pointers with the layouts of pack3d_forward
+ * (page-locked memory makes the copies asynchronous; pageable memory works but
+ * the copies then block the host).  The inputs are copied, in the order the
+ * stages read them, on the pipeline's first copy stream; each stage runs on
+ * `stream` as soon as its own inputs have arrived; the query x summary stage
+ * runs in up to PACK3D_HOST_MAX_CHUNKS token chunks whose outputs are copied
+ * back on the second copy stream while the next chunk computes.  All the work
+ * joins `stream` before the call's work ends there: the output is in `out`
+ * once `stream` is synchronised (pack3d_check_status does that).  workspace:
+ * device, 256-byte aligned, at least pack3d_host_workspace_bytes(cfg) bytes,
+ * not touched by other work until `stream` is synchronised.  err_word:
+ * device int32, as pack3d_forward.  Errors: as pack3d_forward; a pipeline made
+ * on another device -> PACK3D_ERR_INVALID_ARG. */
+pack3d_status pack3d_forward_host(pack3d_pipeline *pipeline, const pack3d_config *cfg,
+                                  const int32_t *coords, const void *q, const void *k_loc,
+                                  const void *v_loc, const void *k_cmp, const void *v_cmp,
+                                  const float *scores, const float *gate, void *out,
+                                  void *workspace, size_t workspace_bytes, int32_t *err_word,
+                                  void *stream);
+
 /* Synchronises `stream`, reads the device error word, resets it to 0 and maps
  * it: COORD_RANGE/DUPLICATE -> PACK3D_ERR_NOT_PERMUTATION, TIMEOUT ->
  * PACK3D_ERR_TIMEOUT, none -> PACK3D_OK.  A failed CUDA call -> PACK3D_ERR_CUDA. */

@@ -86,6 +86,11 @@ def test_host_errors_return_before_launch(p3):
     assert lib.pack3d_forward(cfgp, *args, fake + 16, ws, fake, None) == 6
     assert lib.pack3d_forward(cfgp, *args, fake, ws, None, None) == 1
     assert lib.pack3d_check_status(None, None) == 1
+    # the host-buffer pipeline: no pipeline handle, then a workspace too small for the staging copies
+    hws = p3.host_workspace_bytes(c)
+    assert hws > ws + 50 * 1024 * 1024
+    assert lib.pack3d_forward_host(None, cfgp, *args, fake, hws, fake, None) == 1
+    assert lib.pack3d_forward_host(fake, cfgp, *args, fake, ws, fake, None) == 6
     for st in range(9):
         assert lib.pack3d_status_string(st)
     assert b"sm_100a" in lib.pack3d_backend_info()

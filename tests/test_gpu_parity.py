@@ -167,6 +167,29 @@ def test_rope_qk_equals_two_rope_calls(p3, dtype):
     assert torch.equal(qa, qb) and torch.equal(ka, kb)
 
 
+@pytest.mark.parametrize("name", ["tiny", "small", "65k"])
+def test_forward_host_equals_forward(p3, name):
+    """The host-buffer pipeline (copies overlapped, summary stage in token chunks) gives exactly the
+    device-buffer forward pass's output."""
+    s = {"tiny": synth.CONFIGS["tiny"], "small": small(Z=4, H=16, W=24), "65k": synth.CONFIGS["65k"]}[name]
+    inp = synth.make_inputs(s, s.packing, seed=5)
+    d = to_dev(inp)
+    ref = run_forward(p3, s, d)
+    cfg = p3.config_from_shape(s)
+    names = ("coords", "q", "k_loc", "v_loc", "k_cmp", "v_cmp", "scores", "gate")
+    hin = {k: inp[k].contiguous().pin_memory() for k in names}
+    hout = torch.empty(tuple(ref.shape), dtype=ref.dtype).pin_memory()
+    ws = torch.empty(p3.host_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    pipe = p3.Pipeline()
+    for _ in range(2):   # a second call reuses the pipeline and the staging area
+        hout.zero_()
+        p3.forward_host(pipe, cfg, *(hin[k] for k in names), hout, ws, err)
+        assert p3.check_status(err) == 0
+        assert torch.equal(hout, ref.cpu())
+    pipe.close()
+
+
 @pytest.mark.parametrize("name", ["small", "65k"])
 def test_forward_is_deterministic(p3, name):
     # Every kernel computes each output from a fixed sequence of operations, so
