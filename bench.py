@@ -49,7 +49,7 @@ KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summ
 # DRAM bytes (read + write) of one summary_attn_tc_kernel launch, from an ncu
 # capture of this workload (profiles/summary_attn_tc_65k.md).  Set back to
 # None whenever that kernel changes until it is captured again.
-SUMMARY_ATTN_TRAFFIC = {"65k": 212.698624e6 + 48.737024e6}
+SUMMARY_ATTN_TRAFFIC = {"65k": 212.722432e6 + 48.2944e6}
 
 
 def load_peaks():
