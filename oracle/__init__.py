@@ -58,6 +58,7 @@ def _load():
         lib.orc_build_index.restype = ctypes.c_int
         lib.orc_rotate.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_long]
         lib.orc_summaries.argtypes = [P, P, P, P, P, P, P, P]
+        lib.orc_summaries_center.argtypes = [P, P, P, P, P, P, P]
         lib.orc_local_attn.argtypes = [P, P, P, P, P, P, P, ctypes.c_long, P]
         lib.orc_summary_attn.argtypes = [P, P, P, P, ctypes.c_long, ctypes.c_long, P]
         lib.orc_gate_mix.argtypes = [P, P, P, ctypes.c_long, P, P, P]
@@ -121,15 +122,23 @@ def rotate(s, coords, x, heads: Optional[int] = None) -> np.ndarray:
     return y
 
 
-def summaries(s, coords, members, k_cmp, v_cmp, scores):
-    """Rotate-before-compress summaries (Key design 2, equations k~_j^R and v~_j)."""
+def summaries(s, coords, members, k_cmp, v_cmp, scores, center: bool = False):
+    """Rotate-before-compress summaries (Key design 2, equations k~_j^R and v~_j).
+
+    center=True: the summary-centre variant (contribution 2 and "Future Directions" 3 of the
+    summary page): the pooled key is left unrotated and rotated once by the block's geometric
+    centre (a fractional coordinate); v~ is unchanged."""
     c, m = _i32(coords), _i32(members)
     kc, vc, sc = as_f64(k_cmp), as_f64(v_cmp), as_f64(scores)
     ks = np.empty((s.M, s.Hkv, s.d_h))
     vs = np.empty((s.M, s.Hkv, s.d_h))
     cfg = _cfg(s)
-    _load().orc_summaries(ctypes.byref(cfg), _ptr(c), _ptr(m), _ptr(kc), _ptr(vc), _ptr(sc),
-                          _ptr(ks), _ptr(vs))
+    if center:
+        _load().orc_summaries_center(ctypes.byref(cfg), _ptr(m), _ptr(kc), _ptr(vc), _ptr(sc), _ptr(ks),
+                                     _ptr(vs))
+    else:
+        _load().orc_summaries(ctypes.byref(cfg), _ptr(c), _ptr(m), _ptr(kc), _ptr(vc), _ptr(sc),
+                              _ptr(ks), _ptr(vs))
     return ks, vs
 
 

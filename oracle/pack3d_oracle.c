@@ -14,6 +14,10 @@
  *                                  (a packing is a bijection onto the lattice).
  *   - axial RoPE ................. "Key design 1", equation R(c).
  *   - summaries .................. "Key design 2", equations k~_j^R and v~_j.
+ *   - summary-centre variant ..... the summary's "What This Paper Is About"
+ *                                  (contribution 2) and "Future Directions" 3:
+ *                                  the cheaper variant that rotates the pooled
+ *                                  key by the block centre only.
  *   - local branch ............... "Key design 3" (neighbourhood N(i)); summary
  *                                  "local attention stays exact".
  *   - compressed branch .......... "Key design 3" / summary "every token attends
@@ -81,19 +85,20 @@ int orc_build_index(const orc_cfg *c, const int32_t *coords, int32_t *g2p, int32
 
 /* ---- axial grid RoPE, equation R(c) ------------------------------------ */
 
-/* Angle of rotary pair p for coordinate (z,y,x); returns 0 for untouched dims
- * through *active = 0. */
-static double pair_angle(const orc_cfg *c, int p, int z, int y, int x, int *active)
+/* Angle of rotary pair p for coordinate (z,y,x) (a lattice site, or the
+ * fractional centre of a block); returns 0 for untouched dims through
+ * *active = 0. */
+static double pair_angle(const orc_cfg *c, int p, double z, double y, double x, int *active)
 {
     int axis_pairs[3] = {c->mz, c->my, c->mx};
-    int coord[3] = {z, y, x};
+    double coord[3] = {z, y, x};
     int first = 0;
     for (int a = 0; a < 3; ++a) {
         if (p < first + axis_pairs[a]) {
             int r = p - first;
             double omega = pow(c->base, -(double)r / (double)axis_pairs[a]);
             *active = 1;
-            return omega * (double)coord[a];
+            return omega * coord[a];
         }
         first += axis_pairs[a];
     }
@@ -102,7 +107,7 @@ static double pair_angle(const orc_cfg *c, int p, int z, int y, int x, int *acti
 }
 
 /* y = R(c) x for one head vector of d_h values at coordinate (cz,cy,cx). */
-static void rotate_row(const orc_cfg *c, int cz, int cy, int cx, const double *xi, double *yi)
+static void rotate_row(const orc_cfg *c, double cz, double cy, double cx, const double *xi, double *yi)
 {
     for (int p = 0; p < c->dh / 2; ++p) {
         int active;
@@ -179,6 +184,54 @@ void orc_summaries(const orc_cfg *c, const int32_t *coords, const int32_t *membe
 }
 
 /* ---- exact local branch ------------------------------------------------ */
+
+/* The summary-centre variant: the same block weights a_{j,u}, the pooled
+ * key left unrotated and then rotated once by the block's geometric centre,
+ *   k~_j = R(cbar_j) sum_u a_{j,u} k_u,
+ *   cbar_j = block origin + ((bz-1)/2, (by-1)/2, (bx-1)/2)
+ * (a fractional coordinate); v~_j as in orc_summaries. */
+void orc_summaries_center(const orc_cfg *c, const int32_t *members, const double *kcmp,
+                          const double *vcmp, const double *scores, double *ksum, double *vsum)
+{
+    long N = (long)c->Z * c->H * c->W;
+    int v = c->bz * c->by * c->bx;
+    long M = N / v;
+    int nby = c->H / c->by, nbx = c->W / c->bx;
+    int d = c->dh, Hkv = c->Hkv;
+#pragma omp parallel for schedule(static)
+    for (long j = 0; j < M; ++j) {
+        double *a = (double *)malloc(sizeof(double) * v);
+        double *kp = (double *)malloc(sizeof(double) * d);
+        long jx = j % nbx, jy = (j / nbx) % nby, jz = j / ((long)nbx * nby);
+        double cz = jz * c->bz + 0.5 * (c->bz - 1);
+        double cy = jy * c->by + 0.5 * (c->by - 1);
+        double cx = jx * c->bx + 0.5 * (c->bx - 1);
+        for (int g = 0; g < Hkv; ++g) {
+            double smax = -INFINITY, den = 0.0;
+            for (int t = 0; t < v; ++t) {
+                double s = scores[(long)members[j * v + t] * Hkv + g];
+                if (s > smax) smax = s;
+            }
+            for (int t = 0; t < v; ++t) {
+                a[t] = exp(scores[(long)members[j * v + t] * Hkv + g] - smax);
+                den += a[t];
+            }
+            for (int t = 0; t < v; ++t) a[t] /= den;
+            double *vs = vsum + (j * Hkv + g) * d;
+            for (int e = 0; e < d; ++e) { kp[e] = 0.0; vs[e] = 0.0; }
+            for (int t = 0; t < v; ++t) {
+                long u = members[j * v + t];
+                for (int e = 0; e < d; ++e) {
+                    kp[e] += a[t] * kcmp[(u * Hkv + g) * d + e];
+                    vs[e] += a[t] * vcmp[(u * Hkv + g) * d + e];
+                }
+            }
+            rotate_row(c, cz, cy, cx, kp, ksum + (j * Hkv + g) * d);
+        }
+        free(a);
+        free(kp);
+    }
+}
 
 /* For each sampled packed row i = rows[r] and q head h, with g = kv head of h:
  *   N(i) = tokens at lattice sites within the clipped box of radii (rz,ry,rx)

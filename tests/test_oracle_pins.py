@@ -240,6 +240,60 @@ def test_summaries_uniform_scores_mean_pool_and_unit_blocks():
     assert np.abs(ks1 - rope_complex(s, coords, oracle.as_f64(inp["k_cmp"]))[order]).max() < 1e-12
 
 
+# ------------------------------------------------- summary-centre variant -----
+# The cheaper variant the summary page names (contribution 2, "Future
+# Directions" 3): pooled key unrotated, then rotated by the block centre.
+
+def _block_centres(s):
+    """Geometric centre of every block (raster over the block grid), fractional."""
+    nbz, nby, nbx = s.Z // s.bz, s.H // s.by, s.W // s.bx
+    jz, jy, jx = np.meshgrid(np.arange(nbz), np.arange(nby), np.arange(nbx), indexing="ij")
+    return np.stack([jz.ravel() * s.bz + (s.bz - 1) / 2, jy.ravel() * s.by + (s.by - 1) / 2,
+                     jx.ravel() * s.bx + (s.bx - 1) / 2], axis=1)
+
+
+def test_summary_center_unit_blocks_equal_token_before():
+    s = small(by=1, bx=1)
+    inp, g2p, mem = _summary_case(s)
+    coords = inp["coords"].numpy()
+    kt, vt = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"])
+    kc, vc = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"], center=True)
+    assert np.abs(kc - kt).max() < 1e-12 and np.abs(vc - vt).max() == 0
+
+
+@pytest.mark.parametrize("blocks", [(1, 4, 4), (2, 2, 2), (1, 2, 4)])
+def test_summary_center_is_pooled_key_rotated_at_block_centre(blocks):
+    s = small(Z=4, bz=blocks[0], by=blocks[1], bx=blocks[2])
+    inp, g2p, mem = _summary_case(s, seed=7)
+    coords = inp["coords"].numpy()
+    kc = oracle.as_f64(inp["k_cmp"])
+    a = scipy.special.softmax(oracle.as_f64(inp["scores"])[mem], axis=1)      # [M, v, Hkv]
+    pooled = np.einsum("jug,jugd->jgd", a, kc[mem])
+    expect = rope_complex(s, _block_centres(s), pooled)
+    got, _ = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"], center=True)
+    assert np.abs(got - expect).max() < 1e-12
+
+
+def test_summary_center_error_within_rotation_bound():
+    # Per plane ||R(t1) - R(t2)|| = 2 |sin((t1 - t2) / 2)|, so the key difference of the two
+    # variants is at most sum_u a_u * max_p 2|sin(omega_p (cbar - c_u)_axis(p) / 2)| * ||k_u||.
+    s = small(Z=2, H=8, W=8)
+    inp, g2p, mem = _summary_case(s, seed=9)
+    coords = inp["coords"].numpy()
+    kt, _ = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"])
+    kc, _ = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"], center=True)
+    a = scipy.special.softmax(oracle.as_f64(inp["scores"])[mem], axis=1)
+    knorm = np.linalg.norm(oracle.as_f64(inp["k_cmp"])[mem], axis=-1)          # [M, v, Hkv]
+    omegas = [s.rope_base ** (-np.arange(m) / m) for m in (s.m_z, s.m_y, s.m_x)]
+    delta = _block_centres(s)[:, None, :] - coords[mem].astype(np.float64)       # [M, v, 3]
+    bound_u = np.max(np.stack([np.max(2 * np.abs(np.sin(om[None, None, :] * delta[..., ax:ax + 1] / 2)), axis=-1)
+                               for ax, om in enumerate(omegas)]), axis=0)          # [M, v]
+    bound = np.einsum("jug,ju,jug->jg", a, bound_u, knorm)
+    diff = np.linalg.norm(kc - kt, axis=-1)
+    assert (diff <= bound + 1e-12).all()
+    assert diff.max() > 1e-3          # an approximation, not the identity
+
+
 # ----------------------------------------------------------- branches -------
 
 def _lattice_dist_mask(coords_q, coords_k, s):
