@@ -170,7 +170,7 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def cpu_oracle_sample(s, inp, target_s: float = 12.0):
+def cpu_oracle_sample(s, inp, target_s: float = 12.0, center: bool = False):
     """Times the oracle on this workload: the whole-volume stages (index map, K_loc
     rotation, summaries) once, the per-query stages on a sample of rows sized to
     about ``target_s`` seconds, extrapolated to all N rows.  Returns a dict."""
@@ -181,7 +181,7 @@ def cpu_oracle_sample(s, inp, target_s: float = 12.0):
     st, g2p, mem = oracle.build_index(s, inp["coords"])
     coords = inp["coords"].numpy()
     klr = oracle.rotate(s, coords, inp["k_loc"])
-    ks, vs = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"])
+    ks, vs = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"], center=center)
     t_shared = time.perf_counter() - t0
 
     def per_rows(count, seed):
@@ -229,6 +229,39 @@ def run_reference(args, s):
     print(json.dumps(line), flush=True)
 
 
+def summary_center_error(p3, s, d, q_rot, members, err, stream, rows: int = 2048):
+    """Logit and output error of the summary-centre variant against the exact form, on the GPU
+    outside the timed region: both variants' summaries, the logits of a seeded sample of query rows
+    against every summary, and the two whole forward outputs."""
+    import torch
+    out = {}
+    ks, vs, outs = {}, {}, {}
+    for name, flags in (("exact", 0), ("center", p3.FLAG_SUMMARY_CENTER)):
+        cfg = p3.config_from_shape(s, flags)
+        k = torch.empty(s.M, s.Hkv, s.d_h, dtype=d["q"].dtype, device=d["q"].device)
+        v = torch.empty_like(k)
+        p3.build_summaries(cfg, members, d["k_cmp"], d["v_cmp"], d["scores"], k, v, stream)
+        ks[name] = k.float()
+        op = p3.Pack3D(cfg, d["q"].device)
+        outs[name] = op(d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
+                        d["gate"]).float()
+        op.check()
+    torch.cuda.synchronize()
+    rows = max(64, min(rows, (1 << 27) // (s.Hq * s.M)))   # logits of at most 2^27 floats
+    gen = torch.Generator(device="cpu").manual_seed(0)
+    r = torch.randint(0, s.N, (rows,), generator=gen).to(q_rot.device)
+    q = q_rot[r].float()                                              # [rows, Hq, d]
+    kv = [(h * s.Hkv) // s.Hq for h in range(s.Hq)]
+    le = torch.einsum("rhd,mhd->rhm", q, ks["exact"][:, kv, :]) * s.softmax_scale
+    lc = torch.einsum("rhd,mhd->rhm", q, ks["center"][:, kv, :]) * s.softmax_scale
+    out["logit_rel_rms"] = float((lc - le).norm() / le.norm())
+    out["logit_max_abs_diff"] = float((lc - le).abs().max())
+    out["logit_max_abs"] = float(le.abs().max())
+    out["out_rel_rms"] = float((outs["center"] - outs["exact"]).norm() / outs["exact"].norm())
+    out["query_rows_sampled"] = rows
+    return out
+
+
 def run_ours(args, s):
     import torch
 
@@ -237,7 +270,7 @@ def run_ours(args, s):
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cfg = p3.config_from_shape(s)
+    cfg = p3.config_from_shape(s, p3.FLAG_SUMMARY_CENTER if args.summary_center else 0)
     inp_host = synth.make_inputs(s, s.packing, seed=rank)
     names = ("coords", "q", "k_loc", "v_loc", "k_cmp", "v_cmp", "scores", "gate")
     d = {k: inp_host[k].to(dev) for k in names}
@@ -358,6 +391,7 @@ def run_ours(args, s):
             e["tflops"] = w["flops"] / t / 1e12
             e["tensor_frac"] = e["tflops"] / peaks["bf16_tflops"]
         stages[name] = e
+    variant_err = summary_center_error(p3, s, d, qr, mem, err, stream) if args.summary_center else None
     sa = stages["summary_attn"]
     roof = {"bound": "tensor", "achieved": sa["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": sa["tflops"] / peaks["bf16_tflops"], "traffic": SUMMARY_ATTN_TRAFFIC.get(args.config),
@@ -370,15 +404,19 @@ def run_ours(args, s):
             "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT[args.config], "tokens": s.N, "summaries": s.M,
                        "parallelism": "replicas only" if world > 1 else "single GPU",
+                       "summary_form": "summary-centre variant" if args.summary_center
+                       else "rotate-before-compress (exact)",
                        "l2": "flushed between steps (256 MiB write, outside the timed events)"},
             "e2e": {"value": s.N * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "roofline": roof, "stages": stages, "forward_call_ms": fwd,
             "clocks": clk.summary()}
+    if variant_err is not None:
+        line["summary_center_vs_exact"] = variant_err
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_oracle_sample(s, inp_host, target_s=12.0)
+            cb = cpu_oracle_sample(s, inp_host, target_s=12.0, center=args.summary_center)
             cb.pop("seconds")
             line["cpu_baseline"] = cb
         print(json.dumps(line), flush=True)
@@ -396,6 +434,9 @@ def main():
     ap.add_argument("--config", default="65k", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--summary-center", action="store_true",
+                    help="time the summary-centre variant of the block summaries and report its error "
+                         "against the exact rotate-before-compress form")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

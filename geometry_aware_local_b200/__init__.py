@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libpack3d.so")
 F32, BF16 = 0, 1
 FLAG_SIMT_SUMMARY = 0x1
 FLAG_SIMT_LOCAL = 0x2
+FLAG_SUMMARY_CENTER = 0x4     # summary-centre variant of the block summaries (include/pack3d.h)
 DEVERR_COORD_RANGE, DEVERR_DUPLICATE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: "NOT_PERMUTATION",

@@ -28,6 +28,7 @@ Shape make_shape(const pack3d_config& c) {
   s.tab_entries = c.Z * c.m_z + c.H * c.m_y + c.W * c.m_x;
   s.scale = c.softmax_scale;
   s.scale_log2 = (float)((double)c.softmax_scale * 1.4426950408889634);
+  s.center = (c.flags & PACK3D_FLAG_SUMMARY_CENTER) ? 1 : 0;
   const int m[3] = {c.m_z, c.m_y, c.m_x};
   const int ext[3] = {c.Z, c.H, c.W};
   int p = 0, off = 0;
@@ -130,7 +131,8 @@ pack3d_status pack3d_validate_config(const pack3d_config* c) {
   if (!(c->softmax_scale > 0.f) || !isfinite(c->softmax_scale)) return PACK3D_ERR_INVALID_ARG;
   const long long tab = (long long)c->Z * c->m_z + (long long)c->H * c->m_y + (long long)c->W * c->m_x;
   if (tab * 8 > kMaxTableBytes) return PACK3D_ERR_SHAPE;
-  if (c->flags & ~(PACK3D_FLAG_SIMT_SUMMARY | PACK3D_FLAG_SIMT_LOCAL)) return PACK3D_ERR_INVALID_ARG;
+  if (c->flags & ~(PACK3D_FLAG_SIMT_SUMMARY | PACK3D_FLAG_SIMT_LOCAL | PACK3D_FLAG_SUMMARY_CENTER))
+    return PACK3D_ERR_INVALID_ARG;
   return PACK3D_OK;
 }
 

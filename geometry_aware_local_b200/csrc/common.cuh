@@ -31,6 +31,7 @@ struct Shape {
   double omega[kMaxPairs];        // per rotary plane p: base^(-r/m_axis), 0 if unused
   int pair_axis[kMaxPairs];       // 0 = z, 1 = y, 2 = x, 3 = untouched
   int pair_off[kMaxPairs];        // first table entry of plane p
+  int center;                     // summaries: rotate the pooled key at the block centre
 };
 
 Shape make_shape(const pack3d_config& c);
@@ -137,6 +138,23 @@ struct PlaneLut {
     }
   }
 };
+
+// Rotates the 2*NP values f (planes p0 .. p0+NP-1) by R at the coordinate
+// (z, y, x), which may be fractional (a block centre): the angles are formed
+// directly, without the integer-coordinate tables.
+template <int NP>
+__device__ __forceinline__ void rotate_at(float* f, const Shape& s, int p0, double z, double y, double x) {
+#pragma unroll
+  for (int k = 0; k < NP; ++k) {
+    const int p = p0 + k;
+    if (p >= s.npairs || s.pair_axis[p] == 3) continue;
+    const int a = s.pair_axis[p];
+    const float2 cs = rope_cos_sin(s.omega[p] * (a == 0 ? z : (a == 1 ? y : x)));
+    const float x0 = f[2 * k], x1 = f[2 * k + 1];
+    f[2 * k] = x0 * cs.x - x1 * cs.y;
+    f[2 * k + 1] = x0 * cs.y + x1 * cs.x;
+  }
+}
 
 __device__ __forceinline__ void set_err(int32_t* err, int bits) {
   if (err) atomicOr(err, bits);

@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kSumThreads) summaries_kernel(
         if (t >= vol || mts[b] < 0) continue;
         float f[NE];
         chunk_to_float(rowc[b], f, T());
-        if (!is_v) {
+        if (!is_v && !s.center) {
           const int tz = t / (s.by * s.bx), ty = (t / s.bx) % s.by, tx = t % s.bx;
           lut.rotate(f, tab, jz * s.bz + tz, jy * s.by + ty, jx * s.bx + tx);
         }
@@ -230,6 +230,9 @@ __global__ void __launch_bounds__(kSumThreads) summaries_kernel(
         for (int k = 0; k < NE; ++k) acc[k] = fmaf(ats[b], f[k], acc[k]);
       }
     }
+    if (!is_v && s.center)
+      rotate_at<NP>(acc, s, part * NP, jz * s.bz + 0.5 * (s.bz - 1), jy * s.by + 0.5 * (s.by - 1),
+                    jx * s.bx + 0.5 * (s.bx - 1));
     T* dst = is_v ? vs : ks;
     stg16(dst + ((size_t)j * s.Hkv + g) * kDh + part * NE, float_to_chunk(acc, T()));
   }
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(kSumThreads) summaries_generic_kernel(
       const uint4 c = ldg16(src + ((size_t)m * s.Hkv + g) * kDh + part * NE);
       float f[NE];
       chunk_to_float(c, f, T());
-      if (!is_v) {
+      if (!is_v && !s.center) {
         const int tz = t / (s.by * s.bx), ty = (t / s.bx) % s.by, tx = t % s.bx;
         PlaneLut<NE / 2> lut;
         lut.init(s, part * (NE / 2));
@@ -295,6 +298,9 @@ __global__ void __launch_bounds__(kSumThreads) summaries_generic_kernel(
 #pragma unroll
       for (int k = 0; k < NE; ++k) acc[k] = fmaf(a, f[k], acc[k]);
     }
+    if (!is_v && s.center)
+      rotate_at<NE / 2>(acc, s, part * (NE / 2), jz * s.bz + 0.5 * (s.bz - 1), jy * s.by + 0.5 * (s.by - 1),
+                        jx * s.bx + 0.5 * (s.bx - 1));
     T* dst = is_v ? vs : ks;
     stg16(dst + ((size_t)j * s.Hkv + g) * kDh + part * NE, float_to_chunk(acc, T()));
   }
@@ -329,7 +335,8 @@ __global__ void __launch_bounds__(kSumWarpThreads) summaries_warp_kernel(
   const double my_omega = lane < s.npairs ? s.omega[lane] : 0.0;
   for (int t = threadIdx.x >> 5; t < V; t += kSumWarpThreads / 32) {
     const int d = my_axis == 0 ? t / (s.by * s.bx) : (my_axis == 1 ? (t / s.bx) % s.by : t % s.bx);
-    dtab[t][lane] = my_axis < 3 ? rope_cos_sin(my_omega * (double)d) : make_float2(1.f, 0.f);
+    // (Summary-centre variant: members are pooled unrotated.)
+    dtab[t][lane] = my_axis < 3 && !s.center ? rope_cos_sin(my_omega * (double)d) : make_float2(1.f, 0.f);
   }
   __syncthreads();
   constexpr int NE = Elem<T>::kPerChunk;
@@ -458,9 +465,11 @@ __global__ void __launch_bounds__(kSumWarpThreads) summaries_warp_kernel(
         }
     // R(c_base): lane p evaluates plane p at the block's first site, and every
     // lane takes the pairs of its own planes by shuffle.
-    const float2 cb = my_axis < 3 ? rope_cos_sin(my_omega * (double)(my_axis == 0 ? jz * s.bz
-                                                                     : (my_axis == 1 ? jy * s.by : jx * s.bx)))
-                                  : make_float2(1.f, 0.f);
+    // (Summary-centre variant: at the block's geometric centre instead.)
+    const double half = s.center ? 0.5 : 0.0;
+    const double cpos = my_axis == 0 ? jz * s.bz + half * (s.bz - 1)
+                                     : (my_axis == 1 ? jy * s.by + half * (s.by - 1) : jx * s.bx + half * (s.bx - 1));
+    const float2 cb = my_axis < 3 ? rope_cos_sin(my_omega * cpos) : make_float2(1.f, 0.f);
 #pragma unroll
     for (int i = 0; i < SPL; ++i)
 #pragma unroll

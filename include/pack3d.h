@@ -83,6 +83,13 @@ typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
                                           kernel instead of the tcgen05 one   */
 #define PACK3D_FLAG_SIMT_LOCAL    0x2  /* bf16: use the CUDA-core local-attention
                                           kernel instead of the tcgen05 one   */
+/* The summary-centre variant ("Geometry Matters in Packed 3D Attention",
+ * contribution 2 and "Future Directions" 3: the cheaper approximation that
+ * rotates only at the summary centre): k~_j = R(cbar_j) sum_u a_{j,u} k_u with
+ * cbar_j the block's geometric centre, block origin + ((bz-1)/2, (by-1)/2,
+ * (bx-1)/2), a fractional coordinate; v~_j and every other stage unchanged.
+ * Without the flag the summaries are the exact rotate-before-compress form. */
+#define PACK3D_FLAG_SUMMARY_CENTER 0x4
 
 typedef struct {
     int32_t Z, H, W;          /* lattice extents; N = Z*H*W tokens               */

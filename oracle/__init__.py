@@ -187,8 +187,9 @@ def gate_mix(s, gate, o_loc, o_cmp, rows=None) -> np.ndarray:
     return out
 
 
-def forward(s, inputs: Dict, rows=None) -> Dict[str, np.ndarray]:
+def forward(s, inputs: Dict, rows=None, center: bool = False) -> Dict[str, np.ndarray]:
     """The whole operator, stage by stage in the pages' order, for ``rows`` (default all).
+    ``center`` selects the summary-centre variant of the summaries.
 
     ``inputs`` holds ``coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate`` in
     packed order (numpy or torch; bf16 values are widened exactly).  Only the
@@ -205,7 +206,7 @@ def forward(s, inputs: Dict, rows=None) -> Dict[str, np.ndarray]:
         q = q[_torch_index(r)] if hasattr(q, "detach") else np.asarray(q)[r]
     qr = rotate(s, coords[r], q)
     klr = rotate(s, coords, inputs["k_loc"])
-    ks, vs = summaries(s, coords, mem, inputs["k_cmp"], inputs["v_cmp"], inputs["scores"])
+    ks, vs = summaries(s, coords, mem, inputs["k_cmp"], inputs["v_cmp"], inputs["scores"], center=center)
     ol = local_attn(s, coords, g2p, qr, klr, inputs["v_loc"], r)
     oc = summary_attn(s, qr, ks, vs)
     gate = inputs["gate"]

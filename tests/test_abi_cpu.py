@@ -48,7 +48,7 @@ def test_default_config_matches_pages(p3):
 @pytest.mark.parametrize("field,value,status", [
     ("d_h", 128, 2), ("Hq", 6, 2), ("Hkv", 3, 2), ("W", 63, 2), ("bx", 0, 2), ("rz", -1, 2),
     ("m_z", 20, 2), ("dtype", 7, 4), ("softmax_scale", 0.0, 1), ("flags", 0x100, 1), ("reserved0", 1, 1),
-    ("flags", 0x4, 1),
+    ("flags", 0x8, 1),
     ("rope_base", -1.0, 1), ("Z", 0, 2),
 ])
 def test_validate_rejects(p3, field, value, status):

@@ -111,6 +111,28 @@ def test_stages_match_oracle(p3, name, s, packing):
         assert e <= tol, f"{name}: {key} rel err {e:.3e} > {tol}"
 
 
+CENTER_CASES = [
+    ("bf16-warp", small(), "random"),                                  # warp-per-block kernel
+    ("f32-tiny", synth.CONFIGS["tiny"], "raster"),
+    ("bf16-v4", small(Z=3, H=10, W=14, by=2, bx=2), "morton"),         # block volume 4
+    ("bf16-v32", small(Z=4, H=8, W=8, bz=2), "block"),                 # block volume 32 (generic kernel)
+]
+
+
+@pytest.mark.parametrize("name,s,packing", CENTER_CASES, ids=[c[0] for c in CENTER_CASES])
+def test_summary_center_variant_matches_oracle(p3, name, s, packing):
+    """PACK3D_FLAG_SUMMARY_CENTER: summaries and the whole forward pass against the oracle's variant."""
+    inp = synth.make_inputs(s, packing, seed=13)
+    gpu = run_stages(p3, s, to_dev(inp), flags=p3.FLAG_SUMMARY_CENTER)
+    ref = oracle.forward(s, inp, center=True)
+    tol = TOL[s.dtype]
+    for key in ("k_sum", "v_sum", "o_cmp", "out"):
+        e = rel_err(gpu[key].double().numpy(), ref[key])
+        assert e <= tol, f"{name}: {key} rel err {e:.3e} > {tol}"
+    exact = oracle.forward(s, inp)
+    assert rel_err(ref["k_sum"], exact["k_sum"]) > 2 * tol      # the variant differs from the exact form
+
+
 def test_simt_and_tensor_core_summary_paths_agree(p3):
     s = small(Z=4, H=32, W=40)
     d = to_dev(synth.make_inputs(s, "random", seed=4))
