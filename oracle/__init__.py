@@ -43,7 +43,7 @@ class _Cfg(ctypes.Structure):
                 ("base", ctypes.c_double),
                 ("bz", ctypes.c_int32), ("by", ctypes.c_int32), ("bx", ctypes.c_int32),
                 ("rz", ctypes.c_int32), ("ry", ctypes.c_int32), ("rx", ctypes.c_int32),
-                ("scale", ctypes.c_double)]
+                ("scale", ctypes.c_double), ("cscale", ctypes.c_double * 3)]
 
 
 _lib = None
@@ -75,7 +75,8 @@ def threads() -> int:
 def _cfg(s, scale: Optional[float] = None) -> _Cfg:
     return _Cfg(s.Z, s.H, s.W, s.Hq, s.Hkv, s.d_h, s.m_z, s.m_y, s.m_x, float(s.rope_base),
                 s.bz, s.by, s.bx, s.rz, s.ry, s.rx,
-                float(s.softmax_scale if scale is None else scale))
+                float(s.softmax_scale if scale is None else scale),
+                (ctypes.c_double * 3)(*[float(x) for x in s.coord_scale]))
 
 
 def as_f64(x) -> np.ndarray:

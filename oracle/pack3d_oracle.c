@@ -51,6 +51,7 @@ typedef struct {
     int32_t bz, by, bx;
     int32_t rz, ry, rx;
     double scale;
+    double cscale[3];   /* coordinate scale per axis: angle = omega * cscale[a] * c_a */
 } orc_cfg;
 
 /* ---- lattice and index map ------------------------------------------- */
@@ -98,7 +99,7 @@ static double pair_angle(const orc_cfg *c, int p, double z, double y, double x, 
             int r = p - first;
             double omega = pow(c->base, -(double)r / (double)axis_pairs[a]);
             *active = 1;
-            return omega * coord[a];
+            return omega * (c->cscale[a] * coord[a]);
         }
         first += axis_pairs[a];
     }

@@ -65,6 +65,7 @@ class Pack3DShape:
     dtype: str = "bf16"          # "f32" or "bf16"
     value_scale: float = 0.125   # multiplier on the Q/K/V draws
     packing: str = "raster"
+    coord_scale: tuple = (1.0, 1.0, 1.0)   # per-axis RoPE coordinate scale (z, y, x)
 
     @property
     def N(self) -> int:
@@ -95,9 +96,11 @@ CONFIGS: Dict[str, Pack3DShape] = {
     "262k": Pack3DShape(Z=16, H=128, W=128, Hq=8, Hkv=2, packing="block"),
     "1m": Pack3DShape(Z=64, H=128, W=128, Hq=8, Hkv=2, packing="random"),
     "stress": Pack3DShape(Z=16, H=64, W=64, Hq=8, Hkv=2, packing="raster"),
+    # The shape of the pages' Allen WTC-11 token grid (32 x 128 x 64), synthetic values.
+    "allen": Pack3DShape(Z=32, H=128, W=64, Hq=8, Hkv=2, packing="block"),
 }
 
-PACKINGS = ("raster", "morton", "block", "random")
+PACKINGS = ("raster", "morton", "block", "random", "block_morton")
 
 
 def lattice_sites(Z: int, H: int, W: int) -> np.ndarray:
@@ -106,8 +109,11 @@ def lattice_sites(Z: int, H: int, W: int) -> np.ndarray:
     return np.stack([z.ravel(), y.ravel(), x.ravel()], axis=1).astype(np.int32)
 
 
-def _morton_keys(Z: int, H: int, W: int) -> np.ndarray:
-    s = lattice_sites(Z, H, W).astype(np.int64)
+def _morton_keys(Z: int, H: int, W: int, s: Optional[np.ndarray] = None) -> np.ndarray:
+    """Morton code of each site (raster order by default) of a Z x H x W lattice."""
+    if s is None:
+        s = lattice_sites(Z, H, W)
+    s = np.asarray(s).astype(np.int64)
     nbits = [max(1, (n - 1).bit_length()) for n in (Z, H, W)]
     key = np.zeros(s.shape[0], dtype=np.int64)
     out_bit = 0
@@ -135,6 +141,19 @@ def packing_sites(Z: int, H: int, W: int, packing: str, seed: int = 0,
         bid = ((s[:, 0] // bz) * (H // by) + s[:, 1] // by) * (W // bx) + s[:, 2] // bx
         inner = ((s[:, 0] % bz) * by + s[:, 1] % by) * bx + s[:, 2] % bx
         return np.argsort(bid * (bz * by * bx) + inner, kind="stable").astype(np.int64)
+    if packing == "block_morton":
+        # Two levels: blocks in Morton order over the block grid, sites in
+        # Morton order inside each block.
+        bz, by, bx = block
+        if Z % bz or H % by or W % bx:
+            raise ValueError("block_morton packing needs block dims dividing the lattice")
+        s = lattice_sites(Z, H, W).astype(np.int64)
+        outer = _morton_keys(Z // bz, H // by, W // bx, s // np.array([bz, by, bx]))
+        # Morton rank (0 .. v-1) of each in-block offset, so blocks stay contiguous.
+        rank = np.argsort(np.argsort(_morton_keys(bz, by, bx), kind="stable"), kind="stable")
+        off = s % np.array([bz, by, bx])
+        inner = rank[(off[:, 0] * by + off[:, 1]) * bx + off[:, 2]]
+        return np.argsort(outer * (bz * by * bx) + inner, kind="stable").astype(np.int64)
     if packing == "random":
         return np.random.default_rng(seed + 1).permutation(N).astype(np.int64)
     raise ValueError(f"unknown packing {packing!r}")

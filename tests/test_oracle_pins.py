@@ -128,6 +128,20 @@ def test_rope_matches_complex_form():
     assert np.abs(oracle.rotate(TINY, coords, x) - rope_complex(TINY, coords, x)).max() < 1e-12
 
 
+@pytest.mark.parametrize("scale,m", [((1 / 31, 1 / 127, 1 / 63), (11, 11, 10)),   # normalised coordinates
+                                     ((2.5, 1.0, 1.0), (11, 11, 10)),             # z rescaled
+                                     ((1.0, 1.0, 1.0), (6, 13, 13)),              # z-light allocation
+                                     ((1.0, 1.0, 1.0), (16, 8, 8))])              # z-heavy allocation
+def test_rope_coordinate_scale_and_allocation_match_complex_form(scale, m):
+    # A coordinate scale is the same rotation at the scaled (fractional) coordinate.
+    s = TINY.replace(Z=32, H=128, W=64, m_z=m[0], m_y=m[1], m_x=m[2], coord_scale=scale)
+    rng = np.random.default_rng(5)
+    coords = np.stack([rng.integers(0, n, 40) for n in (s.Z, s.H, s.W)], axis=1).astype(np.int32)
+    x = rng.standard_normal((40, 2, 64))
+    expect = rope_complex(s, coords.astype(np.float64) * np.asarray(scale), x)
+    assert np.abs(oracle.rotate(s, coords, x) - expect).max() < 1e-12
+
+
 # ------------------------------------------------------------ index map -----
 
 @pytest.mark.parametrize("packing", synth.PACKINGS)
@@ -176,6 +190,14 @@ def test_packings_are_bijections_with_expected_locality():
     # Morton: the first 8 slots form the 2x2x2 cube at the origin.
     c = synth.coords_for(s, "morton")
     assert sorted(map(tuple, c[:8])) == sorted(itertools.product(range(2), range(2), range(2)))
+    # Two-level block Morton: every run of v slots is one block, walked in Morton order
+    # inside it; the first four blocks are the 2x2 block square at the origin.
+    c = synth.coords_for(s, "block_morton")
+    blocks = c // np.array([s.bz, s.by, s.bx])
+    for k in range(0, s.N, s.v):
+        assert (blocks[k:k + s.v] == blocks[k]).all()
+    assert sorted(map(tuple, blocks[0:4 * s.v:s.v])) == [(0, 0, 0), (0, 0, 1), (0, 1, 0), (0, 1, 1)]
+    assert [tuple(x) for x in c[:4]] == [(0, 0, 0), (0, 0, 1), (0, 1, 0), (0, 1, 1)]
 
 
 # -------------------------------------------------------------- summaries ---
