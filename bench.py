@@ -43,6 +43,7 @@ WORKLOAD_TEXT = {
     "65k": "16x64x64 lattice (65,536 tokens), Morton packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=4,096), window 3x7x7",
     "262k": "16x128x128 lattice (262,144 tokens), block-contiguous packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=16,384), window 3x7x7",
     "1m": "64x128x128 lattice (1,048,576 tokens), random packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=65,536), window 3x7x7",
+    "allen": "32x128x64 lattice (262,144 tokens; the shape of the Allen WTC-11 token grid, synthetic values), block-contiguous packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=16,384), window 3x7x7",
 }
 STAGES = ("index", "rope", "summaries", "local", "summary_attn")
 KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summary attention

@@ -47,7 +47,8 @@ class Config(ctypes.Structure):
                 ("bz", ctypes.c_int32), ("by", ctypes.c_int32), ("bx", ctypes.c_int32),
                 ("rz", ctypes.c_int32), ("ry", ctypes.c_int32), ("rx", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("flags", ctypes.c_int32), ("reserved1", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("reserved1", ctypes.c_int32),
+                ("coord_scale", ctypes.c_double * 3)]
 
     @property
     def N(self) -> int:
@@ -109,7 +110,8 @@ def backend_info() -> str:
 def make_config(Z: int, H: int, W: int, *, Hq: int = 8, Hkv: int = 2, d_h: int = 64,
                 m: Sequence[int] = (11, 11, 10), rope_base: float = 10000.0,
                 block: Sequence[int] = (1, 4, 4), radius: Sequence[int] = (1, 3, 3),
-                softmax_scale: Optional[float] = None, dtype: str = "bf16", flags: int = 0) -> Config:
+                softmax_scale: Optional[float] = None, dtype: str = "bf16", flags: int = 0,
+                coord_scale: Sequence[float] = (1.0, 1.0, 1.0)) -> Config:
     c = Config()
     c.Z, c.H, c.W = Z, H, W
     c.Hq, c.Hkv, c.d_h = Hq, Hkv, d_h
@@ -120,6 +122,7 @@ def make_config(Z: int, H: int, W: int, *, Hq: int = 8, Hkv: int = 2, d_h: int =
     c.softmax_scale = 1.0 / math.sqrt(d_h) if softmax_scale is None else softmax_scale
     c.dtype = BF16 if dtype in ("bf16", BF16) else F32
     c.flags = flags
+    c.coord_scale[:] = [float(x) for x in coord_scale]
     return c
 
 
@@ -127,7 +130,8 @@ def config_from_shape(s, flags: int = 0) -> Config:
     """Config from any object with the fields of ``synth.Pack3DShape``."""
     return make_config(s.Z, s.H, s.W, Hq=s.Hq, Hkv=s.Hkv, d_h=s.d_h, m=(s.m_z, s.m_y, s.m_x),
                        rope_base=s.rope_base, block=(s.bz, s.by, s.bx), radius=(s.rz, s.ry, s.rx),
-                       softmax_scale=s.softmax_scale, dtype=s.dtype, flags=flags)
+                       softmax_scale=s.softmax_scale, dtype=s.dtype, flags=flags,
+                       coord_scale=getattr(s, "coord_scale", (1.0, 1.0, 1.0)))
 
 
 def validate(cfg: Config) -> int:

@@ -34,7 +34,8 @@ Shape make_shape(const pack3d_config& c) {
   int p = 0, off = 0;
   for (int a = 0; a < 3; ++a)
     for (int r = 0; r < m[a]; ++r) {
-      s.omega[p] = pow(c.rope_base, -(double)r / (double)m[a]);
+      // The coordinate scale of the axis folds into the plane's frequency.
+      s.omega[p] = pow(c.rope_base, -(double)r / (double)m[a]) * c.coord_scale[a];
       s.pair_axis[p] = a;
       s.pair_off[p] = off;
       off += ext[a];
@@ -108,6 +109,7 @@ void pack3d_default_config(pack3d_config* cfg, int32_t Z, int32_t H, int32_t W) 
   cfg->rz = 1; cfg->ry = 3; cfg->rx = 3;
   cfg->softmax_scale = 0.125f;
   cfg->dtype = PACK3D_BF16;
+  cfg->coord_scale[0] = cfg->coord_scale[1] = cfg->coord_scale[2] = 1.0;
 }
 
 pack3d_status pack3d_validate_config(const pack3d_config* c) {
@@ -129,6 +131,8 @@ pack3d_status pack3d_validate_config(const pack3d_config* c) {
   if (c->bz * c->by * c->bx > 64) return PACK3D_ERR_SHAPE;
   if (c->rz < 0 || c->ry < 0 || c->rx < 0) return PACK3D_ERR_SHAPE;
   if (!(c->softmax_scale > 0.f) || !isfinite(c->softmax_scale)) return PACK3D_ERR_INVALID_ARG;
+  for (int a = 0; a < 3; ++a)
+    if (!(c->coord_scale[a] > 0.0) || !isfinite(c->coord_scale[a])) return PACK3D_ERR_INVALID_ARG;
   const long long tab = (long long)c->Z * c->m_z + (long long)c->H * c->m_y + (long long)c->W * c->m_x;
   if (tab * 8 > kMaxTableBytes) return PACK3D_ERR_SHAPE;
   if (c->flags & ~(PACK3D_FLAG_SIMT_SUMMARY | PACK3D_FLAG_SIMT_LOCAL | PACK3D_FLAG_SUMMARY_CENTER))

@@ -103,6 +103,13 @@ typedef struct {
     int32_t dtype;            /* pack3d_dtype of q, k, v, summaries, out         */
     int32_t flags;            /* PACK3D_FLAG_* bits                              */
     int32_t reserved1;        /* must be 0                                       */
+    double  coord_scale[3];   /* per-axis coordinate scale (z, y, x), > 0, 1 by
+                                 default: the rotation angle of axis a is
+                                 omega_{a,r} * coord_scale[a] * c_a, so e.g.
+                                 1/(extent-1) gives normalised coordinates in
+                                 [0, 1] and coord_scale[0] != 1 rescales z (the
+                                 rotary-configuration sweep of the summary page,
+                                 "Main Findings")                                */
 } pack3d_config;
 
 /* Fills cfg with the pages' defaults for a Z x H x W lattice: Hq=8, Hkv=2,

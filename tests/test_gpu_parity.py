@@ -95,6 +95,11 @@ STAGE_CASES = [
     ("hkv4", small(Hq=8, Hkv=4), "random"),
     ("hkv8-f32", small(Hq=8, Hkv=8, dtype="f32", value_scale=1.0), "block"),
     ("hkv4-f32", small(Hq=8, Hkv=4, dtype="f32", value_scale=1.0), "morton"),
+    # rotary configuration knobs: normalised coordinates, z rescaled, z-light and z-heavy pair splits
+    ("coords-normalised", small(Z=4, H=16, W=24, coord_scale=(1 / 3, 1 / 15, 1 / 23)), "block_morton"),
+    ("z-rescaled-f32", small(dtype="f32", value_scale=1.0, coord_scale=(2.5, 1.0, 1.0)), "random"),
+    ("z-light", small(m_z=6, m_y=13, m_x=13), "block_morton"),
+    ("z-heavy", small(m_z=16, m_y=8, m_x=8), "random"),
 ]
 
 
