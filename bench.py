@@ -22,6 +22,8 @@ bounded sample of the same workload (rank 0 only).
 """
 from __future__ import annotations
 
+from typing import Dict
+
 import argparse
 import json
 import os
@@ -263,6 +265,40 @@ def summary_center_error(p3, s, d, q_rot, members, err, stream, rows: int = 2048
     return out
 
 
+def dense_sdpa_ms(s, q_rot, k_rot, v, stream, reps: int = 2) -> Dict:
+    """Comparator: dense softmax attention of every token over every token (torch SDPA, bf16, grouped
+    kv heads) on the same rotated Q/K and V, timed with CUDA events after one warm-up call."""
+    import torch
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    # kv heads repeated to the query heads, so the fused flash kernel runs (no N x N score tensor).
+    rep_kv = [(h * s.Hkv) // s.Hq for h in range(s.Hq)]
+    qt = q_rot.permute(1, 0, 2).unsqueeze(0)
+    kt = k_rot[:, rep_kv, :].permute(1, 0, 2).unsqueeze(0)
+    vt = v[:, rep_kv, :].permute(1, 0, 2).unsqueeze(0)
+
+    def call():
+        with sdpa_kernel(SDPBackend.FLASH_ATTENTION):
+            return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=s.softmax_scale)
+
+    try:
+        call()
+    except RuntimeError as e:
+        return {"unavailable": str(e).splitlines()[0][:200]}
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.mean(ts)
+    flops = 4.0 * s.N * s.N * s.d_h * s.Hq
+    return {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12, "calls_timed": reps,
+            "what": "torch scaled_dot_product_attention (flash backend), bf16, all N x N pairs, kv heads repeated"}
+
+
 def run_ours(args, s):
     import torch
 
@@ -415,6 +451,19 @@ def run_ours(args, s):
             "clocks": clk.summary()}
     if variant_err is not None:
         line["summary_center_vs_exact"] = variant_err
+    # Comparators named by the workloads: a same-window local-only pass at 65k
+    # (index map, RoPE and local attention, the stages that pass runs) and a
+    # dense-attention run of the same shape at 1M.
+    comp = {}
+    if args.config == "65k":
+        comp["local_only_ms"] = st_ms["index"] + st_ms["rope"] + st_ms["local"]
+        comp["local_only_tokens_per_s"] = s.N * world / (comp["local_only_ms"] * 1e-3)
+    if args.config == "1m" and not args.no_dense:
+        comp["dense_sdpa"] = dense_sdpa_ms(s, qr, kr, d["v_loc"], stream)
+        if "ms" in comp["dense_sdpa"]:
+            comp["dense_sdpa"]["speedup_of_pack3d"] = comp["dense_sdpa"]["ms"] / ms
+    if comp:
+        line["comparators"] = comp
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             cb = cpu_oracle_sample(s, inp_host, target_s=12.0, center=args.summary_center)
@@ -435,6 +484,7 @@ def main():
     ap.add_argument("--config", default="65k", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparator at 1M")
     ap.add_argument("--summary-center", action="store_true",
                     help="time the summary-centre variant of the block summaries and report its error "
                          "against the exact rotate-before-compress form")
