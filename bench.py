@@ -50,9 +50,10 @@ WORKLOAD_TEXT = {
 STAGES = ("index", "rope", "summaries", "local", "summary_attn")
 KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summary attention
 # DRAM bytes (read + write) of one summary_attn_tc_kernel launch, from an ncu
-# capture of this workload (profiles/summary_attn_tc_65k.md).  Set back to
-# None whenever that kernel changes until it is captured again.
-SUMMARY_ATTN_TRAFFIC = {"65k": 212.722432e6 + 48.2944e6}
+# capture of this workload (profiles/summary_attn_tc_65k.md; at 65k tokens the
+# one-tile build runs).  Emptied whenever that kernel changes until it is
+# captured again.
+SUMMARY_ATTN_TRAFFIC = {"65k": 212.702976e6 + 48.533504e6}
 
 
 def load_peaks():

@@ -1,0 +1,41 @@
+// Chooses between the two builds of the query x summary kernel.
+//
+// With few summary tiles per query tile, the fixed cost of a CTA (tensor-
+// memory allocation, the first loads, the gate epilogue) is a large share of
+// its time, and one-tile CTAs two per SM hide it behind each other; with many
+// summary tiles the two-tile CTA, which reads every k~ / v~ tile once for both
+// query tiles, is faster.  Measured on B200: 65k tokens (32 summary tiles)
+// 0.78-0.80 ms one-tile vs 0.81 ms two-tile; 262k tokens (128 summary tiles)
+// 11.46 ms vs 10.8-10.9 ms.
+#include "common.cuh"
+#include "internal.h"
+
+namespace pack3d {
+namespace sa_two {
+long token_quantum(const Shape& s);
+cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* vs, const float* oloc,
+                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end);
+}  // namespace sa_two
+namespace sa_one {
+long token_quantum(const Shape& s);
+cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* vs, const float* oloc,
+                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end);
+}  // namespace sa_one
+
+namespace {
+constexpr int kOneTileMaxSummaryTiles = 48;
+bool one_tile(const Shape& s) { return (s.M + 127) / 128 <= kOneTileMaxSummaryTiles; }
+}  // namespace
+
+long summary_attn_tc_token_quantum(const Shape& s) {
+  return one_tile(s) ? sa_one::token_quantum(s) : sa_two::token_quantum(s);
+}
+
+cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
+                                   const float* oloc, const float* gate, void* out, int32_t* err,
+                                   cudaStream_t st, long tok_begin, long tok_end) {
+  return one_tile(s) ? sa_one::launch(s, qr, ks, vs, oloc, gate, out, err, st, tok_begin, tok_end)
+                     : sa_two::launch(s, qr, ks, vs, oloc, gate, out, err, st, tok_begin, tok_end);
+}
+
+}  // namespace pack3d

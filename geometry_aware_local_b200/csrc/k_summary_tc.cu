@@ -30,7 +30,15 @@
 #include "internal.h"
 #include "tc_ptx.cuh"
 
+// The file is compiled twice: as the two-tile kernel (namespace sa_two, the
+// default) and, from k_summary_tc_one.cu, as the one-tile kernel run two
+// CTAs per SM (namespace sa_one); k_summary_dispatch.cu picks per launch.
+#ifndef PACK3D_SA_NS
+#define PACK3D_SA_NS sa_two
+#endif
+
 namespace pack3d {
+namespace PACK3D_SA_NS {
 namespace {
 
 // Compile-time shape of the pipeline: query tiles (softmax warpgroups) per
@@ -52,8 +60,14 @@ constexpr int kColS = 0, kColP = kBN, kColO = kBN + kBN / 2;
 constexpr int kGroupCols = kColO + kDh;       // tensor-memory columns per group
 constexpr int kQBytes = kBM * kDh * 2;        // 16 KiB
 constexpr int kKVBytes = kBN * kDh * 2;
-constexpr int kStages = ((192 * 1024 - kGroups * kQBytes) / (2 * kKVBytes)) < 8
-                            ? ((192 * 1024 - kGroups * kQBytes) / (2 * kKVBytes)) : 8;
+// CTAs per SM: one CTA of two tiles, or two CTAs of one tile each (then an
+// SM runs two independent pipelines, each with half the tensor memory and
+// shared memory).
+constexpr int kCtasPerSm = kGroups == 1 ? 2 : 1;
+constexpr int kSmemBudget = kCtasPerSm == 1 ? 192 * 1024 : 110 * 1024;
+constexpr int kStages = ((kSmemBudget - kGroups * kQBytes) / (2 * kKVBytes)) < 8
+                            ? ((kSmemBudget - kGroups * kQBytes) / (2 * kKVBytes)) : 8;
+constexpr int kTmemCols = kGroups == 1 ? 256 : 512;
 constexpr int kQOff = 0;
 constexpr int kStageOff = kGroups * kQBytes;  // stage s: k~ at +0, v~ at +kKVBytes
 constexpr int kStageBytes = 2 * kKVBytes;
@@ -76,7 +90,7 @@ constexpr int kGroupBars = 3 + 2 * kPChunks;
 constexpr int kNumBars = 2 * kStages + 1 + kGroups * kGroupBars;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
-static_assert(kGroups * kGroupCols <= 512, "tensor memory plan");
+static_assert(kGroups * kGroupCols <= kTmemCols, "tensor memory plan");
 
 constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kBM, kBN, false);      // S: N = kBN summaries
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kDh, true);     // O: N = 64 dims, v~ MN-major
@@ -131,7 +145,7 @@ __device__ __forceinline__ float2 exp2_poly(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -174,7 +188,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     ptx::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 512);
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -429,7 +443,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   __syncthreads();
   if (warp == kMmaWarp) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 512);
+    ptx::tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && *abort_flag) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
 }
@@ -464,13 +478,12 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
 
 }  // namespace
 
-long summary_attn_tc_token_quantum(const Shape& s) { return (long)kGroups * kBM / s.G; }
+long token_quantum(const Shape& s) { return (long)kGroups * kBM / s.G; }
 
-cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
-                                   const float* oloc, const float* gate, void* out, int32_t* err,
-                                   cudaStream_t st, long tok_begin, long tok_end) {
+cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* vs, const float* oloc,
+                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end) {
   if (tok_end < 0) tok_end = s.N;
-  if (tok_begin < 0 || tok_begin >= tok_end || tok_end > s.N || tok_begin % summary_attn_tc_token_quantum(s))
+  if (tok_begin < 0 || tok_begin >= tok_end || tok_end > s.N || tok_begin % token_quantum(s))
     return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   // Q viewed as [N][Hkv][G][64]: a box of 128/G tokens x G heads x 64 dims is one 128-row tile.
@@ -502,4 +515,5 @@ cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* k
   return cudaGetLastError();
 }
 
+}  // namespace PACK3D_SA_NS
 }  // namespace pack3d
