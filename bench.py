@@ -155,23 +155,37 @@ def dist_setup(args):
     return world, rank, local
 
 
+def _reduce_device():
+    """Device of the tensors the process group reduces: the GPU under NCCL, the host under gloo."""
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it); the replicas' step time."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
+def replica_value(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms * 1e-3)
+
+
 def barrier(world):
     import torch
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def cpu_oracle_sample(s, inp, target_s: float = 12.0, center: bool = False):
@@ -372,7 +386,7 @@ def run_ours(args, s):
         raise RuntimeError("device error during the timed steps")
     ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
     st_ms = {k: v / args.steps for k, v in st_ms.items()}
-    value = s.N * world / (ms * 1e-3)
+    value = replica_value(s.N, world, ms)
 
     # pack3d_forward from the device buffers (same kernels, one C-ABI call).
     ws = torch.empty(p3.workspace_bytes(cfg), dtype=torch.uint8, device=dev)
