@@ -45,6 +45,8 @@ WORKLOAD_TEXT = {
     "65k": "16x64x64 lattice (65,536 tokens), Morton packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=4,096), window 3x7x7",
     "262k": "16x128x128 lattice (262,144 tokens), block-contiguous packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=16,384), window 3x7x7",
     "1m": "64x128x128 lattice (1,048,576 tokens), random packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=65,536), window 3x7x7",
+    "4m": "64x256x256 lattice (4,194,304 tokens), Morton packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=262,144), window 3x7x7; values drawn on the device",
+    "8m": "128x256x256 lattice (8,388,608 tokens), Morton packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=524,288), window 3x7x7; values drawn on the device",
     "allen": "32x128x64 lattice (262,144 tokens; the shape of the Allen WTC-11 token grid, synthetic values), block-contiguous packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=16,384), window 3x7x7",
 }
 STAGES = ("index", "rope", "summaries", "local", "summary_attn")
@@ -54,6 +56,9 @@ KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summ
 # one-tile build runs).  Emptied whenever that kernel changes until it is
 # captured again.
 SUMMARY_ATTN_TRAFFIC = {"65k": 212.702976e6 + 48.533504e6}
+
+# Launches at least this long are rated against the sustained bf16 peak.
+SUSTAINED_MS = 1000.0
 
 
 def load_peaks():
@@ -323,9 +328,14 @@ def run_ours(args, s):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cfg = p3.config_from_shape(s, p3.FLAG_SUMMARY_CENTER if args.summary_center else 0)
-    inp_host = synth.make_inputs(s, s.packing, seed=rank)
     names = ("coords", "q", "k_loc", "v_loc", "k_cmp", "v_cmp", "scores", "gate")
-    d = {k: inp_host[k].to(dev) for k in names}
+    if args.config in synth.DEVICE_DRAWN:
+        # Too large for host draws: values drawn on the device, host copies made for the e2e leg.
+        d = synth.make_inputs_on_device(s, s.packing, seed=rank, device=dev)
+        inp_host = {k: d[k].cpu() for k in names}
+    else:
+        inp_host = synth.make_inputs(s, s.packing, seed=rank)
+        d = {k: inp_host[k].to(dev) for k in names}
     dt = d["q"].dtype
     err = torch.zeros(4, dtype=torch.int32, device=dev)
     g2p = torch.empty(s.N, dtype=torch.int32, device=dev)
@@ -445,10 +455,16 @@ def run_ours(args, s):
         stages[name] = e
     variant_err = summary_center_error(p3, s, d, qr, mem, err, stream) if args.summary_center else None
     sa = stages["summary_attn"]
-    roof = {"bound": "tensor", "achieved": sa["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": sa["tflops"] / peaks["bf16_tflops"], "traffic": SUMMARY_ATTN_TRAFFIC.get(args.config),
+    # A launch of a second or more runs under the board's power cap the whole
+    # time, like the measured sustained GEMM loop; shorter ones see burst clocks.
+    sustained = sa["ms"] >= SUSTAINED_MS and peaks.get("bf16_tflops_sustained")
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    roof = {"bound": "tensor", "achieved": sa["tflops"], "peak": peak, "unit": "TFLOP/s",
+            "frac": sa["tflops"] / peak, "traffic": SUMMARY_ATTN_TRAFFIC.get(args.config),
             "kernel": "summary_attn_tc_kernel" if s.dtype == "bf16" else "summary_attn_simt_kernel",
-            "peak_source": peaks["source"] + " burst bf16 (MEASURED_PEAKS.json bf16_tflops)"}
+            "peak_source": peaks["source"] + (" sustained bf16 (MEASURED_PEAKS.json bf16_tflops_sustained)"
+                                              if sustained else " burst bf16 (MEASURED_PEAKS.json bf16_tflops)"),
+            "frac_of_burst": sa["tflops"] / peaks["bf16_tflops"]}
     if s.dtype != "bf16":
         roof["bound"] = "alu"
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -480,7 +496,7 @@ def run_ours(args, s):
     if comp:
         line["comparators"] = comp
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.config not in synth.DEVICE_DRAWN:
             cb = cpu_oracle_sample(s, inp_host, target_s=12.0, center=args.summary_center)
             cb.pop("seconds")
             line["cpu_baseline"] = cb

@@ -98,7 +98,11 @@ CONFIGS: Dict[str, Pack3DShape] = {
     "stress": Pack3DShape(Z=16, H=64, W=64, Hq=8, Hkv=2, packing="raster"),
     # The shape of the pages' Allen WTC-11 token grid (32 x 128 x 64), synthetic values.
     "allen": Pack3DShape(Z=32, H=128, W=64, Hq=8, Hkv=2, packing="block"),
+    # Long query runs (4M and 8M tokens; inputs drawn on the device).
+    "4m": Pack3DShape(Z=64, H=256, W=256, Hq=8, Hkv=2, packing="morton"),
+    "8m": Pack3DShape(Z=128, H=256, W=256, Hq=8, Hkv=2, packing="morton"),
 }
+DEVICE_DRAWN = ("4m", "8m")
 
 PACKINGS = ("raster", "morton", "block", "random", "block_morton")
 
@@ -205,6 +209,33 @@ def make_inputs(shape: Pack3DShape, packing: Optional[str] = None, seed: int = 0
         res[name] = torch.from_numpy(sv[name]).index_select(0, idx).to(tdt).contiguous()
     for name in ("scores", "gate"):
         res[name] = torch.from_numpy(sv[name]).index_select(0, idx).contiguous()
+    return res
+
+
+def make_inputs_on_device(shape: Pack3DShape, packing: Optional[str] = None, seed: int = 0,
+                          device="cuda"):
+    """The same inputs as ``make_inputs`` in kind and distribution, drawn on the device.
+
+    For volumes whose float32 host draws would not fit the host (4M and 8M
+    tokens): the coordinates of ``packing`` come from the host as above, the
+    values are drawn in packed order by a seeded torch generator on ``device``
+    (N(0,1) times ``value_scale`` for Q/K/V, N(0,1) for scores and gate).  The
+    values differ from ``make_inputs``'s; no parity check uses these volumes."""
+    import torch
+    packing = packing or shape.packing
+    sites = packing_sites(shape.Z, shape.H, shape.W, packing, seed, (shape.bz, shape.by, shape.bx))
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=device).manual_seed(seed)
+    N, Hq, Hkv, d = shape.N, shape.Hq, shape.Hkv, shape.d_h
+    res = {"coords": torch.from_numpy(lattice_sites(shape.Z, shape.H, shape.W)[sites].copy()).to(device)}
+    for name, heads in (("q", Hq), ("k_loc", Hkv), ("v_loc", Hkv), ("k_cmp", Hkv), ("v_cmp", Hkv)):
+        x = torch.randn((N, heads, d), generator=gen, device=device, dtype=torch.float32)
+        if shape.value_scale != 1:
+            x *= shape.value_scale
+        res[name] = x.to(tdt)
+        del x
+    res["scores"] = torch.randn((N, Hkv), generator=gen, device=device, dtype=torch.float32)
+    res["gate"] = torch.randn((N, Hq, 2), generator=gen, device=device, dtype=torch.float32)
     return res
 
 
