@@ -23,7 +23,7 @@ _SRC = os.path.join(_HERE, "pack3d_oracle.c")
 _LIB = os.path.join(_HERE, "liborc.so")
 
 __all__ = ["build", "threads", "build_index", "rotate", "summaries", "local_attn",
-           "summary_attn", "gate_mix", "forward", "as_f64"]
+           "summary_attn", "gate_mix", "forward", "as_f64", "rotate_t", "backward"]
 
 
 def build(force: bool = False) -> str:
@@ -62,6 +62,14 @@ def _load():
         lib.orc_local_attn.argtypes = [P, P, P, P, P, P, P, ctypes.c_long, P]
         lib.orc_summary_attn.argtypes = [P, P, P, P, ctypes.c_long, ctypes.c_long, P]
         lib.orc_gate_mix.argtypes = [P, P, P, ctypes.c_long, P, P, P]
+        L = ctypes.c_long
+        lib.orc_rotate_t.argtypes = [P, P, P, P, ctypes.c_int, L]
+        lib.orc_gate_backward.argtypes = [P, P, P, L, P, P, P, P, P, P]
+        lib.orc_local_attn_backward_q.argtypes = [P, P, P, P, P, P, P, P, L, P, P, P]
+        lib.orc_local_attn_backward_kv.argtypes = [P, P, P, P, P, P, P, P, P, P, L, P, P]
+        lib.orc_summary_attn_backward_q.argtypes = [P, P, P, P, L, L, P, P, P, P]
+        lib.orc_summary_attn_backward_kv.argtypes = [P, P, P, P, L, P, P, P, P, L, P, P]
+        lib.orc_summaries_backward.argtypes = [P, P, P, P, P, P, P, P, P, L, P, P, P]
         _lib = lib
     return _lib
 
@@ -219,3 +227,110 @@ def forward(s, inputs: Dict, rows=None, center: bool = False) -> Dict[str, np.nd
 def _torch_index(r):
     import torch
     return torch.from_numpy(r)
+
+
+# ---- backward pass of the training block --------------------------------------
+
+
+def rotate_t(s, coords, y, heads: Optional[int] = None) -> np.ndarray:
+    """``R(c_i)^T y_i`` per head: the RoPE backward (the transpose of equation R(c))."""
+    ya = as_f64(y)
+    n = ya.shape[0]
+    heads = heads if heads is not None else ya.shape[1]
+    c = _i32(coords)
+    x = np.empty_like(ya)
+    cfg = _cfg(s)
+    _load().orc_rotate_t(ctypes.byref(cfg), _ptr(c), _ptr(ya), _ptr(x), heads, n)
+    return x
+
+
+def _ids(x, n):
+    if x is None:
+        return np.arange(n, dtype=np.int64)
+    return np.ascontiguousarray(x, dtype=np.int64)
+
+
+def _scatter(a: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    full = np.empty_like(a)
+    full[idx] = a
+    return full
+
+
+def backward(s, inputs: Dict, dout, keys=None, blocks=None) -> Dict[str, np.ndarray]:
+    """Gradients of L = <dout, out> with respect to every input of the operator.
+
+    The chain rule through the forward stages in reverse: the tokenwise gate
+    (overall framework), both attention branches (Key design 3), the
+    rotate-before-compress summaries (Key design 2) and the axial RoPE (Key
+    design 1).  ``dq`` and ``dgate`` come for every token; ``dk_loc`` and
+    ``dv_loc`` for the tokens ``keys`` (default all, in that order); ``dk_cmp``,
+    ``dv_cmp`` and ``dscores`` for the members of the summary blocks ``blocks``
+    (``cmp_tokens`` = their packed indices, block by block, members in raster
+    order), or, with ``blocks=None``, for every token in packed order.
+    """
+    lib = _load()
+    st, g2p, mem = build_index(s, inputs["coords"])
+    if st != 0:
+        raise ValueError("coordinates are not a bijection onto the lattice (status %d)" % st)
+    coords = _i32(inputs["coords"])
+    N, Hq, Hkv, d = s.N, s.Hq, s.Hkv, s.d_h
+    allr = np.arange(N, dtype=np.int64)
+    cfg = _cfg(s)
+    # forward quantities the backward reads
+    qr = rotate(s, coords, inputs["q"])
+    klr = rotate(s, coords, inputs["k_loc"])
+    vl = as_f64(inputs["v_loc"])
+    ks, vs = summaries(s, coords, mem, inputs["k_cmp"], inputs["v_cmp"], inputs["scores"])
+    ol = local_attn(s, coords, g2p, qr, klr, vl)
+    oc = summary_attn(s, qr, ks, vs)
+    # gate
+    do = as_f64(dout)
+    ga = as_f64(inputs["gate"])
+    dgate = np.empty((N, Hq, 2))
+    dol = np.empty_like(do)
+    doc = np.empty_like(do)
+    lib.orc_gate_backward(ctypes.byref(cfg), _ptr(ga), _ptr(allr), N, _ptr(ol), _ptr(oc), _ptr(do),
+                          _ptr(dgate), _ptr(dol), _ptr(doc))
+    # local branch
+    dqr_l = np.empty_like(qr)
+    lse_l = np.empty((N, Hq))
+    del_l = np.empty((N, Hq))
+    lib.orc_local_attn_backward_q(ctypes.byref(cfg), _ptr(coords), _ptr(g2p), _ptr(qr), _ptr(klr), _ptr(vl),
+                                  _ptr(dol), _ptr(allr), N, _ptr(dqr_l), _ptr(lse_l), _ptr(del_l))
+    kk = _ids(keys, N)
+    dklr = np.empty((kk.shape[0], Hkv, d))
+    dvl = np.empty_like(dklr)
+    lib.orc_local_attn_backward_kv(ctypes.byref(cfg), _ptr(coords), _ptr(g2p), _ptr(qr), _ptr(klr), _ptr(vl),
+                                   _ptr(dol), _ptr(lse_l), _ptr(del_l), _ptr(kk), kk.shape[0], _ptr(dklr),
+                                   _ptr(dvl))
+    # compressed branch
+    dqr_c = np.empty_like(qr)
+    lse_c = np.empty((N, Hq))
+    del_c = np.empty((N, Hq))
+    lib.orc_summary_attn_backward_q(ctypes.byref(cfg), _ptr(qr), _ptr(ks), _ptr(vs), s.M, N, _ptr(doc),
+                                    _ptr(dqr_c), _ptr(lse_c), _ptr(del_c))
+    bb = _ids(blocks, s.M)
+    dks = np.empty((bb.shape[0], Hkv, d))
+    dvs = np.empty_like(dks)
+    lib.orc_summary_attn_backward_kv(ctypes.byref(cfg), _ptr(qr), _ptr(ks), _ptr(vs), N, _ptr(doc),
+                                     _ptr(lse_c), _ptr(del_c), _ptr(bb), bb.shape[0], _ptr(dks), _ptr(dvs))
+    # summaries
+    kc, vc, sc = as_f64(inputs["k_cmp"]), as_f64(inputs["v_cmp"]), as_f64(inputs["scores"])
+    nt = bb.shape[0] * s.v
+    dkc = np.empty((nt, Hkv, d))
+    dvc = np.empty_like(dkc)
+    dsc = np.empty((nt, Hkv))
+    lib.orc_summaries_backward(ctypes.byref(cfg), _ptr(coords), _ptr(mem), _ptr(kc), _ptr(vc), _ptr(sc),
+                               _ptr(dks), _ptr(dvs), _ptr(bb), bb.shape[0], _ptr(dkc), _ptr(dvc), _ptr(dsc))
+    cmp_tokens = mem[bb].reshape(-1).astype(np.int64)
+    if blocks is None:
+        # every token is a member of exactly one block: scatter to packed order
+        dkc, dvc, dsc = (_scatter(a, cmp_tokens) for a in (dkc, dvc, dsc))
+        cmp_tokens = allr
+    # RoPE
+    dq = rotate_t(s, coords, dqr_l + dqr_c)
+    dk_loc = rotate_t(s, coords[kk], dklr)
+    return {"dq": dq, "dk_loc": dk_loc, "dv_loc": dvl, "dk_cmp": dkc, "dv_cmp": dvc, "dscores": dsc,
+            "dgate": dgate, "keys": kk, "cmp_tokens": cmp_tokens, "blocks": bb,
+            "out": gate_mix(s, inputs["gate"], ol, oc), "lse_loc": lse_l, "lse_cmp": lse_c,
+            "dk_sum": dks, "dv_sum": dvs}

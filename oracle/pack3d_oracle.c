@@ -23,6 +23,10 @@
  *   - compressed branch .......... "Key design 3" / summary "every token attends
  *                                  to all M summaries".
  *   - gate ....................... "overall framework" (tokenwise learned gate).
+ *   - backward pass .............. the summary's description of the operator as
+ *                                  a fused forward/backward training block: the
+ *                                  gradients of <dout, out> by the chain rule
+ *                                  through the stages above, in reverse order.
  *
  * Readings where the pages are silent (all listed in the design notes):
  *   omega_{a,r} = base^(-r/m_a); rotary pair p occupies dims (2p, 2p+1); pairs
@@ -340,5 +344,332 @@ void orc_gate_mix(const orc_cfg *c, const double *gate, const int64_t *rows, lon
                 out[k] = w0 * oloc[k] + w1 * ocmp[k];
             }
         }
+    }
+}
+
+/* ======================================================================
+ * Backward pass of the training block (the pages call the operator a fused
+ * forward/backward block; these functions give its gradients).  With
+ * L = <dout, out>, each function applies the chain rule to one forward
+ * stage, in reverse order of the forward pass:
+ *   gate -> both attention branches -> summaries and RoPE.
+ * For a softmax over logits l_j = scale <q, k_j> with o = sum_j P_j v_j,
+ *   dP_j = <do, v_j>,  dl_j = P_j (dP_j - sum_j' P_j' dP_j'),
+ *   dq = scale sum_j dl_j k_j,  dk_j += scale dl_j q,  dv_j += P_j do.
+ * The row quantities lse = log sum_j exp(l_j) and delta = sum_j P_j dP_j
+ * (= <do, o>) are formed in a first pass over the query rows and read by
+ * the second pass, which sums over queries per key; that is the same
+ * arithmetic in another order.
+ * ==================================================================== */
+
+/* x = R(c)^T y: each active pair (y0, y1) becomes
+ * (y0 cos t + y1 sin t, -y0 sin t + y1 cos t). */
+static void rotate_row_t(const orc_cfg *c, double cz, double cy, double cx, const double *yi, double *xi)
+{
+    for (int p = 0; p < c->dh / 2; ++p) {
+        int active;
+        double t = pair_angle(c, p, cz, cy, cx, &active);
+        double y0 = yi[2 * p], y1 = yi[2 * p + 1];
+        if (active) {
+            xi[2 * p] = y0 * cos(t) + y1 * sin(t);
+            xi[2 * p + 1] = -y0 * sin(t) + y1 * cos(t);
+        } else {
+            xi[2 * p] = y0;
+            xi[2 * p + 1] = y1;
+        }
+    }
+}
+
+/* x[i,h,:] = R(c_i)^T y[i,h,:]: the RoPE backward for n tokens. */
+void orc_rotate_t(const orc_cfg *c, const int32_t *coords, const double *y, double *x,
+                  int heads, long n)
+{
+    int d = c->dh;
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; ++i)
+        for (int h = 0; h < heads; ++h)
+            rotate_row_t(c, coords[3 * i], coords[3 * i + 1], coords[3 * i + 2],
+                         y + ((long)i * heads + h) * d, x + ((long)i * heads + h) * d);
+}
+
+/* Gate backward for the sampled rows (r-th entry = token rows[r]):
+ *   gamma = softmax(gate[i,h,:]),  dgamma_c = <dout, o_c>  (o_0 = oloc, o_1 = ocmp)
+ *   dgate_c = gamma_c (dgamma_c - sum_c' gamma_c' dgamma_c')
+ *   dol = gamma_0 dout,  doc = gamma_1 dout.
+ * oloc, ocmp, dout, dol, doc hold the sampled rows in sample order. */
+void orc_gate_backward(const orc_cfg *c, const double *gate, const int64_t *rows, long nrows,
+                       const double *oloc, const double *ocmp, const double *dout,
+                       double *dgate, double *dol, double *doc)
+{
+    int d = c->dh, Hq = c->Hq;
+    for (long r = 0; r < nrows; ++r) {
+        long i = rows[r];
+        for (int h = 0; h < Hq; ++h) {
+            double g0 = gate[(i * Hq + h) * 2], g1 = gate[(i * Hq + h) * 2 + 1];
+            double gm = g0 > g1 ? g0 : g1;
+            double e0 = exp(g0 - gm), e1 = exp(g1 - gm);
+            double w0 = e0 / (e0 + e1), w1 = e1 / (e0 + e1);
+            long k0 = (r * Hq + h) * d;
+            double A = 0.0, B = 0.0;
+            for (int e = 0; e < d; ++e) {
+                A += dout[k0 + e] * oloc[k0 + e];
+                B += dout[k0 + e] * ocmp[k0 + e];
+            }
+            double mean = w0 * A + w1 * B;
+            dgate[(r * Hq + h) * 2] = w0 * (A - mean);
+            dgate[(r * Hq + h) * 2 + 1] = w1 * (B - mean);
+            for (int e = 0; e < d; ++e) {
+                dol[k0 + e] = w0 * dout[k0 + e];
+                doc[k0 + e] = w1 * dout[k0 + e];
+            }
+        }
+    }
+}
+
+/* Packed indices of the tokens in the clipped box of radii (rz,ry,rx)
+ * around site (zi,yi,xi); returns the count.  The box relation is symmetric:
+ * j lies in the window of i exactly when i lies in the window of j. */
+static long window_tokens(const orc_cfg *c, const int32_t *g2p, int zi, int yi, int xi, long *nb)
+{
+    long cnt = 0;
+    for (int z = zi - c->rz; z <= zi + c->rz; ++z)
+        for (int y = yi - c->ry; y <= yi + c->ry; ++y)
+            for (int x = xi - c->rx; x <= xi + c->rx; ++x) {
+                if (z < 0 || z >= c->Z || y < 0 || y >= c->H || x < 0 || x >= c->W) continue;
+                nb[cnt++] = g2p[((long)z * c->H + y) * c->W + x];
+            }
+    return cnt;
+}
+
+/* Local branch, first pass, for the sampled rows (qr, dol, dqr in sample
+ * order): dqr[r,h] = scale sum_j dl_j klr[j,g], and each row's lse and
+ * delta = sum_j P_j <dol, vloc[j,g]>. */
+void orc_local_attn_backward_q(const orc_cfg *c, const int32_t *coords, const int32_t *g2p,
+                               const double *qr, const double *klr, const double *vloc,
+                               const double *dol, const int64_t *rows, long nrows,
+                               double *dqr, double *lse, double *delta)
+{
+    int d = c->dh, Hq = c->Hq, Hkv = c->Hkv;
+    long wmax = (long)(2 * c->rz + 1) * (2 * c->ry + 1) * (2 * c->rx + 1);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long r = 0; r < nrows; ++r) {
+        long i = rows[r];
+        long *nb = (long *)malloc(sizeof(long) * wmax);
+        double *l = (double *)malloc(sizeof(double) * wmax);
+        double *dp = (double *)malloc(sizeof(double) * wmax);
+        long cnt = window_tokens(c, g2p, coords[3 * i], coords[3 * i + 1], coords[3 * i + 2], nb);
+        for (int h = 0; h < Hq; ++h) {
+            int g = (int)(((long)h * Hkv) / Hq);
+            const double *q = qr + (r * Hq + h) * d;
+            const double *dor = dol + (r * Hq + h) * d;
+            double lmax = -INFINITY, den = 0.0, dl_mean = 0.0;
+            for (long k = 0; k < cnt; ++k) {
+                const double *kk = klr + (nb[k] * Hkv + g) * d;
+                const double *vv = vloc + (nb[k] * Hkv + g) * d;
+                double s = 0.0, t = 0.0;
+                for (int e = 0; e < d; ++e) { s += q[e] * kk[e]; t += dor[e] * vv[e]; }
+                l[k] = c->scale * s;
+                dp[k] = t;
+                if (l[k] > lmax) lmax = l[k];
+            }
+            for (long k = 0; k < cnt; ++k) den += exp(l[k] - lmax);
+            double ls = lmax + log(den);
+            for (long k = 0; k < cnt; ++k) dl_mean += exp(l[k] - ls) * dp[k];
+            double *dq = dqr + (r * Hq + h) * d;
+            for (int e = 0; e < d; ++e) dq[e] = 0.0;
+            for (long k = 0; k < cnt; ++k) {
+                double dl = exp(l[k] - ls) * (dp[k] - dl_mean);
+                const double *kk = klr + (nb[k] * Hkv + g) * d;
+                for (int e = 0; e < d; ++e) dq[e] += c->scale * dl * kk[e];
+            }
+            lse[r * Hq + h] = ls;
+            delta[r * Hq + h] = dl_mean;
+        }
+        free(nb);
+        free(l);
+        free(dp);
+    }
+}
+
+/* Local branch, second pass, for the listed keys: for key token j and kv
+ * head g, over every query i whose window holds j (the box around j) and
+ * every q head h of group g,
+ *   dklr[k,g] = scale sum dl_{ih,j} qr[i,h],  dvloc[k,g] = sum P_{ih,j} dol[i,h].
+ * qr, dol, lse, delta hold every token; dklr, dvloc the listed keys in order. */
+void orc_local_attn_backward_kv(const orc_cfg *c, const int32_t *coords, const int32_t *g2p,
+                                const double *qr, const double *klr, const double *vloc,
+                                const double *dol, const double *lse, const double *delta,
+                                const int64_t *keys, long nkeys, double *dklr, double *dvloc)
+{
+    int d = c->dh, Hq = c->Hq, Hkv = c->Hkv;
+    long wmax = (long)(2 * c->rz + 1) * (2 * c->ry + 1) * (2 * c->rx + 1);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long r = 0; r < nkeys; ++r) {
+        long j = keys[r];
+        long *nb = (long *)malloc(sizeof(long) * wmax);
+        long cnt = window_tokens(c, g2p, coords[3 * j], coords[3 * j + 1], coords[3 * j + 2], nb);
+        for (int g = 0; g < Hkv; ++g) {
+            const double *kk = klr + (j * Hkv + g) * d;
+            const double *vv = vloc + (j * Hkv + g) * d;
+            double *dk = dklr + (r * Hkv + g) * d;
+            double *dv = dvloc + (r * Hkv + g) * d;
+            for (int e = 0; e < d; ++e) { dk[e] = 0.0; dv[e] = 0.0; }
+            for (long k = 0; k < cnt; ++k) {
+                long i = nb[k];
+                for (int h = 0; h < Hq; ++h) {
+                    if ((int)(((long)h * Hkv) / Hq) != g) continue;
+                    const double *q = qr + (i * Hq + h) * d;
+                    const double *dor = dol + (i * Hq + h) * d;
+                    double s = 0.0, t = 0.0;
+                    for (int e = 0; e < d; ++e) { s += q[e] * kk[e]; t += dor[e] * vv[e]; }
+                    double P = exp(c->scale * s - lse[i * Hq + h]);
+                    double dl = P * (t - delta[i * Hq + h]);
+                    for (int e = 0; e < d; ++e) {
+                        dk[e] += c->scale * dl * q[e];
+                        dv[e] += P * dor[e];
+                    }
+                }
+            }
+        }
+        free(nb);
+    }
+}
+
+/* Compressed branch, first pass, for nrows query rows (qr, doc in row order)
+ * against all M summaries: each row's lse and delta, and, when dqr is not
+ * NULL, dqr[r,h] = scale sum_j dl_j ksum[j,g]. */
+void orc_summary_attn_backward_q(const orc_cfg *c, const double *qr, const double *ksum,
+                                 const double *vsum, long M, long nrows, const double *doc,
+                                 double *dqr, double *lse, double *delta)
+{
+    int d = c->dh, Hq = c->Hq, Hkv = c->Hkv;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long r = 0; r < nrows; ++r) {
+        double *l = (double *)malloc(sizeof(double) * M);
+        double *dp = (double *)malloc(sizeof(double) * M);
+        for (int h = 0; h < Hq; ++h) {
+            int g = (int)(((long)h * Hkv) / Hq);
+            const double *q = qr + (r * Hq + h) * d;
+            const double *dor = doc + (r * Hq + h) * d;
+            double lmax = -INFINITY, den = 0.0, dl_mean = 0.0;
+            for (long j = 0; j < M; ++j) {
+                const double *kk = ksum + (j * Hkv + g) * d;
+                const double *vv = vsum + (j * Hkv + g) * d;
+                double s = 0.0, t = 0.0;
+                for (int e = 0; e < d; ++e) { s += q[e] * kk[e]; t += dor[e] * vv[e]; }
+                l[j] = c->scale * s;
+                dp[j] = t;
+                if (l[j] > lmax) lmax = l[j];
+            }
+            for (long j = 0; j < M; ++j) den += exp(l[j] - lmax);
+            double ls = lmax + log(den);
+            for (long j = 0; j < M; ++j) dl_mean += exp(l[j] - ls) * dp[j];
+            if (dqr) {
+                double *dq = dqr + (r * Hq + h) * d;
+                for (int e = 0; e < d; ++e) dq[e] = 0.0;
+                for (long j = 0; j < M; ++j) {
+                    double dl = exp(l[j] - ls) * (dp[j] - dl_mean);
+                    const double *kk = ksum + (j * Hkv + g) * d;
+                    for (int e = 0; e < d; ++e) dq[e] += c->scale * dl * kk[e];
+                }
+            }
+            lse[r * Hq + h] = ls;
+            delta[r * Hq + h] = dl_mean;
+        }
+        free(l);
+        free(dp);
+    }
+}
+
+/* Compressed branch, second pass, for the listed summaries js: over every
+ * query row i (all nrows, in row order) and q head h of group g,
+ *   dksum[k,g] = scale sum dl_{ih,j} qr[i,h],  dvsum[k,g] = sum P_{ih,j} doc[i,h]. */
+void orc_summary_attn_backward_kv(const orc_cfg *c, const double *qr, const double *ksum,
+                                  const double *vsum, long nrows, const double *doc,
+                                  const double *lse, const double *delta,
+                                  const int64_t *js, long nj, double *dksum, double *dvsum)
+{
+    int d = c->dh, Hq = c->Hq, Hkv = c->Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long r = 0; r < nj * Hkv; ++r) {
+        long jr = r / Hkv;
+        int g = (int)(r % Hkv);
+        long j = js[jr];
+        const double *kk = ksum + (j * Hkv + g) * d;
+        const double *vv = vsum + (j * Hkv + g) * d;
+        double *dk = dksum + (jr * Hkv + g) * d;
+        double *dv = dvsum + (jr * Hkv + g) * d;
+        for (int e = 0; e < d; ++e) { dk[e] = 0.0; dv[e] = 0.0; }
+        for (long i = 0; i < nrows; ++i)
+            for (int h = 0; h < Hq; ++h) {
+                if ((int)(((long)h * Hkv) / Hq) != g) continue;
+                const double *q = qr + (i * Hq + h) * d;
+                const double *dor = doc + (i * Hq + h) * d;
+                double s = 0.0, t = 0.0;
+                for (int e = 0; e < d; ++e) { s += q[e] * kk[e]; t += dor[e] * vv[e]; }
+                double P = exp(c->scale * s - lse[i * Hq + h]);
+                double dl = P * (t - delta[i * Hq + h]);
+                for (int e = 0; e < d; ++e) {
+                    dk[e] += c->scale * dl * q[e];
+                    dv[e] += P * dor[e];
+                }
+            }
+    }
+}
+
+/* Summaries backward (rotate-before-compress form) for the listed blocks
+ * (dksum, dvsum and the outputs in list order; member t of block jr at
+ * row jr*v + t):
+ *   a_u = softmax over B_j of s_{u,g},  Kcr_u = R(c_u) kcmp[u,g]
+ *   dkcmp[u,g] = R(c_u)^T (a_u dksum[j,g]),  dvcmp[u,g] = a_u dvsum[j,g]
+ *   da_u = <dksum[j,g], Kcr_u> + <dvsum[j,g], vcmp[u,g]>
+ *   dscores[u,g] = a_u (da_u - sum_u' a_u' da_u'). */
+void orc_summaries_backward(const orc_cfg *c, const int32_t *coords, const int32_t *members,
+                            const double *kcmp, const double *vcmp, const double *scores,
+                            const double *dksum, const double *dvsum,
+                            const int64_t *blocks, long nb, double *dkcmp, double *dvcmp,
+                            double *dscores)
+{
+    int v = c->bz * c->by * c->bx;
+    int d = c->dh, Hkv = c->Hkv;
+#pragma omp parallel for schedule(static)
+    for (long jr = 0; jr < nb; ++jr) {
+        long j = blocks[jr];
+        double *a = (double *)malloc(sizeof(double) * v);
+        double *da = (double *)malloc(sizeof(double) * v);
+        double *kr = (double *)malloc(sizeof(double) * d);
+        double *t = (double *)malloc(sizeof(double) * d);
+        for (int g = 0; g < Hkv; ++g) {
+            const double *dk = dksum + (jr * Hkv + g) * d;
+            const double *dv = dvsum + (jr * Hkv + g) * d;
+            double smax = -INFINITY, den = 0.0, mean = 0.0;
+            for (int m = 0; m < v; ++m) {
+                double s = scores[(long)members[j * v + m] * Hkv + g];
+                if (s > smax) smax = s;
+            }
+            for (int m = 0; m < v; ++m) {
+                a[m] = exp(scores[(long)members[j * v + m] * Hkv + g] - smax);
+                den += a[m];
+            }
+            for (int m = 0; m < v; ++m) a[m] /= den;
+            for (int m = 0; m < v; ++m) {
+                long u = members[j * v + m];
+                rotate_row(c, coords[3 * u], coords[3 * u + 1], coords[3 * u + 2],
+                           kcmp + (u * Hkv + g) * d, kr);
+                da[m] = 0.0;
+                for (int e = 0; e < d; ++e)
+                    da[m] += dk[e] * kr[e] + dv[e] * vcmp[(u * Hkv + g) * d + e];
+                mean += a[m] * da[m];
+                for (int e = 0; e < d; ++e) t[e] = a[m] * dk[e];
+                long o = ((jr * v + m) * Hkv + g) * d;
+                rotate_row_t(c, coords[3 * u], coords[3 * u + 1], coords[3 * u + 2], t, dkcmp + o);
+                for (int e = 0; e < d; ++e) dvcmp[o + e] = a[m] * dv[e];
+            }
+            for (int m = 0; m < v; ++m) dscores[(jr * v + m) * Hkv + g] = a[m] * (da[m] - mean);
+        }
+        free(a);
+        free(da);
+        free(kr);
+        free(t);
     }
 }

@@ -11,6 +11,9 @@ method section "Key design 1-3" and the scaling table, Table 4):
   ``numpy.random.default_rng(seed)`` (PCG64), as float32 standard normals via
   ``Generator.standard_normal(dtype=float32)``.  Tensors are drawn in a fixed
   order: Q, K_loc, V_loc, K_cmp, V_cmp, block scores, gate logits.
+* The output gradient dOut of the backward pass (the stress configuration's
+  dOut ~ N(0,1)) is drawn the same way, per site in raster order, from its own
+  generator ``default_rng(seed + 2)``, so the forward inputs do not change.
 * Q/K/V draws are multiplied by ``value_scale`` (1 for the tiny case, 1/8 =
   1/sqrt(d_h) for the large volumes).  Scores and gate logits stay N(0,1).
 * The per-site tensors are then permuted into packed order: packed slot ``p``
@@ -39,7 +42,7 @@ import numpy as np
 
 __all__ = [
     "Pack3DShape", "CONFIGS", "lattice_sites", "packing_sites", "coords_for",
-    "draw_site_values", "make_inputs", "sample_rows",
+    "draw_site_values", "make_inputs", "sample_rows", "make_dout",
 ]
 
 
@@ -210,6 +213,21 @@ def make_inputs(shape: Pack3DShape, packing: Optional[str] = None, seed: int = 0
     for name in ("scores", "gate"):
         res[name] = torch.from_numpy(sv[name]).index_select(0, idx).contiguous()
     return res
+
+
+def make_dout(shape: Pack3DShape, packing: Optional[str] = None, seed: int = 0, scale: float = 1.0):
+    """Packed output gradient dOut [N, Hq, d_h] in ``shape.dtype`` (torch CPU tensor):
+    ``scale`` times N(0,1) float32 draws per lattice site in raster order from
+    ``default_rng(seed + 2)``, permuted like ``make_inputs``'s tensors."""
+    import torch
+    packing = packing or shape.packing
+    rng = np.random.default_rng(seed + 2)
+    a = rng.standard_normal((shape.N, shape.Hq, shape.d_h), dtype=np.float32)
+    if scale != 1:
+        a *= np.float32(scale)
+    sites = packing_sites(shape.Z, shape.H, shape.W, packing, seed, (shape.bz, shape.by, shape.bx))
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    return torch.from_numpy(a).index_select(0, torch.from_numpy(sites)).to(tdt).contiguous()
 
 
 def make_inputs_on_device(shape: Pack3DShape, packing: Optional[str] = None, seed: int = 0,
