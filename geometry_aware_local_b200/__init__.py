@@ -28,7 +28,8 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: 
 ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
                 "pack3d_build_index", "pack3d_rope", "pack3d_rope_qk", "pack3d_build_summaries", "pack3d_local_attn",
                 "pack3d_summary_attn", "pack3d_forward", "pack3d_forward_noalloc", "pack3d_pipeline_create",
-                "pack3d_pipeline_destroy", "pack3d_host_workspace_bytes", "pack3d_forward_host", "pack3d_check_status",
+                "pack3d_pipeline_destroy", "pack3d_host_workspace_bytes", "pack3d_forward_host",
+                "pack3d_train_workspace_bytes", "pack3d_forward_backward", "pack3d_check_status",
                 "pack3d_status_string", "pack3d_backend_info")
 
 
@@ -85,6 +86,8 @@ def _load():
         "pack3d_pipeline_destroy": (None, [P]),
         "pack3d_host_workspace_bytes": (ctypes.c_size_t, [C]),
         "pack3d_forward_host": (ctypes.c_int, [P, C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
+        "pack3d_train_workspace_bytes": (ctypes.c_size_t, [C]),
+        "pack3d_forward_backward": (ctypes.c_int, [C] + [P] * 18 + [ctypes.c_size_t, P, P]),
         "pack3d_check_status": (ctypes.c_int, [P, P]),
         "pack3d_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "pack3d_backend_info": (ctypes.c_char_p, []),
@@ -250,6 +253,33 @@ def forward_host(pipeline, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, g
                                    _host_ptr(k_loc), _host_ptr(v_loc), _host_ptr(k_cmp), _host_ptr(v_cmp),
                                    _host_ptr(scores), _host_ptr(gate), _host_ptr(out), _ptr(workspace), ws_bytes,
                                    _ptr(err), _stream(stream)), "pack3d_forward_host")
+
+
+def train_workspace_bytes(cfg: Config) -> int:
+    return int(lib.pack3d_train_workspace_bytes(ctypes.byref(cfg)))
+
+
+GRAD_NAMES = ("dq", "dk_loc", "dv_loc", "dk_cmp", "dv_cmp", "dscores", "dgate")
+
+
+def forward_backward(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, dout, out, grads, workspace, err,
+                     stream=None):
+    """pack3d_forward_backward: the forward output into `out` and the gradients of <dout, out> into the
+    tensors of the dict `grads` (keys GRAD_NAMES, shapes and dtypes of the matching inputs)."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    g = [grads[k] for k in GRAD_NAMES]
+    _check(lib.pack3d_forward_backward(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc),
+                                       _ptr(k_cmp), _ptr(v_cmp), _ptr(scores), _ptr(gate), _ptr(dout), _ptr(out),
+                                       *[_ptr(x) for x in g], _ptr(workspace), ws_bytes, _ptr(err),
+                                       _stream(stream)), "pack3d_forward_backward")
+
+
+def empty_grads(q, k_loc, scores, gate):
+    """Output tensors for forward_backward, shaped like the inputs they differentiate."""
+    import torch
+    return {"dq": torch.empty_like(q), "dk_loc": torch.empty_like(k_loc), "dv_loc": torch.empty_like(k_loc),
+            "dk_cmp": torch.empty_like(k_loc), "dv_cmp": torch.empty_like(k_loc),
+            "dscores": torch.empty_like(scores), "dgate": torch.empty_like(gate)}
 
 
 def check_status(err, stream=None) -> int:

@@ -94,6 +94,32 @@ Workspace carve(const pack3d_config& c, uintptr_t base) {
   return w;
 }
 
+// Regions of the training block after the forward workspace.
+struct TrainWs {
+  float* stats;   // [N,Hq,4]
+  float* dqr;     // [N,Hq,64]
+  float* dks;     // [M,Hkv,64], followed directly by dvs
+  float* dvs;
+  size_t dkv_bytes;
+  size_t bytes;
+};
+
+TrainWs carve_train(const pack3d_config& c, uintptr_t base) {
+  const size_t N = (size_t)c.Z * c.H * c.W;
+  const size_t M = N / ((size_t)c.bz * c.by * c.bx);
+  const size_t A = 1024;
+  TrainWs t;
+  size_t off = carve(c, 0).bytes;
+  t.stats = reinterpret_cast<float*>(base + off);  off = round_up(off + N * c.Hq * 16, A);
+  t.dqr = reinterpret_cast<float*>(base + off);    off = round_up(off + N * c.Hq * c.d_h * 4, A);
+  t.dkv_bytes = M * c.Hkv * c.d_h * 4;
+  t.dks = reinterpret_cast<float*>(base + off);
+  t.dvs = reinterpret_cast<float*>(base + off + t.dkv_bytes);
+  off = round_up(off + 2 * t.dkv_bytes, A);
+  t.bytes = off;
+  return t;
+}
+
 }  // namespace
 
 extern "C" {
@@ -250,6 +276,62 @@ pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, co
     else
       e = launch_summary_attn_simt(s, cfg->dtype, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, cs);
   }
+  return cuda_status(e);
+}
+
+size_t pack3d_train_workspace_bytes(const pack3d_config* cfg) {
+  if (pack3d_validate_config(cfg) != PACK3D_OK) return 0;
+  return carve_train(*cfg, 0).bytes;
+}
+
+pack3d_status pack3d_forward_backward(const pack3d_config* cfg, const int32_t* coords, const void* q,
+                                      const void* k_loc, const void* v_loc, const void* k_cmp, const void* v_cmp,
+                                      const float* scores, const float* gate, const void* dout, void* out,
+                                      void* dq, void* dk_loc, void* dv_loc, void* dk_cmp, void* dv_cmp,
+                                      float* dscores, float* dgate, void* workspace, size_t workspace_bytes,
+                                      int32_t* err_word, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (cfg->flags & PACK3D_FLAG_SUMMARY_CENTER) return PACK3D_ERR_INVALID_ARG;
+  if (!coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !dout || !out || !dq ||
+      !dk_loc || !dv_loc || !dk_cmp || !dv_cmp || !dscores || !dgate || !err_word)
+    return PACK3D_ERR_INVALID_ARG;
+  if (!workspace || ((uintptr_t)workspace & 255u)) return PACK3D_ERR_WORKSPACE;
+  const Workspace w = carve(*cfg, (uintptr_t)workspace);
+  const TrainWs t = carve_train(*cfg, (uintptr_t)workspace);
+  if (workspace_bytes < t.bytes) return PACK3D_ERR_WORKSPACE;
+  const void* ptrs[] = {coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, dout, out, dq,
+                        dk_loc, dv_loc, dk_cmp, dv_cmp, dscores, dgate};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return PACK3D_ERR_ALIGNMENT;
+  const Shape s = make_shape(*cfg);
+  const int dt = cfg->dtype;
+  const cudaStream_t cs = (cudaStream_t)stream;
+  // Forward, leaving the row statistics and dgate.
+  cudaError_t e = launch_build_index(s, coords, w.g2p, w.members, err_word, cs);
+  if (e == cudaSuccess) e = launch_rope(s, dt, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, cs);
+  if (e == cudaSuccess) e = launch_summaries(s, dt, w.members, k_cmp, v_cmp, scores, w.k_sum, w.v_sum, cs);
+  if (e == cudaSuccess)
+    e = launch_local(s, dt, cfg->flags, w.g2p, w.q_rot, w.k_rot, v_loc, w.o_loc, err_word, cs, t.stats);
+  const Train tr{t.stats, dout, dgate};
+  if (e == cudaSuccess) {
+    if (dt == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
+      e = launch_summary_attn_tc(s, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, err_word, cs, 0, -1, &tr);
+    else
+      e = launch_summary_attn_simt(s, dt, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, cs, &tr);
+  }
+  // Backward: compressed branch, local branch, summaries (RoPE transposes fused).
+  if (e == cudaSuccess) e = cudaMemsetAsync(t.dks, 0, 2 * t.dkv_bytes, cs);
+  if (e == cudaSuccess) e = launch_summary_bwd_dq(s, dt, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dqr, cs);
+  if (e == cudaSuccess)
+    e = launch_summary_bwd_dkv(s, dt, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dks, t.dvs, cs);
+  if (e == cudaSuccess)
+    e = launch_local_bwd_dq(s, dt, w.g2p, w.q_rot, w.k_rot, v_loc, dout, gate, t.stats, t.dqr, dq, cs);
+  if (e == cudaSuccess)
+    e = launch_local_bwd_dkv(s, dt, w.g2p, w.q_rot, w.k_rot, v_loc, dout, gate, t.stats, dk_loc, dv_loc, cs);
+  if (e == cudaSuccess)
+    e = launch_summaries_bwd(s, dt, coords, w.members, k_cmp, v_cmp, scores, t.dks, t.dvs, dk_cmp, dv_cmp,
+                             dscores, cs);
   return cuda_status(e);
 }
 

@@ -156,6 +156,71 @@ __device__ __forceinline__ void rotate_at(float* f, const Shape& s, int p0, doub
   }
 }
 
+// Rotates the 2*np values f (planes p0 .. p0+np-1) of one row at the lattice
+// site (z, y, x) by R(c) (transpose = false) or by R(c)^T (transpose = true),
+// reading the per-CTA table.  R(c)^T is the RoPE backward: each active pair
+// (y0, y1) becomes (y0 cos t + y1 sin t, -y0 sin t + y1 cos t).
+__device__ __forceinline__ void rope_planes(float* f, const Shape& s, const float2* tab, int p0, int np, int z,
+                                            int y, int x, bool transpose) {
+  const float sg = transpose ? -1.f : 1.f;
+#pragma unroll
+  for (int k = 0; k < np; ++k) {
+    const int p = p0 + k;
+    if (p >= s.npairs) break;
+    const int ax = s.pair_axis[p];
+    const int cval = ax == 0 ? z : (ax == 1 ? y : x);
+    const float2 cs = tab[s.pair_off[p] + cval];
+    const float sn = sg * cs.y;
+    const float x0 = f[2 * k], x1 = f[2 * k + 1];
+    f[2 * k] = x0 * cs.x - x1 * sn;
+    f[2 * k + 1] = x0 * sn + x1 * cs.x;
+  }
+}
+
+// Training epilogue of a query x summary row (the gate's backward): with
+// gamma = softmax(gate row), A = <dout, o_loc> and B = <dout, o_cmp>,
+//   dgate = (gamma0 (A - m), gamma1 (B - m)),  m = gamma0 A + gamma1 B,
+// and the row statistics the branches' backward reads: stats[4 row + 1] =
+// lse2 of the compressed softmax, [4 row + 2] = gamma0 A = <gamma0 dout, o_loc>
+// and [4 row + 3] = gamma1 B (the softmax-backward deltas of the two branches;
+// [4 row] holds the local branch's lse2, written by the local kernel).
+template <typename T>
+__device__ __forceinline__ void train_epilogue_row(const float* o_cmp, const float* __restrict__ gate,
+                                                   const float* __restrict__ oloc, const T* __restrict__ dout,
+                                                   size_t row, float lse2, float* __restrict__ stats,
+                                                   float* __restrict__ dgate) {
+  constexpr int NE = Elem<T>::kPerChunk;
+  const float g0 = __ldg(gate + 2 * row), g1 = __ldg(gate + 2 * row + 1);
+  const float gm = fmaxf(g0, g1);
+  const float e0 = expf(g0 - gm), e1 = expf(g1 - gm);
+  const float w0 = e0 / (e0 + e1), w1 = e1 / (e0 + e1);
+  const float* lo = oloc + row * kDh;
+  float A = 0.f, B = 0.f;
+#pragma unroll
+  for (int c = 0; c < kDh / NE; ++c) {
+    float f[NE];
+    chunk_to_float(ldg16(dout + row * kDh + c * NE), f, T());
+#pragma unroll
+    for (int k = 0; k < NE; ++k) {
+      A = fmaf(f[k], __ldg(lo + c * NE + k), A);
+      B = fmaf(f[k], o_cmp[c * NE + k], B);
+    }
+  }
+  const float m = w0 * A + w1 * B;
+  *reinterpret_cast<float2*>(dgate + 2 * row) = make_float2(w0 * (A - m), w1 * (B - m));
+  stats[4 * row + 1] = lse2;
+  stats[4 * row + 2] = w0 * A;
+  stats[4 * row + 3] = w1 * B;
+}
+
+// Gate weights (gamma0, gamma1) = softmax(gate row).
+__device__ __forceinline__ float2 gate_weights(const float* __restrict__ gate, size_t row) {
+  const float g0 = __ldg(gate + 2 * row), g1 = __ldg(gate + 2 * row + 1);
+  const float gm = fmaxf(g0, g1);
+  const float e0 = expf(g0 - gm), e1 = expf(g1 - gm);
+  return make_float2(e0 / (e0 + e1), e1 / (e0 + e1));
+}
+
 __device__ __forceinline__ void set_err(int32_t* err, int bits) {
   if (err) atomicOr(err, bits);
 }

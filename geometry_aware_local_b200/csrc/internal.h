@@ -9,6 +9,16 @@ namespace pack3d {
 
 struct Shape;
 
+// Extra outputs of the forward pass when it runs as the first half of the
+// training block (pack3d_forward_backward): per (token, q head) row four
+// floats of statistics for the backward, the gate gradient, and the output
+// gradient they are formed with.  Null pointers: plain forward.
+struct Train {
+  float* stats;        // [N, Hq, 4]: lse2 local, lse2 compressed, delta local, delta compressed
+  const void* dout;    // [N, Hq, 64] in the operator's dtype
+  float* dgate;        // [N, Hq, 2]
+};
+
 cudaError_t launch_build_index(const Shape& s, const int32_t* coords, int32_t* g2p,
                                int32_t* members, int32_t* err, cudaStream_t st);
 
@@ -20,30 +30,63 @@ cudaError_t launch_summaries(const Shape& s, int dtype, const int32_t* members, 
                              const void* vc, const float* scores, void* ks, void* vs,
                              cudaStream_t st);
 
+// stats (nullable): the local softmax's lse2 (log2 units of the scaled logits)
+// goes to stats[4 row].
 cudaError_t launch_local_attn(const Shape& s, int dtype, const int32_t* g2p, const void* qr,
-                              const void* kr, const void* vl, float* oloc, cudaStream_t st);
+                              const void* kr, const void* vl, float* oloc, cudaStream_t st,
+                              float* stats = nullptr);
 
 // Local attention on the best kernel for the shape: tcgen05 when supported
 // and not disabled by PACK3D_FLAG_SIMT_LOCAL, else CUDA cores.
 cudaError_t launch_local(const Shape& s, int dtype, int flags, const int32_t* g2p, const void* qr,
-                         const void* kr, const void* vl, float* oloc, int32_t* err, cudaStream_t st);
+                         const void* kr, const void* vl, float* oloc, int32_t* err, cudaStream_t st,
+                         float* stats = nullptr);
 
 // tcgen05 local attention (bf16, G = 4, rz = 1, ry <= 3, rx <= 3).
 bool local_attn_tc_supported(const Shape& s, int dtype);
 cudaError_t launch_local_attn_tc(const Shape& s, const int32_t* g2p, const void* qr, const void* kr,
-                                 const void* vl, float* oloc, int32_t* err, cudaStream_t st);
+                                 const void* vl, float* oloc, int32_t* err, cudaStream_t st,
+                                 float* stats = nullptr);
 
 // CUDA-core query x summary kernel (float, or bf16 on request).
 cudaError_t launch_summary_attn_simt(const Shape& s, int dtype, const void* qr, const void* ks,
                                      const void* vs, const float* oloc, const float* gate,
-                                     void* out, cudaStream_t st);
+                                     void* out, cudaStream_t st, const Train* tr = nullptr);
 
 // tcgen05 query x summary kernel (bf16 only), for the tokens [tok_begin,
 // tok_end) (tok_end < 0: to the end); tok_begin must be a multiple of
 // summary_attn_tc_token_quantum(s), the tokens one CTA covers.
 cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
                                    const float* oloc, const float* gate, void* out, int32_t* err,
-                                   cudaStream_t st, long tok_begin = 0, long tok_end = -1);
+                                   cudaStream_t st, long tok_begin = 0, long tok_end = -1,
+                                   const Train* tr = nullptr);
 long summary_attn_tc_token_quantum(const Shape& s);
+
+// ---- backward pass of the training block (k_backward.cu) ----
+// Inputs: the forward's rotated Q / K_loc, summaries, statistics and the
+// output gradient; float accumulators dqr [N,Hq,64] and dks / dvs [M,Hkv,64].
+
+// Compressed branch, query side: dqr = scale * sum_j dS_j k~_j (overwrites dqr).
+cudaError_t launch_summary_bwd_dq(const Shape& s, int dtype, const void* qr, const void* ks, const void* vs,
+                                  const void* dout, const float* gate, const float* stats, float* dqr,
+                                  cudaStream_t st);
+// Compressed branch, summary side: dks += scale * sum_i dS_i q_i, dvs += sum_i P_i do_i
+// (float atomics; dks and dvs must be zeroed first).
+cudaError_t launch_summary_bwd_dkv(const Shape& s, int dtype, const void* qr, const void* ks, const void* vs,
+                                   const void* dout, const float* gate, const float* stats, float* dks,
+                                   float* dvs, cudaStream_t st);
+// Local branch, query side, plus the compressed part from dqr and the RoPE
+// backward: dq = R(c)^T (scale * sum_j dS_j k_j + dqr).
+cudaError_t launch_local_bwd_dq(const Shape& s, int dtype, const int32_t* g2p, const void* qr, const void* kr,
+                                const void* vl, const void* dout, const float* gate, const float* stats,
+                                const float* dqr, void* dq, cudaStream_t st);
+// Local branch, key side, with the RoPE backward: dk_loc = R(c)^T dKlr, dv_loc.
+cudaError_t launch_local_bwd_dkv(const Shape& s, int dtype, const int32_t* g2p, const void* qr, const void* kr,
+                                 const void* vl, const void* dout, const float* gate, const float* stats,
+                                 void* dk, void* dv, cudaStream_t st);
+// Summaries backward: dk_cmp, dv_cmp, dscores from dks, dvs.
+cudaError_t launch_summaries_bwd(const Shape& s, int dtype, const int32_t* coords, const int32_t* members,
+                                 const void* kc, const void* vc, const float* scores, const float* dks,
+                                 const float* dvs, void* dkc, void* dvc, float* dsc, cudaStream_t st);
 
 }  // namespace pack3d

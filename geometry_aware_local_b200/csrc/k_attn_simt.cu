@@ -29,7 +29,7 @@ __device__ __forceinline__ void load_row_f32(const T* p, float* f) {
 template <typename T, int G>
 __global__ void __launch_bounds__(kBrickSites * G) local_attn_kernel(
     Shape s, const int32_t* __restrict__ g2p, const T* __restrict__ qr, const T* __restrict__ kr,
-    const T* __restrict__ vl, float* __restrict__ oloc) {
+    const T* __restrict__ vl, float* __restrict__ oloc, float* __restrict__ stats) {
   constexpr int NE = Elem<T>::kPerChunk;
   const int bricks_x = (s.W + kBrickX - 1) / kBrickX;
   const int bricks_y = (s.H + kBrickY - 1) / kBrickY;
@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kBrickSites * G) local_attn_kernel(
       }
     }
   const float inv = 1.f / l;
+  if (stats) stats[4 * ((size_t)i * s.Hq + h)] = m + log2f(l);
   float* o = oloc + ((size_t)i * s.Hq + h) * kDh;
 #pragma unroll
   for (int c = 0; c < kDh / 4; ++c)
@@ -100,30 +101,30 @@ __global__ void __launch_bounds__(kBrickSites * G) local_attn_kernel(
 
 template <typename T, int G>
 static cudaError_t local_t(const Shape& s, const int32_t* g2p, const void* qr, const void* kr,
-                           const void* vl, float* oloc, cudaStream_t st) {
+                           const void* vl, float* oloc, cudaStream_t st, float* stats) {
   const int bricks = s.Z * ((s.H + kBrickY - 1) / kBrickY) * ((s.W + kBrickX - 1) / kBrickX);
   dim3 grid(bricks, s.Hkv);
   local_attn_kernel<T, G><<<grid, kBrickSites * G, 0, st>>>(s, g2p, (const T*)qr, (const T*)kr,
-                                                            (const T*)vl, oloc);
+                                                            (const T*)vl, oloc, stats);
   return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t local_g(const Shape& s, const int32_t* g2p, const void* qr, const void* kr,
-                           const void* vl, float* oloc, cudaStream_t st) {
+                           const void* vl, float* oloc, cudaStream_t st, float* stats) {
   switch (s.G) {
-    case 1: return local_t<T, 1>(s, g2p, qr, kr, vl, oloc, st);
-    case 2: return local_t<T, 2>(s, g2p, qr, kr, vl, oloc, st);
-    case 4: return local_t<T, 4>(s, g2p, qr, kr, vl, oloc, st);
-    case 8: return local_t<T, 8>(s, g2p, qr, kr, vl, oloc, st);
+    case 1: return local_t<T, 1>(s, g2p, qr, kr, vl, oloc, st, stats);
+    case 2: return local_t<T, 2>(s, g2p, qr, kr, vl, oloc, st, stats);
+    case 4: return local_t<T, 4>(s, g2p, qr, kr, vl, oloc, st, stats);
+    case 8: return local_t<T, 8>(s, g2p, qr, kr, vl, oloc, st, stats);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_local_attn(const Shape& s, int dtype, const int32_t* g2p, const void* qr,
-                              const void* kr, const void* vl, float* oloc, cudaStream_t st) {
-  if (dtype == PACK3D_BF16) return local_g<__nv_bfloat16>(s, g2p, qr, kr, vl, oloc, st);
-  return local_g<float>(s, g2p, qr, kr, vl, oloc, st);
+                              const void* kr, const void* vl, float* oloc, cudaStream_t st, float* stats) {
+  if (dtype == PACK3D_BF16) return local_g<__nv_bfloat16>(s, g2p, qr, kr, vl, oloc, st, stats);
+  return local_g<float>(s, g2p, qr, kr, vl, oloc, st, stats);
 }
 
 // ---- query x summary, CUDA cores ----------------------------------------
@@ -160,7 +161,8 @@ __device__ __forceinline__ void gate_mix_row(float* o, const float* __restrict__
 template <typename T>
 __global__ void __launch_bounds__(kSaRows) summary_attn_simt_kernel(
     Shape s, const T* __restrict__ qr, const T* __restrict__ ks, const T* __restrict__ vs,
-    const float* __restrict__ oloc, const float* __restrict__ gate, T* __restrict__ out) {
+    const float* __restrict__ oloc, const float* __restrict__ gate, T* __restrict__ out,
+    float* __restrict__ stats, const T* __restrict__ dout, float* __restrict__ dgate) {
   __shared__ float Ksh[kSaTile][kDh], Vsh[kSaTile][kDh];
   const int g = blockIdx.y;
   const long rows = (long)s.N * s.G;
@@ -209,23 +211,27 @@ __global__ void __launch_bounds__(kSaRows) summary_attn_simt_kernel(
   const float inv = 1.f / l;
 #pragma unroll
   for (int e = 0; e < kDh; ++e) acc[e] *= inv;
+  if (stats) train_epilogue_row(acc, gate, oloc, dout, orow, m + log2f(l), stats, dgate);
   gate_mix_row(acc, gate, oloc, orow);
   store_row(out + orow * kDh, acc);
 }
 
 cudaError_t launch_summary_attn_simt(const Shape& s, int dtype, const void* qr, const void* ks,
                                      const void* vs, const float* oloc, const float* gate,
-                                     void* out, cudaStream_t st) {
+                                     void* out, cudaStream_t st, const Train* tr) {
   const long rows = (long)s.N * s.G;
   dim3 grid((unsigned)((rows + kSaRows - 1) / kSaRows), s.Hkv);
+  float* stats = tr ? tr->stats : nullptr;
+  float* dgate = tr ? tr->dgate : nullptr;
+  const void* dout = tr ? tr->dout : nullptr;
   if (dtype == PACK3D_BF16)
     summary_attn_simt_kernel<__nv_bfloat16><<<grid, kSaRows, 0, st>>>(
         s, (const __nv_bfloat16*)qr, (const __nv_bfloat16*)ks, (const __nv_bfloat16*)vs, oloc, gate,
-        (__nv_bfloat16*)out);
+        (__nv_bfloat16*)out, stats, (const __nv_bfloat16*)dout, dgate);
   else
     summary_attn_simt_kernel<float><<<grid, kSaRows, 0, st>>>(s, (const float*)qr, (const float*)ks,
                                                               (const float*)vs, oloc, gate,
-                                                              (float*)out);
+                                                              (float*)out, stats, (const float*)dout, dgate);
   return cudaGetLastError();
 }
 

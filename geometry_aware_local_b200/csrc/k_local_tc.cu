@@ -59,6 +59,7 @@ struct LocalArgs {
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
   float* oloc;
+  float* stats;            // nullable: lse2 of each row to stats[4 row]
   int32_t* err;
 };
 
@@ -311,6 +312,7 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
     ptx::tmem_ld64_sync(tO, &r[0][0]);
     if (qi >= 0) {
       const float inv = 1.f / l;
+      if (a.stats) a.stats[4 * ((size_t)qi * a.Hq + h)] = m_used + log2f(l);
       float4* o = reinterpret_cast<float4*>(a.oloc + ((size_t)qi * a.Hq + h) * kDh);
 #pragma unroll
       for (int q = 0; q < kDh / 4; ++q)
@@ -337,10 +339,11 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
 }  // namespace
 
 cudaError_t launch_local(const Shape& s, int dtype, int flags, const int32_t* g2p, const void* qr,
-                         const void* kr, const void* vl, float* oloc, int32_t* err, cudaStream_t st) {
+                         const void* kr, const void* vl, float* oloc, int32_t* err, cudaStream_t st,
+                         float* stats) {
   if (!(flags & PACK3D_FLAG_SIMT_LOCAL) && local_attn_tc_supported(s, dtype))
-    return launch_local_attn_tc(s, g2p, qr, kr, vl, oloc, err, st);
-  return launch_local_attn(s, dtype, g2p, qr, kr, vl, oloc, st);
+    return launch_local_attn_tc(s, g2p, qr, kr, vl, oloc, err, st, stats);
+  return launch_local_attn(s, dtype, g2p, qr, kr, vl, oloc, st, stats);
 }
 
 bool local_attn_tc_supported(const Shape& s, int dtype) {
@@ -348,7 +351,7 @@ bool local_attn_tc_supported(const Shape& s, int dtype) {
 }
 
 cudaError_t launch_local_attn_tc(const Shape& s, const int32_t* g2p, const void* qr, const void* kr,
-                                 const void* vl, float* oloc, int32_t* err, cudaStream_t st) {
+                                 const void* vl, float* oloc, int32_t* err, cudaStream_t st, float* stats) {
   LocalArgs a;
   a.Z = s.Z; a.H = s.H; a.W = s.W; a.Hq = s.Hq; a.Hkv = s.Hkv;
   a.ry = s.ry; a.rx = s.rx;
@@ -360,6 +363,7 @@ cudaError_t launch_local_attn_tc(const Shape& s, const int32_t* g2p, const void*
   a.k = (const __nv_bfloat16*)kr;
   a.v = (const __nv_bfloat16*)vl;
   a.oloc = oloc;
+  a.stats = stats;
   a.err = err;
   cudaError_t e = cudaFuncSetAttribute(local_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;

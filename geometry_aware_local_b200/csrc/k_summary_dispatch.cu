@@ -14,12 +14,14 @@ namespace pack3d {
 namespace sa_two {
 long token_quantum(const Shape& s);
 cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* vs, const float* oloc,
-                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end);
+                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end,
+                   const Train* tr);
 }  // namespace sa_two
 namespace sa_one {
 long token_quantum(const Shape& s);
 cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* vs, const float* oloc,
-                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end);
+                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end,
+                   const Train* tr);
 }  // namespace sa_one
 
 namespace {
@@ -33,9 +35,9 @@ long summary_attn_tc_token_quantum(const Shape& s) {
 
 cudaError_t launch_summary_attn_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
                                    const float* oloc, const float* gate, void* out, int32_t* err,
-                                   cudaStream_t st, long tok_begin, long tok_end) {
-  return one_tile(s) ? sa_one::launch(s, qr, ks, vs, oloc, gate, out, err, st, tok_begin, tok_end)
-                     : sa_two::launch(s, qr, ks, vs, oloc, gate, out, err, st, tok_begin, tok_end);
+                                   cudaStream_t st, long tok_begin, long tok_end, const Train* tr) {
+  return one_tile(s) ? sa_one::launch(s, qr, ks, vs, oloc, gate, out, err, st, tok_begin, tok_end, tr)
+                     : sa_two::launch(s, qr, ks, vs, oloc, gate, out, err, st, tok_begin, tok_end, tr);
 }
 
 }  // namespace pack3d

@@ -116,6 +116,9 @@ struct TcArgs {
   const float* oloc;
   const float* gate;
   __nv_bfloat16* out;
+  float* stats;                 // training: row statistics (nullable)
+  const __nv_bfloat16* dout;    // training: output gradient
+  float* dgate;                 // training: gate gradient
   int32_t* err;
 };
 
@@ -145,6 +148,9 @@ __device__ __forceinline__ float2 exp2_poly(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
+// kTrain: the training block's forward (row statistics and dgate in the
+// epilogue); a separate instantiation so the plain forward's code is unchanged.
+template <bool kTrain>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
@@ -415,6 +421,8 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         float o[kDh];
 #pragma unroll
         for (int e = 0; e < kDh; ++e) o[e] = __uint_as_float(r[e >> 5][e & 31]) * inv;
+        if constexpr (kTrain)
+          train_epilogue_row(o, a.gate, a.oloc, a.dout, orow, m_used + log2f(l), a.stats, a.dgate);
         if (a.gate != nullptr) {
           const float g0 = __ldg(a.gate + 2 * orow), g1 = __ldg(a.gate + 2 * orow + 1);
           const float gm = fmaxf(g0, g1);
@@ -481,7 +489,8 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
 long token_quantum(const Shape& s) { return (long)kGroups * kBM / s.G; }
 
 cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* vs, const float* oloc,
-                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end) {
+                   const float* gate, void* out, int32_t* err, cudaStream_t st, long tok_begin, long tok_end,
+                   const Train* tr) {
   if (tok_end < 0) tok_end = s.N;
   if (tok_begin < 0 || tok_begin >= tok_end || tok_end > s.N || tok_begin % token_quantum(s))
     return cudaErrorInvalidValue;
@@ -495,8 +504,10 @@ cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* v
   const cuuint32_t kb[3] = {(cuuint32_t)kDh, 1, (cuuint32_t)kBN};
   if (!encode(&tq, qr, 4, qd, qs, qb) || !encode(&tk, ks, 3, kd, kst, kb) || !encode(&tv, vs, 3, kd, kst, kb))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(summary_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
+  const bool train = tr != nullptr && tr->stats != nullptr;
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, TcArgs) =
+      train ? summary_attn_tc_kernel<true> : summary_attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   TcArgs a;
   a.M = s.M;
@@ -508,10 +519,13 @@ cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* v
   a.oloc = oloc;
   a.gate = gate;
   a.out = (__nv_bfloat16*)out;
+  a.stats = tr ? tr->stats : nullptr;
+  a.dout = tr ? (const __nv_bfloat16*)tr->dout : nullptr;
+  a.dgate = tr ? tr->dgate : nullptr;
   a.err = err;
   const long tiles = (a.rows - tok_begin * s.G + kBM - 1) / kBM;
   dim3 grid((unsigned)((tiles + kGroups - 1) / kGroups), s.Hkv);
-  summary_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
+  kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

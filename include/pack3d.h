@@ -1,7 +1,8 @@
 /*
  * pack3d.h - C ABI of the B200 (sm_100a) implementation of the PACK3D
- * local-global attention forward pass, from "Geometry Matters in Packed 3D
- * Attention" (method section, Key designs 1-3).
+ * local-global attention forward pass and its backward (the training block),
+ * from "Geometry Matters in Packed 3D Attention" (method section, Key designs
+ * 1-3).
  *
  * The operator maps packed 3D tokens and their lattice coordinates to packed
  * outputs, A(X, c), in five stages:
@@ -274,6 +275,46 @@ pack3d_status pack3d_forward_host(pack3d_pipeline *pipeline, const pack3d_config
                                   const float *scores, const float *gate, void *out,
                                   void *workspace, size_t workspace_bytes, int32_t *err_word,
                                   void *stream);
+
+/* ---- training block: forward and backward in one call ------------------------
+ * The pages call the operator a fused forward/backward training block; this
+ * call runs the forward pass and then the gradients of L = <dout, out> with
+ * respect to every input, by the chain rule through the stages in reverse:
+ *   gate:       dgate = gamma (dgamma - <gamma, dgamma>), dgamma_c = <dout, o_c>
+ *   branches:   for each softmax row, dl_j = P_j (<do, v_j> - <do, o>) with
+ *               do = gamma0 dout (local) or gamma1 dout (compressed);
+ *               dq += scale sum_j dl_j k_j, dk_j += scale dl_j q, dv_j += P_j do
+ *   summaries:  dk_cmp[u] = R(c_u)^T (a_u dk_sum[j]), dv_cmp[u] = a_u dv_sum[j],
+ *               dscores[u] = a_u (da_u - sum_u' a_u' da_u'),
+ *               da_u = <dk_sum[j], R(c_u) k_cmp[u]> + <dv_sum[j], v_cmp[u]>
+ *   RoPE:       dq = R(c)^T dq_rot, dk_loc = R(c)^T dk_rot (Key design 1).
+ * The forward saves per (token, q head) row the log-sum-exp of both softmaxes
+ * and the deltas <do, o> (the query x summary epilogue forms them together
+ * with dgate); the backward recomputes P from them.  Float accumulation
+ * throughout; the compressed summary-side gradients are summed with float
+ * atomics, so their last bits may vary from run to run. */
+
+/* Bytes of device workspace pack3d_forward_backward needs: the pack3d_forward
+ * workspace, then row statistics float [N,Hq,4], the float query gradient of
+ * the compressed branch [N,Hq,d_h] and float dk_sum, dv_sum [M,Hkv,d_h]
+ * (0 on an invalid config). */
+size_t pack3d_train_workspace_bytes(const pack3d_config *cfg);
+
+/* Forward pass and all input gradients.  Inputs as for pack3d_forward plus
+ * dout (T [N,Hq,d_h], the gradient of the loss with respect to out).
+ * Outputs (all required, device, 16-byte aligned): out (T [N,Hq,d_h]), dq
+ * (T [N,Hq,d_h]), dk_loc, dv_loc, dk_cmp, dv_cmp (T [N,Hkv,d_h]), dscores
+ * (float [N,Hkv]) and dgate (float [N,Hq,2]), in packed order.  workspace: at
+ * least pack3d_train_workspace_bytes(cfg) bytes, 256-byte aligned.  The
+ * summary-centre variant has no backward here: PACK3D_FLAG_SUMMARY_CENTER
+ * -> PACK3D_ERR_INVALID_ARG. */
+pack3d_status pack3d_forward_backward(const pack3d_config *cfg, const int32_t *coords, const void *q,
+                                      const void *k_loc, const void *v_loc, const void *k_cmp,
+                                      const void *v_cmp, const float *scores, const float *gate,
+                                      const void *dout, void *out, void *dq, void *dk_loc,
+                                      void *dv_loc, void *dk_cmp, void *dv_cmp, float *dscores,
+                                      float *dgate, void *workspace, size_t workspace_bytes,
+                                      int32_t *err_word, void *stream);
 
 /* Synchronises `stream`, reads the device error word, resets it to 0 and maps
  * it: COORD_RANGE/DUPLICATE -> PACK3D_ERR_NOT_PERMUTATION, TIMEOUT ->

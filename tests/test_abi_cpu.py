@@ -102,3 +102,27 @@ def test_binding_refuses_host_tensors(p3):
     x = torch.zeros(256, 2, 64)
     with pytest.raises(ValueError):
         p3.rope(c, torch.zeros(256, 3, dtype=torch.int32), x, x, 2, stream=0)
+
+
+def test_forward_backward_host_errors(p3):
+    c = p3.make_config(16, 64, 64)
+    lib = p3.lib
+    fake = 1 << 20          # never dereferenced: every call below fails before any launch
+    cfgp = ctypes.byref(c)
+    tws = p3.train_workspace_bytes(c)
+    s = synth.CONFIGS["65k"]
+    # forward workspace + stats [N,Hq,4] + float dQ_rot [N,Hq,64] + float dk~, dv~ [M,Hkv,64]
+    need = p3.workspace_bytes(c) + s.N * s.Hq * 16 + s.N * s.Hq * 64 * 4 + 2 * s.M * s.Hkv * 64 * 4
+    assert need <= tws <= need + 4 * 1024
+    args = [fake] * 17       # coords .. dgate
+    assert lib.pack3d_forward_backward(cfgp, *args, fake, tws - 1, fake, None) == 6
+    assert lib.pack3d_forward_backward(cfgp, *args, fake + 16, tws, fake, None) == 6
+    assert lib.pack3d_forward_backward(cfgp, *args, fake, tws, None, None) == 1
+    nulls = list(args)
+    nulls[8] = None          # dout
+    assert lib.pack3d_forward_backward(cfgp, *nulls, fake, tws, fake, None) == 1
+    bad = list(args)
+    bad[11] = fake + 8       # dk_loc misaligned
+    assert lib.pack3d_forward_backward(cfgp, *bad, fake, tws, fake, None) == 3
+    c.flags = p3.FLAG_SUMMARY_CENTER
+    assert lib.pack3d_forward_backward(cfgp, *args, fake, tws, fake, None) == 1
