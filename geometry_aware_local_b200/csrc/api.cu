@@ -101,6 +101,9 @@ struct TrainWs {
   float* dks;     // [M,Hkv,64], followed directly by dvs
   float* dvs;
   size_t dkv_bytes;
+  float* dkl;     // [N,Hkv,64] local-branch key gradient accumulators, followed directly by dvl
+  float* dvl;
+  size_t dkvl_bytes;
   size_t bytes;
 };
 
@@ -116,6 +119,10 @@ TrainWs carve_train(const pack3d_config& c, uintptr_t base) {
   t.dks = reinterpret_cast<float*>(base + off);
   t.dvs = reinterpret_cast<float*>(base + off + t.dkv_bytes);
   off = round_up(off + 2 * t.dkv_bytes, A);
+  t.dkvl_bytes = N * c.Hkv * c.d_h * 4;
+  t.dkl = reinterpret_cast<float*>(base + off);
+  t.dvl = reinterpret_cast<float*>(base + off + t.dkvl_bytes);
+  off = round_up(off + 2 * t.dkvl_bytes, A);
   t.bytes = off;
   return t;
 }
@@ -322,13 +329,29 @@ pack3d_status pack3d_forward_backward(const pack3d_config* cfg, const int32_t* c
   }
   // Backward: compressed branch, local branch, summaries (RoPE transposes fused).
   if (e == cudaSuccess) e = cudaMemsetAsync(t.dks, 0, 2 * t.dkv_bytes, cs);
-  if (e == cudaSuccess) e = launch_summary_bwd_dq(s, dt, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dqr, cs);
-  if (e == cudaSuccess)
-    e = launch_summary_bwd_dkv(s, dt, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dks, t.dvs, cs);
-  if (e == cudaSuccess)
-    e = launch_local_bwd_dq(s, dt, w.g2p, w.q_rot, w.k_rot, v_loc, dout, gate, t.stats, t.dqr, dq, cs);
-  if (e == cudaSuccess)
-    e = launch_local_bwd_dkv(s, dt, w.g2p, w.q_rot, w.k_rot, v_loc, dout, gate, t.stats, dk_loc, dv_loc, cs);
+  if (dt == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY)) {
+    if (e == cudaSuccess)
+      e = launch_summary_bwd_dq_tc(s, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dqr, err_word, cs);
+    if (e == cudaSuccess)
+      e = launch_summary_bwd_dkv_tc(s, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dks, t.dvs, err_word, cs);
+  } else {
+    if (e == cudaSuccess)
+      e = launch_summary_bwd_dq(s, dt, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dqr, cs);
+    if (e == cudaSuccess)
+      e = launch_summary_bwd_dkv(s, dt, w.q_rot, w.k_sum, w.v_sum, dout, gate, t.stats, t.dks, t.dvs, cs);
+  }
+  if (!(cfg->flags & PACK3D_FLAG_SIMT_LOCAL) && local_attn_tc_supported(s, dt)) {
+    if (e == cudaSuccess) e = cudaMemsetAsync(t.dkl, 0, 2 * t.dkvl_bytes, cs);
+    if (e == cudaSuccess)
+      e = launch_local_bwd_tc(s, w.g2p, w.q_rot, w.k_rot, v_loc, dout, gate, t.stats, t.dqr, t.dkl, t.dvl,
+                              err_word, cs);
+    if (e == cudaSuccess) e = launch_local_bwd_finalize(s, dt, coords, t.dqr, t.dkl, t.dvl, dq, dk_loc, dv_loc, cs);
+  } else {
+    if (e == cudaSuccess)
+      e = launch_local_bwd_dq(s, dt, w.g2p, w.q_rot, w.k_rot, v_loc, dout, gate, t.stats, t.dqr, dq, cs);
+    if (e == cudaSuccess)
+      e = launch_local_bwd_dkv(s, dt, w.g2p, w.q_rot, w.k_rot, v_loc, dout, gate, t.stats, dk_loc, dv_loc, cs);
+  }
   if (e == cudaSuccess)
     e = launch_summaries_bwd(s, dt, coords, w.members, k_cmp, v_cmp, scores, t.dks, t.dvs, dk_cmp, dv_cmp,
                              dscores, cs);

@@ -75,6 +75,13 @@ cudaError_t launch_summary_bwd_dq(const Shape& s, int dtype, const void* qr, con
 cudaError_t launch_summary_bwd_dkv(const Shape& s, int dtype, const void* qr, const void* ks, const void* vs,
                                    const void* dout, const float* gate, const float* stats, float* dks,
                                    float* dvs, cudaStream_t st);
+// The same two steps on tcgen05 tensor cores (bf16, k_summary_bwd_tc.cu).
+cudaError_t launch_summary_bwd_dq_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
+                                     const void* dout, const float* gate, const float* stats, float* dqr,
+                                     int32_t* err, cudaStream_t st);
+cudaError_t launch_summary_bwd_dkv_tc(const Shape& s, const void* qr, const void* ks, const void* vs,
+                                      const void* dout, const float* gate, const float* stats, float* dks,
+                                      float* dvs, int32_t* err, cudaStream_t st);
 // Local branch, query side, plus the compressed part from dqr and the RoPE
 // backward: dq = R(c)^T (scale * sum_j dS_j k_j + dqr).
 cudaError_t launch_local_bwd_dq(const Shape& s, int dtype, const int32_t* g2p, const void* qr, const void* kr,
@@ -84,6 +91,17 @@ cudaError_t launch_local_bwd_dq(const Shape& s, int dtype, const int32_t* g2p, c
 cudaError_t launch_local_bwd_dkv(const Shape& s, int dtype, const int32_t* g2p, const void* qr, const void* kr,
                                  const void* vl, const void* dout, const float* gate, const float* stats,
                                  void* dk, void* dv, cudaStream_t st);
+// Local branch on tcgen05 tensor cores (k_local_bwd_tc.cu; shapes of
+// local_attn_tc_supported): dqr += scale * dQ_loc, and the rotated-frame key
+// gradients added to the float accumulators dk_acc, dv_acc [N,Hkv,64]
+// (zeroed first); then the finalize kernel: dq = R(c)^T dqr,
+// dk_loc = R(c)^T dk_acc, dv_loc = dv_acc in the operator's dtype.
+cudaError_t launch_local_bwd_tc(const Shape& s, const int32_t* g2p, const void* qr, const void* kr, const void* vl,
+                                const void* dout, const float* gate, const float* stats, float* dqr, float* dk_acc,
+                                float* dv_acc, int32_t* err, cudaStream_t st);
+cudaError_t launch_local_bwd_finalize(const Shape& s, int dtype, const int32_t* coords, const float* dqr,
+                                      const float* dka, const float* dva, void* dq, void* dk, void* dv,
+                                      cudaStream_t st);
 // Summaries backward: dk_cmp, dv_cmp, dscores from dks, dvs.
 cudaError_t launch_summaries_bwd(const Shape& s, int dtype, const int32_t* coords, const int32_t* members,
                                  const void* kc, const void* vc, const float* scores, const float* dks,

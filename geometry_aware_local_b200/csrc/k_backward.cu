@@ -430,6 +430,41 @@ __global__ void __launch_bounds__(kSbThreads) summaries_bwd_kernel(
   }
 }
 
+// ---- finalize of the tensor-core local backward ----------------------------
+
+// dq = R(c)^T dqr, dk_loc = R(c)^T dk_acc, dv_loc = dv_acc (float accumulators
+// to the operator's dtype); blockIdx.y picks the tensor, thread = 16 dims of a row.
+template <typename T>
+__global__ void __launch_bounds__(256) local_bwd_finalize_kernel(
+    Shape s, const int32_t* __restrict__ coords, const float* __restrict__ dqr, const float* __restrict__ dka,
+    const float* __restrict__ dva, T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv) {
+  extern __shared__ float2 tab[];
+  build_rope_table(tab, s);
+  __syncthreads();
+  const int which = blockIdx.y;
+  const int heads = which == 0 ? s.Hq : s.Hkv;
+  const float* src = which == 0 ? dqr : (which == 1 ? dka : dva);
+  T* dst = which == 0 ? dq : (which == 1 ? dk : dv);
+  const long n = (long)s.N * heads * 4;
+  for (long t = (long)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += (long)gridDim.x * blockDim.x) {
+    const long row = t >> 2;
+    const int qd = (int)(t & 3);
+    float f[16];
+    const float4* s4 = reinterpret_cast<const float4*>(src + row * kDh + qd * 16);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float4 v = __ldg(s4 + c);
+      f[4 * c] = v.x; f[4 * c + 1] = v.y; f[4 * c + 2] = v.z; f[4 * c + 3] = v.w;
+    }
+    if (which < 2) {
+      const long tok = row / heads;
+      rope_planes(f, s, tab, qd * 8, 8, __ldg(coords + 3 * tok), __ldg(coords + 3 * tok + 1),
+                  __ldg(coords + 3 * tok + 2), true);
+    }
+    store_f32(dst + row * kDh + qd * 16, f, 16);
+  }
+}
+
 // ---- launchers --------------------------------------------------------------
 
 template <typename T>
@@ -537,6 +572,25 @@ cudaError_t launch_local_bwd_dkv(const Shape& s, int dtype, const int32_t* g2p, 
                                  void* dk, void* dv, cudaStream_t st) {
   if (dtype == PACK3D_BF16) return local_dkv_t<__nv_bfloat16>(s, g2p, qr, kr, vl, dout, gate, stats, dk, dv, st);
   return local_dkv_t<float>(s, g2p, qr, kr, vl, dout, gate, stats, dk, dv, st);
+}
+
+cudaError_t launch_local_bwd_finalize(const Shape& s, int dtype, const int32_t* coords, const float* dqr,
+                                      const float* dka, const float* dva, void* dq, void* dk, void* dv,
+                                      cudaStream_t st) {
+  const size_t smem = (size_t)s.tab_entries * sizeof(float2);
+  dim3 grid(148 * 8, 3);
+  if (dtype == PACK3D_BF16) {
+    cudaError_t e = set_table_smem((const void*)local_bwd_finalize_kernel<__nv_bfloat16>, smem);
+    if (e != cudaSuccess) return e;
+    local_bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(
+        s, coords, dqr, dka, dva, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv);
+  } else {
+    cudaError_t e = set_table_smem((const void*)local_bwd_finalize_kernel<float>, smem);
+    if (e != cudaSuccess) return e;
+    local_bwd_finalize_kernel<float><<<grid, 256, smem, st>>>(s, coords, dqr, dka, dva, (float*)dq, (float*)dk,
+                                                              (float*)dv);
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_summaries_bwd(const Shape& s, int dtype, const int32_t* coords, const int32_t* members,

@@ -247,6 +247,22 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// The same with A's major-ness as well (bit 15, 1 = MN major): for A read
+// from shared memory with the M dimension contiguous.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// Byte offset of element (r, e) (e < 64 bf16) in a 128-byte-swizzled tile of
+// 128-byte rows: the 16-byte chunk e / 8 of row r sits at chunk (e / 8) ^ (r % 8).
+__host__ __device__ constexpr uint32_t sw128_offset(uint32_t r, uint32_t e) {
+  return r * 128u + ((((e >> 3) ^ (r & 7u)) << 4) | ((e & 7u) << 1));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -291,13 +291,14 @@ pack3d_status pack3d_forward_host(pack3d_pipeline *pipeline, const pack3d_config
  * The forward saves per (token, q head) row the log-sum-exp of both softmaxes
  * and the deltas <do, o> (the query x summary epilogue forms them together
  * with dgate); the backward recomputes P from them.  Float accumulation
- * throughout; the compressed summary-side gradients are summed with float
- * atomics, so their last bits may vary from run to run. */
+ * throughout; the summary-side gradients of the compressed branch (and, on
+ * the tensor-core local path, the local key and value gradients) are summed
+ * with float atomics, so their last bits may vary from run to run. */
 
 /* Bytes of device workspace pack3d_forward_backward needs: the pack3d_forward
- * workspace, then row statistics float [N,Hq,4], the float query gradient of
- * the compressed branch [N,Hq,d_h] and float dk_sum, dv_sum [M,Hkv,d_h]
- * (0 on an invalid config). */
+ * workspace, then row statistics float [N,Hq,4], the float query gradient
+ * [N,Hq,d_h], float dk_sum, dv_sum [M,Hkv,d_h] and float local key / value
+ * gradient accumulators [N,Hkv,d_h] (0 on an invalid config). */
 size_t pack3d_train_workspace_bytes(const pack3d_config *cfg);
 
 /* Forward pass and all input gradients.  Inputs as for pack3d_forward plus

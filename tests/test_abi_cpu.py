@@ -112,7 +112,9 @@ def test_forward_backward_host_errors(p3):
     tws = p3.train_workspace_bytes(c)
     s = synth.CONFIGS["65k"]
     # forward workspace + stats [N,Hq,4] + float dQ_rot [N,Hq,64] + float dk~, dv~ [M,Hkv,64]
-    need = p3.workspace_bytes(c) + s.N * s.Hq * 16 + s.N * s.Hq * 64 * 4 + 2 * s.M * s.Hkv * 64 * 4
+    # + float local dK, dV accumulators [N,Hkv,64]
+    need = (p3.workspace_bytes(c) + s.N * s.Hq * 16 + s.N * s.Hq * 64 * 4 + 2 * s.M * s.Hkv * 64 * 4
+            + 2 * s.N * s.Hkv * 64 * 4)
     assert need <= tws <= need + 4 * 1024
     args = [fake] * 17       # coords .. dgate
     assert lib.pack3d_forward_backward(cfgp, *args, fake, tws - 1, fake, None) == 6

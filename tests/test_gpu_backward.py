@@ -110,16 +110,19 @@ def test_gate_pinned_local_gives_zero_compressed_gradients(p3):
 
 
 def test_backward_is_deterministic_where_no_atomics(p3):
-    """dq, dk_loc, dv_loc, dgate and out are written without atomics: identical across calls."""
+    """dq, dgate and out are written without atomics: identical across calls.  The key-side
+    gradients are summed with float atomics and may differ in their last bits."""
     s = small(Z=4, H=32, W=40)
     inp = synth.make_inputs(s, "random", seed=8)
     dout = synth.make_dout(s, "random", seed=8)
     a = run_fwd_bwd(p3, s, inp, dout)
     b = run_fwd_bwd(p3, s, inp, dout)
-    for k in ("dq", "dk_loc", "dv_loc", "dgate", "out"):
+    for k in ("dq", "dgate", "out"):
         assert torch.equal(a[k], b[k]), k
-    for k in ("dk_cmp", "dv_cmp", "dscores"):
-        assert rel_err(a[k].double().numpy(), b[k].double().numpy()) <= 1e-3, k
+    # a different float summation order can move a bf16 result by one unit in the last place,
+    # at most 2^-7 of its magnitude
+    for k in ("dk_loc", "dv_loc", "dk_cmp", "dv_cmp", "dscores"):
+        assert rel_err(a[k].double().numpy(), b[k].double().numpy()) <= 2.0 ** -7, k
 
 
 def test_gradients_permute_with_the_packing(p3):
