@@ -21,7 +21,8 @@
 // summary_bwd_dkv_tc_kernel (summary side): one 128-summary tile per CTA and a
 //   range of the kv group's query rows, 128 rows per step, one CTA per SM.
 //   Per step S = Q k~^T and dP = dout v~^T (M=128 rows, N=128 summaries) go to
-//   tensor memory; the softmax warps write dS and gamma1 P as bf16 into one of
+//   tensor memory; two softmax warpgroups (one per 64-summary half) write dS
+//   and gamma1 P as bf16 into one of
 //   two shared-memory buffers (alternate steps) in the 128-byte-swizzled
 //   MN-major layout, and the MMA warp
 //   accumulates dk~ += dS^T Q and dv~ += (gamma1 P)^T dout (M=128 summaries,
@@ -284,8 +285,12 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 namespace k_side {
 
 constexpr int kBS = 128;                        // summaries per CTA (M of the dk~ / dv~ accumulators)
-constexpr int kThreads = 192;                   // 4 softmax warps, MMA warp, TMA warp
-constexpr int kMmaWarp = 4, kTmaWarp = 5;
+// Two softmax warpgroups (warps 0-3: summaries 0-63 of the tile, warps 4-7:
+// 64-127; a warp reads the tensor-memory lanes of its warp index mod 4), then
+// the MMA warp and the TMA warp.
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+constexpr int kMmaWarp = kSoftmaxWarps, kTmaWarp = kSoftmaxWarps + 1;
 constexpr int kColS = 0, kColDP = 128, kColDK = 256, kColDV = 320, kTmemCols = 512;
 constexpr int kSumTileBytes = kBS * kDh * 2;    // 16 KiB
 constexpr int kStages = 2;
@@ -336,10 +341,10 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     }
     ptx::mbar_init(kvfull, 1);
     ptx::mbar_init(s_full, 1);
-    ptx::mbar_init(s_free, 4);
+    ptx::mbar_init(s_free, kSoftmaxWarps);
     ptx::mbar_init(o_final, 1);
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(p_full(b), 4);
+      ptx::mbar_init(p_full(b), kSoftmaxWarps);
       ptx::mbar_init(p_free(b), 1);
     }
     *abort_flag = 0;
@@ -438,7 +443,8 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     __syncwarp();
   } else {
     // ---------------- softmax warps: thread = query row of the step ----------------
-    const int lane_base = warp * 32;
+    const int wg = warp >> 2;                    // summary half of the tile this warpgroup covers
+    const int lane_base = (warp & 3) * 32;
     const int rl = lane_base + lane;             // row inside the step's tile
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
     const float2 c2 = make_float2(a.scale_log2, a.scale_log2);
@@ -454,11 +460,11 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       const float2 nl2 = make_float2(-lse2, -lse2), w2 = make_float2(w1, w1), nd2 = make_float2(-delta, -delta);
       if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, t & 1, abort_flag)))) break;
       ptx::tc_fence_after();
-      for (int c = 0; c < kBS / 32; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * wg + cc;               // 32-summary chunk of the tile
         uint32_t sv[32], dv[32];
-        ptx::tmem_ld32_sync(trow + kColS + 32 * c, sv);
-        ptx::tmem_ld32_sync(trow + kColDP + 32 * c, dv);
-        if (c == kBS / 32 - 1) warp_arrive(s_free);
+        ptx::tmem_ld32x2_sync(trow + kColS + 32 * c, trow + kColDP + 32 * c, sv, dv);
+        if (cc == 1) warp_arrive(s_free);
         uint32_t pd[16], pp[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -472,16 +478,16 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         }
         // Step t-2's dk~ / dv~ MMAs read this buffer: wait for them only now,
         // so this step's first exponentials overlap them.
-        if (c == 0 && t >= 2) {
+        if (cc == 0 && t >= 2) {
           if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(t & 1), ((t >> 1) - 1) & 1, abort_flag))))
             break;
         }
         // Row rl of the MN-major operands: summaries 32c .. 32c+31 are 16-byte
-        // chunks (c & 1) * 4 + m of half c / 2.
-        const uint32_t op = sbase + kOpOff + (t & 1) * kOpBytes + (uint32_t)(c >> 1) * kQTileBytes;
+        // chunks (c & 1) * 4 + m of half c / 2 (= wg).
+        const uint32_t op = sbase + kOpOff + (t & 1) * kOpBytes + (uint32_t)wg * kQTileBytes;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const uint32_t off = ptx::sw128_offset((uint32_t)rl, (uint32_t)(((c & 1) * 4 + m) * 8));
+          const uint32_t off = ptx::sw128_offset((uint32_t)rl, (uint32_t)((cc * 4 + m) * 8));
           ptx::st_shared_v4(op + off, pd[4 * m], pd[4 * m + 1], pd[4 * m + 2], pd[4 * m + 3]);
           ptx::st_shared_v4(op + kPInOp + off, pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
         }
@@ -492,22 +498,17 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     }
     if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final, 0, abort_flag))) {
       ptx::tc_fence_after();
-      // Accumulator lane = summary of this tile.
+      // Accumulator lane = summary of this tile; warpgroup 0 adds dk~, warpgroup 1 dv~.
       const int j = stile * kBS + rl;
-      uint32_t rk[kDh], rv[kDh];
-      ptx::tmem_ld64_sync(tmem + ((uint32_t)lane_base << 16) + kColDK, rk);
-      ptx::tmem_ld64_sync(tmem + ((uint32_t)lane_base << 16) + kColDV, rv);
+      uint32_t r[kDh];
+      ptx::tmem_ld64_sync(trow + (wg == 0 ? kColDK : kColDV), r);
       if (j < a.M) {
-        float4* dk = reinterpret_cast<float4*>(a.dks + ((size_t)j * gridDim.y + g) * kDh);
-        float4* dv = reinterpret_cast<float4*>(a.dvs + ((size_t)j * gridDim.y + g) * kDh);
+        const float f = wg == 0 ? a.scale : 1.f;
+        float4* dst = reinterpret_cast<float4*>((wg == 0 ? a.dks : a.dvs) + ((size_t)j * gridDim.y + g) * kDh);
 #pragma unroll
-        for (int q = 0; q < kDh / 4; ++q) {
-          atomicAdd(dk + q, make_float4(a.scale * __uint_as_float(rk[4 * q]), a.scale * __uint_as_float(rk[4 * q + 1]),
-                                        a.scale * __uint_as_float(rk[4 * q + 2]),
-                                        a.scale * __uint_as_float(rk[4 * q + 3])));
-          atomicAdd(dv + q, make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
-                                        __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3])));
-        }
+        for (int q = 0; q < kDh / 4; ++q)
+          atomicAdd(dst + q, make_float4(f * __uint_as_float(r[4 * q]), f * __uint_as_float(r[4 * q + 1]),
+                                         f * __uint_as_float(r[4 * q + 2]), f * __uint_as_float(r[4 * q + 3])));
       }
     }
   }

@@ -210,6 +210,25 @@ __device__ __forceinline__ void tmem_ld48_sync(uint32_t taddr, uint32_t* r) {
       : "r"(taddr)
       : "memory");
 }
+// Two 32-column loads from different column ranges (taddr0, taddr1) in
+// flight, then one wait: r0 <- taddr0 .. +31, r1 <- taddr1 .. +31.
+__device__ __forceinline__ void tmem_ld32x2_sync(uint32_t taddr0, uint32_t taddr1, uint32_t* r0, uint32_t* r1) {
+  uint32_t* r = r0;
+  uint32_t* s = r1;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : P3_R16(0), P3_R16(16), "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]),
+        "=r"(s[6]), "=r"(s[7]), "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]), "=r"(s[12]), "=r"(s[13]),
+        "=r"(s[14]), "=r"(s[15]), "=r"(s[16]), "=r"(s[17]), "=r"(s[18]), "=r"(s[19]), "=r"(s[20]), "=r"(s[21]),
+        "=r"(s[22]), "=r"(s[23]), "=r"(s[24]), "=r"(s[25]), "=r"(s[26]), "=r"(s[27]), "=r"(s[28]), "=r"(s[29]),
+        "=r"(s[30]), "=r"(s[31])
+      : "r"(taddr0), "r"(taddr1)
+      : "memory");
+}
 #undef P3_R16
 #undef P3_R8
 #undef P3_W8
