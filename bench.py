@@ -17,6 +17,11 @@ Under torchrun (N > 1) every rank runs an independent replica of the volume
 (the operator is single-GPU; ranks exchange nothing on the data path), the
 time is the max over ranks and ``value`` counts every rank's tokens.
 
+``train`` times the training block, pack3d_forward_backward (the forward
+pass saving its softmax statistics, then the gradients of <dOut, out> with
+respect to every input), on the same volume with dOut drawn N(0,1) per site;
+tokens/s there count one forward and one backward per token.
+
 ``--impl reference`` times the float64 CPU oracle on the host cores on a
 bounded sample of the same workload (rank 0 only).
 """
@@ -47,6 +52,7 @@ WORKLOAD_TEXT = {
     "1m": "64x128x128 lattice (1,048,576 tokens), random packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=65,536), window 3x7x7",
     "4m": "64x256x256 lattice (4,194,304 tokens), Morton packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=262,144), window 3x7x7; values drawn on the device",
     "8m": "128x256x256 lattice (8,388,608 tokens), Morton packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=524,288), window 3x7x7; values drawn on the device",
+    "stress": "16x64x64 lattice (65,536 tokens), raster packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=4,096), window 3x7x7 (the repacking stress case)",
     "allen": "32x128x64 lattice (262,144 tokens; the shape of the Allen WTC-11 token grid, synthetic values), block-contiguous packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=16,384), window 3x7x7",
 }
 STAGES = ("index", "rope", "summaries", "local", "summary_attn")
@@ -319,6 +325,38 @@ def dense_sdpa_ms(s, q_rot, k_rot, v, stream, reps: int = 2) -> Dict:
             "what": "torch scaled_dot_product_attention (flash backend), bf16, all N x N pairs, kv heads repeated"}
 
 
+def time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world, rank, dev) -> Dict:
+    """pack3d_forward_backward on the resident inputs: W untimed calls, then K
+    timed ones with CUDA events on the launching stream, L2 flushed between
+    calls outside the events; the max over ranks."""
+    import torch
+    if args.config in synth.DEVICE_DRAWN:
+        gen = torch.Generator(device=dev).manual_seed(rank + 2)
+        dout = torch.randn(d["q"].shape, generator=gen, device=dev, dtype=torch.float32).to(d["q"].dtype)
+    else:
+        dout = synth.make_dout(s, s.packing, seed=rank).to(dev)
+    out = torch.empty_like(d["q"])
+    grads = p3.empty_grads(d["q"], d["k_loc"], d["scores"], d["gate"])
+    tws = torch.empty(p3.train_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    evs = []
+    for k in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        p3.forward_backward(cfg, d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
+                            d["gate"], dout, out, grads, tws, err)
+        e1.record(stream)
+        if k >= args.warmup:
+            evs.append((e0, e1))
+    torch.cuda.synchronize()
+    if p3.check_status(err) != 0:
+        raise RuntimeError("device error during the training-block steps")
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
+    return {"ms_per_step": ms, "tokens_per_s": replica_value(s.N, world, ms),
+            "call": "pack3d_forward_backward (forward saving statistics + every input gradient)",
+            "dout": "N(0,1) per lattice site", "l2": "flushed between calls (outside the timed events)"}
+
+
 def run_ours(args, s):
     import torch
 
@@ -439,6 +477,10 @@ def run_ours(args, s):
     if p3.check_status(err) != 0:
         raise RuntimeError("device error during the e2e steps")
 
+    train = None
+    if not args.summary_center and (args.config not in synth.DEVICE_DRAWN or args.train):
+        train = time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world, rank, dev)
+
     peaks = load_peaks()
     work = algorithmic_work(s)
     stages = {}
@@ -482,6 +524,8 @@ def run_ours(args, s):
             "clocks": clk.summary()}
     if variant_err is not None:
         line["summary_center_vs_exact"] = variant_err
+    if train is not None:
+        line["train"] = train
     # Comparators named by the workloads: a same-window local-only pass at 65k
     # (index map, RoPE and local attention, the stages that pass runs) and a
     # dense-attention run of the same shape at 1M.
@@ -516,6 +560,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparator at 1M")
+    ap.add_argument("--train", action="store_true",
+                    help="also time the training block on the device-drawn 4m / 8m volumes")
     ap.add_argument("--summary-center", action="store_true",
                     help="time the summary-centre variant of the block summaries and report its error "
                          "against the exact rotate-before-compress form")
