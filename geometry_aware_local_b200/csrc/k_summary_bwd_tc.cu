@@ -288,9 +288,12 @@ constexpr int kBS = 128;                        // summaries per CTA (M of the d
 // Two softmax warpgroups (warps 0-3: summaries 0-63 of the tile, warps 4-7:
 // 64-127; a warp reads the tensor-memory lanes of its warp index mod 4), then
 // the MMA warp and the TMA warp.
+// Two MMA warps: the first issues each step's S and dP, the second its
+// dk~ / dv~ accumulation, so that S and dP of the next step never queue
+// behind the slower accumulation issue.
 constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
-constexpr int kMmaWarp = kSoftmaxWarps, kTmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
+constexpr int kMmaWarp = kSoftmaxWarps, kMmaWarp2 = kSoftmaxWarps + 1, kTmaWarp = kSoftmaxWarps + 2;
 constexpr int kColS = 0, kColDP = 128, kColDK = 256, kColDV = 320, kTmemCols = 512;
 constexpr int kSumTileBytes = kBS * kDh * 2;    // 16 KiB
 constexpr int kStages = 2;
@@ -386,7 +389,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
     if (lane == 0) {
       const uint32_t tS = tmem + kColS, tDP = tmem + kColDP, tDK = tmem + kColDK, tDV = tmem + kColDV;
       auto issue_sdp = [&](int t) {
@@ -418,26 +421,34 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         ptx::tc_commit(empty(t % kStages));
         if (t == nsteps - 1) ptx::tc_commit(o_final);
       };
-      bool ok = ptx::mbar_wait(kvfull, 0, abort_flag) && ptx::mbar_wait(full(0), 0, abort_flag);
-      if (ok) {
-        ptx::tc_fence_after();
-        issue_sdp(0);
-      }
-      for (int t = 0; ok && t < nsteps; ++t) {
-        if (t + 1 < nsteps) {
-          if (!(ok = ptx::mbar_wait(s_free, t & 1, abort_flag) &&
-                     ptx::mbar_wait(full((t + 1) % kStages), ((t + 1) / kStages) & 1, abort_flag)))
-            break;
+      bool ok = true;
+      if (warp == kMmaWarp) {
+        ok = ptx::mbar_wait(kvfull, 0, abort_flag);
+        int issued = 0;
+        for (int t = 0; ok && t < nsteps; ++t) {
+          // S and dP of step t: stage t landed, and step t-1's softmax read S and dP.
+          if (!(ok = ptx::mbar_wait(full(t % kStages), (t / kStages) & 1, abort_flag))) break;
+          if (t > 0 && !(ok = ptx::mbar_wait(s_free, (t - 1) & 1, abort_flag))) break;
           ptx::tc_fence_after();
-          issue_sdp(t + 1);
+          issue_sdp(t);
+          issued = t + 1;
         }
-        if (!(ok = ptx::mbar_wait(p_full(t & 1), (t >> 1) & 1, abort_flag))) break;
-        ptx::tc_fence_after();
-        issue_dkv(t);
-      }
-      if (!ok) {
-        ptx::tc_commit(o_final);
-        ptx::mbar_wait(o_final, 0, abort_flag);
+        if (!ok) {
+          // Drain this warp's MMAs before tensor memory is released (the
+          // commit tracks every earlier MMA of this thread).
+          ptx::tc_commit(s_full);
+          ptx::mbar_wait(s_full, issued & 1, abort_flag);
+        }
+      } else {
+        for (int t = 0; ok && t < nsteps; ++t) {
+          if (!(ok = ptx::mbar_wait(p_full(t & 1), (t >> 1) & 1, abort_flag))) break;
+          ptx::tc_fence_after();
+          issue_dkv(t);
+        }
+        if (!ok) {
+          ptx::tc_commit(o_final);
+          ptx::mbar_wait(o_final, 0, abort_flag);
+        }
       }
     }
     __syncwarp();
