@@ -1,7 +1,7 @@
 """Benchmark of the PACK3D forward pass on B200: tokens/s, per-stage roofline.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 65k|262k|1m|tiny]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 65k|262k|1m|stress|...]
+                    [--impl ours|reference] [--train-only]
 
 One step = one pass of the whole hot path over one synthetic volume: index
 map, axial RoPE on Q and K_loc, block summaries, local attention, query x
@@ -325,12 +325,13 @@ def dense_sdpa_ms(s, q_rot, k_rot, v, stream, reps: int = 2) -> Dict:
             "what": "torch scaled_dot_product_attention (flash backend), bf16, all N x N pairs, kv heads repeated"}
 
 
-def time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world, rank, dev) -> Dict:
+def time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world, rank, dev,
+                        device_dout: bool = False) -> Dict:
     """pack3d_forward_backward on the resident inputs: W untimed calls, then K
     timed ones with CUDA events on the launching stream, L2 flushed between
     calls outside the events; the max over ranks."""
     import torch
-    if args.config in synth.DEVICE_DRAWN:
+    if device_dout or args.config in synth.DEVICE_DRAWN:
         gen = torch.Generator(device=dev).manual_seed(rank + 2)
         dout = torch.randn(d["q"].shape, generator=gen, device=dev, dtype=torch.float32).to(d["q"].dtype)
     else:
@@ -355,6 +356,37 @@ def time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world
     return {"ms_per_step": ms, "tokens_per_s": replica_value(s.N, world, ms),
             "call": "pack3d_forward_backward (forward saving statistics + every input gradient)",
             "dout": "N(0,1) per lattice site", "l2": "flushed between calls (outside the timed events)"}
+
+
+def run_train_only(args, s):
+    """--train-only: the training block alone (no forward legs), one JSON line."""
+    import torch
+
+    import geometry_aware_local_b200 as p3
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = p3.config_from_shape(s)
+    d = synth.make_inputs_on_device(s, s.packing, seed=rank, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    err = torch.zeros(4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    barrier(world)
+    with ClockSampler(local) as clk:
+        train = time_training_block(p3, args, s, cfg, d, None, flush, stream, err, world, rank, dev, device_dout=True)
+    if rank == 0:
+        line = {"metric": "PACK3D forward+backward tokens/s (training block), 1 B200", "value": train["tokens_per_s"],
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": train["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": s.dtype, "data": "synthetic (values drawn on the device)",
+                "config": {"workload": WORKLOAD_TEXT[args.config], "tokens": s.N, "summaries": s.M}, "train": train,
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def run_ours(args, s):
@@ -562,6 +594,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparator at 1M")
     ap.add_argument("--train", action="store_true",
                     help="also time the training block on the device-drawn 4m / 8m volumes")
+    ap.add_argument("--train-only", action="store_true",
+                    help="time only the training block (pack3d_forward_backward), inputs drawn on the device")
     ap.add_argument("--summary-center", action="store_true",
                     help="time the summary-centre variant of the block summaries and report its error "
                          "against the exact rotate-before-compress form")
@@ -571,6 +605,8 @@ def main():
     s = synth.CONFIGS[args.config]
     if args.impl == "reference":
         run_reference(args, s)
+    elif args.train_only:
+        run_train_only(args, s)
     else:
         run_ours(args, s)
 
