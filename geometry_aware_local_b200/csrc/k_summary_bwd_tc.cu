@@ -44,6 +44,7 @@ namespace pack3d {
 namespace {
 
 constexpr int kRowsPerTile = 128;
+constexpr long kSmCount = 148;                        // B200
 constexpr int kQTileBytes = kRowsPerTile * kDh * 2;   // 16 KiB: 128 rows x 64 bf16
 
 struct BwdArgs {
@@ -296,19 +297,27 @@ constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
 constexpr int kMmaWarp = kSoftmaxWarps, kMmaWarp2 = kSoftmaxWarps + 1, kTmaWarp = kSoftmaxWarps + 2;
 constexpr int kColS = 0, kColDP = 128, kColDK = 256, kColDV = 320, kTmemCols = 512;
 constexpr int kSumTileBytes = kBS * kDh * 2;    // 16 KiB
-constexpr int kStages = 2;
+// Operand buffers: buffer b holds dS^T (two 16 KiB halves: summaries 0-63,
+// 64-127) and then (gamma1 P)^T; step t uses buffer t % kOpBufs.  With two
+// buffers a step's softmax writes while the previous step's dk~ / dv~ MMAs
+// still read; with one, shared memory holds two more Q / dout stages (four).
+// Measured on B200, forward+backward: 65k 4.86 ms (two) vs 4.81 ms (one);
+// 262k 56.8 vs 56.6 ms.
+#ifndef PACK3D_BKV_OPBUFS
+#define PACK3D_BKV_OPBUFS 1
+#endif
+constexpr int kOpBufs = PACK3D_BKV_OPBUFS;
+constexpr int kOpBytes = 4 * kQTileBytes;
+constexpr int kPInOp = 2 * kQTileBytes;
 constexpr int kKOff = 0, kVOff = kSumTileBytes;
 constexpr int kStageOff = 2 * kSumTileBytes;
 constexpr int kStageBytes = 2 * kQTileBytes;    // Q at +0, dout at +kQTileBytes
-// Two operand buffers, used by alternate steps, so that a step's softmax
-// writes while the previous step's dk~ / dv~ MMAs still read: buffer b holds
-// dS^T (two 16 KiB halves: summaries 0-63, 64-127) and then (gamma1 P)^T.
+constexpr int kStages = (224 * 1024 - kStageOff - kOpBufs * kOpBytes) / kStageBytes;
 constexpr int kOpOff = kStageOff + kStages * kStageBytes;
-constexpr int kOpBytes = 4 * kQTileBytes;
-constexpr int kPInOp = 2 * kQTileBytes;
-constexpr int kBarOff = kOpOff + 2 * kOpBytes;
-// barriers: full[S], empty[S], kvfull, s_full, s_free, o_final, p_full[2], p_free[2]
-constexpr int kNumBars = 2 * kStages + 8;
+constexpr int kBarOff = kOpOff + kOpBufs * kOpBytes;
+// barriers: full[S], empty[S], kvfull, s_full, s_free, o_final, p_full[kOpBufs], p_free[kOpBufs]
+constexpr int kNumBars = 2 * kStages + 4 + 2 * kOpBufs;
+static_assert(kStages >= 2, "at least two Q / dout stages");
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kRowsPerTile, kBS, false);        // S, dP: N = 128 summaries
@@ -333,7 +342,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
   const uint32_t kvfull = bar0 + 8 * (2 * kStages);
   const uint32_t s_full = kvfull + 8, s_free = kvfull + 16, o_final = kvfull + 24;
   auto p_full = [&](int b) { return kvfull + 32 + 8 * b; };
-  auto p_free = [&](int b) { return kvfull + 48 + 8 * b; };
+  auto p_free = [&](int b) { return kvfull + 32 + 8 * kOpBufs + 8 * b; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -346,7 +355,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(s_free, kSoftmaxWarps);
     ptx::mbar_init(o_final, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kOpBufs; ++b) {
       ptx::mbar_init(p_full(b), kSoftmaxWarps);
       ptx::mbar_init(p_free(b), 1);
     }
@@ -408,7 +417,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       auto issue_dkv = [&](int t) {
         const uint32_t qaddr = sbase + kStageOff + (t % kStages) * kStageBytes;
         const uint32_t oaddr = qaddr + kQTileBytes;
-        const uint32_t op = sbase + kOpOff + (t & 1) * kOpBytes;
+        const uint32_t op = sbase + kOpOff + (t % kOpBufs) * kOpBytes;
 #pragma unroll
         for (int kk = 0; kk < kRowsPerTile / 16; ++kk)
           ptx::mma_ss(tDK, ptx::smem_desc_sw128(op + kk * 2048, 2 * 8192, 1024),
@@ -417,7 +426,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         for (int kk = 0; kk < kRowsPerTile / 16; ++kk)
           ptx::mma_ss(tDV, ptx::smem_desc_sw128(op + kPInOp + kk * 2048, 2 * 8192, 1024),
                       ptx::smem_desc_sw128(oaddr + kk * 2048, 8192, 1024), kIdescKV, (t > 0 || kk > 0) ? 1u : 0u);
-        ptx::tc_commit(p_free(t & 1));
+        ptx::tc_commit(p_free(t % kOpBufs));
         ptx::tc_commit(empty(t % kStages));
         if (t == nsteps - 1) ptx::tc_commit(o_final);
       };
@@ -441,7 +450,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         }
       } else {
         for (int t = 0; ok && t < nsteps; ++t) {
-          if (!(ok = ptx::mbar_wait(p_full(t & 1), (t >> 1) & 1, abort_flag))) break;
+          if (!(ok = ptx::mbar_wait(p_full(t % kOpBufs), (t / kOpBufs) & 1, abort_flag))) break;
           ptx::tc_fence_after();
           issue_dkv(t);
         }
@@ -487,15 +496,16 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
           pd[k] = pack_bf16x2(ds.x, ds.y);
           pp[k] = pack_bf16x2(pw.x, pw.y);
         }
-        // Step t-2's dk~ / dv~ MMAs read this buffer: wait for them only now,
-        // so this step's first exponentials overlap them.
-        if (cc == 0 && t >= 2) {
-          if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(t & 1), ((t >> 1) - 1) & 1, abort_flag))))
+        // Step (t - kOpBufs)'s dk~ / dv~ MMAs read this buffer: wait for them
+        // only now, so this step's first exponentials overlap them.
+        if (cc == 0 && t >= kOpBufs) {
+          if (!(ok = __all_sync(0xffffffffu,
+                                ptx::mbar_wait(p_free(t % kOpBufs), ((t / kOpBufs) - 1) & 1, abort_flag))))
             break;
         }
         // Row rl of the MN-major operands: summaries 32c .. 32c+31 are 16-byte
         // chunks (c & 1) * 4 + m of half c / 2 (= wg).
-        const uint32_t op = sbase + kOpOff + (t & 1) * kOpBytes + (uint32_t)wg * kQTileBytes;
+        const uint32_t op = sbase + kOpOff + (t % kOpBufs) * kOpBytes + (uint32_t)wg * kQTileBytes;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const uint32_t off = ptx::sw128_offset((uint32_t)rl, (uint32_t)((cc * 4 + m) * 8));
@@ -505,7 +515,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       }
       if (!ok) break;
       ptx::fence_proxy_async_smem();
-      warp_arrive(p_full(t & 1));
+      warp_arrive(p_full(t % kOpBufs));
     }
     if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final, 0, abort_flag))) {
       ptx::tc_fence_after();
@@ -603,12 +613,26 @@ cudaError_t launch_summary_bwd_dkv_tc(const Shape& s, const void* qr, const void
   BwdArgs a = make_args(s, gate, stats, err);
   a.dks = dks;
   a.dvs = dvs;
-  // Split the kv group's rows so that the grid covers every SM about four
-  // times; each CTA keeps at least eight 128-row steps.
+  // Split the kv group's rows over grid.z: at least four CTAs per SM over
+  // the grid, each CTA keeping at least eight 128-row steps, and among the
+  // split counts up to twice that, the one whose last wave of CTAs leaves the
+  // fewest SMs idle.
   const int tiles = (s.M + k_side::kBS - 1) / k_side::kBS;
   const long steps = (a.rows + kRowsPerTile - 1) / kRowsPerTile;
-  long splits = (4L * 148 + (long)tiles * s.Hkv - 1) / ((long)tiles * s.Hkv);
-  splits = max(1L, min(splits, steps / 8));
+  const long units = (long)tiles * s.Hkv;
+  const long lo = max(1L, min((4L * kSmCount + units - 1) / units, steps / 8));
+  long splits = lo;
+  double best = 2.0;
+  for (long c = lo; c <= max(lo, min(2 * lo, steps / 8)); ++c) {
+    const long per = (steps + c - 1) / c;
+    const long used = (steps + per - 1) / per;          // splits that get rows
+    const long ctas = units * used;
+    const double idle = (double)((ctas + kSmCount - 1) / kSmCount * kSmCount - ctas) / (double)ctas;
+    if (idle < best - 1e-9) {
+      best = idle;
+      splits = c;
+    }
+  }
   const long per_steps = (steps + splits - 1) / splits;
   a.rows_per_split = per_steps * kRowsPerTile;
   splits = (a.rows + a.rows_per_split - 1) / a.rows_per_split;
