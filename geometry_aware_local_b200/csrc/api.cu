@@ -299,7 +299,6 @@ pack3d_status pack3d_forward_backward(const pack3d_config* cfg, const int32_t* c
                                       int32_t* err_word, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
-  if (cfg->flags & PACK3D_FLAG_SUMMARY_CENTER) return PACK3D_ERR_INVALID_ARG;
   if (!coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !dout || !out || !dq ||
       !dk_loc || !dv_loc || !dk_cmp || !dv_cmp || !dscores || !dgate || !err_word)
     return PACK3D_ERR_INVALID_ARG;

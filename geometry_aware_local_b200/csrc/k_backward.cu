@@ -30,7 +30,10 @@
 //                    applies R(c)^T: dK_loc, and dV_loc.
 //   summaries_bwd    one thread per (block, kv head): dK_cmp = R(c_u)^T
 //                    (a_u dk~), dV_cmp = a_u dv~, dscores = a_u (da_u - sum a da)
-//                    with da_u = <dk~, R(c_u) k_u> + <dv~, v_u>.
+//                    with da_u = <dk~, R(c_u) k_u> + <dv~, v_u>; for the
+//                    summary-centre variant R(c_u) is replaced by one R(cbar)
+//                    on the pooled key: dK_cmp = a_u R(cbar)^T dk~ and
+//                    da_u = <R(cbar)^T dk~, k_u> + <dv~, v_u>.
 #include "common.cuh"
 #include "internal.h"
 
@@ -391,6 +394,13 @@ __global__ void __launch_bounds__(kSbThreads) summaries_bwd_kernel(
     }
   }
   const int32_t* mem = members + (size_t)j * s.v;
+  if (s.center) {
+    // Summary-centre variant: k~ = R(cbar) sum_u a_u k_u, so the pooled key's
+    // gradient is R(cbar)^T dk~ = R(-cbar) dk~ and the members are unrotated.
+    const int jx = j % s.nbx, jy = (j / s.nbx) % s.nby, jz = j / (s.nbx * s.nby);
+    rotate_at<kMaxPairs>(dk, s, 0, -(jz * s.bz + 0.5 * (s.bz - 1)), -(jy * s.by + 0.5 * (s.by - 1)),
+                         -(jx * s.bx + 0.5 * (s.bx - 1)));
+  }
   float a[kMaxBlockVolume], da[kMaxBlockVolume];
   float smax = -INFINITY, den = 0.f, mean = 0.f;
   for (int m = 0; m < s.v; ++m) smax = fmaxf(smax, __ldg(scores + (size_t)__ldg(mem + m) * s.Hkv + g));
@@ -405,7 +415,7 @@ __global__ void __launch_bounds__(kSbThreads) summaries_bwd_kernel(
     const int cz = __ldg(coords + 3 * u), cy = __ldg(coords + 3 * u + 1), cx = __ldg(coords + 3 * u + 2);
     float f[kDh];
     load_f32(kc + (u * s.Hkv + g) * kDh, f, kDh);
-    rope_planes(f, s, tab, 0, kMaxPairs, cz, cy, cx, false);
+    if (!s.center) rope_planes(f, s, tab, 0, kMaxPairs, cz, cy, cx, false);
     float acc = 0.f;
 #pragma unroll
     for (int e = 0; e < kDh; ++e) acc = fmaf(dk[e], f[e], acc);
@@ -422,7 +432,7 @@ __global__ void __launch_bounds__(kSbThreads) summaries_bwd_kernel(
     float f[kDh];
 #pragma unroll
     for (int e = 0; e < kDh; ++e) f[e] = a[m] * dk[e];
-    rope_planes(f, s, tab, 0, kMaxPairs, cz, cy, cx, true);
+    if (!s.center) rope_planes(f, s, tab, 0, kMaxPairs, cz, cy, cx, true);
     store_f32(dkc + (u * s.Hkv + g) * kDh, f, kDh);
 #pragma unroll
     for (int e = 0; e < kDh; ++e) f[e] = a[m] * dv[e];

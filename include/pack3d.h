@@ -306,9 +306,11 @@ size_t pack3d_train_workspace_bytes(const pack3d_config *cfg);
  * Outputs (all required, device, 16-byte aligned): out (T [N,Hq,d_h]), dq
  * (T [N,Hq,d_h]), dk_loc, dv_loc, dk_cmp, dv_cmp (T [N,Hkv,d_h]), dscores
  * (float [N,Hkv]) and dgate (float [N,Hq,2]), in packed order.  workspace: at
- * least pack3d_train_workspace_bytes(cfg) bytes, 256-byte aligned.  The
- * summary-centre variant has no backward here: PACK3D_FLAG_SUMMARY_CENTER
- * -> PACK3D_ERR_INVALID_ARG. */
+ * least pack3d_train_workspace_bytes(cfg) bytes, 256-byte aligned.  With
+ * PACK3D_FLAG_SUMMARY_CENTER the forward and the summaries' backward follow
+ * the summary-centre variant (the pooled key rotated once by R(cbar_j)):
+ * dk_cmp[u] = a_u R(cbar_j)^T dk_sum[j] and
+ * da_u = <R(cbar_j)^T dk_sum[j], k_cmp[u]> + <dv_sum[j], v_cmp[u]>. */
 pack3d_status pack3d_forward_backward(const pack3d_config *cfg, const int32_t *coords, const void *q,
                                       const void *k_loc, const void *v_loc, const void *k_cmp,
                                       const void *v_cmp, const float *scores, const float *gate,

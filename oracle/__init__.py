@@ -70,6 +70,7 @@ def _load():
         lib.orc_summary_attn_backward_q.argtypes = [P, P, P, P, L, L, P, P, P, P]
         lib.orc_summary_attn_backward_kv.argtypes = [P, P, P, P, L, P, P, P, P, L, P, P]
         lib.orc_summaries_backward.argtypes = [P, P, P, P, P, P, P, P, P, L, P, P, P]
+        lib.orc_summaries_center_backward.argtypes = [P, P, P, P, P, P, P, P, L, P, P, P]
         _lib = lib
     return _lib
 
@@ -256,7 +257,7 @@ def _scatter(a: np.ndarray, idx: np.ndarray) -> np.ndarray:
     return full
 
 
-def backward(s, inputs: Dict, dout, keys=None, blocks=None) -> Dict[str, np.ndarray]:
+def backward(s, inputs: Dict, dout, keys=None, blocks=None, center: bool = False) -> Dict[str, np.ndarray]:
     """Gradients of L = <dout, out> with respect to every input of the operator.
 
     The chain rule through the forward stages in reverse: the tokenwise gate
@@ -267,6 +268,7 @@ def backward(s, inputs: Dict, dout, keys=None, blocks=None) -> Dict[str, np.ndar
     ``dv_cmp`` and ``dscores`` for the members of the summary blocks ``blocks``
     (``cmp_tokens`` = their packed indices, block by block, members in raster
     order), or, with ``blocks=None``, for every token in packed order.
+    ``center`` differentiates the summary-centre variant of the summaries.
     """
     lib = _load()
     st, g2p, mem = build_index(s, inputs["coords"])
@@ -280,7 +282,7 @@ def backward(s, inputs: Dict, dout, keys=None, blocks=None) -> Dict[str, np.ndar
     qr = rotate(s, coords, inputs["q"])
     klr = rotate(s, coords, inputs["k_loc"])
     vl = as_f64(inputs["v_loc"])
-    ks, vs = summaries(s, coords, mem, inputs["k_cmp"], inputs["v_cmp"], inputs["scores"])
+    ks, vs = summaries(s, coords, mem, inputs["k_cmp"], inputs["v_cmp"], inputs["scores"], center=center)
     ol = local_attn(s, coords, g2p, qr, klr, vl)
     oc = summary_attn(s, qr, ks, vs)
     # gate
@@ -320,8 +322,12 @@ def backward(s, inputs: Dict, dout, keys=None, blocks=None) -> Dict[str, np.ndar
     dkc = np.empty((nt, Hkv, d))
     dvc = np.empty_like(dkc)
     dsc = np.empty((nt, Hkv))
-    lib.orc_summaries_backward(ctypes.byref(cfg), _ptr(coords), _ptr(mem), _ptr(kc), _ptr(vc), _ptr(sc),
-                               _ptr(dks), _ptr(dvs), _ptr(bb), bb.shape[0], _ptr(dkc), _ptr(dvc), _ptr(dsc))
+    if center:
+        lib.orc_summaries_center_backward(ctypes.byref(cfg), _ptr(mem), _ptr(kc), _ptr(vc), _ptr(sc), _ptr(dks),
+                                          _ptr(dvs), _ptr(bb), bb.shape[0], _ptr(dkc), _ptr(dvc), _ptr(dsc))
+    else:
+        lib.orc_summaries_backward(ctypes.byref(cfg), _ptr(coords), _ptr(mem), _ptr(kc), _ptr(vc), _ptr(sc),
+                                   _ptr(dks), _ptr(dvs), _ptr(bb), bb.shape[0], _ptr(dkc), _ptr(dvc), _ptr(dsc))
     cmp_tokens = mem[bb].reshape(-1).astype(np.int64)
     if blocks is None:
         # every token is a member of exactly one block: scatter to packed order

@@ -673,3 +673,61 @@ void orc_summaries_backward(const orc_cfg *c, const int32_t *coords, const int32
         free(t);
     }
 }
+
+/* Summary-centre variant backward, for the listed blocks (layout as
+ * orc_summaries_backward): with kp_j = sum_u a_u kcmp[u,g] and
+ * ksum = R(cbar_j) kp_j,
+ *   dkp = R(cbar_j)^T dksum[j,g]
+ *   dkcmp[u,g] = a_u dkp,  dvcmp[u,g] = a_u dvsum[j,g]
+ *   da_u = <dkp, kcmp[u,g]> + <dvsum[j,g], vcmp[u,g]>
+ *   dscores[u,g] = a_u (da_u - sum_u' a_u' da_u'). */
+void orc_summaries_center_backward(const orc_cfg *c, const int32_t *members, const double *kcmp,
+                                   const double *vcmp, const double *scores, const double *dksum,
+                                   const double *dvsum, const int64_t *blocks, long nb,
+                                   double *dkcmp, double *dvcmp, double *dscores)
+{
+    int v = c->bz * c->by * c->bx;
+    int nby = c->H / c->by, nbx = c->W / c->bx;
+    int d = c->dh, Hkv = c->Hkv;
+#pragma omp parallel for schedule(static)
+    for (long jr = 0; jr < nb; ++jr) {
+        long j = blocks[jr];
+        long jx = j % nbx, jy = (j / nbx) % nby, jz = j / ((long)nbx * nby);
+        double cz = jz * c->bz + 0.5 * (c->bz - 1);
+        double cy = jy * c->by + 0.5 * (c->by - 1);
+        double cx = jx * c->bx + 0.5 * (c->bx - 1);
+        double *a = (double *)malloc(sizeof(double) * v);
+        double *da = (double *)malloc(sizeof(double) * v);
+        double *dkp = (double *)malloc(sizeof(double) * d);
+        for (int g = 0; g < Hkv; ++g) {
+            const double *dv = dvsum + (jr * Hkv + g) * d;
+            rotate_row_t(c, cz, cy, cx, dksum + (jr * Hkv + g) * d, dkp);
+            double smax = -INFINITY, den = 0.0, mean = 0.0;
+            for (int m = 0; m < v; ++m) {
+                double s = scores[(long)members[j * v + m] * Hkv + g];
+                if (s > smax) smax = s;
+            }
+            for (int m = 0; m < v; ++m) {
+                a[m] = exp(scores[(long)members[j * v + m] * Hkv + g] - smax);
+                den += a[m];
+            }
+            for (int m = 0; m < v; ++m) a[m] /= den;
+            for (int m = 0; m < v; ++m) {
+                long u = members[j * v + m];
+                da[m] = 0.0;
+                for (int e = 0; e < d; ++e)
+                    da[m] += dkp[e] * kcmp[(u * Hkv + g) * d + e] + dv[e] * vcmp[(u * Hkv + g) * d + e];
+                mean += a[m] * da[m];
+                long o = ((jr * v + m) * Hkv + g) * d;
+                for (int e = 0; e < d; ++e) {
+                    dkcmp[o + e] = a[m] * dkp[e];
+                    dvcmp[o + e] = a[m] * dv[e];
+                }
+            }
+            for (int m = 0; m < v; ++m) dscores[(jr * v + m) * Hkv + g] = a[m] * (da[m] - mean);
+        }
+        free(a);
+        free(da);
+        free(dkp);
+    }
+}

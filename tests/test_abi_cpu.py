@@ -126,5 +126,3 @@ def test_forward_backward_host_errors(p3):
     bad = list(args)
     bad[11] = fake + 8       # dk_loc misaligned
     assert lib.pack3d_forward_backward(cfgp, *bad, fake, tws, fake, None) == 3
-    c.flags = p3.FLAG_SUMMARY_CENTER
-    assert lib.pack3d_forward_backward(cfgp, *args, fake, tws, fake, None) == 1

@@ -83,6 +83,26 @@ def test_forward_backward_matches_oracle(p3, name, s, packing, flags):
         assert e <= tol, f"{name}: {key} rel err {e:.3e} > {tol}"
 
 
+CENTER_CASES = [
+    ("center-bf16", small(), "random", 0),
+    ("center-f32", small(dtype="f32", value_scale=1.0), "morton", 0),
+    ("center-blocks222-bf16", small(Z=4, H=12, W=16, bz=2, by=2, bx=2), "block", 0),
+]
+
+
+@pytest.mark.parametrize("name,s,packing,flags", CENTER_CASES, ids=[c[0] for c in CENTER_CASES])
+def test_summary_center_forward_backward_matches_oracle(p3, name, s, packing, flags):
+    """The summary-centre variant through the training block against the oracle's centre backward."""
+    inp = synth.make_inputs(s, packing, seed=4)
+    dout = synth.make_dout(s, packing, seed=4)
+    gpu = run_fwd_bwd(p3, s, inp, dout, flags | p3.FLAG_SUMMARY_CENTER)
+    ref = oracle.backward(s, inp, dout, center=True)
+    tol = TOL[s.dtype]
+    for key in GRADS + ("out",):
+        e = rel_err(gpu[key].double().numpy(), ref[key])
+        assert e <= tol, f"{name}: {key} rel err {e:.3e} > {tol}"
+
+
 @pytest.mark.parametrize("flags", [0, 0x3])
 def test_training_forward_output_equals_forward(p3, flags):
     """The training forward (statistics saved in the epilogue) leaves `out` bit for bit as pack3d_forward."""

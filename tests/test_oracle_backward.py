@@ -139,3 +139,34 @@ def test_sampled_keys_and_blocks_equal_the_full_backward():
     tok = part["cmp_tokens"]
     for k in ("dk_cmp", "dv_cmp", "dscores"):
         np.testing.assert_array_equal(part[k], full[k][tok])
+
+
+@pytest.mark.parametrize("name", INPUTS)
+def test_summary_center_variant_directional_derivatives(name):
+    """The summary-centre variant's backward against finite differences of its forward."""
+    s, packing = CASES[1][1], "random"
+    inp = f64_inputs(s, packing)
+    dout = synth.make_dout(s, packing, seed=5).double().numpy()
+    grads = oracle.backward(s, inp, dout, center=True)
+    rng = np.random.default_rng(23)
+    delta = rng.standard_normal(inp[name].shape)
+    eps = 1e-6
+
+    def loss_c(x):
+        return float(np.sum(oracle.forward(s, x, center=True)["out"] * dout))
+
+    fd = (loss_c(dict(inp, **{name: inp[name] + eps * delta})) -
+          loss_c(dict(inp, **{name: inp[name] - eps * delta}))) / (2 * eps)
+    an = float(np.sum(grads[GRAD[name]] * delta))
+    assert abs(fd - an) <= 1e-6 * max(abs(an), 1e-3), f"{name}: fd {fd!r} vs analytic {an!r}"
+
+
+def test_summary_center_backward_equals_exact_on_unit_blocks():
+    """With 1x1x1 blocks the centre is the token's own site: both forms and their gradients coincide."""
+    s = CASES[1][1].replace(bz=1, by=1, bx=1)
+    inp = f64_inputs(s, "morton")
+    dout = synth.make_dout(s, "morton", seed=5).double().numpy()
+    a = oracle.backward(s, inp, dout)
+    b = oracle.backward(s, inp, dout, center=True)
+    for k in GRAD.values():
+        np.testing.assert_allclose(b[k], a[k], rtol=0, atol=1e-12 * max(np.abs(a[k]).max(), 1.0))
