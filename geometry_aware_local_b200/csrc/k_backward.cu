@@ -28,7 +28,7 @@
 //                    whose box holds it (the box around the key: the window
 //                    relation is symmetric), all q heads of the kv head;
 //                    applies R(c)^T: dK_loc, and dV_loc.
-//   summaries_bwd    one thread per (block, kv head): dK_cmp = R(c_u)^T
+//   summaries_bwd    one warp per (block, kv head), lane = rotary plane: dK_cmp = R(c_u)^T
 //                    (a_u dk~), dV_cmp = a_u dv~, dscores = a_u (da_u - sum a da)
 //                    with da_u = <dk~, R(c_u) k_u> + <dv~, v_u>; for the
 //                    summary-centre variant R(c_u) is replaced by one R(cbar)
@@ -368,7 +368,33 @@ __global__ void __launch_bounds__(2 * kBSites) local_bwd_dkv_kernel(
 
 // ---- summaries ------------------------------------------------------------
 
-constexpr int kSbThreads = 128, kMaxBlockVolume = 64;
+constexpr int kSbThreads = 256, kMaxBlockVolume = 64;
+
+// One warp per (block, kv head); lane p owns rotary plane p, i.e. dims 2p and
+// 2p+1 of every row, so R(c) and R(c)^T act lane-locally and every load and
+// store of a 64-dim row is one coalesced warp access.
+template <typename T>
+__device__ __forceinline__ float2 load_pair(const T* p);
+template <>
+__device__ __forceinline__ float2 load_pair<float>(const float* p) {
+  return __ldg(reinterpret_cast<const float2*>(p));
+}
+template <>
+__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint32_t w = __ldg(reinterpret_cast<const unsigned int*>(p));
+  return make_float2(bf16_lo(w), bf16_hi(w));
+}
+__device__ __forceinline__ void store_pair(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+__device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
+  *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(v.x, v.y);
+}
+
+// (x0, x1) of plane p at coordinate value cval: R (sg = +1) or R^T (sg = -1).
+__device__ __forceinline__ float2 rot_pair(float2 f, const float2* tab, int off, int cval, float sg) {
+  const float2 cs = tab[off + cval];
+  const float sn = sg * cs.y;
+  return make_float2(f.x * cs.x - f.y * sn, f.x * sn + f.y * cs.x);
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kSbThreads) summaries_bwd_kernel(
@@ -379,64 +405,67 @@ __global__ void __launch_bounds__(kSbThreads) summaries_bwd_kernel(
   extern __shared__ float2 tab[];
   build_rope_table(tab, s);
   __syncthreads();
-  const long t = (long)blockIdx.x * kSbThreads + threadIdx.x;
-  if (t >= (long)s.M * s.Hkv) return;
-  const int j = (int)(t / s.Hkv), g = (int)(t % s.Hkv);
-  float dk[kDh], dv[kDh];
-  {
-    const float4* a = reinterpret_cast<const float4*>(dks + ((size_t)j * s.Hkv + g) * kDh);
-    const float4* b = reinterpret_cast<const float4*>(dvs + ((size_t)j * s.Hkv + g) * kDh);
-#pragma unroll
-    for (int c = 0; c < kDh / 4; ++c) {
-      const float4 x = __ldg(a + c), y = __ldg(b + c);
-      dk[4 * c] = x.x; dk[4 * c + 1] = x.y; dk[4 * c + 2] = x.z; dk[4 * c + 3] = x.w;
-      dv[4 * c] = y.x; dv[4 * c + 1] = y.y; dv[4 * c + 2] = y.z; dv[4 * c + 3] = y.w;
-    }
-  }
-  const int32_t* mem = members + (size_t)j * s.v;
+  const int lane = threadIdx.x & 31;
+  const long w = (long)blockIdx.x * (kSbThreads / 32) + (threadIdx.x >> 5);
+  if (w >= (long)s.M * s.Hkv) return;
+  const int j = (int)(w / s.Hkv), g = (int)(w % s.Hkv);
+  // This lane's rotary plane: axis and first table entry (untouched planes: identity).
+  const int ax = lane < s.npairs ? s.pair_axis[lane] : 3;
+  const int toff = lane < s.npairs ? s.pair_off[lane] : 0;
+  const size_t srow = ((size_t)j * s.Hkv + g) * kDh + 2 * lane;
+  float2 dk = __ldg(reinterpret_cast<const float2*>(dks + srow));
+  const float2 dv = __ldg(reinterpret_cast<const float2*>(dvs + srow));
   if (s.center) {
     // Summary-centre variant: k~ = R(cbar) sum_u a_u k_u, so the pooled key's
     // gradient is R(cbar)^T dk~ = R(-cbar) dk~ and the members are unrotated.
+    float f[2] = {dk.x, dk.y};
     const int jx = j % s.nbx, jy = (j / s.nbx) % s.nby, jz = j / (s.nbx * s.nby);
-    rotate_at<kMaxPairs>(dk, s, 0, -(jz * s.bz + 0.5 * (s.bz - 1)), -(jy * s.by + 0.5 * (s.by - 1)),
-                         -(jx * s.bx + 0.5 * (s.bx - 1)));
+    if (lane < s.npairs)
+      rotate_at<1>(f, s, lane, -(jz * s.bz + 0.5 * (s.bz - 1)), -(jy * s.by + 0.5 * (s.by - 1)),
+                   -(jx * s.bx + 0.5 * (s.bx - 1)));
+    dk = make_float2(f[0], f[1]);
   }
-  float a[kMaxBlockVolume], da[kMaxBlockVolume];
-  float smax = -INFINITY, den = 0.f, mean = 0.f;
-  for (int m = 0; m < s.v; ++m) smax = fmaxf(smax, __ldg(scores + (size_t)__ldg(mem + m) * s.Hkv + g));
-  for (int m = 0; m < s.v; ++m) {
-    a[m] = expf(__ldg(scores + (size_t)__ldg(mem + m) * s.Hkv + g) - smax);
-    den += a[m];
-  }
+  const int32_t* mem = members + (size_t)j * s.v;
+  // Block weights: the scores of the block's members (lanes hold two members each).
+  float smax = -INFINITY;
+  for (int m = lane; m < s.v; m += 32) smax = fmaxf(smax, __ldg(scores + (size_t)__ldg(mem + m) * s.Hkv + g));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+  float den = 0.f;
+  for (int m = lane; m < s.v; m += 32) den += expf(__ldg(scores + (size_t)__ldg(mem + m) * s.Hkv + g) - smax);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   const float inv = 1.f / den;
+  // da_u for every member, then the mean sum_u a_u da_u.
+  float a[kMaxBlockVolume], da[kMaxBlockVolume];
+  float mean = 0.f;
   for (int m = 0; m < s.v; ++m) {
-    a[m] *= inv;
     const size_t u = (size_t)__ldg(mem + m);
-    const int cz = __ldg(coords + 3 * u), cy = __ldg(coords + 3 * u + 1), cx = __ldg(coords + 3 * u + 2);
-    float f[kDh];
-    load_f32(kc + (u * s.Hkv + g) * kDh, f, kDh);
-    if (!s.center) rope_planes(f, s, tab, 0, kMaxPairs, cz, cy, cx, false);
-    float acc = 0.f;
+    a[m] = expf(__ldg(scores + u * s.Hkv + g) - smax) * inv;
+    const size_t row = (u * s.Hkv + g) * kDh + 2 * lane;
+    float2 kr = load_pair(kc + row);
+    if (!s.center && ax < 3) {
+      const int cval = __ldg(coords + 3 * u + ax);
+      kr = rot_pair(kr, tab, toff, cval, 1.f);
+    }
+    const float2 vv = load_pair(vc + row);
+    float acc = dk.x * kr.x + dk.y * kr.y + dv.x * vv.x + dv.y * vv.y;
 #pragma unroll
-    for (int e = 0; e < kDh; ++e) acc = fmaf(dk[e], f[e], acc);
-    load_f32(vc + (u * s.Hkv + g) * kDh, f, kDh);
-#pragma unroll
-    for (int e = 0; e < kDh; ++e) acc = fmaf(dv[e], f[e], acc);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     da[m] = acc;
     mean = fmaf(a[m], acc, mean);
   }
   for (int m = 0; m < s.v; ++m) {
     const size_t u = (size_t)__ldg(mem + m);
-    const int cz = __ldg(coords + 3 * u), cy = __ldg(coords + 3 * u + 1), cx = __ldg(coords + 3 * u + 2);
-    dsc[u * s.Hkv + g] = a[m] * (da[m] - mean);
-    float f[kDh];
-#pragma unroll
-    for (int e = 0; e < kDh; ++e) f[e] = a[m] * dk[e];
-    if (!s.center) rope_planes(f, s, tab, 0, kMaxPairs, cz, cy, cx, true);
-    store_f32(dkc + (u * s.Hkv + g) * kDh, f, kDh);
-#pragma unroll
-    for (int e = 0; e < kDh; ++e) f[e] = a[m] * dv[e];
-    store_f32(dvc + (u * s.Hkv + g) * kDh, f, kDh);
+    if (lane == 0) dsc[u * s.Hkv + g] = a[m] * (da[m] - mean);
+    const size_t row = (u * s.Hkv + g) * kDh + 2 * lane;
+    float2 k2 = make_float2(a[m] * dk.x, a[m] * dk.y);
+    if (!s.center && ax < 3) {
+      const int cval = __ldg(coords + 3 * u + ax);
+      k2 = rot_pair(k2, tab, toff, cval, -1.f);
+    }
+    store_pair(dkc + row, k2);
+    store_pair(dvc + row, make_float2(a[m] * dv.x, a[m] * dv.y));
   }
 }
 
@@ -548,8 +577,9 @@ cudaError_t summaries_bwd_t(const Shape& s, const int32_t* coords, const int32_t
   const size_t smem = (size_t)s.tab_entries * sizeof(float2);
   cudaError_t e = set_table_smem((const void*)summaries_bwd_kernel<T>, smem);
   if (e != cudaSuccess) return e;
-  const long n = (long)s.M * s.Hkv;
-  summaries_bwd_kernel<T><<<(unsigned)((n + kSbThreads - 1) / kSbThreads), kSbThreads, smem, st>>>(
+  const long warps = (long)s.M * s.Hkv;
+  const long per_cta = kSbThreads / 32;
+  summaries_bwd_kernel<T><<<(unsigned)((warps + per_cta - 1) / per_cta), kSbThreads, smem, st>>>(
       s, coords, members, (const T*)kc, (const T*)vc, scores, dks, dvs, (T*)dkc, (T*)dvc, dsc);
   return cudaGetLastError();
 }
