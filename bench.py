@@ -380,7 +380,8 @@ def run_train_only(args, s):
                 "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": train["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": s.dtype, "data": "synthetic (values drawn on the device)",
-                "config": {"workload": WORKLOAD_TEXT[args.config], "tokens": s.N, "summaries": s.M}, "train": train,
+                "config": {"workload": WORKLOAD_TEXT[args.config], "tokens": s.N, "summaries": s.M,
+                           "packing": s.packing}, "train": train,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -545,6 +546,7 @@ def run_ours(args, s):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT[args.config], "tokens": s.N, "summaries": s.M,
+                       "packing": s.packing,
                        "parallelism": "replicas only" if world > 1 else "single GPU",
                        "summary_form": "summary-centre variant" if args.summary_center
                        else "rotate-before-compress (exact)",
@@ -596,6 +598,8 @@ def main():
                     help="also time the training block on the device-drawn 4m / 8m volumes")
     ap.add_argument("--train-only", action="store_true",
                     help="time only the training block (pack3d_forward_backward), inputs drawn on the device")
+    ap.add_argument("--packing", choices=synth.PACKINGS, default=None,
+                    help="override the workload's packing (the stress case times all of them)")
     ap.add_argument("--summary-center", action="store_true",
                     help="time the summary-centre variant of the block summaries and report its error "
                          "against the exact rotate-before-compress form")
@@ -603,6 +607,8 @@ def main():
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     s = synth.CONFIGS[args.config]
+    if args.packing is not None:
+        s = s.replace(packing=args.packing)
     if args.impl == "reference":
         run_reference(args, s)
     elif args.train_only:
