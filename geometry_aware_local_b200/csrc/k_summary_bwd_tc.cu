@@ -44,7 +44,6 @@ namespace pack3d {
 namespace {
 
 constexpr int kRowsPerTile = 128;
-constexpr long kSmCount = 148;                        // B200
 constexpr int kQTileBytes = kRowsPerTile * kDh * 2;   // 16 KiB: 128 rows x 64 bf16
 
 struct BwdArgs {
@@ -633,6 +632,9 @@ cudaError_t launch_summary_bwd_dkv_tc(const Shape& s, const void* qr, const void
   // the grid, each CTA keeping at least eight 128-row steps, and among the
   // split counts up to twice that, the one whose last wave of CTAs leaves the
   // fewest SMs idle.
+  int dev = 0, sm_count = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
+  const long kSmCount = max(1, sm_count);
   const int tiles = (s.M + k_side::kBS - 1) / k_side::kBS;
   const long steps = (a.rows + kRowsPerTile - 1) / kRowsPerTile;
   const long units = (long)tiles * s.Hkv;
