@@ -634,18 +634,18 @@ cudaError_t launch_summary_bwd_dkv_tc(const Shape& s, const void* qr, const void
   // fewest SMs idle.
   int dev = 0, sm_count = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
-  const long kSmCount = max(1, sm_count);
+  const long sms = max(1, sm_count);
   const int tiles = (s.M + k_side::kBS - 1) / k_side::kBS;
   const long steps = (a.rows + kRowsPerTile - 1) / kRowsPerTile;
   const long units = (long)tiles * s.Hkv;
-  const long lo = max(1L, min((4L * kSmCount + units - 1) / units, steps / 8));
+  const long lo = max(1L, min((4L * sms + units - 1) / units, steps / 8));
   long splits = lo;
   double best = 2.0;
   for (long c = lo; c <= max(lo, min(2 * lo, steps / 8)); ++c) {
     const long per = (steps + c - 1) / c;
     const long used = (steps + per - 1) / per;          // splits that get rows
     const long ctas = units * used;
-    const double idle = (double)((ctas + kSmCount - 1) / kSmCount * kSmCount - ctas) / (double)ctas;
+    const double idle = (double)((ctas + sms - 1) / sms * sms - ctas) / (double)ctas;
     if (idle < best - 1e-9) {
       best = idle;
       splits = c;
