@@ -246,25 +246,34 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         ptx::tmem_ld64_sync(trow + kColDP + 64 * h, dv);
         if (h == kBN / 64 - 1) warp_arrive(s_free);
         const int lim = a.M - j * kBN - 64 * h;   // columns >= lim are past the last summary
+        uint32_t pk[32];
+        if (lim >= 64) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), c2, nl2);
+            const float2 t = __ffma2_rn(make_float2(__uint_as_float(dv[2 * k]), __uint_as_float(dv[2 * k + 1])), w2, nd2);
+            const float2 ds = __fmul2_rn(make_float2(ptx::ex2(x.x), ptx::ex2(x.y)), t);
+            pk[k] = pack_bf16x2(ds.x, ds.y);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), c2, nl2);
+            const float2 t = __ffma2_rn(make_float2(__uint_as_float(dv[2 * k]), __uint_as_float(dv[2 * k + 1])), w2, nd2);
+            float2 ds = __fmul2_rn(make_float2(ptx::ex2(x.x), ptx::ex2(x.y)), t);
+            if (2 * k >= lim) ds.x = 0.f;
+            if (2 * k + 1 >= lim) ds.y = 0.f;
+            pk[k] = pack_bf16x2(ds.x, ds.y);
+          }
+        }
+        // dS of the previous step is read by its dQ MMAs until p_free: wait
+        // only now, so this step's exponentials overlap them.
         if (h == 0 && j > 0) {
           if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free, (j - 1) & 1, abort_flag)))) break;
           ptx::tc_fence_after();
         }
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int c = 32 * q + 2 * k;
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2, nl2);
-            const float2 t = __ffma2_rn(make_float2(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])), w2, nd2);
-            float2 ds = __fmul2_rn(make_float2(ptx::ex2(x.x), ptx::ex2(x.y)), t);
-            if (c >= lim) ds.x = 0.f;
-            if (c + 1 >= lim) ds.y = 0.f;
-            pk[k] = pack_bf16x2(ds.x, ds.y);
-          }
-          ptx::tmem_st16(trow + kColDS + 32 * h + 16 * q, pk);
-        }
+        ptx::tmem_st16(trow + kColDS + 32 * h, pk);
+        ptx::tmem_st16(trow + kColDS + 32 * h + 16, pk + 16);
       }
       if (!ok) break;
       ptx::tmem_wait_st();
