@@ -311,3 +311,65 @@ class Pack3D:
         st = check_status(self.err)
         if st != 0:
             raise Pack3DError(st, "pack3d_forward")
+
+
+def attention(cfg: Config, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate):
+    """The PACK3D operator as a differentiable PyTorch op.
+
+    Forward: pack3d_forward.  Backward: pack3d_forward_backward, which reruns
+    the forward to save its softmax statistics and returns the gradients of
+    every differentiable input (q, k_loc, v_loc, k_cmp, v_cmp, scores, gate;
+    coords is integer).  Tensors are CUDA, contiguous, in the layouts of
+    include/pack3d.h; the work runs on the current stream.
+    """
+    return _Pack3DAutograd.apply(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate)
+
+
+def _make_autograd():
+    import torch
+
+    class Pack3DAutograd(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate):
+            st = validate(cfg)
+            if st != 0:
+                raise Pack3DError(st, "pack3d_validate_config")
+            out = torch.empty_like(q)
+            ws = torch.empty(workspace_bytes(cfg), dtype=torch.uint8, device=q.device)
+            err = torch.zeros(4, dtype=torch.int32, device=q.device)
+            forward(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, ws, err)
+            ctx.cfg = cfg
+            ctx.err = err
+            ctx.save_for_backward(coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate)
+            return out
+
+        @staticmethod
+        def backward(ctx, dout):
+            coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate = ctx.saved_tensors
+            dout = dout.to(q.dtype).contiguous()
+            grads = empty_grads(q, k_loc, scores, gate)
+            out = torch.empty_like(q)
+            ws = torch.empty(train_workspace_bytes(ctx.cfg), dtype=torch.uint8, device=q.device)
+            forward_backward(ctx.cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, dout, out, grads, ws,
+                             ctx.err)
+            st = check_status(ctx.err)
+            if st != 0:
+                raise Pack3DError(st, "pack3d_forward_backward")
+            return (None, None, grads["dq"], grads["dk_loc"], grads["dv_loc"], grads["dk_cmp"], grads["dv_cmp"],
+                    grads["dscores"], grads["dgate"])
+
+    return Pack3DAutograd
+
+
+class _LazyAutograd:
+    """Defers the torch import until the differentiable op is first used."""
+    _cls = None
+
+    @classmethod
+    def apply(cls, *args):
+        if cls._cls is None:
+            cls._cls = _make_autograd()
+        return cls._cls.apply(*args)
+
+
+_Pack3DAutograd = _LazyAutograd

@@ -179,3 +179,24 @@ def test_forward_backward_65k_sampled(p3):
     for k, (a, b) in checks.items():
         e = rel_err(a.double().numpy(), b)
         assert e <= tol, f"65k: {k} rel err {e:.3e} > {tol}"
+
+
+def test_autograd_op_matches_forward_backward(p3):
+    """geometry_aware_local_b200.attention: torch.autograd gradients equal pack3d_forward_backward's,
+    and the forward output equals pack3d_forward's; the gradients match the oracle."""
+    s = small(Z=4, H=16, W=24)
+    inp = synth.make_inputs(s, "random", seed=12)
+    dout = synth.make_dout(s, "random", seed=12)
+    cfg = p3.config_from_shape(s)
+    names = ("q", "k_loc", "v_loc", "k_cmp", "v_cmp", "scores", "gate")
+    d = {k: inp[k].cuda().requires_grad_(k in names) for k in ("coords",) + names}
+    out = p3.attention(cfg, d["coords"], *[d[k] for k in names])
+    out.backward(dout.cuda())
+    ref = run_fwd_bwd(p3, s, inp, dout)
+    assert torch.equal(out.detach().cpu(), ref["out"])
+    grad_of = dict(zip(names, ("dq", "dk_loc", "dv_loc", "dk_cmp", "dv_cmp", "dscores", "dgate")))
+    oref = oracle.backward(s, inp, dout)
+    for k, gname in grad_of.items():
+        g = d[k].grad.cpu()
+        assert rel_err(g.double().numpy(), ref[gname].double().numpy()) <= 2.0 ** -7, k
+        assert rel_err(g.double().numpy(), oref[gname]) <= TOL["bf16"], k
