@@ -21,13 +21,11 @@
 // summary_bwd_dkv_tc_kernel (summary side): one 128-summary tile per CTA and a
 //   range of the kv group's query rows, 128 rows per step, one CTA per SM.
 //   Per step S = Q k~^T and dP = dout v~^T (M=128 rows, N=128 summaries) go to
-//   tensor memory; two softmax warpgroups (one per 64-summary half) write dS
-//   and gamma1 P as bf16 into one of
-//   two shared-memory buffers (alternate steps) in the 128-byte-swizzled
-//   MN-major layout, and the MMA warp
-//   accumulates dk~ += dS^T Q and dv~ += (gamma1 P)^T dout (M=128 summaries,
-//   N=64, K=128 rows; A MN-major from shared memory, B = the Q / dout tiles
-//   read MN-major) in tensor memory.  Each CTA adds its partial dk~ / dv~ to
+//   tensor memory; four softmax warpgroups (one per 32-summary chunk) write
+//   dS and gamma1 P as bf16 into shared memory in the 128-byte-swizzled
+//   MN-major layout, and a second MMA warp accumulates dk~ += dS^T Q and
+//   dv~ += (gamma1 P)^T dout (M=128 summaries, N=64, K=128 rows; A MN-major
+//   from shared memory, B = the Q / dout tiles read MN-major) in tensor memory.  Each CTA adds its partial dk~ / dv~ to
 //   the float outputs with vector atomics.
 //
 // Every mbarrier wait is bounded; a CTA that gives up raises
@@ -310,13 +308,22 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 namespace k_side {
 
 constexpr int kBS = 128;                        // summaries per CTA (M of the dk~ / dv~ accumulators)
-// Two softmax warpgroups (warps 0-3: summaries 0-63 of the tile, warps 4-7:
-// 64-127; a warp reads the tensor-memory lanes of its warp index mod 4), then
-// the MMA warp and the TMA warp.
+// Softmax warpgroups first (warpgroup w covers 32-summary chunks of the tile;
+// a warp reads the tensor-memory lanes of its warp index mod 4), then two MMA
+// warps and the TMA warp.
 // Two MMA warps: the first issues each step's S and dP, the second its
 // dk~ / dv~ accumulation, so that S and dP of the next step never queue
 // behind the slower accumulation issue.
-constexpr int kSoftmaxWarps = 8;
+#ifndef PACK3D_BKV_SMWARPS
+#define PACK3D_BKV_SMWARPS 16
+#endif
+// Softmax warps: 16 (four warpgroups, one 32-summary chunk per thread and
+// step) or 8 (two chunks).  Measured on B200, forward+backward: 65k 4.45 ms
+// (16) vs 4.62 ms (8); 262k 52.6 vs 55.4 ms.  With two warps per
+// sub-partition the softmax's waits were exposed.
+constexpr int kSoftmaxWarps = PACK3D_BKV_SMWARPS;
+constexpr int kWarpgroups = kSoftmaxWarps / 4;
+constexpr int kChunksPerWg = 4 / kWarpgroups;      // 32-summary chunks per thread and step
 constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
 constexpr int kMmaWarp = kSoftmaxWarps, kMmaWarp2 = kSoftmaxWarps + 1, kTmaWarp = kSoftmaxWarps + 2;
 constexpr int kColS = 0, kColDP = 128, kColDK = 256, kColDV = 320, kTmemCols = 512;
@@ -339,7 +346,7 @@ constexpr int kStageBytes = 2 * kQTileBytes;    // Q at +0, dout at +kQTileBytes
 constexpr int kStages = (224 * 1024 - kStageOff - kOpBufs * kOpBytes) / kStageBytes;
 constexpr int kOpOff = kStageOff + kStages * kStageBytes;
 constexpr int kBarOff = kOpOff + kOpBufs * kOpBytes;
-// barriers: full[S], empty[S], kvfull, s_full, s_free, o_final, p_full[kOpBufs], p_free[kOpBufs]
+// barriers: full[S], empty[S], kvfull, o_final, s_full, s_free, p_full[kOpBufs], p_free[kOpBufs]
 constexpr int kNumBars = 2 * kStages + 4 + 2 * kOpBufs;
 static_assert(kStages >= 2, "at least two Q / dout stages");
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
@@ -364,7 +371,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
   auto full = [&](int s) { return bar0 + 8 * s; };
   auto empty = [&](int s) { return bar0 + 8 * (kStages + s); };
   const uint32_t kvfull = bar0 + 8 * (2 * kStages);
-  const uint32_t s_full = kvfull + 8, s_free = kvfull + 16, o_final = kvfull + 24;
+  const uint32_t o_final = kvfull + 8, s_full = kvfull + 16, s_free = kvfull + 24;
   auto p_full = [&](int b) { return kvfull + 32 + 8 * b; };
   auto p_free = [&](int b) { return kvfull + 32 + 8 * kOpBufs + 8 * b; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
@@ -487,7 +494,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     __syncwarp();
   } else {
     // ---------------- softmax warps: thread = query row of the step ----------------
-    const int wg = warp >> 2;                    // summary half of the tile this warpgroup covers
+    const int wg = warp >> 2;                    // summary chunks [kChunksPerWg wg, +kChunksPerWg) of the tile
     const int lane_base = (warp & 3) * 32;
     const int rl = lane_base + lane;             // row inside the step's tile
     const uint32_t trow = tmem + ((uint32_t)lane_base << 16);
@@ -504,11 +511,11 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       const float2 nl2 = make_float2(-lse2, -lse2), w2 = make_float2(w1, w1), nd2 = make_float2(-delta, -delta);
       if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, t & 1, abort_flag)))) break;
       ptx::tc_fence_after();
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * wg + cc;               // 32-summary chunk of the tile
+      for (int cc = 0; cc < kChunksPerWg; ++cc) {
+        const int c = kChunksPerWg * wg + cc;    // 32-summary chunk of the tile
         uint32_t sv[32], dv[32];
         ptx::tmem_ld32x2_sync(trow + kColS + 32 * c, trow + kColDP + 32 * c, sv, dv);
-        if (cc == 1) warp_arrive(s_free);
+        if (cc == kChunksPerWg - 1) warp_arrive(s_free);
         uint32_t pd[16], pp[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -528,11 +535,11 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             break;
         }
         // Row rl of the MN-major operands: summaries 32c .. 32c+31 are 16-byte
-        // chunks (c & 1) * 4 + m of half c / 2 (= wg).
-        const uint32_t op = sbase + kOpOff + (t % kOpBufs) * kOpBytes + (uint32_t)wg * kQTileBytes;
+        // chunks (c & 1) * 4 + m of half c / 2.
+        const uint32_t op = sbase + kOpOff + (t % kOpBufs) * kOpBytes + (uint32_t)(c >> 1) * kQTileBytes;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const uint32_t off = ptx::sw128_offset((uint32_t)rl, (uint32_t)((cc * 4 + m) * 8));
+          const uint32_t off = ptx::sw128_offset((uint32_t)rl, (uint32_t)(((c & 1) * 4 + m) * 8));
           ptx::st_shared_v4(op + off, pd[4 * m], pd[4 * m + 1], pd[4 * m + 2], pd[4 * m + 3]);
           ptx::st_shared_v4(op + kPInOp + off, pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
         }
@@ -543,15 +550,23 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     }
     if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final, 0, abort_flag))) {
       ptx::tc_fence_after();
-      // Accumulator lane = summary of this tile; warpgroup 0 adds dk~, warpgroup 1 dv~.
+      // Accumulator lane = summary of this tile.  The warpgroups share the
+      // 128 accumulator columns (dk~ 64, then dv~ 64) evenly.
       const int j = stile * kBS + rl;
-      uint32_t r[kDh];
-      ptx::tmem_ld64_sync(trow + (wg == 0 ? kColDK : kColDV), r);
+      constexpr int kCols = 2 * kDh / kWarpgroups;   // 64 or 32
+      const int col0 = wg * kCols;                   // in [0, 128): dk~ below 64, dv~ from 64
+      const bool is_k = col0 < kDh;
+      uint32_t r[kCols];
+      if constexpr (kCols == 64)
+        ptx::tmem_ld64_sync(trow + kColDK + col0, r);
+      else
+        ptx::tmem_ld32_sync(trow + kColDK + col0, r);
       if (j < a.M) {
-        const float f = wg == 0 ? a.scale : 1.f;
-        float4* dst = reinterpret_cast<float4*>((wg == 0 ? a.dks : a.dvs) + ((size_t)j * gridDim.y + g) * kDh);
+        const float f = is_k ? a.scale : 1.f;
+        float4* dst = reinterpret_cast<float4*>((is_k ? a.dks : a.dvs) + ((size_t)j * gridDim.y + g) * kDh +
+                                                (col0 % kDh));
 #pragma unroll
-        for (int q = 0; q < kDh / 4; ++q)
+        for (int q = 0; q < kCols / 4; ++q)
           atomicAdd(dst + q, make_float4(f * __uint_as_float(r[4 * q]), f * __uint_as_float(r[4 * q + 1]),
                                          f * __uint_as_float(r[4 * q + 2]), f * __uint_as_float(r[4 * q + 3])));
       }
