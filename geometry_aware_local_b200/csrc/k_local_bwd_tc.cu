@@ -34,7 +34,16 @@ namespace pack3d {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kThreads = 128;
+// Warpgroups: each covers the CTA's 128 rows (a warp serves the tensor-memory
+// lanes of its index mod 4); they split the softmax's column units, the
+// per-plane dK / dV flush and the dQ epilogue.  Warpgroup 0 also does the
+// gathers.  Measured on B200, forward+backward at 65k / 262k: one warpgroup
+// 4.436 / 52.30 ms, two 4.399 / 52.58, four 4.416 / 51.90 (no clear gain).
+#ifndef PACK3D_LBWD_WG
+#define PACK3D_LBWD_WG 1
+#endif
+constexpr int kWG = PACK3D_LBWD_WG;
+constexpr int kThreads = 128 * kWG;
 constexpr int kMaxKeys = 112;                     // padded keys per plane
 constexpr int kMaxPlanes = 4;                     // 2 brick layers + r_z = 1 on each side
 constexpr int kRowTileBytes = kRows * kDh * 2;    // 16 KiB
@@ -82,17 +91,15 @@ __device__ __forceinline__ void gather_row(uint32_t tile, int r, const __nv_bflo
   }
 }
 
-// Packed index of this thread's row of the padded plane zp, or -1.
-__device__ __forceinline__ int plane_row_index(const LocalBwdArgs& a, int zp, int y0, int x0) {
-  const int r = threadIdx.x;
+// Packed index of row r of the padded plane zp, or -1.
+__device__ __forceinline__ int plane_row_index(const LocalBwdArgs& a, int r, int zp, int y0, int x0) {
   if (r >= a.PH * a.PW) return -1;
   const int y = y0 - a.ry + r / a.PW, x = x0 - a.rx + r % a.PW;
   if (y < 0 || y >= a.H || x < 0 || x >= a.W) return -1;
   return __ldg(a.g2p + ((size_t)zp * a.H + y) * a.W + x);
 }
 
-__device__ __forceinline__ void gather_plane(const LocalBwdArgs& a, uint32_t kt, int g, int j) {
-  const int r = threadIdx.x;
+__device__ __forceinline__ void gather_plane(const LocalBwdArgs& a, int r, uint32_t kt, int g, int j) {
   if (r >= a.NP) return;
   gather_row(kt, r, j >= 0 ? a.k + ((size_t)j * a.Hkv + g) * kDh : nullptr, a.k);
   gather_row(kt + kPlaneTileBytes, r, j >= 0 ? a.v + ((size_t)j * a.Hkv + g) * kDh : nullptr, a.v);
@@ -107,12 +114,13 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + 20);
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & (kRows - 1), wg = tid >> 7;   // tensor-memory lane and warpgroup
   const int g = blockIdx.y;
 
   const int nbx = (a.W + 3) / 4, nby = (a.H + 3) / 4;
   const int b = blockIdx.x;
   const int x0 = (b % nbx) * 4, y0 = ((b / nbx) % nby) * 4, z0 = (b / (nbx * nby)) * 2;
-  const int site = tid >> 2, hh = tid & 3;
+  const int site = row >> 2, hh = row & 3;
   const int lz = site >> 4, ly = (site >> 2) & 3, lx = site & 3;
   const int qz = z0 + lz, qy = y0 + ly, qx = x0 + lx;
   const bool qvalid = qz < a.Z && qy < a.H && qx < a.W;
@@ -134,14 +142,16 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
   const int qi = qvalid ? __ldg(a.g2p + ((size_t)qz * a.H + qy) * a.W + qx) : -1;
   int gi[kMaxPlanes];
 #pragma unroll
-  for (int p = 0; p < kMaxPlanes; ++p) gi[p] = p < nplanes ? plane_row_index(a, zlo + p, y0, x0) : -1;
+  for (int p = 0; p < kMaxPlanes; ++p) gi[p] = p < nplanes ? plane_row_index(a, row, zlo + p, y0, x0) : -1;
 
   auto kt_of = [&](int p) { return sbase + kBufOff + (p % kBufs) * kBufBytes; };
   const size_t orow = qi >= 0 ? (size_t)qi * a.Hq + h : 0;
-  gather_row(sbase + kQOff, tid, qi >= 0 ? a.q + orow * kDh : nullptr, a.q);
-  gather_row(sbase + kDOOff, tid, qi >= 0 ? a.dout + orow * kDh : nullptr, a.dout);
-  gather_plane(a, kt_of(0), g, gi[0]);
-  if (nplanes > 1) gather_plane(a, kt_of(1), g, gi[1]);
+  if (wg == 0) {
+    gather_row(sbase + kQOff, row, qi >= 0 ? a.q + orow * kDh : nullptr, a.q);
+    gather_row(sbase + kDOOff, row, qi >= 0 ? a.dout + orow * kDh : nullptr, a.dout);
+    gather_plane(a, row, kt_of(0), g, gi[0]);
+    if (nplanes > 1) gather_plane(a, row, kt_of(1), g, gi[1]);
+  }
   ptx::cp_async_commit();
 
   // Row statistics; rows of sites outside the volume keep P = 0 through an empty mask.
@@ -176,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const uint32_t idescS = ptx::idesc_bf16_f32(kRows, a.NP, false);
   const float2 c2 = make_float2(a.scale_log2, a.scale_log2), nl2 = make_float2(-lse2, -lse2);
   const float2 w2 = make_float2(w0, w0), nd2 = make_float2(-delta, -delta);
@@ -208,27 +218,31 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
                   ptx::smem_desc_sw128(sbase + kDOOff + kk * 2048, 8192, 1024), kIdescKV, kk > 0);
     ptx::tc_commit(mma_done);
   };
-  // Adds plane p's dK / dV rows (tensor-memory lane = key row of the plane) to the accumulators.
+  // Adds plane p's dK / dV rows (tensor-memory lane = key row of the plane) to
+  // the accumulators; the warpgroups share the 128 columns (dK 64, then dV 64).
   auto flush_plane = [&](int p) {
     const int j = gi[p];
-    const bool mine = tid < a.NP && j >= 0;
-    uint32_t r[kDh];
-    ptx::tmem_ld64_sync(trow + kColDK, r);
-    if (mine) {
-      float4* dst = reinterpret_cast<float4*>(a.dk_acc + ((size_t)j * a.Hkv + g) * kDh);
+    const bool mine = row < a.NP && j >= 0;
+    constexpr int kCols = 2 * kDh / kWG;          // 128, 64 or 32
+    constexpr int kLoad = kCols < 64 ? kCols : 64;
 #pragma unroll
-      for (int q = 0; q < kDh / 4; ++q)
-        atomicAdd(dst + q, make_float4(a.scale * __uint_as_float(r[4 * q]), a.scale * __uint_as_float(r[4 * q + 1]),
-                                       a.scale * __uint_as_float(r[4 * q + 2]),
-                                       a.scale * __uint_as_float(r[4 * q + 3])));
-    }
-    ptx::tmem_ld64_sync(trow + kColDV, r);
-    if (mine) {
-      float4* dst = reinterpret_cast<float4*>(a.dv_acc + ((size_t)j * a.Hkv + g) * kDh);
+    for (int part = 0; part < kCols / kLoad; ++part) {
+      const int col0 = wg * kCols + part * kLoad;   // in [0, 128): dK below 64, dV from 64
+      uint32_t r[kLoad];
+      if constexpr (kLoad == 64)
+        ptx::tmem_ld64_sync(trow + kColDK + col0, r);
+      else
+        ptx::tmem_ld32_sync(trow + kColDK + col0, r);
+      if (mine) {
+        const bool is_k = col0 < kDh;
+        const float f = is_k ? a.scale : 1.f;
+        float4* dst = reinterpret_cast<float4*>((is_k ? a.dk_acc : a.dv_acc) + ((size_t)j * a.Hkv + g) * kDh +
+                                                (col0 % kDh));
 #pragma unroll
-      for (int q = 0; q < kDh / 4; ++q)
-        atomicAdd(dst + q, make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                       __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])));
+        for (int q = 0; q < kLoad / 4; ++q)
+          atomicAdd(dst + q, make_float4(f * __uint_as_float(r[4 * q]), f * __uint_as_float(r[4 * q + 1]),
+                                         f * __uint_as_float(r[4 * q + 2]), f * __uint_as_float(r[4 * q + 3])));
+      }
     }
   };
 
@@ -245,14 +259,13 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
     if (p > 0) {
       flush_plane(p - 1);
       // Plane p-1's buffer is free again (its MMAs completed): gather plane p+1 into it.
-      if (p + 1 < nplanes) gather_plane(a, kt_of(p + 1), g, gi[p + 1]);
+      if (p + 1 < nplanes && wg == 0) gather_plane(a, row, kt_of(p + 1), g, gi[p + 1]);
       ptx::cp_async_commit();
     }
-    // One pass over the plane's columns, 16 at a time.
-    for (int u = 0; u < a.NP / 16; ++u) {
+    // One pass over the plane's columns, 16 at a time, units split over the warpgroups.
+    for (int u = wg; u < a.NP / 16; u += kWG) {
       uint32_t sv[16], dv[16];
-      ptx::tmem_ld16_sync(trow + kColS + 16 * u, sv);
-      ptx::tmem_ld16_sync(trow + kColDP + 16 * u, dv);
+      ptx::tmem_ld16x2_sync(trow + kColS + 16 * u, trow + kColDP + 16 * u, sv, dv);
       const uint32_t bits = uses ? (mask[u >> 1] >> ((u & 1) * 16)) & 0xffffu : 0u;
       uint32_t pd[8], pw[8];
 #pragma unroll
@@ -268,10 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
         pw[k] = pack_bf16x2(pwv.x, pwv.y);
       }
       ptx::tmem_st8(trow + kColDS + 8 * u, pd);
-      // keys 16u .. 16u+15: chunks ((16u) % 64) / 8 and +1 of half (16u) / 64, row tid
+      // keys 16u .. 16u+15: chunks ((16u) % 64) / 8 and +1 of half (16u) / 64, this row
       const uint32_t half = (uint32_t)(16 * u) >> 6, e0 = (uint32_t)(16 * u) & 63u;
-      const uint32_t o0 = half * kRowTileBytes + ptx::sw128_offset((uint32_t)tid, e0);
-      const uint32_t o1 = half * kRowTileBytes + ptx::sw128_offset((uint32_t)tid, e0 + 8);
+      const uint32_t o0 = half * kRowTileBytes + ptx::sw128_offset((uint32_t)row, e0);
+      const uint32_t o1 = half * kRowTileBytes + ptx::sw128_offset((uint32_t)row, e0 + 8);
       ptx::st_shared_v4(sbase + kDSOff + o0, pd[0], pd[1], pd[2], pd[3]);
       ptx::st_shared_v4(sbase + kDSOff + o1, pd[4], pd[5], pd[6], pd[7]);
       ptx::st_shared_v4(sbase + kPWOff + o0, pw[0], pw[1], pw[2], pw[3]);
@@ -294,12 +307,18 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
   if (ok) {
     ptx::tc_fence_after();
     flush_plane(nplanes - 1);
-    uint32_t r[kDh];
-    ptx::tmem_ld64_sync(trow + kColDQ, r);
+    constexpr int kQCols = kDh / kWG;             // 64, 32 or 16 columns of dQ per warpgroup
+    uint32_t r[kQCols];
+    if constexpr (kQCols == 64)
+      ptx::tmem_ld64_sync(trow + kColDQ, r);
+    else if constexpr (kQCols == 32)
+      ptx::tmem_ld32_sync(trow + kColDQ + wg * 32, r);
+    else
+      ptx::tmem_ld16_sync(trow + kColDQ + wg * 16, r);
     if (qi >= 0) {
-      float4* dst = reinterpret_cast<float4*>(a.dqr + orow * kDh);
+      float4* dst = reinterpret_cast<float4*>(a.dqr + orow * kDh + wg * kQCols);
 #pragma unroll
-      for (int q = 0; q < kDh / 4; ++q) {
+      for (int q = 0; q < kQCols / 4; ++q) {
         float4 v = dst[q];
         v.x = fmaf(a.scale, __uint_as_float(r[4 * q]), v.x);
         v.y = fmaf(a.scale, __uint_as_float(r[4 * q + 1]), v.y);

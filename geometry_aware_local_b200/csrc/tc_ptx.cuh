@@ -210,6 +210,20 @@ __device__ __forceinline__ void tmem_ld48_sync(uint32_t taddr, uint32_t* r) {
       : "r"(taddr)
       : "memory");
 }
+// Two 16-column loads from different column ranges in flight, then one wait.
+__device__ __forceinline__ void tmem_ld16x2_sync(uint32_t taddr0, uint32_t taddr1, uint32_t* r0, uint32_t* r1) {
+  uint32_t* r = r0;
+  uint32_t* s = r1;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, "
+      "[%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : P3_R16(0), "=r"(s[0]), "=r"(s[1]), "=r"(s[2]), "=r"(s[3]), "=r"(s[4]), "=r"(s[5]), "=r"(s[6]), "=r"(s[7]),
+        "=r"(s[8]), "=r"(s[9]), "=r"(s[10]), "=r"(s[11]), "=r"(s[12]), "=r"(s[13]), "=r"(s[14]), "=r"(s[15])
+      : "r"(taddr0), "r"(taddr1)
+      : "memory");
+}
 // Two 32-column loads from different column ranges (taddr0, taddr1) in
 // flight, then one wait: r0 <- taddr0 .. +31, r1 <- taddr1 .. +31.
 __device__ __forceinline__ void tmem_ld32x2_sync(uint32_t taddr0, uint32_t taddr1, uint32_t* r0, uint32_t* r1) {
