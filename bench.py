@@ -1,14 +1,17 @@
 """Benchmark of the PACK3D forward pass on B200: tokens/s, per-stage roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config 65k|262k|1m|stress|...]
-                    [--impl ours|reference] [--train-only]
+                    [--impl ours|reference] [--train-only] [--flush write-read|write]
 
 One step = one pass of the whole hot path over one synthetic volume: index
-map, axial RoPE on Q and K_loc, block summaries, local attention, query x
+map, block summaries, axial RoPE on Q and K_loc, local attention, query x
 summary attention with the gate.  The timed step calls the C ABI stage entry
 points in the order pack3d_forward runs them, with CUDA events between stages
 on the launching stream, so each kernel's live duration is known.  L2 is
-flushed (a 256 MiB write) between steps, outside the timed events.  ``e2e``
+flushed between steps, outside the timed events: a 256 MiB write, then a
+256 MiB read of another buffer, so that no input is left in L2 and none of
+the flush's dirty lines is written back inside a timed kernel (``--flush
+write`` drops the read).  ``e2e``
 times pack3d_forward_host, the C-ABI call that takes pinned host buffers
 (inputs copied in and the output copied out inside the timed region, the
 copies overlapped with the stages by the library).
@@ -55,7 +58,7 @@ WORKLOAD_TEXT = {
     "stress": "16x64x64 lattice (65,536 tokens), raster packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=4,096), window 3x7x7 (the repacking stress case)",
     "allen": "32x128x64 lattice (262,144 tokens; the shape of the Allen WTC-11 token grid, synthetic values), block-contiguous packing, bf16, Hq=8, Hkv=2, d_h=64, blocks 1x4x4 (M=16,384), window 3x7x7",
 }
-STAGES = ("index", "rope", "summaries", "local", "summary_attn")
+STAGES = ("index", "summaries", "rope", "local", "summary_attn")
 KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summary attention
 # DRAM bytes (read + write) of one summary_attn_tc_kernel launch, from an ncu
 # capture of this workload (profiles/summary_attn_tc_65k.md; at 65k tokens the
@@ -325,6 +328,32 @@ def dense_sdpa_ms(s, q_rot, k_rot, v, stream, reps: int = 2) -> Dict:
             "what": "torch scaled_dot_product_attention (flash backend), bf16, all N x N pairs, kv heads repeated"}
 
 
+class L2Flush:
+    """Empties L2 between timed steps (outside the timed events): a 256 MiB
+    write and, in the default mode, a 256 MiB read of a second buffer, which
+    evicts the write's dirty lines so their write-back is not charged to the
+    first timed kernel."""
+
+    TEXT = {"write-read": "flushed between steps (256 MiB write, then a 256 MiB read; outside the timed events)",
+            "write": "flushed between steps (256 MiB write; outside the timed events)"}
+
+    def __init__(self, dev, mode: str):
+        import torch
+        self.mode = mode
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.rd = torch.zeros(64 << 20, dtype=torch.int32, device=dev) if mode == "write-read" else None
+
+    def __call__(self):
+        import torch
+        self.buf.zero_()
+        if self.rd is not None:
+            torch.sum(self.rd, dtype=torch.int64)
+
+    @property
+    def text(self) -> str:
+        return self.TEXT[self.mode]
+
+
 def time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world, rank, dev,
                         device_dout: bool = False) -> Dict:
     """pack3d_forward_backward on the resident inputs: W untimed calls, then K
@@ -341,7 +370,7 @@ def time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world
     tws = torch.empty(p3.train_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
     evs = []
     for k in range(args.warmup + args.steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         p3.forward_backward(cfg, d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
@@ -355,7 +384,7 @@ def time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world
     ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
     return {"ms_per_step": ms, "tokens_per_s": replica_value(s.N, world, ms),
             "call": "pack3d_forward_backward (forward saving statistics + every input gradient)",
-            "dout": "N(0,1) per lattice site", "l2": "flushed between calls (outside the timed events)"}
+            "dout": "N(0,1) per lattice site", "l2": flush.text}
 
 
 def run_train_only(args, s):
@@ -369,7 +398,7 @@ def run_train_only(args, s):
     torch.cuda.set_device(dev)
     cfg = p3.config_from_shape(s)
     d = synth.make_inputs_on_device(s, s.packing, seed=rank, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev, args.flush)
     err = torch.zeros(4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     barrier(world)
@@ -416,7 +445,7 @@ def run_ours(args, s):
     vs = torch.empty_like(ks)
     ol = torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device=dev)
     out = torch.empty_like(d["q"])
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev, args.flush)
     stream = torch.cuda.current_stream(dev)
 
     lib = p3.lib
@@ -430,10 +459,10 @@ def run_ours(args, s):
         ev[0].record(stream)
         st = lib.pack3d_build_index(cfgp, P(d["coords"]), P(g2p), P(mem), P(err), sh)
         ev[1].record(stream)
-        st |= lib.pack3d_rope_qk(cfgp, P(d["coords"]), P(d["q"]), P(qr), P(d["k_loc"]), P(kr), sh)
-        ev[2].record(stream)
         st |= lib.pack3d_build_summaries(cfgp, P(mem), P(d["k_cmp"]), P(d["v_cmp"]), P(d["scores"]), P(ks),
                                          P(vs), sh)
+        ev[2].record(stream)
+        st |= lib.pack3d_rope_qk(cfgp, P(d["coords"]), P(d["q"]), P(qr), P(d["k_loc"]), P(kr), sh)
         ev[3].record(stream)
         st |= lib.pack3d_local_attn(cfgp, P(g2p), P(qr), P(kr), P(d["v_loc"]), P(ol), P(err), sh)
         ev[4].record(stream)
@@ -454,7 +483,7 @@ def run_ours(args, s):
     barrier(world)
     with ClockSampler(local) as clk:
         for k in range(args.steps):
-            flush.zero_()
+            flush()
             step(evs[k])
         barrier(world)
     st_ms = {name: 0.0 for name in STAGES}
@@ -473,7 +502,7 @@ def run_ours(args, s):
     ws = torch.empty(p3.workspace_bytes(cfg), dtype=torch.uint8, device=dev)
     fwd_ms = []
     for k in range(args.warmup + args.steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         p3.forward(cfg, d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
@@ -496,7 +525,7 @@ def run_ours(args, s):
     pipe = p3.Pipeline()
     e2e = []
     for k in range(args.warmup + args.steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         p3.forward_host(pipe, cfg, hin["coords"], hin["q"], hin["k_loc"], hin["v_loc"], hin["k_cmp"],
@@ -550,7 +579,7 @@ def run_ours(args, s):
                        "parallelism": "replicas only" if world > 1 else "single GPU",
                        "summary_form": "summary-centre variant" if args.summary_center
                        else "rotate-before-compress (exact)",
-                       "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+                       "l2": flush.text},
             "e2e": {"value": s.N * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
@@ -593,6 +622,8 @@ def main():
     ap.add_argument("--config", default="65k", choices=sorted(WORKLOAD_TEXT))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush", default="write-read", choices=sorted(L2Flush.TEXT),
+                    help="L2 flush between steps: a write then a read (default), or the write alone")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparator at 1M")
     ap.add_argument("--train", action="store_true",
                     help="also time the training block on the device-drawn 4m / 8m volumes")

@@ -193,7 +193,7 @@ pack3d_status pack3d_summary_attn(const pack3d_config *cfg, const void *q_rot,
                                   const float *gate, void *out, int32_t *err_word,
                                   void *stream);
 
-/* The whole forward pass: index map, RoPE on Q and K_loc, summaries, local
+/* The whole forward pass: index map, summaries, RoPE on Q and K_loc, local
  * branch, query-summary branch with the gate, all stream-ordered on `stream`.
  * workspace: device buffer of at least pack3d_workspace_bytes(cfg) bytes,
  * 256-byte aligned; its contents on entry do not matter.  err_word: device int32
