@@ -68,6 +68,14 @@ CASES = [
     ("simt-forward-bf16", small(), "random", 0x3),                # CUDA-core forward kernels on bf16
     ("coords-scaled-f32", small(dtype="f32", value_scale=1.0, coord_scale=(2.5, 0.5, 1.0)), "random", 0),
     ("z-light-bf16", small(m_z=6, m_y=13, m_x=13), "block", 0),
+    # degenerate volumes with M >= 2 and blocks of >= 2 members (with one summary,
+    # or one member per block, dk~ and dscores are zero by the softmax's invariance
+    # and a tolerance relative to them is meaningless): two blocks whose window
+    # covers nearly the whole volume, a one-row line, a column of 4x4 planes
+    ("two-blocks-bf16", small(Z=1, H=4, W=8), "block", 0),
+    ("two-blocks-f32", small(Z=1, H=4, W=8, dtype="f32", value_scale=1.0), "raster", 0),
+    ("line-1x1x64-bf16", small(Z=1, H=1, W=64, by=1, bx=4), "morton", 0),
+    ("z-column-bf16", small(Z=16, H=4, W=4), "random", 0),
 ]
 
 

@@ -100,6 +100,14 @@ STAGE_CASES = [
     ("z-rescaled-f32", small(dtype="f32", value_scale=1.0, coord_scale=(2.5, 1.0, 1.0)), "random"),
     ("z-light", small(m_z=6, m_y=13, m_x=13), "block_morton"),
     ("z-heavy", small(m_z=16, m_y=8, m_x=8), "random"),
+    # degenerate volumes: one block (M = 1, so every query's summary softmax has a
+    # single term, and the 3x7x7 window covers the whole 1x4x4 volume), one token,
+    # a one-row line (the y window clipped to a single row), a column of 4x4 planes
+    ("one-block-bf16", small(Z=1, H=4, W=4), "random"),
+    ("one-block-f32", small(Z=1, H=4, W=4, dtype="f32", value_scale=1.0), "raster"),
+    ("one-token", small(Z=1, H=1, W=1, bz=1, by=1, bx=1), "raster"),
+    ("line-1x1x64", small(Z=1, H=1, W=64, by=1, bx=4), "morton"),
+    ("z-column", small(Z=16, H=4, W=4), "random"),
 ]
 
 
