@@ -54,6 +54,10 @@ namespace {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// A lattice with a zero extent holds no token: every entry point returns at
+// once, before reading a pointer or launching anything.
+bool empty_volume(const pack3d_config& c) { return c.Z == 0 || c.H == 0 || c.W == 0; }
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int elem_bytes(int dtype) { return dtype == PACK3D_BF16 ? 2 : 4; }
@@ -149,7 +153,7 @@ pack3d_status pack3d_validate_config(const pack3d_config* c) {
   if (!c) return PACK3D_ERR_INVALID_ARG;
   if (c->reserved0 != 0 || c->reserved1 != 0) return PACK3D_ERR_INVALID_ARG;
   if (c->dtype != PACK3D_F32 && c->dtype != PACK3D_BF16) return PACK3D_ERR_DTYPE;
-  if (c->Z <= 0 || c->H <= 0 || c->W <= 0) return PACK3D_ERR_SHAPE;
+  if (c->Z < 0 || c->H < 0 || c->W < 0) return PACK3D_ERR_SHAPE;   // a zero extent is an empty volume
   const long long N = (long long)c->Z * c->H * c->W;
   if (N >= (1LL << 31) / 128) return PACK3D_ERR_SHAPE;  // keeps every element index in 32 bits
   if (c->d_h != kDh) return PACK3D_ERR_SHAPE;
@@ -182,6 +186,7 @@ pack3d_status pack3d_build_index(const pack3d_config* cfg, const int32_t* coords
                                  int32_t* members, int32_t* err_word, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!coords || !g2p || !members || !err_word) return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(coords) || !aligned16(g2p) || !aligned16(members)) return PACK3D_ERR_ALIGNMENT;
   const Shape s = make_shape(*cfg);
@@ -192,6 +197,7 @@ pack3d_status pack3d_rope(const pack3d_config* cfg, const int32_t* coords, const
                           int32_t heads, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!coords || !x || !y || heads <= 0) return PACK3D_ERR_INVALID_ARG;
   if ((long long)cfg->Z * cfg->H * cfg->W * heads >= (1LL << 31) / 16) return PACK3D_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(y)) return PACK3D_ERR_ALIGNMENT;
@@ -204,6 +210,7 @@ pack3d_status pack3d_rope_qk(const pack3d_config* cfg, const int32_t* coords, co
                              const void* k, void* k_rot, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!coords || !q || !q_rot || !k || !k_rot) return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(q_rot) || !aligned16(k) || !aligned16(k_rot)) return PACK3D_ERR_ALIGNMENT;
   const Shape s = make_shape(*cfg);
@@ -215,6 +222,7 @@ pack3d_status pack3d_build_summaries(const pack3d_config* cfg, const int32_t* me
                                      void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!members || !k_cmp || !v_cmp || !scores || !k_sum || !v_sum) return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(k_sum) || !aligned16(v_sum))
     return PACK3D_ERR_ALIGNMENT;
@@ -228,6 +236,7 @@ pack3d_status pack3d_local_attn(const pack3d_config* cfg, const int32_t* g2p, co
                                 void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!g2p || !q_rot || !k_rot || !v_loc || !o_loc) return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(q_rot) || !aligned16(k_rot) || !aligned16(v_loc) || !aligned16(o_loc))
     return PACK3D_ERR_ALIGNMENT;
@@ -241,6 +250,7 @@ pack3d_status pack3d_summary_attn(const pack3d_config* cfg, const void* q_rot, c
                                   int32_t* err_word, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!q_rot || !k_sum || !v_sum || !out || (gate && !o_loc)) return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(q_rot) || !aligned16(k_sum) || !aligned16(v_sum) || !aligned16(out) ||
       (o_loc && !aligned16(o_loc)))
@@ -260,6 +270,7 @@ pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, co
                              int32_t* err_word, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !out || !err_word)
     return PACK3D_ERR_INVALID_ARG;
   if (!workspace || ((uintptr_t)workspace & 255u)) return PACK3D_ERR_WORKSPACE;
@@ -303,6 +314,7 @@ pack3d_status pack3d_forward_backward(const pack3d_config* cfg, const int32_t* c
                                       int32_t* err_word, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !dout || !out || !dq ||
       !dk_loc || !dv_loc || !dk_cmp || !dv_cmp || !dscores || !dgate || !err_word)
     return PACK3D_ERR_INVALID_ARG;
@@ -451,6 +463,7 @@ pack3d_status pack3d_forward_host(pack3d_pipeline* pl, const pack3d_config* cfg,
                                   void* workspace, size_t workspace_bytes, int32_t* err_word, void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;
   if (!pl || !coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !out || !err_word)
     return PACK3D_ERR_INVALID_ARG;
   if (!workspace || ((uintptr_t)workspace & 255u)) return PACK3D_ERR_WORKSPACE;

@@ -81,6 +81,8 @@ cudaError_t scratch_address(uint8_t** out) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+bool empty_volume(const pack3d_config& c) { return c.Z == 0 || c.H == 0 || c.W == 0; }
+
 }  // namespace
 
 using namespace pack3d;
@@ -92,6 +94,7 @@ extern "C" pack3d_status pack3d_forward_noalloc(const pack3d_config* cfg, const 
                                                 void* stream) {
   pack3d_status st = pack3d_validate_config(cfg);
   if (st != PACK3D_OK) return st;
+  if (empty_volume(*cfg)) return PACK3D_OK;   // no token: nothing to read or launch
   if (!coords || !q || !k_loc || !v_loc || !k_cmp || !v_cmp || !scores || !gate || !out)
     return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(coords) || !aligned16(q) || !aligned16(k_loc) || !aligned16(v_loc) || !aligned16(k_cmp) ||

@@ -48,7 +48,11 @@
  *   two <= 8; 2*(m_z+m_y+m_x) <= 64; block dims dividing the lattice, block
  *   volume <= 64; lattice extents small enough that the per-axis cos/sin
  *   tables (Z*m_z + H*m_y + W*m_x entries) fit 96 KiB of shared memory;
- *   N < 2^31.
+ *   N < 2^24 (16,777,216 tokens).
+ * - Empty volumes: a lattice with Z, H or W equal to 0 (N = 0) is valid.  Every
+ *   entry point then returns PACK3D_OK at once, without reading any pointer
+ *   (NULL is fine) or launching anything, and the workspace sizes are those
+ *   of no token.
  */
 #ifndef PACK3D_H
 #define PACK3D_H

@@ -49,12 +49,41 @@ def test_default_config_matches_pages(p3):
     ("d_h", 128, 2), ("Hq", 6, 2), ("Hkv", 3, 2), ("W", 63, 2), ("bx", 0, 2), ("rz", -1, 2),
     ("m_z", 20, 2), ("dtype", 7, 4), ("softmax_scale", 0.0, 1), ("flags", 0x100, 1), ("reserved0", 1, 1),
     ("flags", 0x8, 1),
-    ("rope_base", -1.0, 1), ("Z", 0, 2),
+    ("rope_base", -1.0, 1), ("Z", -1, 2), ("W", -4, 2),
 ])
 def test_validate_rejects(p3, field, value, status):
     c = p3.make_config(16, 64, 64)
     setattr(c, field, value)
     assert p3.validate(c) == status
+
+
+@pytest.mark.parametrize("dims", [(0, 64, 64), (16, 0, 64), (16, 64, 0), (0, 0, 0)])
+def test_empty_volume_is_a_no_op(p3, dims):
+    """A lattice with a zero extent holds no token: it validates, needs no
+    workspace, and every entry point returns PACK3D_OK before reading a pointer
+    (all NULL here) or touching the device."""
+    c = p3.make_config(*dims)
+    assert p3.validate(c) == 0 and c.N == 0 and c.M == 0
+    assert p3.workspace_bytes(c) == 0
+    assert p3.train_workspace_bytes(c) == 0
+    assert p3.host_workspace_bytes(c) == 0
+    cp, L = ctypes.byref(c), p3.lib
+    assert L.pack3d_build_index(cp, None, None, None, None, None) == 0
+    assert L.pack3d_rope(cp, None, None, None, 8, None) == 0
+    assert L.pack3d_rope_qk(cp, None, None, None, None, None, None) == 0
+    assert L.pack3d_build_summaries(cp, None, None, None, None, None, None, None) == 0
+    assert L.pack3d_local_attn(cp, None, None, None, None, None, None, None) == 0
+    assert L.pack3d_summary_attn(cp, None, None, None, None, None, None, None, None) == 0
+    assert L.pack3d_forward(cp, *[None] * 10, 0, None, None) == 0
+    assert L.pack3d_forward_noalloc(cp, *[None] * 11) == 0
+    assert L.pack3d_forward_host(None, cp, *[None] * 10, 0, None, None) == 0
+    assert L.pack3d_forward_backward(cp, *[None] * 18, 0, None, None) == 0
+
+
+def test_volume_size_limit(p3):
+    """N = Z*H*W must stay below 2^24 tokens."""
+    assert p3.validate(p3.make_config(255, 256, 256)) == 0      # 16,711,680 tokens
+    assert p3.validate(p3.make_config(256, 256, 256)) == 2      # 2^24
 
 
 def test_table_limit_and_sizes(p3):

@@ -225,6 +225,39 @@ def test_forward_host_equals_forward(p3, name):
     pipe.close()
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_empty_volume(p3, dtype):
+    """N = 0 (a zero lattice extent): the forward op, the host-buffer pipeline and
+    the differentiable op return empty outputs and empty gradients, status OK."""
+    cfg = p3.make_config(0, 64, 64, dtype=dtype)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    dev = "cuda"
+    coords = torch.empty(0, 3, dtype=torch.int32, device=dev)
+    q = torch.empty(0, 8, 64, dtype=tdt, device=dev)
+    kv = [torch.empty(0, 2, 64, dtype=tdt, device=dev) for _ in range(4)]
+    scores = torch.empty(0, 2, dtype=torch.float32, device=dev)
+    gate = torch.empty(0, 8, 2, dtype=torch.float32, device=dev)
+    op = p3.Pack3D(cfg, dev)
+    out = op(coords, q, *kv, scores, gate)
+    op.check()
+    assert out.shape == (0, 8, 64)
+
+    hin = [t.cpu().pin_memory() for t in (coords, q, *kv, scores, gate)]
+    hout = torch.empty(0, 8, 64, dtype=tdt).pin_memory()
+    ws = torch.empty(p3.host_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    err = torch.zeros(4, dtype=torch.int32, device=dev)
+    pipe = p3.Pipeline()
+    p3.forward_host(pipe, cfg, *hin, hout, ws, err)
+    pipe.close()
+    assert p3.check_status(err) == 0
+
+    leaves = [t.clone().requires_grad_(True) for t in (q, *kv, scores, gate)]
+    y = p3.attention(cfg, coords, *leaves)
+    y.float().sum().backward()
+    for t in leaves:
+        assert t.grad is not None and t.grad.shape == t.shape
+
+
 @pytest.mark.parametrize("name", ["small", "65k"])
 def test_forward_is_deterministic(p3, name):
     # Every kernel computes each output from a fixed sequence of operations, so
