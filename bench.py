@@ -60,10 +60,10 @@ WORKLOAD_TEXT = {
 }
 STAGES = ("index", "summaries", "rope", "local", "summary_attn")
 KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summary attention
-# DRAM bytes (read + write) of one summary_attn_tc_kernel launch, from an ncu
-# capture of this workload (profiles/summary_attn_tc_65k.md; at 65k tokens the
-# one-tile build runs).  Emptied whenever that kernel changes until it is
-# captured again.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# summary_attn_tc_kernel launch, from an ncu capture of the 65k workload (where
+# the one-tile build runs); the summary of that capture is kept under
+# profiles/.  Emptied whenever that kernel changes until it is captured again.
 SUMMARY_ATTN_TRAFFIC = {"65k": 212.771072e6 + 48.423168e6}
 
 # Launches at least this long are rated against the sustained bf16 peak.
@@ -87,7 +87,10 @@ def mean_window(s) -> float:
 
 
 def algorithmic_work(s):
-    """Per-launch algorithmic bytes / flops of each stage (the design doc derives them)."""
+    """Per-launch algorithmic bytes / flops of each stage: the bytes every stage
+    must read and write once (inputs, outputs, the o_loc hand-over) and the
+    useful flops of the two attention branches (4 d per query-key pair and
+    head; w̄ = the mean clipped window size)."""
     eb = 2 if s.dtype == "bf16" else 4
     d = s.d_h
     N, M = s.N, s.M
