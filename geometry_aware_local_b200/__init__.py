@@ -157,6 +157,57 @@ def _ptr(t) -> Optional[int]:
     return t.data_ptr()
 
 
+# Element type and element count of every tensor argument, from the layouts of
+# include/pack3d.h: "T" is the operator's dtype (config.dtype).
+_LAYOUT = {
+    "coords": ("i32", lambda c: c.N * 3),
+    "q": ("T", lambda c: c.N * c.Hq * c.d_h),          # also q_rot, out, dout, dq
+    "kv": ("T", lambda c: c.N * c.Hkv * c.d_h),        # k_loc, v_loc, k_cmp, v_cmp, k_rot and their gradients
+    "scores": ("f32", lambda c: c.N * c.Hkv),
+    "gate": ("f32", lambda c: c.N * c.Hq * 2),
+    "g2p": ("i32", lambda c: c.N),
+    "members": ("i32", lambda c: c.M * c.v),
+    "sum": ("T", lambda c: c.M * c.Hkv * c.d_h),       # k_sum, v_sum
+    "o_loc": ("f32", lambda c: c.N * c.Hq * c.d_h),
+}
+
+
+def _check_layout(what: str, cfg, **tensors):
+    """Refuses, before anything runs, a tensor whose element type or element count
+    does not match the config: the kernels trust the sizes the config implies,
+    so a short buffer would be read or written out of bounds.  Arguments are
+    given as kind=(name, tensor); None (a nullable argument) and raw integer
+    pointers are not checked.  An invalid config is left to the C ABI to report."""
+    import torch
+    if validate(cfg) != 0:
+        return
+    types = {"T": torch.bfloat16 if cfg.dtype == BF16 else torch.float32, "f32": torch.float32,
+             "i32": torch.int32}
+    for kind, items in tensors.items():
+        base = kind.rstrip("0123456789")
+        if base == "rope":                      # x / y of pack3d_rope: T [N, heads, d_h]
+            heads = items[0]
+            items = items[1:]
+            dt, count = types["T"], cfg.N * heads * cfg.d_h
+        else:
+            code, size = _LAYOUT[base]
+            dt, count = types[code], size(cfg)
+        for name, t in items:
+            if t is None or isinstance(t, int):
+                continue
+            if t.dtype != dt:
+                raise ValueError(f"{what}: {name} must be {dt}, got {t.dtype}")
+            if t.numel() != count:
+                raise ValueError(f"{what}: {name} must hold {count} elements for this config, "
+                                 f"got {t.numel()} (shape {tuple(t.shape)})")
+
+
+def _check_err(what: str, err):
+    import torch
+    if err is not None and not isinstance(err, int) and (err.dtype != torch.int32 or err.numel() < 1):
+        raise ValueError(f"{what}: the error word must be an int32 tensor of at least one element")
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         import torch
@@ -170,37 +221,59 @@ def _check(st: int, what: str):
 
 
 def build_index(cfg, coords, g2p, members, err, stream=None):
+    _check_layout("build_index", cfg, coords=[("coords", coords)], g2p=[("g2p", g2p)],
+                  members=[("members", members)])
+    _check_err("build_index", err)
     _check(lib.pack3d_build_index(ctypes.byref(cfg), _ptr(coords), _ptr(g2p), _ptr(members), _ptr(err),
                                   _stream(stream)), "pack3d_build_index")
 
 
 def rope(cfg, coords, x, y, heads: int, stream=None):
+    _check_layout("rope", cfg, coords=[("coords", coords)], rope=[heads, ("x", x), ("y", y)])
     _check(lib.pack3d_rope(ctypes.byref(cfg), _ptr(coords), _ptr(x), _ptr(y), heads, _stream(stream)),
            "pack3d_rope")
 
 
 def rope_qk(cfg, coords, q, q_rot, k, k_rot, stream=None):
+    _check_layout("rope_qk", cfg, coords=[("coords", coords)], q=[("q", q), ("q_rot", q_rot)],
+                  kv=[("k", k), ("k_rot", k_rot)])
     _check(lib.pack3d_rope_qk(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(q_rot), _ptr(k), _ptr(k_rot),
                               _stream(stream)), "pack3d_rope_qk")
 
 
 def build_summaries(cfg, members, k_cmp, v_cmp, scores, k_sum, v_sum, stream=None):
+    _check_layout("build_summaries", cfg, members=[("members", members)], kv=[("k_cmp", k_cmp), ("v_cmp", v_cmp)],
+                  scores=[("scores", scores)], sum=[("k_sum", k_sum), ("v_sum", v_sum)])
     _check(lib.pack3d_build_summaries(ctypes.byref(cfg), _ptr(members), _ptr(k_cmp), _ptr(v_cmp),
                                       _ptr(scores), _ptr(k_sum), _ptr(v_sum), _stream(stream)),
            "pack3d_build_summaries")
 
 
 def local_attn(cfg, g2p, q_rot, k_rot, v_loc, o_loc, err=None, stream=None):
+    _check_layout("local_attn", cfg, g2p=[("g2p", g2p)], q=[("q_rot", q_rot)], kv=[("k_rot", k_rot), ("v_loc", v_loc)],
+                  o_loc=[("o_loc", o_loc)])
+    _check_err("local_attn", err)
     _check(lib.pack3d_local_attn(ctypes.byref(cfg), _ptr(g2p), _ptr(q_rot), _ptr(k_rot), _ptr(v_loc),
                                  _ptr(o_loc), _ptr(err), _stream(stream)), "pack3d_local_attn")
 
 
 def summary_attn(cfg, q_rot, k_sum, v_sum, o_loc, gate, out, err=None, stream=None):
+    _check_layout("summary_attn", cfg, q=[("q_rot", q_rot), ("out", out)], sum=[("k_sum", k_sum), ("v_sum", v_sum)],
+                  o_loc=[("o_loc", o_loc)], gate=[("gate", gate)])
+    _check_err("summary_attn", err)
     _check(lib.pack3d_summary_attn(ctypes.byref(cfg), _ptr(q_rot), _ptr(k_sum), _ptr(v_sum), _ptr(o_loc),
                                    _ptr(gate), _ptr(out), _ptr(err), _stream(stream)), "pack3d_summary_attn")
 
 
+def _check_forward_args(what, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err):
+    _check_layout(what, cfg, coords=[("coords", coords)], q=[("q", q), ("out", out)],
+                  kv=[("k_loc", k_loc), ("v_loc", v_loc), ("k_cmp", k_cmp), ("v_cmp", v_cmp)],
+                  scores=[("scores", scores)], gate=[("gate", gate)])
+    _check_err(what, err)
+
+
 def forward(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, workspace, err, stream=None):
+    _check_forward_args("forward", cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.pack3d_forward(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc), _ptr(k_cmp),
                               _ptr(v_cmp), _ptr(scores), _ptr(gate), _ptr(out), _ptr(workspace), ws_bytes,
@@ -210,6 +283,7 @@ def forward(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, works
 def forward_noalloc(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err=None, stream=None):
     """pack3d_forward with the library's built-in scratch array instead of a workspace (for
     callers that cannot allocate device memory); see include/pack3d.h for its limit and rules."""
+    _check_forward_args("forward_noalloc", cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err)
     _check(lib.pack3d_forward_noalloc(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc),
                                       _ptr(k_cmp), _ptr(v_cmp), _ptr(scores), _ptr(gate), _ptr(out), _ptr(err),
                                       _stream(stream)), "pack3d_forward_noalloc")
@@ -248,6 +322,7 @@ def forward_host(pipeline, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, g
                  stream=None):
     """pack3d_forward from host tensors (inputs and `out`), copies overlapped with the stages; the result
     is in `out` once the stream is synchronised."""
+    _check_forward_args("forward_host", cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.pack3d_forward_host(pipeline.handle, ctypes.byref(cfg), _host_ptr(coords), _host_ptr(q),
                                    _host_ptr(k_loc), _host_ptr(v_loc), _host_ptr(k_cmp), _host_ptr(v_cmp),
@@ -266,6 +341,10 @@ def forward_backward(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, d
                      stream=None):
     """pack3d_forward_backward: the forward output into `out` and the gradients of <dout, out> into the
     tensors of the dict `grads` (keys GRAD_NAMES, shapes and dtypes of the matching inputs)."""
+    _check_forward_args("forward_backward", cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err)
+    _check_layout("forward_backward", cfg, q=[("dout", dout), ("dq", grads["dq"])],
+                  kv=[(k, grads[k]) for k in ("dk_loc", "dv_loc", "dk_cmp", "dv_cmp")],
+                  scores=[("dscores", grads["dscores"])], gate=[("dgate", grads["dgate"])])
     ws_bytes = workspace.numel() * workspace.element_size()
     g = [grads[k] for k in GRAD_NAMES]
     _check(lib.pack3d_forward_backward(ctypes.byref(cfg), _ptr(coords), _ptr(q), _ptr(k_loc), _ptr(v_loc),

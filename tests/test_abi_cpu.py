@@ -133,6 +133,45 @@ def test_binding_refuses_host_tensors(p3):
         p3.rope(c, torch.zeros(256, 3, dtype=torch.int32), x, x, 2, stream=0)
 
 
+def test_binding_checks_layouts_before_anything_runs(p3):
+    """A tensor whose element type or count does not match the config is refused by
+    the binding before any pointer reaches the library (the kernels trust the
+    sizes the config implies)."""
+    import torch
+    c = p3.make_config(4, 8, 8, Hq=2, Hkv=1, radius=(1, 1, 1), dtype="f32")   # N = 256, M = 16
+    N, M = 256, 16
+
+    def f(*shape, dt=torch.float32):
+        return torch.zeros(*shape, dtype=dt)
+
+    good = dict(coords=f(N, 3, dt=torch.int32), q=f(N, 2, 64), k_loc=f(N, 1, 64), v_loc=f(N, 1, 64),
+                k_cmp=f(N, 1, 64), v_cmp=f(N, 1, 64), scores=f(N, 1), gate=f(N, 2, 2))
+    out, err, ws = f(N, 2, 64), f(4, dt=torch.int32), torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):        # well-formed: stopped only by the device check
+        p3.forward(c, *good.values(), out, ws, err)
+    for name, t, msg in [("q", f(N - 1, 2, 64), "elements"), ("k_cmp", f(N, 2, 64), "elements"),
+                         ("scores", f(N, 1, dt=torch.float64), "float32"), ("coords", f(N, 3), "int32"),
+                         ("gate", f(N, 2), "elements"), ("v_loc", f(N, 1, 64, dt=torch.bfloat16), "float32")]:
+        args = dict(good, **{name: t})
+        with pytest.raises(ValueError, match=msg):
+            p3.forward(c, *args.values(), out, ws, err)
+    with pytest.raises(ValueError, match="out"):
+        p3.forward(c, *good.values(), f(N, 2, 63), ws, err)
+    with pytest.raises(ValueError, match="error word"):
+        p3.forward(c, *good.values(), out, ws, f(4))
+    with pytest.raises(ValueError, match="members"):
+        p3.build_index(c, good["coords"], f(N, dt=torch.int32), f(M, 8, dt=torch.int32), err)
+    with pytest.raises(ValueError, match="k_sum"):
+        p3.build_summaries(c, f(M, 16, dt=torch.int32), good["k_cmp"], good["v_cmp"], good["scores"],
+                           f(M - 1, 1, 64), f(M, 1, 64))
+    with pytest.raises(ValueError, match="y"):
+        p3.rope(c, good["coords"], good["q"], f(N, 1, 64), 2)
+    grads = p3.empty_grads(good["q"], good["k_loc"], good["scores"], good["gate"])
+    grads["dgate"] = f(N, 2, 1)
+    with pytest.raises(ValueError, match="dgate"):
+        p3.forward_backward(c, *good.values(), f(N, 2, 64), out, grads, ws, err)
+
+
 def test_forward_backward_host_errors(p3):
     c = p3.make_config(16, 64, 64)
     lib = p3.lib
