@@ -5,6 +5,22 @@ declared in ``include/pack3d.h`` ("Geometry Matters in Packed 3D Attention",
 Key designs 1-3).  Tensors must be CUDA, contiguous and 16-byte aligned; calls
 are asynchronous on torch's current stream.  There is no CPU fallback: if the
 library was not built, importing the binding raises.
+
+Typical use (packed order throughout; coords are each token's lattice site)::
+
+    import geometry_aware_local_b200 as p3
+    cfg = p3.make_config(Z, H, W)    # Hq=8, Hkv=2, d_h=64, 1x4x4 blocks, 3x7x7 window, bf16
+    # coords int32 [N,3]; q [N,8,64]; k_loc, v_loc, k_cmp, v_cmp [N,2,64] (bf16);
+    # scores float [N,2]; gate float [N,8,2]
+    out = p3.attention(cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate)
+    out.backward(dout)               # gradients of every float input
+
+``Pack3D(cfg)`` runs the forward pass with a workspace it keeps;
+``forward`` / ``forward_backward`` / ``forward_host`` take caller-owned
+buffers; the stage entry points (``build_index``, ``rope_qk``,
+``build_summaries``, ``local_attn``, ``summary_attn``) run one stage each.
+Every wrapper checks its tensors' dtypes and element counts against the
+config before calling the library.
 """
 from __future__ import annotations
 
