@@ -36,6 +36,9 @@ F32, BF16 = 0, 1
 FLAG_SIMT_SUMMARY = 0x1
 FLAG_SIMT_LOCAL = 0x2
 FLAG_SUMMARY_CENTER = 0x4     # summary-centre variant of the block summaries (include/pack3d.h)
+FLAG_DIAG_STALL = 0x8         # diagnostic: each tensor-core kernel withholds one pipeline step (timeout path)
+FLAG_SUMMARY_ONE_TILE = 0x10  # force the one-tile build of the tensor-core query x summary kernel
+FLAG_SUMMARY_TWO_TILE = 0x20  # force the two-tile build
 DEVERR_COORD_RANGE, DEVERR_DUPLICATE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: "NOT_PERMUTATION",
@@ -64,7 +67,7 @@ class Config(ctypes.Structure):
                 ("bz", ctypes.c_int32), ("by", ctypes.c_int32), ("bx", ctypes.c_int32),
                 ("rz", ctypes.c_int32), ("ry", ctypes.c_int32), ("rx", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("flags", ctypes.c_int32), ("reserved1", ctypes.c_int32),
+                ("flags", ctypes.c_int32), ("wait_limit_us", ctypes.c_int32),
                 ("coord_scale", ctypes.c_double * 3)]
 
     @property
@@ -130,7 +133,7 @@ def make_config(Z: int, H: int, W: int, *, Hq: int = 8, Hkv: int = 2, d_h: int =
                 m: Sequence[int] = (11, 11, 10), rope_base: float = 10000.0,
                 block: Sequence[int] = (1, 4, 4), radius: Sequence[int] = (1, 3, 3),
                 softmax_scale: Optional[float] = None, dtype: str = "bf16", flags: int = 0,
-                coord_scale: Sequence[float] = (1.0, 1.0, 1.0)) -> Config:
+                coord_scale: Sequence[float] = (1.0, 1.0, 1.0), wait_limit_us: int = 0) -> Config:
     c = Config()
     c.Z, c.H, c.W = Z, H, W
     c.Hq, c.Hkv, c.d_h = Hq, Hkv, d_h
@@ -141,16 +144,17 @@ def make_config(Z: int, H: int, W: int, *, Hq: int = 8, Hkv: int = 2, d_h: int =
     c.softmax_scale = 1.0 / math.sqrt(d_h) if softmax_scale is None else softmax_scale
     c.dtype = BF16 if dtype in ("bf16", BF16) else F32
     c.flags = flags
+    c.wait_limit_us = wait_limit_us
     c.coord_scale[:] = [float(x) for x in coord_scale]
     return c
 
 
-def config_from_shape(s, flags: int = 0) -> Config:
+def config_from_shape(s, flags: int = 0, wait_limit_us: int = 0) -> Config:
     """Config from any object with the fields of ``synth.Pack3DShape``."""
     return make_config(s.Z, s.H, s.W, Hq=s.Hq, Hkv=s.Hkv, d_h=s.d_h, m=(s.m_z, s.m_y, s.m_x),
                        rope_base=s.rope_base, block=(s.bz, s.by, s.bx), radius=(s.rz, s.ry, s.rx),
                        softmax_scale=s.softmax_scale, dtype=s.dtype, flags=flags,
-                       coord_scale=getattr(s, "coord_scale", (1.0, 1.0, 1.0)))
+                       coord_scale=getattr(s, "coord_scale", (1.0, 1.0, 1.0)), wait_limit_us=wait_limit_us)
 
 
 def validate(cfg: Config) -> int:

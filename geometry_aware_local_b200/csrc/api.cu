@@ -29,6 +29,9 @@ Shape make_shape(const pack3d_config& c) {
   s.scale = c.softmax_scale;
   s.scale_log2 = (float)((double)c.softmax_scale * 1.4426950408889634);
   s.center = (c.flags & PACK3D_FLAG_SUMMARY_CENTER) ? 1 : 0;
+  s.wait_ns = c.wait_limit_us > 0 ? (unsigned long long)c.wait_limit_us * 1000ull : 2000000000ull;
+  s.stall = (c.flags & PACK3D_FLAG_DIAG_STALL) ? 1 : 0;
+  s.sa_build = (c.flags & PACK3D_FLAG_SUMMARY_ONE_TILE) ? 1 : ((c.flags & PACK3D_FLAG_SUMMARY_TWO_TILE) ? 2 : 0);
   const int m[3] = {c.m_z, c.m_y, c.m_x};
   const int ext[3] = {c.Z, c.H, c.W};
   int p = 0, off = 0;
@@ -44,6 +47,48 @@ Shape make_shape(const pack3d_config& c) {
   s.npairs = p;
   for (; p < kMaxPairs; ++p) s.pair_axis[p] = 3;
   return s;
+}
+
+ForwardWs carve_forward(const pack3d_config& c, uintptr_t base) {
+  const size_t N = (size_t)c.Z * c.H * c.W;
+  const size_t v = (size_t)c.bz * c.by * c.bx;
+  const size_t M = N / v;
+  const size_t eb = c.dtype == PACK3D_BF16 ? 2 : 4;
+  const size_t A = 1024;
+  auto up = [&](size_t x) { return (x + A - 1) / A * A; };
+  ForwardWs w;
+  size_t off = 0;
+  w.g2p = reinterpret_cast<int32_t*>(base + off);      off = up(off + N * 4);
+  w.members = reinterpret_cast<int32_t*>(base + off);  off = up(off + M * v * 4);
+  w.q_rot = reinterpret_cast<void*>(base + off);       off = up(off + N * c.Hq * c.d_h * eb);
+  w.k_rot = reinterpret_cast<void*>(base + off);       off = up(off + N * c.Hkv * c.d_h * eb);
+  w.k_sum = reinterpret_cast<void*>(base + off);       off = up(off + M * c.Hkv * c.d_h * eb);
+  w.v_sum = reinterpret_cast<void*>(base + off);       off = up(off + M * c.Hkv * c.d_h * eb);
+  w.o_loc = reinterpret_cast<float*>(base + off);      off = up(off + N * c.Hq * c.d_h * 4);
+  w.bytes = off;
+  return w;
+}
+
+cudaError_t enqueue_forward(const pack3d_config& c, const Shape& s, const ForwardWs& w, const int32_t* coords,
+                            const void* q, const void* k_loc, const void* v_loc, const void* k_cmp,
+                            const void* v_cmp, const float* scores, const float* gate, void* out, int32_t* err,
+                            cudaStream_t cs) {
+  // The summaries run before RoPE: both stream from HBM and are independent,
+  // and the summaries write 1/16 of what they read, so RoPE starts with few
+  // dirty L2 lines to evict; in the other order the summaries stage would
+  // pay for writing back RoPE's output (about 10 % of its time at 262k tokens).
+  cudaError_t e = launch_build_index(s, coords, w.g2p, w.members, err, cs);
+  if (e == cudaSuccess) e = launch_summaries(s, c.dtype, w.members, k_cmp, v_cmp, scores, w.k_sum, w.v_sum, cs);
+  if (e == cudaSuccess) e = launch_rope(s, c.dtype, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, cs);
+  if (e == cudaSuccess)
+    e = launch_local(s, c.dtype, c.flags, w.g2p, w.q_rot, w.k_rot, v_loc, w.o_loc, err, cs);
+  if (e == cudaSuccess) {
+    if (c.dtype == PACK3D_BF16 && !(c.flags & PACK3D_FLAG_SIMT_SUMMARY))
+      e = launch_summary_attn_tc(s, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, err, cs);
+    else
+      e = launch_summary_attn_simt(s, c.dtype, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, cs);
+  }
+  return e;
 }
 
 }  // namespace pack3d
@@ -68,35 +113,9 @@ pack3d_status cuda_status(cudaError_t e) {
   return PACK3D_ERR_CUDA;
 }
 
-struct Workspace {
-  int32_t* g2p;
-  int32_t* members;
-  void* q_rot;
-  void* k_rot;
-  void* k_sum;
-  void* v_sum;
-  float* o_loc;
-  size_t bytes;
-};
+typedef ForwardWs Workspace;
 
-Workspace carve(const pack3d_config& c, uintptr_t base) {
-  const size_t N = (size_t)c.Z * c.H * c.W;
-  const size_t v = (size_t)c.bz * c.by * c.bx;
-  const size_t M = N / v;
-  const size_t eb = elem_bytes(c.dtype);
-  const size_t A = 1024;
-  Workspace w;
-  size_t off = 0;
-  w.g2p = reinterpret_cast<int32_t*>(base + off);      off = round_up(off + N * 4, A);
-  w.members = reinterpret_cast<int32_t*>(base + off);  off = round_up(off + M * v * 4, A);
-  w.q_rot = reinterpret_cast<void*>(base + off);                off = round_up(off + N * c.Hq * c.d_h * eb, A);
-  w.k_rot = reinterpret_cast<void*>(base + off);                off = round_up(off + N * c.Hkv * c.d_h * eb, A);
-  w.k_sum = reinterpret_cast<void*>(base + off);                off = round_up(off + M * c.Hkv * c.d_h * eb, A);
-  w.v_sum = reinterpret_cast<void*>(base + off);                off = round_up(off + M * c.Hkv * c.d_h * eb, A);
-  w.o_loc = reinterpret_cast<float*>(base + off);      off = round_up(off + N * c.Hq * c.d_h * 4, A);
-  w.bytes = off;
-  return w;
-}
+Workspace carve(const pack3d_config& c, uintptr_t base) { return carve_forward(c, base); }
 
 // Regions of the training block after the forward workspace.
 struct TrainWs {
@@ -151,7 +170,7 @@ void pack3d_default_config(pack3d_config* cfg, int32_t Z, int32_t H, int32_t W) 
 
 pack3d_status pack3d_validate_config(const pack3d_config* c) {
   if (!c) return PACK3D_ERR_INVALID_ARG;
-  if (c->reserved0 != 0 || c->reserved1 != 0) return PACK3D_ERR_INVALID_ARG;
+  if (c->reserved0 != 0 || c->wait_limit_us < 0) return PACK3D_ERR_INVALID_ARG;
   if (c->dtype != PACK3D_F32 && c->dtype != PACK3D_BF16) return PACK3D_ERR_DTYPE;
   if (c->Z < 0 || c->H < 0 || c->W < 0) return PACK3D_ERR_SHAPE;   // a zero extent is an empty volume
   const long long N = (long long)c->Z * c->H * c->W;
@@ -172,7 +191,10 @@ pack3d_status pack3d_validate_config(const pack3d_config* c) {
     if (!(c->coord_scale[a] > 0.0) || !isfinite(c->coord_scale[a])) return PACK3D_ERR_INVALID_ARG;
   const long long tab = (long long)c->Z * c->m_z + (long long)c->H * c->m_y + (long long)c->W * c->m_x;
   if (tab * 8 > kMaxTableBytes) return PACK3D_ERR_SHAPE;
-  if (c->flags & ~(PACK3D_FLAG_SIMT_SUMMARY | PACK3D_FLAG_SIMT_LOCAL | PACK3D_FLAG_SUMMARY_CENTER))
+  if (c->flags & ~(PACK3D_FLAG_SIMT_SUMMARY | PACK3D_FLAG_SIMT_LOCAL | PACK3D_FLAG_SUMMARY_CENTER |
+                   PACK3D_FLAG_DIAG_STALL | PACK3D_FLAG_SUMMARY_ONE_TILE | PACK3D_FLAG_SUMMARY_TWO_TILE))
+    return PACK3D_ERR_INVALID_ARG;
+  if ((c->flags & PACK3D_FLAG_SUMMARY_ONE_TILE) && (c->flags & PACK3D_FLAG_SUMMARY_TWO_TILE))
     return PACK3D_ERR_INVALID_ARG;
   return PACK3D_OK;
 }
@@ -280,25 +302,8 @@ pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, co
       !aligned16(v_cmp) || !aligned16(out))
     return PACK3D_ERR_ALIGNMENT;
   const Shape s = make_shape(*cfg);
-  const cudaStream_t cs = (cudaStream_t)stream;
-  // The summaries run before RoPE: both stream from HBM and are independent,
-  // and the summaries write 1/16 of what they read, so RoPE starts with few
-  // dirty L2 lines to evict; in the other order the summaries stage would
-  // pay for writing back RoPE's output (about 10 % of its time at 262k tokens).
-  cudaError_t e = launch_build_index(s, coords, w.g2p, w.members, err_word, cs);
-  if (e == cudaSuccess)
-    e = launch_summaries(s, cfg->dtype, w.members, k_cmp, v_cmp, scores, w.k_sum, w.v_sum, cs);
-  if (e == cudaSuccess)
-    e = launch_rope(s, cfg->dtype, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, cs);
-  if (e == cudaSuccess)
-    e = launch_local(s, cfg->dtype, cfg->flags, w.g2p, w.q_rot, w.k_rot, v_loc, w.o_loc, err_word, cs);
-  if (e == cudaSuccess) {
-    if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
-      e = launch_summary_attn_tc(s, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, err_word, cs);
-    else
-      e = launch_summary_attn_simt(s, cfg->dtype, w.q_rot, w.k_sum, w.v_sum, w.o_loc, gate, out, cs);
-  }
-  return cuda_status(e);
+  return cuda_status(enqueue_forward(*cfg, s, w, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out,
+                                     err_word, (cudaStream_t)stream));
 }
 
 size_t pack3d_train_workspace_bytes(const pack3d_config* cfg) {

@@ -14,7 +14,10 @@
 //
 // Set-up: the first call on a device looks up the array's device address with
 // cudaGetSymbolAddress (with that device current) and caches it per device;
-// make that first call before any stream capture.  All calls share the one
+// make that first call before any stream capture.  The cached address belongs
+// to the device's current context: after cudaDeviceReset the module may be
+// loaded again at another address, so a process that resets a device must not
+// call this entry point on it again.  All calls share the one
 // array, so calls whose work overlaps on the GPU (for example on two streams)
 // race and must be serialised by the caller.  Each region of the scratch is
 // fully written by this call's kernels before it is read (the index maps are
@@ -36,31 +39,6 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes]
 
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
-
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-// Same regions as pack3d_forward's workspace, carved from the static array.
-struct Regions {
-  size_t g2p, members, q_rot, k_rot, k_sum, v_sum, o_loc, bytes;
-};
-
-Regions plan(const pack3d_config& c) {
-  const size_t N = (size_t)c.Z * c.H * c.W;
-  const size_t v = (size_t)c.bz * c.by * c.bx;
-  const size_t M = N / v;
-  const size_t eb = c.dtype == PACK3D_BF16 ? 2 : 4;
-  Regions r;
-  size_t off = 0;
-  r.g2p = off;     off = align_up(off + N * 4, 1024);
-  r.members = off; off = align_up(off + M * v * 4, 1024);
-  r.q_rot = off;   off = align_up(off + N * c.Hq * c.d_h * eb, 1024);
-  r.k_rot = off;   off = align_up(off + N * c.Hkv * c.d_h * eb, 1024);
-  r.k_sum = off;   off = align_up(off + M * c.Hkv * c.d_h * eb, 1024);
-  r.v_sum = off;   off = align_up(off + M * c.Hkv * c.d_h * eb, 1024);
-  r.o_loc = off;   off = align_up(off + N * c.Hq * c.d_h * 4, 1024);
-  r.bytes = off;
-  return r;
-}
 
 // Device address of the scratch array on the current device (looked up once).
 cudaError_t scratch_address(uint8_t** out) {
@@ -100,33 +78,17 @@ extern "C" pack3d_status pack3d_forward_noalloc(const pack3d_config* cfg, const 
   if (!aligned16(coords) || !aligned16(q) || !aligned16(k_loc) || !aligned16(v_loc) || !aligned16(k_cmp) ||
       !aligned16(v_cmp) || !aligned16(out))
     return PACK3D_ERR_ALIGNMENT;
-  const Regions r = plan(*cfg);
-  if (r.bytes > kNoallocScratchBytes) return PACK3D_ERR_WORKSPACE;  // volume too large for the array
+  // The same regions (and the same size check) as pack3d_forward's workspace.
+  if (carve_forward(*cfg, 0).bytes > kNoallocScratchBytes) return PACK3D_ERR_WORKSPACE;  // too large
   uint8_t* base = nullptr;
   if (scratch_address(&base) != cudaSuccess) {
     cudaGetLastError();
     return PACK3D_ERR_CUDA;
   }
-  int32_t* g2p = reinterpret_cast<int32_t*>(base + r.g2p);
-  int32_t* members = reinterpret_cast<int32_t*>(base + r.members);
-  void* q_rot = base + r.q_rot;
-  void* k_rot = base + r.k_rot;
-  void* k_sum = base + r.k_sum;
-  void* v_sum = base + r.v_sum;
-  float* o_loc = reinterpret_cast<float*>(base + r.o_loc);
-
+  const ForwardWs w = carve_forward(*cfg, (uintptr_t)base);
   const Shape s = make_shape(*cfg);
-  const cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e = launch_build_index(s, coords, g2p, members, err_word, cs);
-  if (e == cudaSuccess) e = launch_rope(s, cfg->dtype, coords, q, q_rot, s.Hq, k_loc, k_rot, s.Hkv, cs);
-  if (e == cudaSuccess) e = launch_summaries(s, cfg->dtype, members, k_cmp, v_cmp, scores, k_sum, v_sum, cs);
-  if (e == cudaSuccess) e = launch_local(s, cfg->dtype, cfg->flags, g2p, q_rot, k_rot, v_loc, o_loc, err_word, cs);
-  if (e == cudaSuccess) {
-    if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
-      e = launch_summary_attn_tc(s, q_rot, k_sum, v_sum, o_loc, gate, out, err_word, cs);
-    else
-      e = launch_summary_attn_simt(s, cfg->dtype, q_rot, k_sum, v_sum, o_loc, gate, out, cs);
-  }
+  const cudaError_t e = enqueue_forward(*cfg, s, w, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out,
+                                        err_word, (cudaStream_t)stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return PACK3D_ERR_CUDA;

@@ -32,6 +32,9 @@ struct Shape {
   int pair_axis[kMaxPairs];       // 0 = z, 1 = y, 2 = x, 3 = untouched
   int pair_off[kMaxPairs];        // first table entry of plane p
   int center;                     // summaries: rotate the pooled key at the block centre
+  unsigned long long wait_ns;     // limit of every bounded pipeline wait
+  int stall;                      // diagnostic: withhold one pipeline step (PACK3D_FLAG_DIAG_STALL)
+  int sa_build;                   // query x summary build: 0 by size, 1 one-tile, 2 two-tile
 };
 
 Shape make_shape(const pack3d_config& c);

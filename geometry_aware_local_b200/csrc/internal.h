@@ -3,11 +3,36 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
+
+#include "pack3d.h"
 
 namespace pack3d {
 
 struct Shape;
+
+// Regions of the pack3d_forward workspace, each at a 1 KiB offset from base:
+// g2p int32 [N], members int32 [M,v], q_rot, k_rot (operator dtype), k_sum,
+// v_sum [M,Hkv,64], o_loc float [N,Hq,64].  `bytes` is the total size.
+struct ForwardWs {
+  int32_t* g2p;
+  int32_t* members;
+  void* q_rot;
+  void* k_rot;
+  void* k_sum;
+  void* v_sum;
+  float* o_loc;
+  size_t bytes;
+};
+ForwardWs carve_forward(const pack3d_config& c, uintptr_t base);
+
+// The forward pass's launches, stream-ordered on st, on a carved workspace
+// (pack3d_forward and pack3d_forward_noalloc both run exactly this).
+cudaError_t enqueue_forward(const pack3d_config& c, const Shape& s, const ForwardWs& w, const int32_t* coords,
+                            const void* q, const void* k_loc, const void* v_loc, const void* k_cmp,
+                            const void* v_cmp, const float* scores, const float* gate, void* out, int32_t* err,
+                            cudaStream_t st);
 
 // Extra outputs of the forward pass when it runs as the first half of the
 // training block (pack3d_forward_backward): per (token, q head) row four

@@ -76,6 +76,8 @@ struct LocalBwdArgs {
   float* dk_acc;               // [N, Hkv, 64]: += scale * dK (rotated frame)
   float* dv_acc;               // [N, Hkv, 64]
   int32_t* err;
+  unsigned long long wait_ns;  // limit of every pipeline wait
+  int stall;                   // diagnostic: the S / dP MMAs of the last plane are never issued
 };
 
 // One 128-byte row into a 128-byte-swizzled tile at row r (zeros if src == nullptr).
@@ -111,8 +113,10 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
   const uint32_t sbase = ptx::smem_u32(smem);
   const uint32_t s_full = sbase + kBarOff;        // S and dP of the current plane are in tensor memory
   const uint32_t mma_done = sbase + kBarOff + 8;  // dQ / dK / dV MMAs of the last issued plane completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + 20);
+  const uint32_t drain = sbase + kBarOff + 16;    // abort path: every MMA issued so far has completed
+  volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + 24);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 24 + sizeof(ptx::WaitCtl));
+  auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row = tid & (kRows - 1), wg = tid >> 7;   // tensor-memory lane and warpgroup
   const int g = blockIdx.y;
@@ -129,7 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
   if (tid == 0) {
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(mma_done, 1);
-    *abort_flag = 0;
+    ptx::mbar_init(drain, 1);
+    ctl->abort = 0;
+    ctl->limit_ns = a.wait_ns;
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -246,14 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
     }
   };
 
-  if (tid == 0) issue_sdp(0);
+  // (PACK3D_FLAG_DIAG_STALL withholds the S / dP MMAs of the last plane.)
+  if (tid == 0 && !(a.stall && nplanes == 1)) issue_sdp(0);
   bool ok = true;
-  int issued = 0;   // planes whose gradient MMAs were issued
   for (int p = 0; p < nplanes; ++p) {
     const int zp = zlo + p;
     const bool uses = zp >= z0 + lz - 1 && zp <= z0 + lz + 1;   // warp-uniform (layer = warp / 2)
-    bool w_ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, p & 1, abort_flag));
-    if (w_ok && p > 0) w_ok = __all_sync(0xffffffffu, ptx::mbar_wait(mma_done, (p - 1) & 1, abort_flag));
+    bool w_ok = __all_sync(0xffffffffu, wait(s_full, p & 1));
+    if (w_ok && p > 0) w_ok = __all_sync(0xffffffffu, wait(mma_done, (p - 1) & 1));
     if (!(ok = __syncthreads_and(w_ok))) break;
     ptx::tc_fence_after();
     if (p > 0) {
@@ -298,12 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
     if (tid == 0) {
       ptx::tc_fence_after();
       issue_grads(p);
-      if (p + 1 < nplanes) issue_sdp(p + 1);
+      if (p + 1 < nplanes && !(a.stall && p + 2 == nplanes)) issue_sdp(p + 1);
     }
-    issued = p + 1;
   }
 
-  if (ok) ok = __syncthreads_and(__all_sync(0xffffffffu, ptx::mbar_wait(mma_done, (nplanes - 1) & 1, abort_flag)));
+  if (ok) ok = __syncthreads_and(__all_sync(0xffffffffu, wait(mma_done, (nplanes - 1) & 1)));
   if (ok) {
     ptx::tc_fence_after();
     flush_plane(nplanes - 1);
@@ -327,19 +332,25 @@ __global__ void __launch_bounds__(kThreads, 1) local_bwd_tc_kernel(const LocalBw
         dst[q] = v;
       }
     }
-  } else if (tid == 0) {
-    // Drain whatever was issued before tensor memory is released.
-    ptx::tc_commit(mma_done);
-    ptx::mbar_wait(mma_done, issued & 1, abort_flag);
   }
   ptx::cp_async_wait_all();
   ptx::tc_fence_before();
   __syncthreads();
+  if (ctl->abort) {
+    // The flag is final here: the MMAs thread 0 issued complete before
+    // tensor memory is released.
+    if (tid == 0) {
+      ptx::tc_commit(drain);
+      ptx::mbar_wait_drain(drain, 0, ctl->limit_ns);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 0) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
-  if (tid == 0 && *abort_flag) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
+  if (tid == 0 && ctl->abort) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
 }
 
 }  // namespace
@@ -365,6 +376,8 @@ cudaError_t launch_local_bwd_tc(const Shape& s, const int32_t* g2p, const void* 
   a.dk_acc = dk_acc;
   a.dv_acc = dv_acc;
   a.err = err;
+  a.wait_ns = s.wait_ns;
+  a.stall = s.stall;
   cudaError_t e = cudaFuncSetAttribute(local_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(((s.Z + 1) / 2) * ((s.H + 3) / 4) * ((s.W + 3) / 4)), s.Hkv);

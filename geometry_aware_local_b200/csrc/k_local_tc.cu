@@ -46,7 +46,7 @@ constexpr int kKV0 = kRows * kDh * 2;             // plane buffers: K at +0, V a
 constexpr int kBufs = 3;
 constexpr int kBufBytes = 2 * kTileBytes;
 constexpr int kBarOff = kKV0 + kBufs * kBufBytes;
-constexpr int kSmemBytes = kBarOff + 64 + 1024;   // + barriers, + alignment slack
+constexpr int kSmemBytes = kBarOff + 64 + 1024;   // + barriers and flags, + alignment slack
 static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -61,6 +61,8 @@ struct LocalArgs {
   float* oloc;
   float* stats;            // nullable: lse2 of each row to stats[4 row]
   int32_t* err;
+  unsigned long long wait_ns;  // limit of every pipeline wait
+  int stall;               // diagnostic: the score MMA of the last plane is never issued
 };
 
 // Copies one 128-byte row into a 128-byte-swizzled tile at row r (zeros if src == nullptr).
@@ -100,8 +102,10 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
   const uint32_t sbase = ptx::smem_u32(smem);
   const uint32_t s_full = sbase + kBarOff;        // S of the current plane is in tensor memory
   const uint32_t pv_done = sbase + kBarOff + 8;   // O += P V of the last issued plane has completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + 20);
+  const uint32_t drain = sbase + kBarOff + 16;    // abort path: every MMA issued so far has completed
+  volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + 24);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 24 + sizeof(ptx::WaitCtl));
+  auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
   const int tid = threadIdx.x, warp = tid >> 5;
   const int g = blockIdx.y;
 
@@ -120,7 +124,9 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
   if (tid == 0) {
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(pv_done, 1);
-    *abort_flag = 0;
+    ptx::mbar_init(drain, 1);
+    ctl->abort = 0;
+    ctl->limit_ns = a.wait_ns;
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -194,16 +200,16 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
   ptx::cp_async_wait_two();
   ptx::fence_proxy_async_smem();
   __syncthreads();
-  if (tid == 0) issue_s(0);
+  // (PACK3D_FLAG_DIAG_STALL withholds the score MMA of the last plane.)
+  if (tid == 0 && !(a.stall && nplanes == 1)) issue_s(0);
 
   float m_used = -INFINITY, l = 0.f;
   bool ok = true;
-  int issued_pv = 0;
   for (int p = 0; p < nplanes; ++p) {
     const int zp = zlo + p;
     const bool uses = zp >= z0 + lz - 1 && zp <= z0 + lz + 1;  // warp-uniform (layer = warp / 2)
     // S of plane p; each using warp keeps its rows in registers.
-    bool w_ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, p & 1, abort_flag));
+    bool w_ok = __all_sync(0xffffffffu, wait(s_full, p & 1));
     uint32_t sv[kMaxKeys];
     if (w_ok) {
       ptx::tc_fence_after();
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
     if (!(ok = __syncthreads_and(w_ok))) break;
     // Every warp has read S(p): S(p+1) may overwrite it and run under this
     // plane's exponentials.
-    if (tid == 0 && p + 1 < nplanes) issue_s(p + 1);
+    if (tid == 0 && p + 1 < nplanes && !(a.stall && p + 2 == nplanes)) issue_s(p + 1);
 
     float f = 1.f, rs = 0.f;
     if (uses) {
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
     }
     // P and O are free again once O += P V of plane p-1 has completed.
     if (p > 0) {
-      w_ok = __all_sync(0xffffffffu, ptx::mbar_wait(pv_done, (p - 1) & 1, abort_flag));
+      w_ok = __all_sync(0xffffffffu, wait(pv_done, (p - 1) & 1));
       if (w_ok) ptx::tc_fence_after();
     }
     if (p == 1 && nplanes > 3 && w_ok) {
@@ -302,10 +308,9 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
                     (p > 0 || kk > 0) ? 1u : 0u);
       ptx::tc_commit(pv_done);
     }
-    issued_pv = p + 1;
   }
 
-  if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(pv_done, (nplanes - 1) & 1, abort_flag));
+  if (ok) ok = __all_sync(0xffffffffu, wait(pv_done, (nplanes - 1) & 1));
   if (ok) {
     ptx::tc_fence_after();
     uint32_t r[2][32];
@@ -321,19 +326,25 @@ __global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalA
                            __uint_as_float(r[q / 8][(4 * q + 2) % 32]) * inv,
                            __uint_as_float(r[q / 8][(4 * q + 3) % 32]) * inv);
     }
-  } else if (tid == 0) {
-    // Let whatever was issued drain before tensor memory is released.
-    ptx::tc_commit(pv_done);
-    ptx::mbar_wait(pv_done, issued_pv & 1, abort_flag);
   }
   ptx::cp_async_wait_all();
   ptx::tc_fence_before();
   __syncthreads();
+  if (ctl->abort) {
+    // The flag is final here (every thread has left the plane loop).  The
+    // MMAs thread 0 issued complete before tensor memory is released.
+    if (tid == 0) {
+      ptx::tc_commit(drain);
+      ptx::mbar_wait_drain(drain, 0, ctl->limit_ns);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 0) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 256);
   }
-  if (tid == 0 && *abort_flag) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
+  if (tid == 0 && ctl->abort) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
 }
 
 }  // namespace
@@ -365,6 +376,8 @@ cudaError_t launch_local_attn_tc(const Shape& s, const int32_t* g2p, const void*
   a.oloc = oloc;
   a.stats = stats;
   a.err = err;
+  a.wait_ns = s.wait_ns;
+  a.stall = s.stall;
   cudaError_t e = cudaFuncSetAttribute(local_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(((s.Z + 1) / 2) * ((s.H + 3) / 4) * ((s.W + 3) / 4)), s.Hkv);

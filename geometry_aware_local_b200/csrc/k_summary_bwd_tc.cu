@@ -56,6 +56,8 @@ struct BwdArgs {
   float* dks;          // summary side outputs [M, Hkv, 64] float (accumulated)
   float* dvs;
   int32_t* err;
+  unsigned long long wait_ns;  // limit of every pipeline wait
+  int stall;                   // diagnostic: the last operand tile is never loaded
 };
 
 // Row of the kv group's row space -> (token * Hq + head).
@@ -93,9 +95,9 @@ constexpr int kStages = 4;
 constexpr int kQOff = 0, kDOOff = kQTileBytes, kStageOff = 2 * kQTileBytes;
 constexpr int kStageBytes = 2 * kKVBytes;       // k~ at +0, v~ at +kKVBytes
 constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-// barriers: full[S], empty[S], qfull, s_full, s_free, p_full, p_free, o_final
-constexpr int kNumBars = 2 * kStages + 6;
-constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+// barriers: full[S], empty[S], qfull, s_full, s_free, p_full, p_free, o_final, drain
+constexpr int kNumBars = 2 * kStages + 7;
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;
 static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "CTAs per SM");
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kRowsPerTile, kBN, false);  // S, dP: N = 64 summaries
 constexpr uint32_t kIdescDQ = ptx::idesc_bf16_f32(kRowsPerTile, kDh, true);  // dQ: N = 64 dims, k~ MN-major
@@ -116,9 +118,10 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
   auto empty = [&](int s) { return bar0 + 8 * (kStages + s); };
   const uint32_t qfull = bar0 + 8 * (2 * kStages);
   const uint32_t s_full = qfull + 8, s_free = qfull + 16, p_full = qfull + 24, p_free = qfull + 32,
-                 o_final = qfull + 40;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+                 o_final = qfull + 40, drain = qfull + 48;
+  volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + kNumBars * 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8 + sizeof(ptx::WaitCtl));
+  auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -131,7 +134,9 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
     ptx::mbar_init(p_full, 4);
     ptx::mbar_init(p_free, 1);
     ptx::mbar_init(o_final, 1);
-    *abort_flag = 0;
+    ptx::mbar_init(drain, 1);
+    ctl->abort = 0;
+    ctl->limit_ns = a.wait_ns;
     ptx::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -142,6 +147,7 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int issued = 0;   // producer: summary tiles whose loads were issued
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
@@ -153,19 +159,15 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
       ptx::mbar_expect_tx(qfull, 2 * kQTileBytes);
       ptx::tma_load_4d(sbase + kQOff, &tmQ, 0, 0, g, tok0, qfull);
       ptx::tma_load_4d(sbase + kDOOff, &tmO, 0, 0, g, tok0, qfull);
-      int issued = 0;
-      for (int j = 0; j < T; ++j) {
+      const int T_load = a.stall ? T - 1 : T;
+      for (int j = 0; j < T_load; ++j) {
         const int st = j % kStages;
-        if (j >= kStages && !ptx::mbar_wait(empty(st), ((j / kStages) - 1) & 1, abort_flag)) break;
+        if (j >= kStages && !wait(empty(st), ((j / kStages) - 1) & 1)) break;
         const uint32_t dst = sbase + kStageOff + st * kStageBytes;
         ptx::mbar_expect_tx(full(st), kStageBytes);
         ptx::tma_load_3d(dst, &tmK, 0, g, j * kBN, full(st));
         ptx::tma_load_3d(dst + kKVBytes, &tmV, 0, g, j * kBN, full(st));
         issued = j + 1;
-      }
-      if (*abort_flag) {
-        for (int j = max(0, issued - kStages); j < issued; ++j)
-          ptx::mbar_wait(full(j % kStages), (j / kStages) & 1, abort_flag);
       }
     }
     __syncwarp();
@@ -195,26 +197,20 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         ptx::tc_commit(empty(j % kStages));
         if (j == T - 1) ptx::tc_commit(o_final);
       };
-      bool ok = ptx::mbar_wait(qfull, 0, abort_flag) && ptx::mbar_wait(full(0), 0, abort_flag);
+      bool ok = wait(qfull, 0) && wait(full(0), 0);
       if (ok) {
         ptx::tc_fence_after();
         issue_sdp(0);
       }
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
-          if (!(ok = ptx::mbar_wait(s_free, j & 1, abort_flag) &&
-                     ptx::mbar_wait(full((j + 1) % kStages), ((j + 1) / kStages) & 1, abort_flag)))
-            break;
+          if (!(ok = wait(s_free, j & 1) && wait(full((j + 1) % kStages), ((j + 1) / kStages) & 1))) break;
           ptx::tc_fence_after();
           issue_sdp(j + 1);
         }
-        if (!(ok = ptx::mbar_wait(p_full, j & 1, abort_flag))) break;
+        if (!(ok = wait(p_full, j & 1))) break;
         ptx::tc_fence_after();
         issue_dq(j);
-      }
-      if (!ok) {
-        ptx::tc_commit(o_final);
-        ptx::mbar_wait(o_final, 0, abort_flag);
       }
     }
     __syncwarp();
@@ -233,7 +229,7 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
     const float2 w2 = make_float2(w1, w1), nd2 = make_float2(-delta, -delta);
     bool ok = true;
     for (int j = 0; j < T; ++j) {
-      if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, j & 1, abort_flag)))) break;
+      if (!(ok = __all_sync(0xffffffffu, wait(s_full, j & 1)))) break;
       ptx::tc_fence_after();
       // 64 columns of S and dP at a time; the tensor memory is released after
       // the last chunk is read.
@@ -267,7 +263,7 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         // dS of the previous step is read by its dQ MMAs until p_free: wait
         // only now, so this step's exponentials overlap them.
         if (h == 0 && j > 0) {
-          if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free, (j - 1) & 1, abort_flag)))) break;
+          if (!(ok = __all_sync(0xffffffffu, wait(p_free, (j - 1) & 1)))) break;
           ptx::tc_fence_after();
         }
         ptx::tmem_st16(trow + kColDS + 32 * h, pk);
@@ -277,7 +273,7 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
       ptx::tmem_wait_st();
       warp_arrive(p_full);
     }
-    if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final, 0, abort_flag))) {
+    if (ok && __all_sync(0xffffffffu, wait(o_final, 0))) {
       ptx::tc_fence_after();
       uint32_t r[kDh];
       ptx::tmem_ld64_sync(trow + kColDQ, r);
@@ -293,11 +289,26 @@ summary_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 
   ptx::tc_fence_before();
   __syncthreads();
+  if (ctl->abort) {
+    // Final once every role has finished: the MMAs and loads this CTA
+    // started complete before its tensor and shared memory are released.
+    if (warp == kMmaWarp && lane == 0) {
+      ptx::tc_commit(drain);
+      ptx::mbar_wait_drain(drain, 0, ctl->limit_ns);
+    }
+    if (warp == kTmaWarp && lane == 0) {
+      ptx::mbar_wait_drain(qfull, 0, ctl->limit_ns);
+      for (int j = max(0, issued - kStages); j < issued; ++j)
+        ptx::mbar_wait_drain(full(j % kStages), (j / kStages) & 1, ctl->limit_ns);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
+  if (threadIdx.x == 0 && ctl->abort) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
 }
 
 }  // namespace q_side
@@ -346,10 +357,11 @@ constexpr int kStageBytes = 2 * kQTileBytes;    // Q at +0, dout at +kQTileBytes
 constexpr int kStages = (224 * 1024 - kStageOff - kOpBufs * kOpBytes) / kStageBytes;
 constexpr int kOpOff = kStageOff + kStages * kStageBytes;
 constexpr int kBarOff = kOpOff + kOpBufs * kOpBytes;
-// barriers: full[S], empty[S], kvfull, o_final, s_full, s_free, p_full[kOpBufs], p_free[kOpBufs]
-constexpr int kNumBars = 2 * kStages + 4 + 2 * kOpBufs;
+// barriers: full[S], empty[S], kvfull, o_final, s_full, s_free, p_full[kOpBufs], p_free[kOpBufs],
+// drain[2] (the abort path's MMA drain of each issuing warp)
+constexpr int kNumBars = 2 * kStages + 6 + 2 * kOpBufs;
 static_assert(kStages >= 2, "at least two Q / dout stages");
-constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kRowsPerTile, kBS, false);        // S, dP: N = 128 summaries
 constexpr uint32_t kIdescKV = ptx::idesc_bf16_f32_ab(kBS, kDh, true, true);        // dk~, dv~: A, B MN-major
@@ -374,8 +386,10 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
   const uint32_t o_final = kvfull + 8, s_full = kvfull + 16, s_free = kvfull + 24;
   auto p_full = [&](int b) { return kvfull + 32 + 8 * b; };
   auto p_free = [&](int b) { return kvfull + 32 + 8 * kOpBufs + 8 * b; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto drain = [&](int i) { return kvfull + 32 + 16 * kOpBufs + 8 * i; };
+  volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + kNumBars * 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8 + sizeof(ptx::WaitCtl));
+  auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -390,7 +404,10 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       ptx::mbar_init(p_full(b), kSoftmaxWarps);
       ptx::mbar_init(p_free(b), 1);
     }
-    *abort_flag = 0;
+    ptx::mbar_init(drain(0), 1);
+    ptx::mbar_init(drain(1), 1);
+    ctl->abort = 0;
+    ctl->limit_ns = a.wait_ns;
     ptx::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -401,6 +418,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int issued = 0;   // producer: steps whose Q / dout loads were issued
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
@@ -411,21 +429,16 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       ptx::mbar_expect_tx(kvfull, 2 * kSumTileBytes);
       ptx::tma_load_3d(sbase + kKOff, &tmK, 0, g, stile * kBS, kvfull);
       ptx::tma_load_3d(sbase + kVOff, &tmV, 0, g, stile * kBS, kvfull);
-      int issued = 0;
-      for (int t = 0; t < nsteps; ++t) {
+      const int nsteps_load = a.stall ? nsteps - 1 : nsteps;
+      for (int t = 0; t < nsteps_load; ++t) {
         const int st = t % kStages;
-        if (t >= kStages && !ptx::mbar_wait(empty(st), ((t / kStages) - 1) & 1, abort_flag)) break;
+        if (t >= kStages && !wait(empty(st), ((t / kStages) - 1) & 1)) break;
         const uint32_t dst = sbase + kStageOff + st * kStageBytes;
         const int tok0 = (int)((r0 + (long)t * kRowsPerTile) / a.G);
         ptx::mbar_expect_tx(full(st), kStageBytes);
         ptx::tma_load_4d(dst, &tmQ, 0, 0, g, tok0, full(st));
         ptx::tma_load_4d(dst + kQTileBytes, &tmO, 0, 0, g, tok0, full(st));
         issued = t + 1;
-      }
-      if (*abort_flag) {
-        ptx::mbar_wait(kvfull, 0, abort_flag);
-        for (int t = max(0, issued - kStages); t < issued; ++t)
-          ptx::mbar_wait(full(t % kStages), (t / kStages) & 1, abort_flag);
       }
     }
     __syncwarp();
@@ -463,31 +476,19 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       };
       bool ok = true;
       if (warp == kMmaWarp) {
-        ok = ptx::mbar_wait(kvfull, 0, abort_flag);
-        int issued = 0;
+        ok = wait(kvfull, 0);
         for (int t = 0; ok && t < nsteps; ++t) {
           // S and dP of step t: stage t landed, and step t-1's softmax read S and dP.
-          if (!(ok = ptx::mbar_wait(full(t % kStages), (t / kStages) & 1, abort_flag))) break;
-          if (t > 0 && !(ok = ptx::mbar_wait(s_free, (t - 1) & 1, abort_flag))) break;
+          if (!(ok = wait(full(t % kStages), (t / kStages) & 1))) break;
+          if (t > 0 && !(ok = wait(s_free, (t - 1) & 1))) break;
           ptx::tc_fence_after();
           issue_sdp(t);
-          issued = t + 1;
-        }
-        if (!ok) {
-          // Drain this warp's MMAs before tensor memory is released (the
-          // commit tracks every earlier MMA of this thread).
-          ptx::tc_commit(s_full);
-          ptx::mbar_wait(s_full, issued & 1, abort_flag);
         }
       } else {
         for (int t = 0; ok && t < nsteps; ++t) {
-          if (!(ok = ptx::mbar_wait(p_full(t % kOpBufs), (t / kOpBufs) & 1, abort_flag))) break;
+          if (!(ok = wait(p_full(t % kOpBufs), (t / kOpBufs) & 1))) break;
           ptx::tc_fence_after();
           issue_dkv(t);
-        }
-        if (!ok) {
-          ptx::tc_commit(o_final);
-          ptx::mbar_wait(o_final, 0, abort_flag);
         }
       }
     }
@@ -509,7 +510,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       // Rows outside this CTA's range contribute nothing: gamma1 = 0 zeroes gamma1 P and dS.
       const float w1 = valid ? gate_weights(a.gate, orow).y : 0.f;
       const float2 nl2 = make_float2(-lse2, -lse2), w2 = make_float2(w1, w1), nd2 = make_float2(-delta, -delta);
-      if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, t & 1, abort_flag)))) break;
+      if (!(ok = __all_sync(0xffffffffu, wait(s_full, t & 1)))) break;
       ptx::tc_fence_after();
       for (int cc = 0; cc < kChunksPerWg; ++cc) {
         const int c = kChunksPerWg * wg + cc;    // 32-summary chunk of the tile
@@ -530,9 +531,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         // Step (t - kOpBufs)'s dk~ / dv~ MMAs read this buffer: wait for them
         // only now, so this step's first exponentials overlap them.
         if (cc == 0 && t >= kOpBufs) {
-          if (!(ok = __all_sync(0xffffffffu,
-                                ptx::mbar_wait(p_free(t % kOpBufs), ((t / kOpBufs) - 1) & 1, abort_flag))))
-            break;
+          if (!(ok = __all_sync(0xffffffffu, wait(p_free(t % kOpBufs), ((t / kOpBufs) - 1) & 1)))) break;
         }
         // Row rl of the MN-major operands: summaries 32c .. 32c+31 are 16-byte
         // chunks (c & 1) * 4 + m of half c / 2.
@@ -548,7 +547,7 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
       ptx::fence_proxy_async_smem();
       warp_arrive(p_full(t % kOpBufs));
     }
-    if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final, 0, abort_flag))) {
+    if (ok && __all_sync(0xffffffffu, wait(o_final, 0))) {
       ptx::tc_fence_after();
       // Accumulator lane = summary of this tile.  The warpgroups share the
       // 128 accumulator columns (dk~ 64, then dv~ 64) evenly.
@@ -575,11 +574,27 @@ summary_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
 
   ptx::tc_fence_before();
   __syncthreads();
+  if (ctl->abort) {
+    // Final once every role has finished: the MMAs of both issuing warps and
+    // the producer's loads complete before tensor and shared memory are released.
+    if ((warp == kMmaWarp || warp == kMmaWarp2) && lane == 0) {
+      const uint32_t d = drain(warp - kMmaWarp);
+      ptx::tc_commit(d);
+      ptx::mbar_wait_drain(d, 0, ctl->limit_ns);
+    }
+    if (warp == kTmaWarp && lane == 0) {
+      ptx::mbar_wait_drain(kvfull, 0, ctl->limit_ns);
+      for (int t = max(0, issued - kStages); t < issued; ++t)
+        ptx::mbar_wait_drain(full(t % kStages), (t / kStages) & 1, ctl->limit_ns);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
+  if (threadIdx.x == 0 && ctl->abort) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
 }
 
 }  // namespace k_side
@@ -617,6 +632,8 @@ BwdArgs make_args(const Shape& s, const float* gate, const float* stats, int32_t
   a.dqr = nullptr;
   a.dks = a.dvs = nullptr;
   a.err = err;
+  a.wait_ns = s.wait_ns;
+  a.stall = s.stall;
   return a;
 }
 

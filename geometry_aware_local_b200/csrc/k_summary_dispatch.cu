@@ -26,7 +26,11 @@ cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* v
 
 namespace {
 constexpr int kOneTileMaxSummaryTiles = 48;
-bool one_tile(const Shape& s) { return (s.M + 127) / 128 <= kOneTileMaxSummaryTiles; }
+// s.sa_build forces a build (PACK3D_FLAG_SUMMARY_ONE_TILE / _TWO_TILE); 0 picks by size.
+bool one_tile(const Shape& s) {
+  if (s.sa_build != 0) return s.sa_build == 1;
+  return (s.M + 127) / 128 <= kOneTileMaxSummaryTiles;
+}
 }  // namespace
 
 long summary_attn_tc_token_quantum(const Shape& s) {

@@ -19,9 +19,8 @@
 //   * warps 0 .. 4*kGroups-1 are the softmax warpgroups, one per query tile,
 //     thread = row = TMEM lane.
 // At d_h = 64 each exponential pairs with only 256 MMA flops, so the softmax
-// sets the pace: packed f32x2 FMA/add, a three-input max and MUFU.ex2, with a
-// fixed share of the exponentials optionally evaluated by a cubic on the FMA
-// pipe.  O is rescaled lazily (only when a row maximum grows by more than
+// sets the pace: packed f32x2 FMA/add, a three-input max and MUFU.ex2.  O is
+// rescaled lazily (only when a row maximum grows by more than
 // 2^8).  Tensor memory (512 columns), group w at w*kGroupCols: S, P (packed
 // bf16), O.
 #include <cuda.h>
@@ -85,26 +84,15 @@ constexpr int kPairsPerChunk = kBN / 2 / kPChunks;   // packed P columns per chu
 constexpr int kMmasPerChunk = kBN / 16 / kPChunks;   // K = 16 steps of O += P v~ per chunk
 static_assert(kPairsPerChunk % 16 == 0, "P chunks are stored 16 columns at a time");
 // barriers: full[S], empty[S], qfull, then per group: s_full, s_free, o_final,
-// p_full[kPChunks], p_free[kPChunks]
-constexpr int kGroupBars = 3 + 2 * kPChunks;
+// p_full[kPChunks], p_free[kPChunks], drain (the abort path's MMA drain)
+constexpr int kGroupBars = 4 + 2 * kPChunks;
 constexpr int kNumBars = 2 * kStages + 1 + kGroups * kGroupBars;
-constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 static_assert(kGroups * kGroupCols <= kTmemCols, "tensor memory plan");
 
 constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kBM, kBN, false);      // S: N = kBN summaries
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, kDh, true);     // O: N = 64 dims, v~ MN-major
-
-// Pair k of the 32 column pairs of a tile uses the FMA-pipe exponential when
-// this holds; the others use MUFU.ex2.
-// PACK3D_SA_POLY of every 16 pairs (spread evenly) take the cubic; 0 by
-// default, since every share tried (2, 3, 4 and 6 of 16) was slower on B200.
-#ifndef PACK3D_SA_POLY
-#define PACK3D_SA_POLY 0
-#endif
-__host__ __device__ constexpr bool poly_pair(int k) {
-  return PACK3D_SA_POLY > 0 && ((k % 16) * PACK3D_SA_POLY) % 16 < PACK3D_SA_POLY;
-}
 
 struct TcArgs {
   int M;             // summaries
@@ -120,32 +108,14 @@ struct TcArgs {
   const __nv_bfloat16* dout;    // training: output gradient
   float* dgate;                 // training: gate gradient
   int32_t* err;
+  unsigned long long wait_ns;   // limit of every pipeline wait
+  int stall;                    // diagnostic: the last summary tile is never loaded
 };
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x for a pair, on the FMA pipe: x = n + f with n = rint(x) (added to the
-// exponent field) and f in [-1/2, 1/2], 2^f from a cubic fitted here by a
-// Remez exchange on the relative error (max 7.5e-5, well under bf16's 3.9e-3).
-// Inputs are clamped at -125 so the result stays a normal float (~1e-38 in
-// place of 0 for masked columns).
-__device__ __forceinline__ float2 exp2_poly(float2 x) {
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
-  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // kTrain: the training block's forward (row statistics and dgate in the
@@ -172,8 +142,10 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   auto o_final = [&](int w) { return gbar(w, 2); };
   auto p_full = [&](int w, int c) { return gbar(w, 3 + c); };
   auto p_free = [&](int w, int c) { return gbar(w, 3 + kPChunks + c); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto drain = [&](int w) { return gbar(w, 3 + 2 * kPChunks); };
+  volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + kNumBars * 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8 + sizeof(ptx::WaitCtl));
+  auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -185,12 +157,14 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ptx::mbar_init(s_full(w), 1);
       ptx::mbar_init(s_free(w), 4);       // one arrival per softmax warp
       ptx::mbar_init(o_final(w), 1);
+      ptx::mbar_init(drain(w), 1);
       for (int c = 0; c < kPChunks; ++c) {
         ptx::mbar_init(p_full(w, c), 4);
         ptx::mbar_init(p_free(w, c), 1);
       }
     }
-    *abort_flag = 0;
+    ctl->abort = 0;
+    ctl->limit_ns = a.wait_ns;
     ptx::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -201,6 +175,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int issued = 0;   // producer: summary tiles whose loads were issued
 
   if (warp == kTmaWarp) {
     // ---------------- TMA producer ----------------
@@ -212,20 +187,15 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ptx::mbar_expect_tx(qfull, kGroups * kQBytes);
       for (int w = 0; w < kGroups; ++w)
         ptx::tma_load_4d(sbase + kQOff + w * kQBytes, &tmQ, 0, 0, g, (tile0 + w) * tok_per_tile, qfull);
-      int issued = 0;
-      for (int j = 0; j < T; ++j) {
+      const int T_load = a.stall ? T - 1 : T;
+      for (int j = 0; j < T_load; ++j) {
         const int st = j % kStages;
-        if (j >= kStages && !ptx::mbar_wait(empty(st), ((j / kStages) - 1) & 1, abort_flag)) break;
+        if (j >= kStages && !wait(empty(st), ((j / kStages) - 1) & 1)) break;
         const uint32_t dst = sbase + kStageOff + st * kStageBytes;
         ptx::mbar_expect_tx(full(st), kStageBytes);
         ptx::tma_load_3d(dst, &tmK, 0, g, j * kBN, full(st));
         ptx::tma_load_3d(dst + kKVBytes, &tmV, 0, g, j * kBN, full(st));
         issued = j + 1;
-      }
-      if (*abort_flag) {
-        // Let copies already in flight land before the CTA's shared memory is released.
-        for (int j = max(0, issued - kStages); j < issued; ++j)
-          ptx::mbar_wait(full(j % kStages), (j / kStages) & 1, abort_flag);
       }
     }
     __syncwarp();
@@ -264,29 +234,23 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           if (j == T - 1) ptx::tc_commit(o_final(w));
         }
       };
-      bool ok = ptx::mbar_wait(qfull, 0, abort_flag) && ptx::mbar_wait(full(0), 0, abort_flag);
+      bool ok = wait(qfull, 0) && wait(full(0), 0);
       if (ok) {
         ptx::tc_fence_after();
         issue_s(0);
       }
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
-          if (!(ok = ptx::mbar_wait(s_free(w), j & 1, abort_flag) &&
-                     ptx::mbar_wait(full((j + 1) % kStages), ((j + 1) / kStages) & 1, abort_flag)))
+          if (!(ok = wait(s_free(w), j & 1) && wait(full((j + 1) % kStages), ((j + 1) / kStages) & 1)))
             break;
           ptx::tc_fence_after();
           issue_s(j + 1);
         }
         for (int c = 0; ok && c < kPChunks; ++c) {
-          if (!(ok = ptx::mbar_wait(p_full(w, c), j & 1, abort_flag))) break;
+          if (!(ok = wait(p_full(w, c), j & 1))) break;
           ptx::tc_fence_after();
           issue_pv(j, c);
         }
-      }
-      if (!ok) {
-        // Drain whatever this warp issued before tensor memory is released.
-        ptx::tc_commit(o_final(w));
-        ptx::mbar_wait(o_final(w), 0, abort_flag);
       }
     }
     __syncwarp();
@@ -340,13 +304,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           const int pair = cc * kPairsPerChunk + q * 16 + k;
           const float2 x =
               __ffma2_rn(make_float2(__uint_as_float(sv[2 * pair]), __uint_as_float(sv[2 * pair + 1])), c2, nm2);
-          float2 p;
-          if (poly_pair(pair)) {
-            p = exp2_poly(x);
-          } else {
-            p.x = ptx::ex2(x.x);
-            p.y = ptx::ex2(x.y);
-          }
+          const float2 p = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
           rs[k & 1] = __fadd2_rn(rs[k & 1], p);
           pk[k] = pack_bf16x2(p.x, p.y);
         }
@@ -362,7 +320,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       if (lane == 0) ptx::mbar_arrive(bar);
     };
     for (int j = 0; j < T; ++j) {
-      if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full(w), j & 1, abort_flag)))) break;
+      if (!(ok = __all_sync(0xffffffffu, wait(s_full(w), j & 1)))) break;
       ptx::tc_fence_after();
       float f = 1.f;
       float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -380,7 +338,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll
         for (int cc = 0; cc < kPChunks; ++cc) {
           if (j > 0) {
-            if (!(ok = __all_sync(0xffffffffu, ptx::mbar_wait(p_free(w, cc), (j - 1) & 1, abort_flag)))) break;
+            if (!(ok = __all_sync(0xffffffffu, wait(p_free(w, cc), (j - 1) & 1)))) break;
             ptx::tc_fence_after();
           }
           exps_chunk(sv, cc, rs);
@@ -388,8 +346,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             // O is rescaled before this tile's first O += P v~ is issued and
             // after the previous tile's last one has completed (its commit
             // covers all earlier MMAs of the group).
-            if (!(ok = __all_sync(0xffffffffu,
-                                  ptx::mbar_wait(p_free(w, kPChunks - 1), (j - 1) & 1, abort_flag))))
+            if (!(ok = __all_sync(0xffffffffu, wait(p_free(w, kPChunks - 1), (j - 1) & 1))))
               break;
             ptx::tc_fence_after();
             uint32_t r[16];
@@ -408,7 +365,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       }
       l = l * f + ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y));
     }
-    if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(o_final(w), 0, abort_flag))) {
+    if (ok && __all_sync(0xffffffffu, wait(o_final(w), 0))) {
       ptx::tc_fence_after();
       uint32_t r[2][32];
       ptx::tmem_ld64_sync(tO, &r[0][0]);
@@ -449,11 +406,27 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
   ptx::tc_fence_before();
   __syncthreads();
+  if (ctl->abort) {
+    // Every role has finished, so the flag is final and the same for all
+    // threads.  Before tensor memory and shared memory are released, the MMAs
+    // each issuing warp started and the loads the producer started complete.
+    if (warp >= kMmaWarp && warp < kTmaWarp && lane == 0) {
+      ptx::tc_commit(drain(warp - kMmaWarp));
+      ptx::mbar_wait_drain(drain(warp - kMmaWarp), 0, ctl->limit_ns);
+    }
+    if (warp == kTmaWarp && lane == 0) {
+      ptx::mbar_wait_drain(qfull, 0, ctl->limit_ns);
+      for (int j = max(0, issued - kStages); j < issued; ++j)
+        ptx::mbar_wait_drain(full(j % kStages), (j / kStages) & 1, ctl->limit_ns);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
+  if (threadIdx.x == 0 && ctl->abort) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
 }
 
 // ---- host side -------------------------------------------------------------
@@ -523,6 +496,8 @@ cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* v
   a.dout = tr ? (const __nv_bfloat16*)tr->dout : nullptr;
   a.dgate = tr ? tr->dgate : nullptr;
   a.err = err;
+  a.wait_ns = s.wait_ns;
+  a.stall = s.stall;
   const long tiles = (a.rows - tok_begin * s.G + kBM - 1) / kBM;
   dim3 grid((unsigned)((tiles + kGroups - 1) / kGroups), s.Hkv);
   kern<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);

@@ -53,20 +53,43 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Waits for phase `parity` of `bar`.  Gives up after ~2 s (or as soon as
-// another role of the CTA gave up), raising *abort; returns false then.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// Per-CTA state of the bounded waits, in shared memory: the abort flag every
+// role polls, and the wait limit (kept here rather than in registers, since it
+// is read only on the slow path of a wait).
+struct WaitCtl {
+  int abort;
+  int pad;
+  unsigned long long limit_ns;
+};
+
+// Waits for phase `parity` of `bar`.  Gives up after ctl->limit_ns of
+// %globaltimer (or as soon as another role of the CTA gave up), raising
+// ctl->abort; returns false then.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile WaitCtl* ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > 2000000000ull) {
-        *abort = 1;
+      if (ctl->abort) return false;
+      if (globaltimer_ns() - t0 > ctl->limit_ns) {
+        ctl->abort = 1;
         return false;
       }
     }
+  }
+}
+
+// Wait of the abort path: the CTA has given up, and before it frees tensor
+// memory or exits it lets the asynchronous work it issued (TMA loads into its
+// shared memory, MMAs into its tensor memory) complete.  Ignores the abort
+// flag; gives up after `limit_ns` all the same, so the CTA always ends.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -95,6 +95,26 @@ typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
  * (bx-1)/2), a fractional coordinate; v~_j and every other stage unchanged.
  * Without the flag the summaries are the exact rotate-before-compress form. */
 #define PACK3D_FLAG_SUMMARY_CENTER 0x4
+/* Diagnostic: every tensor-core kernel withholds one step of its pipeline
+ * (the query x summary kernels the load of their last summary tile, the
+ * local-attention kernel the score MMA of its last key plane), so that the
+ * waits that depend on it run out after wait_limit_us.  The call then reports
+ * PACK3D_DEVERR_TIMEOUT in err_word (PACK3D_ERR_TIMEOUT from
+ * pack3d_check_status) and its outputs are unspecified; the kernels still let
+ * their issued loads and MMAs complete, free their tensor memory and return,
+ * so the next call on the stream runs normally.  It exists to test that error
+ * path; nothing else sets it.  No entry point that takes it runs on CUDA cores
+ * only (float, PACK3D_FLAG_SIMT_*): those have no pipeline waits. */
+#define PACK3D_FLAG_DIAG_STALL    0x8
+/* The tensor-core query x summary kernel comes in two builds: one 128-row query
+ * tile per CTA with two CTAs per SM, and two tiles per CTA with one CTA per SM
+ * (every summary tile read once for both).  By default the library picks the
+ * one-tile build up to 48 summary tiles (M <= 6,144) and the two-tile build
+ * above; these flags force one of them (setting both is an error).  Both
+ * builds compute every row with the same sequence of operations, so their
+ * outputs are identical bit for bit; the flags only move the cost. */
+#define PACK3D_FLAG_SUMMARY_ONE_TILE 0x10
+#define PACK3D_FLAG_SUMMARY_TWO_TILE 0x20
 
 typedef struct {
     int32_t Z, H, W;          /* lattice extents; N = Z*H*W tokens               */
@@ -107,7 +127,12 @@ typedef struct {
     float   softmax_scale;    /* logit scale in both branches (1/sqrt(d_h))      */
     int32_t dtype;            /* pack3d_dtype of q, k, v, summaries, out         */
     int32_t flags;            /* PACK3D_FLAG_* bits                              */
-    int32_t reserved1;        /* must be 0                                       */
+    int32_t wait_limit_us;    /* limit of every bounded device-side pipeline wait,
+                                 in microseconds, >= 0; 0 = the default of 2 s.
+                                 A wait that runs out makes its CTA give up
+                                 (PACK3D_DEVERR_TIMEOUT); a limit far below a
+                                 kernel's normal step time turns healthy calls
+                                 into timeouts                                  */
     double  coord_scale[3];   /* per-axis coordinate scale (z, y, x), > 0, 1 by
                                  default: the rotation angle of axis a is
                                  omega_{a,r} * coord_scale[a] * c_a, so e.g.
@@ -228,7 +253,9 @@ pack3d_status pack3d_forward(const pack3d_config *cfg, const int32_t *coords, co
  *     reported;
  *   - the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it: make
- *     that first call before any stream capture;
+ *     that first call before any stream capture.  The cache belongs to the
+ *     device's context: after cudaDeviceReset the library may load at another
+ *     address, so do not call this entry point on a device that was reset;
  *   - every call shares the one array, so calls whose work overlaps on the
  *     GPU (e.g. on two streams) race; the caller must serialise them.
  * Nothing is allocated or freed. */

@@ -48,13 +48,24 @@ def test_default_config_matches_pages(p3):
 @pytest.mark.parametrize("field,value,status", [
     ("d_h", 128, 2), ("Hq", 6, 2), ("Hkv", 3, 2), ("W", 63, 2), ("bx", 0, 2), ("rz", -1, 2),
     ("m_z", 20, 2), ("dtype", 7, 4), ("softmax_scale", 0.0, 1), ("flags", 0x100, 1), ("reserved0", 1, 1),
-    ("flags", 0x8, 1),
+    ("flags", 0x40, 1), ("flags", 0x30, 1), ("wait_limit_us", -1, 1),
     ("rope_base", -1.0, 1), ("Z", -1, 2), ("W", -4, 2),
 ])
 def test_validate_rejects(p3, field, value, status):
     c = p3.make_config(16, 64, 64)
     setattr(c, field, value)
     assert p3.validate(c) == status
+
+
+@pytest.mark.parametrize("field,value", [
+    ("flags", 0x8), ("flags", 0x10), ("flags", 0x20), ("flags", 0x8 | 0x20 | 0x4), ("wait_limit_us", 0),
+    ("wait_limit_us", 1), ("wait_limit_us", 2_000_000),
+])
+def test_validate_accepts(p3, field, value):
+    """The diagnostic stall, the two forced query x summary builds and any non-negative wait limit."""
+    c = p3.make_config(16, 64, 64)
+    setattr(c, field, value)
+    assert p3.validate(c) == 0
 
 
 @pytest.mark.parametrize("dims", [(0, 64, 64), (16, 0, 64), (16, 64, 0), (0, 0, 0)])

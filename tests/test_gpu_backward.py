@@ -91,6 +91,49 @@ def test_forward_backward_matches_oracle(p3, name, s, packing, flags):
         assert e <= tol, f"{name}: {key} rel err {e:.3e} > {tol}"
 
 
+TWO_TILE_CASES = [c for c in CASES if c[1].dtype == "bf16" and not c[3]]
+
+
+@pytest.mark.parametrize("name,s,packing,flags", TWO_TILE_CASES, ids=[c[0] for c in TWO_TILE_CASES])
+def test_two_tile_training_forward_matches_oracle(p3, name, s, packing, flags):
+    """The training instantiation of the two-tile query x summary build (statistics and dgate in its
+    epilogue), forced at small M, through every bf16 case: all gradients against the oracle."""
+    inp = synth.make_inputs(s, packing, seed=4)
+    dout = synth.make_dout(s, packing, seed=4)
+    gpu = run_fwd_bwd(p3, s, inp, dout, flags | p3.FLAG_SUMMARY_TWO_TILE)
+    ref = oracle.backward(s, inp, dout)
+    for key in GRADS + ("out",):
+        e = rel_err(gpu[key].double().numpy(), ref[key])
+        assert e <= TOL["bf16"], f"{name}: {key} rel err {e:.3e}"
+
+
+def test_forward_backward_large_m_sharp(p3):
+    """Above the one-tile limit by size: 28,672 tokens in 1x2x2 blocks, so M = 7,168 (56 summary tiles),
+    with Q x 8 and K_loc / 8 (exact in bf16) making the summary softmax sharp.  Every gradient against the
+    oracle's chain rule: dq, dgate and out on every row, the local key gradients on sampled keys, the
+    summary-side ones on sampled blocks."""
+    s = small(Z=4, H=64, W=112, by=2, bx=2, value_scale=1.0)
+    assert (s.M + 127) // 128 > 48
+    inp = synth.make_inputs(s, "morton", seed=17)
+    inp["q"] = (inp["q"].float() * 8.0).bfloat16()
+    inp["k_loc"] = (inp["k_loc"].float() * 0.125).bfloat16()
+    dout = synth.make_dout(s, "morton", seed=17)
+    gpu = run_fwd_bwd(p3, s, inp, dout)
+    rng = np.random.default_rng(23)
+    keys = np.unique(np.concatenate([[0, s.N - 1], rng.choice(s.N, 254, replace=False)]))
+    blocks = np.unique(np.concatenate([[0, s.M - 1], rng.choice(s.M, 62, replace=False)]))
+    ref = oracle.backward(s, inp, dout, keys=keys, blocks=blocks)
+    kt, tok = torch.from_numpy(keys), torch.from_numpy(ref["cmp_tokens"])
+    checks = {"dq": (gpu["dq"], ref["dq"]), "dgate": (gpu["dgate"], ref["dgate"]), "out": (gpu["out"], ref["out"]),
+              "dk_loc": (gpu["dk_loc"].index_select(0, kt), ref["dk_loc"]),
+              "dv_loc": (gpu["dv_loc"].index_select(0, kt), ref["dv_loc"])}
+    for k in ("dk_cmp", "dv_cmp", "dscores"):
+        checks[k] = (gpu[k].index_select(0, tok), ref[k])
+    for k, (a, b) in checks.items():
+        e = rel_err(a.double().numpy(), b)
+        assert e <= TOL["bf16"], f"{k} rel err {e:.3e}"
+
+
 CENTER_CASES = [
     ("center-bf16", small(), "random", 0),
     ("center-f32", small(dtype="f32", value_scale=1.0), "morton", 0),

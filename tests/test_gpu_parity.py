@@ -124,6 +124,81 @@ def test_stages_match_oracle(p3, name, s, packing):
         assert e <= tol, f"{name}: {key} rel err {e:.3e} > {tol}"
 
 
+BF16_STAGE_CASES = [c for c in STAGE_CASES if c[1].dtype == "bf16"]
+
+
+@pytest.mark.parametrize("name,s,packing", BF16_STAGE_CASES, ids=[c[0] for c in BF16_STAGE_CASES])
+def test_two_tile_build_matches_oracle(p3, name, s, packing):
+    """The two-tile query x summary build (one CTA per SM, chosen by size only above 48 summary
+    tiles) forced on every bf16 stage case: its compressed branch and gate against the oracle."""
+    inp = synth.make_inputs(s, packing, seed=3)
+    gpu = run_stages(p3, s, to_dev(inp), flags=p3.FLAG_SUMMARY_TWO_TILE)
+    ref = oracle.forward(s, inp)
+    for key in ("o_cmp", "out"):
+        e = rel_err(gpu[key].double().numpy(), ref[key])
+        assert e <= TOL["bf16"], f"{name}: {key} rel err {e:.3e}"
+
+
+@pytest.mark.parametrize("s", [small(Z=4, H=32, W=40), small(Z=3, H=10, W=14, by=2, bx=2), small(Hq=8, Hkv=1)],
+                         ids=["m-multi", "ragged-brick", "g8"])
+def test_one_and_two_tile_builds_are_bit_identical(p3, s):
+    """Both builds run every row through the same operations: o_cmp and the gated output agree bit for
+    bit, and so do the training forward's output and gate gradient."""
+    d = to_dev(synth.make_inputs(s, "random", seed=14))
+    a = run_stages(p3, s, d, flags=p3.FLAG_SUMMARY_ONE_TILE)
+    b = run_stages(p3, s, d, flags=p3.FLAG_SUMMARY_TWO_TILE)
+    assert torch.equal(a["o_cmp"], b["o_cmp"]) and torch.equal(a["out"], b["out"])
+    dout = synth.make_dout(s, "random", seed=14).cuda()
+    res = []
+    for flags in (p3.FLAG_SUMMARY_ONE_TILE, p3.FLAG_SUMMARY_TWO_TILE):
+        cfg = p3.config_from_shape(s, flags)
+        out = torch.empty_like(d["q"])
+        grads = p3.empty_grads(d["q"], d["k_loc"], d["scores"], d["gate"])
+        ws = torch.empty(p3.train_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+        err = torch.zeros(4, dtype=torch.int32, device="cuda")
+        p3.forward_backward(cfg, d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
+                            d["gate"], dout, out, grads, ws, err)
+        assert p3.check_status(err) == 0
+        res.append((out.cpu(), grads["dgate"].cpu(), grads["dq"].cpu()))
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    assert torch.equal(res[0][2], res[1][2])
+
+
+def sharp_inputs(s, packing, seed):
+    """Inputs whose summary softmax is sharp: Q x 8 and K_loc / 8 (exact in bf16) on top of value_scale 1,
+    so the compressed logits have a standard deviation of about 3 (a few summaries carry each row) while
+    the local logits stay about N(0,1).  A wrong summary tile, ring stage or rescale then moves o_cmp by
+    the size of a summary value instead of by a fraction of a flat average."""
+    inp = synth.make_inputs(s, packing, seed=seed)
+    inp["q"] = (inp["q"].float() * 8.0).to(inp["q"].dtype)
+    inp["k_loc"] = (inp["k_loc"].float() * 0.125).to(inp["k_loc"].dtype)
+    return inp
+
+
+def test_large_m_two_tile_build_sharp_logits(p3):
+    """131,072 tokens, M = 8,192 (64 summary tiles, the two-tile build by size) with a sharp summary
+    softmax: o_cmp and out on every row of the first, a middle and the last CTA's query tiles (two
+    128-row tiles per kv head each) and on 1,024 sampled tokens, element by element."""
+    s = synth.Pack3DShape(Z=8, H=64, W=256, Hq=8, Hkv=2, value_scale=1.0)
+    assert (s.M + 127) // 128 > 48
+    inp = sharp_inputs(s, "random", seed=7)
+    gpu = run_stages(p3, s, to_dev(inp))
+    per_cta = 2 * 128 // (s.Hq // s.Hkv)        # tokens of one two-tile CTA (both kv heads run it)
+    mid = (s.N // 2) // per_cta * per_cta
+    full_tiles = np.concatenate([np.arange(0, per_cta), np.arange(mid, mid + per_cta),
+                                 np.arange(s.N - per_cta, s.N)])
+    rows = np.unique(np.concatenate([full_tiles, synth.sample_rows(s.N, 1024, seed=5)]))
+    ref = oracle.forward(s, inp, rows)
+    # the softmax really is sharp: a few dozen of the 8,192 summaries carry each row
+    logits = np.einsum("rd,md->rm", ref["q_rot"][:64, 0], ref["k_sum"][:, 0]) * s.softmax_scale
+    pr = np.exp(logits - logits.max(1, keepdims=True))
+    pr /= pr.sum(1, keepdims=True)
+    assert np.median(1.0 / (pr ** 2).sum(1)) < 64
+    for key in ("o_cmp", "out"):
+        e = rel_err(gpu[key][rows].double().numpy(), ref[key])
+        assert e <= TOL["bf16"], f"{key} rel err {e:.3e}"
+
+
 CENTER_CASES = [
     ("bf16-warp", small(), "random"),                                  # warp-per-block kernel
     ("f32-tiny", synth.CONFIGS["tiny"], "raster"),
@@ -332,7 +407,7 @@ def test_stress_packing_equivariance_65k(p3):
     rows = synth.sample_rows(s.N, 256, seed=2)
     oref = oracle.forward(s, base, rows)["out"]
     assert rel_err(ref[rows].numpy(), oref) <= TOL["bf16"]
-    for packing in ("morton", "block", "random"):
+    for packing in ("morton", "block", "random", "block_morton"):
         inp = synth.make_inputs(s, packing, 5, sv)
         out = run_forward(p3, s, to_dev(inp)).double()
         sites = inp["sites"]
