@@ -25,6 +25,11 @@ pass saving its softmax statistics, then the gradients of <dOut, out> with
 respect to every input), on the same volume with dOut drawn N(0,1) per site;
 tokens/s there count one forward and one backward per token.
 
+``sizes`` (single-GPU runs of the default workload) times the same stages
+on the 262k- and 1M-token volumes, where the stage targets are set, with
+their values drawn on the device (same distributions; no parity is taken
+from them), each with its own clock record.
+
 ``--impl reference`` times the float64 CPU oracle on the host cores on a
 bounded sample of the same workload (rank 0 only).
 """
@@ -61,10 +66,16 @@ WORKLOAD_TEXT = {
 STAGES = ("index", "summaries", "rope", "local", "summary_attn")
 KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summary attention
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
-# summary_attn_tc_kernel launch, from an ncu capture of the 65k workload (where
-# the one-tile build runs); the summary of that capture is kept under
-# profiles/.  Emptied whenever that kernel changes until it is captured again.
-SUMMARY_ATTN_TRAFFIC = {"65k": 212.771072e6 + 48.423168e6}
+# summary_attn_tc_kernel launch per workload, from an ncu capture of that
+# workload, with the capture it came from; the summary of the capture is kept
+# under profiles/.  Emptied whenever that kernel changes until it is captured
+# again (a workload without an entry reports null).
+SUMMARY_ATTN_TRAFFIC: Dict[str, tuple] = {}
+# The benchmark spec's nominal HBM bandwidth, reported beside the measured copy peak.
+HBM_NOMINAL_GBS = 8000.0
+# Volumes timed in the `sizes` block of a default single-GPU run.
+SIZES = ("262k", "1m")
+SIZE_STEPS = {"262k": (3, 8), "1m": (3, 3)}   # (warm-up, timed) steps
 
 # Launches at least this long are rated against the sustained bf16 peak.
 SUSTAINED_MS = 1000.0
@@ -422,6 +433,120 @@ def run_train_only(args, s):
         dist.destroy_process_group()
 
 
+def stage_fractions(s, st_ms, peaks) -> Dict:
+    """Per-stage ms with achieved GB/s and TFLOP/s against the measured peaks (and the nominal HBM)."""
+    work = algorithmic_work(s)
+    stages = {}
+    for name in STAGES:
+        t = st_ms[name] * 1e-3
+        w = work[name]
+        e = {"ms": st_ms[name]}
+        if "bytes" in w:
+            e["hbm_gbs"] = w["bytes"] / t / 1e9
+            e["hbm_frac"] = e["hbm_gbs"] / peaks["hbm_gbs"]
+            e["hbm_frac_nominal"] = e["hbm_gbs"] / HBM_NOMINAL_GBS
+        if "flops" in w:
+            e["tflops"] = w["flops"] / t / 1e12
+            e["tensor_frac"] = e["tflops"] / peaks["bf16_tflops"]
+        stages[name] = e
+    return stages
+
+
+class StageTimer:
+    """One step = the C-ABI stage entry points in the order pack3d_forward launches them, CUDA events
+    between the stages on the launching stream."""
+
+    def __init__(self, p3, s, cfg, d, stream, err):
+        import torch
+        dev, dt = d["q"].device, d["q"].dtype
+        self.p3, self.s, self.cfg, self.d, self.stream, self.err = p3, s, cfg, d, stream, err
+        self.g2p = torch.empty(s.N, dtype=torch.int32, device=dev)
+        self.mem = torch.empty(s.M, s.v, dtype=torch.int32, device=dev)
+        self.qr, self.kr = torch.empty_like(d["q"]), torch.empty_like(d["k_loc"])
+        self.ks = torch.empty(s.M, s.Hkv, s.d_h, dtype=dt, device=dev)
+        self.vs = torch.empty_like(self.ks)
+        self.ol = torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device=dev)
+        self.out = torch.empty_like(d["q"])
+
+    def step(self, ev):
+        import ctypes
+        lib, d, sh = self.p3.lib, self.d, self.stream.cuda_stream
+        cfgp = ctypes.byref(self.cfg)
+        P = lambda t: t.data_ptr()  # noqa: E731
+        ev[0].record(self.stream)
+        st = lib.pack3d_build_index(cfgp, P(d["coords"]), P(self.g2p), P(self.mem), P(self.err), sh)
+        ev[1].record(self.stream)
+        st |= lib.pack3d_build_summaries(cfgp, P(self.mem), P(d["k_cmp"]), P(d["v_cmp"]), P(d["scores"]),
+                                         P(self.ks), P(self.vs), sh)
+        ev[2].record(self.stream)
+        st |= lib.pack3d_rope_qk(cfgp, P(d["coords"]), P(d["q"]), P(self.qr), P(d["k_loc"]), P(self.kr), sh)
+        ev[3].record(self.stream)
+        st |= lib.pack3d_local_attn(cfgp, P(self.g2p), P(self.qr), P(self.kr), P(d["v_loc"]), P(self.ol),
+                                    P(self.err), sh)
+        ev[4].record(self.stream)
+        st |= lib.pack3d_summary_attn(cfgp, P(self.qr), P(self.ks), P(self.vs), P(self.ol), P(d["gate"]),
+                                      P(self.out), P(self.err), sh)
+        ev[5].record(self.stream)
+        if st:
+            raise RuntimeError("a PACK3D entry point failed")
+
+    @staticmethod
+    def events():
+        import torch
+        return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    def run(self, warmup, steps, flush, world, clock_gpu):
+        """W untimed steps, then K timed ones (L2 flushed before each, outside the events) inside a
+        clock record; returns the mean stage ms, the mean step ms (max over ranks) and the clocks."""
+        for _ in range(warmup):
+            self.step(self.events())
+        if self.p3.check_status(self.err) != 0:
+            raise RuntimeError("device error during warm-up")
+        evs = [self.events() for _ in range(steps)]
+        barrier(world)
+        with ClockSampler(clock_gpu) as clk:
+            for k in range(steps):
+                flush()
+                self.step(evs[k])
+            barrier(world)
+        st_ms = {name: 0.0 for name in STAGES}
+        step_ms = []
+        for ev in evs:
+            for i, name in enumerate(STAGES):
+                st_ms[name] += ev[i].elapsed_time(ev[i + 1])
+            step_ms.append(ev[0].elapsed_time(ev[5]))
+        if self.p3.check_status(self.err) != 0:
+            raise RuntimeError("device error during the timed steps")
+        ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+        return {k: v / steps for k, v in st_ms.items()}, ms, clk.summary()
+
+
+def time_sizes(p3, flush, stream, dev, peaks) -> Dict:
+    """The `sizes` block: the stages at 262k and 1M tokens (values drawn on the device)."""
+    import torch
+    res = {}
+    for name in SIZES:
+        s = synth.CONFIGS[name]
+        cfg = p3.config_from_shape(s)
+        d = synth.make_inputs_on_device(s, s.packing, seed=0, device=dev)
+        err = torch.zeros(4, dtype=torch.int32, device=dev)
+        warm, steps = SIZE_STEPS[name]
+        timer = StageTimer(p3, s, cfg, d, stream, err)
+        st_ms, ms, clocks = timer.run(warm, steps, flush, 1, dev.index or 0)
+        stages = stage_fractions(s, st_ms, peaks)
+        res[name] = {"workload": WORKLOAD_TEXT[name], "tokens": s.N, "summaries": s.M, "value": s.N / (ms * 1e-3),
+                     "unit": "tokens/s", "ms_per_step": ms, "steps": steps, "warmup": warm,
+                     "stages": stages, "clocks": clocks,
+                     "query_x_summary_tensor_frac": stages["summary_attn"]["tensor_frac"],
+                     "summaries_hbm_frac": stages["summaries"]["hbm_frac"],
+                     "rope_hbm_frac": stages["rope"]["hbm_frac"],
+                     "data": "synthetic, values drawn on the device (same distributions as the host recipe)",
+                     "l2": flush.text}
+        del timer, d
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, s):
     import torch
 
@@ -439,67 +564,13 @@ def run_ours(args, s):
     else:
         inp_host = synth.make_inputs(s, s.packing, seed=rank)
         d = {k: inp_host[k].to(dev) for k in names}
-    dt = d["q"].dtype
     err = torch.zeros(4, dtype=torch.int32, device=dev)
-    g2p = torch.empty(s.N, dtype=torch.int32, device=dev)
-    mem = torch.empty(s.M, s.v, dtype=torch.int32, device=dev)
-    qr, kr = torch.empty_like(d["q"]), torch.empty_like(d["k_loc"])
-    ks = torch.empty(s.M, s.Hkv, s.d_h, dtype=dt, device=dev)
-    vs = torch.empty_like(ks)
-    ol = torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device=dev)
-    out = torch.empty_like(d["q"])
     flush = L2Flush(dev, args.flush)
     stream = torch.cuda.current_stream(dev)
-
-    lib = p3.lib
-    import ctypes
-    cfgp = ctypes.byref(cfg)
-    sh = stream.cuda_stream
-    P = lambda t: t.data_ptr()  # noqa: E731
-
-    def step(ev):
-        # The same launches pack3d_forward makes, one entry point per stage.
-        ev[0].record(stream)
-        st = lib.pack3d_build_index(cfgp, P(d["coords"]), P(g2p), P(mem), P(err), sh)
-        ev[1].record(stream)
-        st |= lib.pack3d_build_summaries(cfgp, P(mem), P(d["k_cmp"]), P(d["v_cmp"]), P(d["scores"]), P(ks),
-                                         P(vs), sh)
-        ev[2].record(stream)
-        st |= lib.pack3d_rope_qk(cfgp, P(d["coords"]), P(d["q"]), P(qr), P(d["k_loc"]), P(kr), sh)
-        ev[3].record(stream)
-        st |= lib.pack3d_local_attn(cfgp, P(g2p), P(qr), P(kr), P(d["v_loc"]), P(ol), P(err), sh)
-        ev[4].record(stream)
-        st |= lib.pack3d_summary_attn(cfgp, P(qr), P(ks), P(vs), P(ol), P(d["gate"]), P(out), P(err), sh)
-        ev[5].record(stream)
-        if st:
-            raise RuntimeError("a PACK3D entry point failed")
-
-    def events():
-        return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-
-    for _ in range(args.warmup):
-        step(events())
-    if p3.check_status(err) != 0:
-        raise RuntimeError("device error during warm-up")
-
-    evs = [events() for _ in range(args.steps)]
-    barrier(world)
-    with ClockSampler(local) as clk:
-        for k in range(args.steps):
-            flush()
-            step(evs[k])
-        barrier(world)
-    st_ms = {name: 0.0 for name in STAGES}
-    step_ms = []
-    for ev in evs:
-        for i, name in enumerate(STAGES):
-            st_ms[name] += ev[i].elapsed_time(ev[i + 1])
-        step_ms.append(ev[0].elapsed_time(ev[5]))
-    if p3.check_status(err) != 0:
-        raise RuntimeError("device error during the timed steps")
-    ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
-    st_ms = {k: v / args.steps for k, v in st_ms.items()}
+    timer = StageTimer(p3, s, cfg, d, stream, err)
+    st_ms, ms, clock_rec = timer.run(args.warmup, args.steps, flush, world, local)
     value = replica_value(s.N, world, ms)
+    qr, kr, mem, out = timer.qr, timer.kr, timer.mem, timer.out
 
     # pack3d_forward from the device buffers (same kernels, one C-ABI call).
     ws = torch.empty(p3.workspace_bytes(cfg), dtype=torch.uint8, device=dev)
@@ -547,27 +618,17 @@ def run_ours(args, s):
         train = time_training_block(p3, args, s, cfg, d, inp_host, flush, stream, err, world, rank, dev)
 
     peaks = load_peaks()
-    work = algorithmic_work(s)
-    stages = {}
-    for name in STAGES:
-        t = st_ms[name] * 1e-3
-        w = work[name]
-        e = {"ms": st_ms[name]}
-        if "bytes" in w:
-            e["hbm_gbs"] = w["bytes"] / t / 1e9
-            e["hbm_frac"] = e["hbm_gbs"] / peaks["hbm_gbs"]
-        if "flops" in w:
-            e["tflops"] = w["flops"] / t / 1e12
-            e["tensor_frac"] = e["tflops"] / peaks["bf16_tflops"]
-        stages[name] = e
+    stages = stage_fractions(s, st_ms, peaks)
     variant_err = summary_center_error(p3, s, d, qr, mem, err, stream) if args.summary_center else None
     sa = stages["summary_attn"]
     # A launch of a second or more runs under the board's power cap the whole
     # time, like the measured sustained GEMM loop; shorter ones see burst clocks.
     sustained = sa["ms"] >= SUSTAINED_MS and peaks.get("bf16_tflops_sustained")
     peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    traffic = SUMMARY_ATTN_TRAFFIC.get(args.config)
     roof = {"bound": "tensor", "achieved": sa["tflops"], "peak": peak, "unit": "TFLOP/s",
-            "frac": sa["tflops"] / peak, "traffic": SUMMARY_ATTN_TRAFFIC.get(args.config),
+            "frac": sa["tflops"] / peak, "traffic": traffic[0] if traffic else None,
+            "traffic_source": traffic[1] if traffic else "not captured since the kernel last changed",
             "kernel": "summary_attn_tc_kernel" if s.dtype == "bf16" else "summary_attn_simt_kernel",
             "peak_source": peaks["source"] + (" sustained bf16 (MEASURED_PEAKS.json bf16_tflops_sustained)"
                                               if sustained else " burst bf16 (MEASURED_PEAKS.json bf16_tflops)"),
@@ -587,7 +648,7 @@ def run_ours(args, s):
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "roofline": roof, "stages": stages, "forward_call_ms": fwd,
-            "clocks": clk.summary()}
+            "clocks": clock_rec}
     if variant_err is not None:
         line["summary_center_vs_exact"] = variant_err
     if train is not None:
@@ -605,6 +666,11 @@ def run_ours(args, s):
             comp["dense_sdpa"]["speedup_of_pack3d"] = comp["dense_sdpa"]["ms"] / ms
     if comp:
         line["comparators"] = comp
+    if world == 1 and args.config == "65k" and not args.no_sizes and not args.summary_center:
+        del timer
+        torch.cuda.empty_cache()
+        line["sizes"] = time_sizes(p3, flush, stream, dev, peaks)
+        line["gpu_launches"] += sum(KERNELS_PER_STEP * SIZE_STEPS[n][1] for n in SIZES)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline and args.config not in synth.DEVICE_DRAWN:
             cb = cpu_oracle_sample(s, inp_host, target_s=12.0, center=args.summary_center)
@@ -631,6 +697,8 @@ def main():
     ap.add_argument("--train", action="store_true",
                     help="also time the training block on the device-drawn 4m / 8m volumes")
     ap.add_argument("--no-train", action="store_true", help="skip the training-block leg")
+    ap.add_argument("--no-sizes", action="store_true",
+                    help="skip the 262k / 1M stage timings a default single-GPU run adds")
     ap.add_argument("--train-only", action="store_true",
                     help="time only the training block (pack3d_forward_backward), inputs drawn on the device")
     ap.add_argument("--packing", choices=synth.PACKINGS, default=None,

@@ -3,30 +3,46 @@
 // its clipped lattice box, found through the grid-to-packed map, with no
 // gathered neighbour tensor in global memory).
 //
-// One CTA = one 2 x 4 x 4 brick of query sites of one kv head; with the G = 4
-// query heads of a kv head stacked, that is 128 rows = one tcgen05 M tile
+// Work item = one 2 x 4 x 4 brick of query sites and one kv head; with the
+// G = 4 query heads of a kv head stacked, that is 128 rows = one tcgen05 M tile
 // (row = site * 4 + head, sites z-major, so rows 0-63 are the brick's first
 // z layer and rows 64-127 its second).  The keys of the brick's halo are
-// processed one lattice z-plane at a time: a plane of (4 + 2ry) x (4 + 2rx) <=
-// 10 x 10 sites, padded to NP <= 112 rows, is gathered through the index map
-// with cp.async (keys outside the volume are zero-filled) into a 128-byte-
-// swizzled K tile and V tile.  Per plane:
-//   S = Q K^T  (M=128, N=NP, K=64; A, B from shared memory)
-//   softmax on the rows whose z window contains the plane (the other layer's
-//   warps write P = 0): the lattice-box mask is a per-row bit mask, the
-//   running maximum moves lazily (only by more than 2^8) and O is rescaled in
-//   tensor memory when it does;
-//   O += P V   (M=128, N=64, K=NP; A = P from tensor memory, B = V from
-//   shared memory, MN-major).
-// Pipelining inside the CTA: every index-map lookup of the CTA (its query row
-// and its gather row of each plane) is issued at the start; three plane
-// buffers hold planes 0-2 from the start and plane 3 once plane 0's MMAs are
-// done; S of plane p+1 is issued as soon as every warp has read S of plane p
-// into registers, so it runs under plane p's exponentials.  Two CTAs share an
-// SM (256 tensor-memory columns each: S 0-111, P 128-183, O 192-255).
+// taken one key unit at a time: half of a lattice z-plane of the halo, i.e.
+// (2 + ry) rows of (4 + 2rx) sites (at most 5 x 10 = 50 keys), padded to
+// NU <= 64 keys.  Per unit:
+//   S = Q K^T  (M=128, N=NU, K=64; A, B from shared memory) into one of two
+//   S / P buffers of tensor memory;
+//   softmax on the rows whose z window contains the unit's plane (the other
+//   layer's warps write P = 0): the lattice-box mask is a per-row bit mask of
+//   the unit (the same for every plane of the brick), the running maximum
+//   moves lazily (only by more than 2^8) and O is rescaled in tensor memory
+//   when it does; P (packed bf16) is written over the columns S occupied;
+//   O += P V  (M=128, N=64, K=NU; A = P from tensor memory, B = V from shared
+//   memory, MN-major).
+// The kernel is persistent: CTA c takes items c, c + grid, c + 2 grid, ...,
+// and the units of its items form one stream, so the gathers and MMAs of the
+// next item start while the current one's last units and epilogue run.  The
+// query tile is triple-buffered and the O accumulator double-buffered by item.
+// Warp roles (224 threads, two CTAs per SM):
+//   * warps 0-3, softmax: thread = row = tensor-memory lane;
+//   * warp 4, S: issues S of unit t+2 once O += P V of unit t has freed its
+//     S / P buffer and the unit's keys (and, at an item's first unit, its query
+//     tile) have landed;
+//   * warp 5, P V: issues O += P V of unit t once P(t) is written, never held
+//     up by the S of a later item;
+//   * warp 6, gather: the next item's query rows at the start of each item,
+//     then each unit's K and V rows, through the index map into shared memory
+//     with cp.async (keys outside the volume and padding zero-filled, 128-byte
+//     swizzle), completion signalled on mbarriers; a K / V slot is refilled
+//     once O += P V has read it.
+// An item's output rows leave through its own query tile (no longer read by
+// then): each softmax warp stages its 32 rows there, half a row at a time, and
+// writes them back as whole 128-byte segments, instead of every thread
+// storing its own 256-byte row (32 cache lines per warp instruction).
+// Tensor memory: S / P buffers at columns 0 and 64, O buffers at 128 and 192.
 // Supported: bf16, G = 4, rz = 1, ry <= 3, rx <= 3 (the SIMT kernel covers the
-// rest).  Every mbarrier wait is bounded, and the CTA leaves the plane loop
-// only all together (barrier votes).
+// rest).  Every mbarrier wait is bounded; a CTA that gives up lets its issued
+// copies and MMAs complete before it frees tensor memory.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -37,22 +53,30 @@ namespace pack3d {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kThreads = 128;
-constexpr int kMaxKeys = 112;                     // padded keys per plane
-constexpr int kMaxPlanes = 4;                     // 2 brick layers + r_z = 1 on each side
-constexpr int kTileBytes = kMaxKeys * kDh * 2;    // 14 KiB, a multiple of 1 KiB
-constexpr int kQOff = 0;                          // 16 KiB query tile
-constexpr int kKV0 = kRows * kDh * 2;             // plane buffers: K at +0, V at +kTileBytes
-constexpr int kBufs = 3;
-constexpr int kBufBytes = 2 * kTileBytes;
-constexpr int kBarOff = kKV0 + kBufs * kBufBytes;
-constexpr int kSmemBytes = kBarOff + 64 + 1024;   // + barriers and flags, + alignment slack
-static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+constexpr int kSWarp = 4, kPVWarp = 5, kGatherWarp = 6;
+constexpr int kThreads = 32 * 7;
+constexpr int kUnitKeys = 64;                     // padded keys per unit (half a halo plane)
+constexpr int kTileBytes = kUnitKeys * kDh * 2;   // 8 KiB
+constexpr int kSlots = 3;                         // K / V unit slots
+constexpr int kQBufs = 3;                         // query tiles
+constexpr int kQBytes = kRows * kDh * 2;          // 16 KiB query tile
+constexpr int kSlotOff = kQBufs * kQBytes;        // slot s: K at kSlotOff + 2 s kTileBytes, V after it
+constexpr int kBarOff = kSlotOff + kSlots * 2 * kTileBytes;
+// barriers: q_full[3], q_free[3], kv_full[kSlots], slot_free[kSlots], s_full[2], p_full[2],
+// pv_done[2], o_free[2], drain[2]
+constexpr int kNumBars = 2 * kQBufs + 2 * kSlots + 2 + 2 + 2 + 2 + 2;
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;   // + barriers, wait control, alignment slack
+constexpr int kCtasPerSm = 2;
+static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+constexpr int kTmemCols = 256;                    // S / P buffer b at 64 b, O buffer c at 128 + 64 c
+constexpr int kColO = 128;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct LocalArgs {
   int Z, H, W, Hq, Hkv;
-  int ry, rx, PH, PW, NP;  // plane height/width and padded key count
+  int ry, rx, PW;          // window radii in y and x, halo plane width (4 + 2rx)
+  int UR, UK, NU;          // plane rows per unit (2 + ry), keys per unit, padded to NU (multiple of 16)
+  int nitems;              // bricks x kv heads
   float scale_log2;
   const int32_t* g2p;
   const __nv_bfloat16* q;
@@ -62,8 +86,27 @@ struct LocalArgs {
   float* stats;            // nullable: lse2 of each row to stats[4 row]
   int32_t* err;
   unsigned long long wait_ns;  // limit of every pipeline wait
-  int stall;               // diagnostic: the score MMA of the last plane is never issued
+  int stall;               // diagnostic: the score MMA of the CTA's last unit is never issued
 };
+
+// One work item: brick origin, kv head, the in-volume planes z0-1 .. z0+2 of
+// its halo (unit u = half u % 2 of plane zlo + u / 2).
+struct Item {
+  int g, x0, y0, z0, zlo, nunits;
+};
+
+__device__ __forceinline__ Item decode_item(const LocalArgs& a, int i) {
+  Item it;
+  it.g = i % a.Hkv;
+  const int b = i / a.Hkv;
+  const int nbx = (a.W + 3) / 4, nby = (a.H + 3) / 4;
+  it.x0 = (b % nbx) * 4;
+  it.y0 = ((b / nbx) % nby) * 4;
+  it.z0 = (b / (nbx * nby)) * 2;
+  it.zlo = max(0, it.z0 - 1);
+  it.nunits = 2 * (min(a.Z - 1, it.z0 + 2) - it.zlo + 1);
+  return it;
+}
 
 // Copies one 128-byte row into a 128-byte-swizzled tile at row r (zeros if src == nullptr).
 __device__ __forceinline__ void gather_row(uint32_t tile, int r, const __nv_bfloat16* src,
@@ -78,271 +121,346 @@ __device__ __forceinline__ void gather_row(uint32_t tile, int r, const __nv_bflo
   }
 }
 
-// Packed index of this thread's gather row (row r = threadIdx.x of the padded
-// plane) in lattice plane zp, or -1 (padding or outside the volume).
-__device__ __forceinline__ int plane_row_index(const LocalArgs& a, int zp, int y0, int x0) {
-  const int r = threadIdx.x;
-  if (r >= a.PH * a.PW) return -1;
-  const int y = y0 - a.ry + r / a.PW, x = x0 - a.rx + r % a.PW;
-  if (y < 0 || y >= a.H || x < 0 || x >= a.W) return -1;
-  return __ldg(a.g2p + ((size_t)zp * a.H + y) * a.W + x);
+// Packed index of query row `row` of an item (site row / 4 of the brick), or -1 outside the volume.
+__device__ __forceinline__ int query_index(const LocalArgs& a, const Item& it, int row) {
+  const int site = row >> 2;
+  const int qz = it.z0 + (site >> 4), qy = it.y0 + ((site >> 2) & 3), qx = it.x0 + (site & 3);
+  return (qz < a.Z && qy < a.H && qx < a.W) ? __ldg(a.g2p + ((size_t)qz * a.H + qy) * a.W + qx) : -1;
 }
 
-// K and V rows of this thread's gather row into plane buffer (kt, vt).
-__device__ __forceinline__ void gather_plane(const LocalArgs& a, uint32_t kt, uint32_t vt, int g, int j) {
-  const int r = threadIdx.x;
-  if (r >= a.NP) return;
-  gather_row(kt, r, j >= 0 ? a.k + ((size_t)j * a.Hkv + g) * kDh : nullptr, a.k);
-  gather_row(vt, r, j >= 0 ? a.v + ((size_t)j * a.Hkv + g) * kDh : nullptr, a.v);
-}
-
-__global__ void __launch_bounds__(kThreads, 2) local_attn_tc_kernel(const LocalArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(const LocalArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
-  const uint32_t s_full = sbase + kBarOff;        // S of the current plane is in tensor memory
-  const uint32_t pv_done = sbase + kBarOff + 8;   // O += P V of the last issued plane has completed
-  const uint32_t drain = sbase + kBarOff + 16;    // abort path: every MMA issued so far has completed
-  volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + 24);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 24 + sizeof(ptx::WaitCtl));
+  const uint32_t bar0 = sbase + kBarOff;
+  constexpr int kB = 2 * kQBufs + 2 * kSlots;
+  auto q_full = [&](int c) { return bar0 + 8 * c; };                   // query tile c loaded
+  auto q_free = [&](int c) { return bar0 + 8 * (kQBufs + c); };        // S MMAs done reading tile c
+  auto kv_full = [&](int s) { return bar0 + 8 * (2 * kQBufs + s); };   // slot s holds K and V
+  auto slot_free = [&](int s) { return bar0 + 8 * (2 * kQBufs + kSlots + s); };  // O += P V read slot s
+  auto s_full = [&](int b) { return bar0 + 8 * (kB + b); };            // S in buffer b
+  auto p_full = [&](int b) { return bar0 + 8 * (kB + 2 + b); };        // P in buffer b, O rescaled
+  auto pv_done = [&](int b) { return bar0 + 8 * (kB + 4 + b); };       // O += P V from buffer b done
+  auto o_free = [&](int c) { return bar0 + 8 * (kB + 6 + c); };        // O buffer c read out
+  auto drain = [&](int w) { return bar0 + 8 * (kB + 8 + w); };         // abort path: warp w's MMAs completed
+  volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + 8 * kNumBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * kNumBars + sizeof(ptx::WaitCtl));
   auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int g = blockIdx.y;
-
-  // Brick origin.
-  const int nbx = (a.W + 3) / 4, nby = (a.H + 3) / 4;
-  const int b = blockIdx.x;
-  const int x0 = (b % nbx) * 4, y0 = ((b / nbx) % nby) * 4, z0 = (b / (nbx * nby)) * 2;
-
-  // This thread's row: site (lz, ly, lx) of the brick, head hh.
-  const int site = tid >> 2, hh = tid & 3;
-  const int lz = site >> 4, ly = (site >> 2) & 3, lx = site & 3;
-  const int qz = z0 + lz, qy = y0 + ly, qx = x0 + lx;
-  const bool qvalid = qz < a.Z && qy < a.H && qx < a.W;
-  const int h = g * 4 + hh;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    ptx::mbar_init(s_full, 1);
-    ptx::mbar_init(pv_done, 1);
-    ptx::mbar_init(drain, 1);
+    for (int c = 0; c < kQBufs; ++c) {
+      ptx::mbar_init(q_full(c), 32);           // one cp.async arrival per gather thread
+      ptx::mbar_init(q_free(c), 1);
+    }
+    for (int c = 0; c < 2; ++c) {
+      ptx::mbar_init(s_full(c), 1);
+      ptx::mbar_init(p_full(c), 4);            // one arrival per softmax warp
+      ptx::mbar_init(pv_done(c), 1);
+      ptx::mbar_init(o_free(c), 4);
+    }
+    for (int s = 0; s < kSlots; ++s) {
+      ptx::mbar_init(kv_full(s), 32);
+      ptx::mbar_init(slot_free(s), 1);
+    }
+    ptx::mbar_init(drain(0), 1);
+    ptx::mbar_init(drain(1), 1);
     ctl->abort = 0;
+    ctl->issued = 0;
     ctl->limit_ns = a.wait_ns;
     ptx::fence_mbar_init();
   }
-  if (warp == 0) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 256);
+  if (warp == kSWarp) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
     ptx::tmem_relinquish();
   }
-
-  // Every index-map lookup of the CTA at once: the query row and this
-  // thread's gather row of each plane z0-1 .. z0+2 inside the volume.
-  const int zlo = max(0, z0 - 1), zhi = min(a.Z - 1, z0 + 2);
-  const int nplanes = zhi - zlo + 1;
-  const int qi = qvalid ? __ldg(a.g2p + ((size_t)qz * a.H + qy) * a.W + qx) : -1;
-  int gi[kMaxPlanes];
-#pragma unroll
-  for (int p = 0; p < kMaxPlanes; ++p) gi[p] = p < nplanes ? plane_row_index(a, zlo + p, y0, x0) : -1;
-
-  // cp.async groups: {Q, plane 0}, {plane 1}, {plane 2} (possibly empty), and
-  // later {plane 3} into plane 0's buffer.
-  auto kt_of = [&](int p) { return sbase + kKV0 + (p % kBufs) * kBufBytes; };
-  gather_row(sbase + kQOff, tid, qi >= 0 ? a.q + ((size_t)qi * a.Hq + h) * kDh : nullptr, a.q);
-  gather_plane(a, kt_of(0), kt_of(0) + kTileBytes, g, gi[0]);
-  ptx::cp_async_commit();
-  if (nplanes > 1) gather_plane(a, kt_of(1), kt_of(1) + kTileBytes, g, gi[1]);
-  ptx::cp_async_commit();
-  if (nplanes > 2) gather_plane(a, kt_of(2), kt_of(2) + kTileBytes, g, gi[2]);
-  ptx::cp_async_commit();
-
-  // Lattice-box mask of this row over the padded plane (bit k = key k
-  // allowed): the row's x run [lx, lx + 2rx] limited to in-volume columns,
-  // repeated on the plane rows [ly, ly + 2ry] that lie inside the volume.
-  uint32_t mask[4];
-  {
-    uint32_t xvalid = 0;
-    for (int kx = 0; kx < a.PW; ++kx) {
-      const int x = x0 - a.rx + kx;
-      if (x >= 0 && x < a.W) xvalid |= 1u << kx;
-    }
-    const uint32_t xbits = (((1u << (2 * a.rx + 1)) - 1u) << lx) & xvalid;
-    unsigned __int128 m = 0;
-    for (int dy = 0; dy <= 2 * a.ry; ++dy) {
-      const int ky = ly + dy, y = y0 - a.ry + ky;
-      if (y >= 0 && y < a.H) m |= (unsigned __int128)xbits << (ky * a.PW);
-    }
-    mask[0] = (uint32_t)m;
-    mask[1] = (uint32_t)(m >> 32);
-    mask[2] = (uint32_t)(m >> 64);
-    mask[3] = (uint32_t)(m >> 96);
-  }
-
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-  const uint32_t tS = trow, tP = trow + 128, tO = trow + 192;
-  const uint32_t idescS = ptx::idesc_bf16_f32(kRows, a.NP, false);
-  const uint32_t idescPV = ptx::idesc_bf16_f32(kRows, kDh, true);
-  const float c = a.scale_log2;
+  auto q_tile = [&](int k) { return sbase + (k % kQBufs) * kQBytes; };
+  auto k_tile = [&](int t) { return sbase + kSlotOff + (t % kSlots) * 2 * kTileBytes; };
 
-  auto issue_s = [&](int p) {
-    ptx::tc_fence_after();
-    const uint32_t kt = kt_of(p);
+  if (warp == kGatherWarp) {
+    // ---------------- gather: query rows lane + 32 i, K / V rows lane and lane + 32 ----------------
+    int r[2], kyr[2], kxo[2];
 #pragma unroll
-    for (int kk = 0; kk < kDh / 16; ++kk)
-      ptx::mma_ss(tmem, ptx::smem_desc_sw128(sbase + kQOff + kk * 32, 16, 1024),
-                  ptx::smem_desc_sw128(kt + kk * 32, 16, 1024), idescS, kk > 0);
-    ptx::tc_commit(s_full);
-  };
-
-  // S of plane 0 once Q and plane 0 are in shared memory (group 0 of 3).
-  ptx::cp_async_wait_two();
-  ptx::fence_proxy_async_smem();
-  __syncthreads();
-  // (PACK3D_FLAG_DIAG_STALL withholds the score MMA of the last plane.)
-  if (tid == 0 && !(a.stall && nplanes == 1)) issue_s(0);
-
-  float m_used = -INFINITY, l = 0.f;
-  bool ok = true;
-  for (int p = 0; p < nplanes; ++p) {
-    const int zp = zlo + p;
-    const bool uses = zp >= z0 + lz - 1 && zp <= z0 + lz + 1;  // warp-uniform (layer = warp / 2)
-    // S of plane p; each using warp keeps its rows in registers.
-    bool w_ok = __all_sync(0xffffffffu, wait(s_full, p & 1));
-    uint32_t sv[kMaxKeys];
-    if (w_ok) {
-      ptx::tc_fence_after();
-      if (uses) {
-        ptx::tmem_ld64_sync(tS, sv);
-        ptx::tmem_ld48_sync(tS + 64, sv + 64);
-      }
+    for (int i = 0; i < 2; ++i) {
+      r[i] = lane + 32 * i;
+      kyr[i] = r[i] / a.PW;
+      kxo[i] = r[i] % a.PW;
     }
-    // Plane p+1 landed (groups: after plane 0 one more may be pending, later none).
-    if (p == 0) ptx::cp_async_wait_one(); else ptx::cp_async_wait_all();
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    if (!(ok = __syncthreads_and(w_ok))) break;
-    // Every warp has read S(p): S(p+1) may overwrite it and run under this
-    // plane's exponentials.
-    if (tid == 0 && p + 1 < nplanes && !(a.stall && p + 2 == nplanes)) issue_s(p + 1);
-
-    float f = 1.f, rs = 0.f;
-    if (uses) {
-      // Masked row maximum: 8 independent max3 chains.
-      float m8[8];
+    auto key_index = [&](const Item& it, int u, int i) {
+      const int y = it.y0 - a.ry + (u & 1) * a.UR + kyr[i];
+      const int x = it.x0 - a.rx + kxo[i];
+      return (r[i] < a.UK && x >= 0 && x < a.W && y >= 0 && y < a.H)
+                 ? __ldg(a.g2p + ((size_t)(it.zlo + (u >> 1)) * a.H + y) * a.W + x)
+                 : -1;
+    };
+    // Query rows of item k (lane + 32 rr) into query tile k % kQBufs, once the S
+    // MMAs of item k - kQBufs have finished reading that tile.
+    auto load_query = [&](int k, int i) {
+      // The tile's previous item: its S MMAs are done and its output has left the tile.
+      if (k >= kQBufs && !(wait(q_free(k % kQBufs), ((k / kQBufs) - 1) & 1) &&
+                           wait(o_free((k - kQBufs) & 1), ((k - kQBufs) >> 1) & 1)))
+        return false;
+      const Item it = decode_item(a, i);
+      int qi[4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+      for (int rr = 0; rr < 4; ++rr) qi[rr] = query_index(a, it, lane + 32 * rr);
 #pragma unroll
-      for (int k = 0; k < kMaxKeys; k += 2) {
-        const float s0 = (mask[k >> 5] >> (k & 31)) & 1u ? __uint_as_float(sv[k]) : -INFINITY;
-        const float s1 = (mask[(k + 1) >> 5] >> ((k + 1) & 31)) & 1u ? __uint_as_float(sv[k + 1]) : -INFINITY;
-        sv[k] = __float_as_uint(s0);
-        sv[k + 1] = __float_as_uint(s1);
-        float& mq = m8[(k >> 1) & 7];
-        asm("max.f32 %0, %0, %1, %2;" : "+f"(mq) : "f"(s0), "f"(s1));
+      for (int rr = 0; rr < 4; ++rr) {
+        const int row = lane + 32 * rr;
+        const int h = it.g * 4 + (row & 3);
+        gather_row(q_tile(k), row, qi[rr] >= 0 ? a.q + ((size_t)qi[rr] * a.Hq + h) * kDh : nullptr, a.q);
       }
-      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      const float mxs = mx * c;
-      if (m_used == -INFINITY) {
-        m_used = mxs;            // first plane this row sees: its O row is still zero
-      } else if (mxs > m_used + kRescaleThreshold) {
-        f = ptx::ex2(m_used - mxs);
-        m_used = mxs;
-      }
-    }
-    // P and O are free again once O += P V of plane p-1 has completed.
-    if (p > 0) {
-      w_ok = __all_sync(0xffffffffu, wait(pv_done, (p - 1) & 1));
-      if (w_ok) ptx::tc_fence_after();
-    }
-    if (p == 1 && nplanes > 3 && w_ok) {
-      // Plane 0's buffer (read by S(0) and O += P V of plane 0, both done) takes plane 3.
-      gather_plane(a, kt_of(3), kt_of(3) + kTileBytes, g, gi[3]);
-    }
-    if (p == 1) ptx::cp_async_commit();
-    if (uses && w_ok) {
-      // A row with no allowed key yet (only rows of sites outside the volume)
-      // keeps P = 0 instead of exp2(-inf + inf).
-      const float nm = m_used == -INFINITY ? 0.f : -m_used;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(nm, nm);
-      float2 r2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int q = 0; q < kMaxKeys / 16; ++q) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int i = 16 * q + 2 * k;
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), c2, nm2);
-          const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
-          r2[k & 1] = __fadd2_rn(r2[k & 1], pe);
-          pk[k] = pack_bf16x2(pe.x, pe.y);
-        }
-        ptx::tmem_st8(tP + 8 * q, pk);
-      }
-      rs = (r2[0].x + r2[0].y) + (r2[1].x + r2[1].y);
-      if (__any_sync(0xffffffffu, f != 1.f)) {
-        uint32_t r[32];
+      ptx::cp_async_mbar_arrive(q_full(k % kQBufs));
+      return true;
+    };
+    bool ok = blockIdx.x < a.nitems ? load_query(0, blockIdx.x) : true;
+    int t = 0;
+    for (int k = 0, i = blockIdx.x; ok && i < a.nitems; ++k, i += gridDim.x) {
+      const Item it = decode_item(a, i);
+      int j[2] = {key_index(it, 0, 0), key_index(it, 0, 1)};
+      if (i + gridDim.x < a.nitems && !(ok = load_query(k + 1, i + gridDim.x))) break;
+      for (int u = 0; u < it.nunits; ++u, ++t) {
+        if (t >= kSlots && !(ok = wait(slot_free(t % kSlots), ((t / kSlots) - 1) & 1))) break;
+        const uint32_t kt = k_tile(t), vt = kt + kTileBytes;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          ptx::tmem_ld32_sync(tO + 32 * q, r);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
-          ptx::tmem_st32(tO + 32 * q, r);
+          gather_row(kt, r[q], j[q] >= 0 ? a.k + ((size_t)j[q] * a.Hkv + it.g) * kDh : nullptr, a.k);
+          gather_row(vt, r[q], j[q] >= 0 ? a.v + ((size_t)j[q] * a.Hkv + it.g) * kDh : nullptr, a.v);
+        }
+        ptx::cp_async_mbar_arrive(kv_full(t % kSlots));
+        if (u + 1 < it.nunits) {
+          j[0] = key_index(it, u + 1, 0);
+          j[1] = key_index(it, u + 1, 1);
         }
       }
-      l = l * f + rs;
-    } else if (w_ok) {
-      uint32_t zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-      for (int q = 0; q < kMaxKeys / 16; ++q) ptx::tmem_st8(tP + 8 * q, zero);
     }
-    ptx::tmem_wait_st();
-    ptx::tc_fence_before();
-    if (!(ok = __syncthreads_and(w_ok))) break;
-    if (tid == 0) {
+  } else if (warp == kSWarp || warp == kPVWarp) {
+    // ---------------- MMA issue (lane 0 of the S warp and of the P V warp) ----------------
+    if (lane == 0) {
+      const uint32_t idescS = ptx::idesc_bf16_f32(kRows, a.NU, false);
+      const uint32_t idescPV = ptx::idesc_bf16_f32(kRows, kDh, true);
+      // Cursor over the CTA's unit stream: item number k, item index i, unit u, global unit t.
+      int k = 0, i = blockIdx.x, u = 0, t = 0;
+      int n = i < a.nitems ? decode_item(a, i).nunits : 0;
+      auto next = [&]() {
+        ++t;
+        if (++u == n) {
+          ++k;
+          i += gridDim.x;
+          u = 0;
+          n = i < a.nitems ? decode_item(a, i).nunits : 0;
+        }
+      };
+      int total = 0;
+      for (int ii = blockIdx.x; ii < a.nitems; ii += gridDim.x) total += decode_item(a, ii).nunits;
+      bool ok = true;
+      if (warp == kSWarp) {
+        // S(t) into buffer t % 2 once K(t) (and, at an item's first unit, its query tile) has
+        // landed and O += P V(t-2) has read that buffer's P.  (PACK3D_FLAG_DIAG_STALL
+        // withholds the S of the CTA's last unit.)
+        const int s_units = a.stall ? total - 1 : total;
+        for (; ok && t < s_units; next()) {
+          if (!(ok = wait(kv_full(t % kSlots), (t / kSlots) & 1))) break;
+          if (u == 0 && !(ok = wait(q_full(k % kQBufs), (k / kQBufs) & 1))) break;
+          if (t >= 2 && !(ok = wait(pv_done(t & 1), ((t >> 1) - 1) & 1))) break;
+          ptx::tc_fence_after();
+          const uint32_t kt = k_tile(t), qt = q_tile(k);
+#pragma unroll
+          for (int kk = 0; kk < kDh / 16; ++kk)
+            ptx::mma_ss(tmem + 64 * (t & 1), ptx::smem_desc_sw128(qt + kk * 32, 16, 1024),
+                        ptx::smem_desc_sw128(kt + kk * 32, 16, 1024), idescS, kk > 0);
+          ptx::tc_commit(s_full(t & 1));
+          if (u == n - 1) ptx::tc_commit(q_free(k % kQBufs));   // the item's last read of its query tile
+        }
+      } else {
+        // O(item) += P(t) V(t) once the softmax warps have written P(t); an item's first unit
+        // starts its O buffer afresh once the softmax warps have read out the item two back.
+        for (; ok && t < total; next()) {
+          if (!(ok = wait(p_full(t & 1), (t >> 1) & 1))) break;
+          if (u == 0 && k >= 2 && !(ok = wait(o_free(k & 1), ((k >> 1) - 1) & 1))) break;
+          ptx::tc_fence_after();
+          const uint32_t vt = k_tile(t) + kTileBytes;
+          const uint32_t tO = tmem + kColO + 64 * (k & 1);
+          for (int kk = 0; kk < a.NU / 16; ++kk)
+            ptx::mma_ts(tO, tmem + 64 * (t & 1) + kk * 8, ptx::smem_desc_sw128(vt + kk * 2048, 8192, 1024),
+                        idescPV, (u > 0 || kk > 0) ? 1u : 0u);
+          ptx::tc_commit(pv_done(t & 1));
+          ptx::tc_commit(slot_free(t % kSlots));
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax warps: thread = row = tensor-memory lane ----------------
+    const int site = tid >> 2, hh = tid & 3;
+    const int lz = site >> 4, ly = (site >> 2) & 3, lx = site & 3;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const float c = a.scale_log2;
+    bool ok = true;
+    int t = 0;
+    for (int k = 0, i = blockIdx.x; ok && i < a.nitems; ++k, i += gridDim.x) {
+      const Item it = decode_item(a, i);
+      const int qi = query_index(a, it, tid);   // where this row's output goes (read at the item's end)
+      const bool qvalid = it.z0 + lz < a.Z && it.y0 + ly < a.H && it.x0 + lx < a.W;
+      // Lattice-box mask of this row over each half's unit (bit k = key k of the
+      // unit allowed): plane row ky = half * UR + k / PW and column kx = k % PW
+      // must lie in [ly, ly + 2ry] x [lx, lx + 2rx] and inside the volume.  It is
+      // the same for every plane of the brick.
+      uint32_t mask0[2], mask1[2];   // half 0 / half 1 of a plane, bits 0-31 and 32-63
+      {
+        uint32_t xvalid = 0;
+        for (int kx = 0; kx < a.PW; ++kx) {
+          const int x = it.x0 - a.rx + kx;
+          if (x >= 0 && x < a.W) xvalid |= 1u << kx;
+        }
+        const uint32_t xbits = qvalid ? (((1u << (2 * a.rx + 1)) - 1u) << lx) & xvalid : 0u;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint64_t m = 0;
+          for (int kr = 0; kr < a.UR; ++kr) {
+            const int ky = half * a.UR + kr, y = it.y0 - a.ry + ky;
+            if (ky >= ly && ky <= ly + 2 * a.ry && y >= 0 && y < a.H) m |= (uint64_t)xbits << (kr * a.PW);
+          }
+          (half ? mask1 : mask0)[0] = (uint32_t)m;
+          (half ? mask1 : mask0)[1] = (uint32_t)(m >> 32);
+        }
+      }
+      const uint32_t tO = trow + kColO + 64 * (k & 1);
+      float m_used = -INFINITY, l = 0.f;
+      for (int u = 0; u < it.nunits; ++u, ++t) {
+        const int zp = it.zlo + (u >> 1);
+        const bool uses = zp >= it.z0 + lz - 1 && zp <= it.z0 + lz + 1;  // warp-uniform (layer = warp / 2)
+        const uint32_t tS = trow + 64 * (t & 1);
+        if (!(ok = __all_sync(0xffffffffu, wait(s_full(t & 1), (t >> 1) & 1)))) break;
+        ptx::tc_fence_after();
+        if (uses) {
+          uint32_t sv[kUnitKeys];
+          ptx::tmem_ld64_sync(tS, sv);
+          // Masked row maximum: 8 independent max3 chains.
+          const uint32_t mk[2] = {(u & 1) ? mask1[0] : mask0[0], (u & 1) ? mask1[1] : mask0[1]};
+          float m8[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+          for (int kk = 0; kk < kUnitKeys; kk += 2) {
+            const float s0 = (mk[kk >> 5] >> (kk & 31)) & 1u ? __uint_as_float(sv[kk]) : -INFINITY;
+            const float s1 = (mk[kk >> 5] >> ((kk + 1) & 31)) & 1u ? __uint_as_float(sv[kk + 1]) : -INFINITY;
+            sv[kk] = __float_as_uint(s0);
+            sv[kk + 1] = __float_as_uint(s1);
+            float& mq = m8[(kk >> 1) & 7];
+            asm("max.f32 %0, %0, %1, %2;" : "+f"(mq) : "f"(s0), "f"(s1));
+          }
+          const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          const float mxs = mx * c;
+          float f = 1.f;
+          if (m_used == -INFINITY) {
+            m_used = mxs;            // first unit this row sees a key in: its O row is still zero
+          } else if (mxs > m_used + kRescaleThreshold) {
+            f = ptx::ex2(m_used - mxs);
+            m_used = mxs;
+          }
+          // A row with no allowed key yet (only rows of sites outside the volume)
+          // keeps P = 0 instead of exp2(-inf + inf).
+          const float nm = m_used == -INFINITY ? 0.f : -m_used;
+          const float2 c2 = make_float2(c, c), nm2 = make_float2(nm, nm);
+          float2 r2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int q = 0; q < kUnitKeys / 16; ++q) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const int e = 16 * q + 2 * kk;
+              const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2, nm2);
+              const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+              r2[kk & 1] = __fadd2_rn(r2[kk & 1], pe);
+              pk[kk] = pack_bf16x2(pe.x, pe.y);
+            }
+            ptx::tmem_st8(tS + 8 * q, pk);   // P over the S columns this warp has read
+          }
+          if (__any_sync(0xffffffffu, f != 1.f)) {
+            // O is rescaled once O += P V of the item's previous unit has completed,
+            // before this unit's O += P V is issued.
+            if (!(ok = __all_sync(0xffffffffu, wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1)))) break;
+            ptx::tc_fence_after();
+            uint32_t o[32];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              ptx::tmem_ld32_sync(tO + 32 * q, o);
+#pragma unroll
+              for (int kk = 0; kk < 32; ++kk) o[kk] = __float_as_uint(__uint_as_float(o[kk]) * f);
+              ptx::tmem_st32(tO + 32 * q, o);
+            }
+          }
+          l = l * f + ((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y));
+        } else {
+          const uint32_t zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+          for (int q = 0; q < kUnitKeys / 16; ++q) ptx::tmem_st8(tS + 8 * q, zero);
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(p_full(t & 1));
+      }
+      if (!ok) break;
+      // The item's output: its last O += P V has completed.
+      if (!(ok = __all_sync(0xffffffffu, wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1)))) break;
       ptx::tc_fence_after();
-      const uint32_t vt = kt_of(p) + kTileBytes;
-      for (int kk = 0; kk < a.NP / 16; ++kk)
-        ptx::mma_ts(tO, tmem + 128 + kk * 8, ptx::smem_desc_sw128(vt + kk * 2048, 8192, 1024), idescPV,
-                    (p > 0 || kk > 0) ? 1u : 0u);
-      ptx::tc_commit(pv_done);
+      uint32_t o[2][32];
+      ptx::tmem_ld64_sync(tO, &o[0][0]);
+      const float inv = 1.f / l;
+      if (a.stats && qi >= 0) a.stats[4 * ((size_t)qi * a.Hq + it.g * 4 + hh)] = m_used + log2f(l);
+      // Rows 32 warp .. 32 warp + 31 of the item's query tile hold this warp's
+      // staging: row r, 16-byte chunk c at r * 128 + (c ^ (r % 8)) * 16.
+      const uint32_t stg = q_tile(k) + warp * 32 * 128;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          ptx::st_shared_v4(stg + lane * 128 + ((cc ^ (lane & 7)) << 4),
+                            __float_as_uint(__uint_as_float(o[half][4 * cc]) * inv),
+                            __float_as_uint(__uint_as_float(o[half][4 * cc + 1]) * inv),
+                            __float_as_uint(__uint_as_float(o[half][4 * cc + 2]) * inv),
+                            __float_as_uint(__uint_as_float(o[half][4 * cc + 3]) * inv));
+        __syncwarp();
+        // Four rows per instruction: lanes 8 r' .. 8 r' + 7 write row 4 s + r' of the warp.
+#pragma unroll
+        for (int s4 = 0; s4 < 8; ++s4) {
+          const int rw = 4 * s4 + (lane >> 3), cc = lane & 7;
+          const int dst_i = __shfl_sync(0xffffffffu, qi, rw);
+          const uint4 v = ptx::ld_shared_v4(stg + rw * 128 + ((cc ^ (rw & 7)) << 4));
+          if (dst_i >= 0)
+            *reinterpret_cast<uint4*>(a.oloc + ((size_t)dst_i * a.Hq + it.g * 4 + (rw & 3)) * kDh + 32 * half +
+                                      4 * cc) = v;
+        }
+        __syncwarp();
+      }
+      ptx::tc_fence_before();
+      if (lane == 0) ptx::mbar_arrive(o_free(k & 1));
     }
   }
 
-  if (ok) ok = __all_sync(0xffffffffu, wait(pv_done, (nplanes - 1) & 1));
-  if (ok) {
-    ptx::tc_fence_after();
-    uint32_t r[2][32];
-    ptx::tmem_ld64_sync(tO, &r[0][0]);
-    if (qi >= 0) {
-      const float inv = 1.f / l;
-      if (a.stats) a.stats[4 * ((size_t)qi * a.Hq + h)] = m_used + log2f(l);
-      float4* o = reinterpret_cast<float4*>(a.oloc + ((size_t)qi * a.Hq + h) * kDh);
-#pragma unroll
-      for (int q = 0; q < kDh / 4; ++q)
-        o[q] = make_float4(__uint_as_float(r[q / 8][(4 * q) % 32]) * inv,
-                           __uint_as_float(r[q / 8][(4 * q + 1) % 32]) * inv,
-                           __uint_as_float(r[q / 8][(4 * q + 2) % 32]) * inv,
-                           __uint_as_float(r[q / 8][(4 * q + 3) % 32]) * inv);
-    }
-  }
-  ptx::cp_async_wait_all();
+  ptx::cp_async_wait_all();            // the gather warp's copies
   ptx::tc_fence_before();
   __syncthreads();
   if (ctl->abort) {
-    // The flag is final here (every thread has left the plane loop).  The
-    // MMAs thread 0 issued complete before tensor memory is released.
-    if (tid == 0) {
-      ptx::tc_commit(drain);
-      ptx::mbar_wait_drain(drain, 0, ctl->limit_ns);
+    // The flag is final here (every role has finished).  The MMAs each issuing
+    // warp started complete before tensor memory is released.
+    if ((warp == kSWarp || warp == kPVWarp) && lane == 0) {
+      ptx::tc_commit(drain(warp - kSWarp));
+      ptx::mbar_wait_drain(drain(warp - kSWarp), 0, ctl->limit_ns);
     }
     ptx::tc_fence_before();
     __syncthreads();
   }
-  if (warp == 0) {
+  if (warp == kSWarp) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 256);
+    ptx::tmem_dealloc(tmem, kTmemCols);
   }
   if (tid == 0 && ctl->abort) set_err(a.err, PACK3D_DEVERR_TIMEOUT);
 }
@@ -366,8 +484,11 @@ cudaError_t launch_local_attn_tc(const Shape& s, const int32_t* g2p, const void*
   LocalArgs a;
   a.Z = s.Z; a.H = s.H; a.W = s.W; a.Hq = s.Hq; a.Hkv = s.Hkv;
   a.ry = s.ry; a.rx = s.rx;
-  a.PH = 4 + 2 * s.ry; a.PW = 4 + 2 * s.rx;
-  a.NP = (a.PH * a.PW + 15) / 16 * 16;
+  a.PW = 4 + 2 * s.rx;
+  a.UR = 2 + s.ry;                        // half of the 4 + 2ry plane rows
+  a.UK = a.UR * a.PW;                     // <= 50 keys
+  a.NU = (a.UK + 15) / 16 * 16;           // <= 64
+  a.nitems = ((s.Z + 1) / 2) * ((s.H + 3) / 4) * ((s.W + 3) / 4) * s.Hkv;
   a.scale_log2 = s.scale_log2;
   a.g2p = g2p;
   a.q = (const __nv_bfloat16*)qr;
@@ -380,7 +501,9 @@ cudaError_t launch_local_attn_tc(const Shape& s, const int32_t* g2p, const void*
   a.stall = s.stall;
   cudaError_t e = cudaFuncSetAttribute(local_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(((s.Z + 1) / 2) * ((s.H + 3) / 4) * ((s.W + 3) / 4)), s.Hkv);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = min(a.nitems, kCtasPerSm * max(1, sms));
   local_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(a);
   return cudaGetLastError();
 }

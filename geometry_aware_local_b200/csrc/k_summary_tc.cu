@@ -164,6 +164,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       }
     }
     ctl->abort = 0;
+    ctl->issued = 0;
     ctl->limit_ns = a.wait_ns;
     ptx::fence_mbar_init();
   }
@@ -175,7 +176,6 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  int issued = 0;   // producer: summary tiles whose loads were issued
 
   if (warp == kTmaWarp) {
     // ---------------- TMA producer ----------------
@@ -188,6 +188,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       for (int w = 0; w < kGroups; ++w)
         ptx::tma_load_4d(sbase + kQOff + w * kQBytes, &tmQ, 0, 0, g, (tile0 + w) * tok_per_tile, qfull);
       const int T_load = a.stall ? T - 1 : T;
+      int issued = 0;
       for (int j = 0; j < T_load; ++j) {
         const int st = j % kStages;
         if (j >= kStages && !wait(empty(st), ((j / kStages) - 1) & 1)) break;
@@ -197,6 +198,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         ptx::tma_load_3d(dst + kKVBytes, &tmV, 0, g, j * kBN, full(st));
         issued = j + 1;
       }
+      ctl->issued = issued;
     }
     __syncwarp();
   } else if (warp >= kMmaWarp) {
@@ -251,6 +253,12 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           ptx::tc_fence_after();
           issue_pv(j, c);
         }
+      }
+      if (!ok) {
+        // Gave up: let this warp's MMAs complete now (phase 0 of drain(w);
+        // the end of the kernel then finds it done and skips its own drain).
+        ptx::tc_commit(drain(w));
+        ptx::mbar_wait_drain(drain(w), 0, ctl->limit_ns);
       }
     }
     __syncwarp();
@@ -410,12 +418,13 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     // Every role has finished, so the flag is final and the same for all
     // threads.  Before tensor memory and shared memory are released, the MMAs
     // each issuing warp started and the loads the producer started complete.
-    if (warp >= kMmaWarp && warp < kTmaWarp && lane == 0) {
+    if (warp >= kMmaWarp && warp < kTmaWarp && lane == 0 && !ptx::mbar_test_wait(drain(warp - kMmaWarp), 0)) {
       ptx::tc_commit(drain(warp - kMmaWarp));
       ptx::mbar_wait_drain(drain(warp - kMmaWarp), 0, ctl->limit_ns);
     }
     if (warp == kTmaWarp && lane == 0) {
       ptx::mbar_wait_drain(qfull, 0, ctl->limit_ns);
+      const int issued = ctl->issued;
       for (int j = max(0, issued - kStages); j < issued; ++j)
         ptx::mbar_wait_drain(full(j % kStages), (j / kStages) & 1, ctl->limit_ns);
     }

@@ -54,11 +54,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Per-CTA state of the bounded waits, in shared memory: the abort flag every
-// role polls, and the wait limit (kept here rather than in registers, since it
-// is read only on the slow path of a wait).
+// role polls, the wait limit (kept here rather than in registers, since it is
+// read only on the slow path of a wait) and, for kernels with a TMA producer,
+// how many stages' loads it issued (read by the abort path's drain).
 struct WaitCtl {
   int abort;
-  int pad;
+  int issued;
   unsigned long long limit_ns;
 };
 
@@ -276,6 +277,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Arrives on mbarrier `bar` once every cp.async this thread issued before has
+// completed (the arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_two() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
@@ -317,6 +323,11 @@ __host__ __device__ constexpr uint32_t sw128_offset(uint32_t r, uint32_t e) {
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ float ex2(float x) {
