@@ -70,7 +70,10 @@ KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summ
 # workload, with the capture it came from; the summary of the capture is kept
 # under profiles/.  Emptied whenever that kernel changes until it is captured
 # again (a workload without an entry reports null).
-SUMMARY_ATTN_TRAFFIC: Dict[str, tuple] = {}
+SUMMARY_ATTN_TRAFFIC: Dict[str, tuple] = {
+    "65k": (212.776704e6 + 48.349696e6,
+            "ncu capture of summary_attn_tc_kernel<0> on the 65k volume (profiles/summary_attn_tc_65k.md)"),
+}
 # The benchmark spec's nominal HBM bandwidth, reported beside the measured copy peak.
 HBM_NOMINAL_GBS = 8000.0
 # Volumes timed in the `sizes` block of a default single-GPU run.
