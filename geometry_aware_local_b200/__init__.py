@@ -46,7 +46,8 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: 
 
 ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
                 "pack3d_build_index", "pack3d_rope", "pack3d_rope_qk", "pack3d_build_summaries", "pack3d_local_attn",
-                "pack3d_summary_attn", "pack3d_forward", "pack3d_forward_noalloc", "pack3d_pipeline_create",
+                "pack3d_summary_attn", "pack3d_summary_attn_rows", "pack3d_forward", "pack3d_forward_noalloc",
+                "pack3d_pipeline_create",
                 "pack3d_pipeline_destroy", "pack3d_host_workspace_bytes", "pack3d_forward_host",
                 "pack3d_train_workspace_bytes", "pack3d_forward_backward", "pack3d_check_status",
                 "pack3d_status_string", "pack3d_backend_info")
@@ -68,7 +69,8 @@ class Config(ctypes.Structure):
                 ("rz", ctypes.c_int32), ("ry", ctypes.c_int32), ("rx", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("dtype", ctypes.c_int32),
                 ("flags", ctypes.c_int32), ("wait_limit_us", ctypes.c_int32),
-                ("coord_scale", ctypes.c_double * 3)]
+                ("coord_scale", ctypes.c_double * 3), ("origin", ctypes.c_int32 * 3),
+                ("reserved2", ctypes.c_int32)]
 
     @property
     def N(self) -> int:
@@ -99,6 +101,7 @@ def _load():
         "pack3d_build_summaries": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
         "pack3d_local_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
         "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
+        "pack3d_summary_attn_rows": (ctypes.c_int, [C, ctypes.c_int64, ctypes.c_int64] + [P] * 8),
         "pack3d_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
         "pack3d_forward_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
         "pack3d_pipeline_create": (ctypes.c_int, [ctypes.POINTER(P)]),
@@ -133,7 +136,8 @@ def make_config(Z: int, H: int, W: int, *, Hq: int = 8, Hkv: int = 2, d_h: int =
                 m: Sequence[int] = (11, 11, 10), rope_base: float = 10000.0,
                 block: Sequence[int] = (1, 4, 4), radius: Sequence[int] = (1, 3, 3),
                 softmax_scale: Optional[float] = None, dtype: str = "bf16", flags: int = 0,
-                coord_scale: Sequence[float] = (1.0, 1.0, 1.0), wait_limit_us: int = 0) -> Config:
+                coord_scale: Sequence[float] = (1.0, 1.0, 1.0), wait_limit_us: int = 0,
+                origin: Sequence[int] = (0, 0, 0)) -> Config:
     c = Config()
     c.Z, c.H, c.W = Z, H, W
     c.Hq, c.Hkv, c.d_h = Hq, Hkv, d_h
@@ -146,6 +150,7 @@ def make_config(Z: int, H: int, W: int, *, Hq: int = 8, Hkv: int = 2, d_h: int =
     c.flags = flags
     c.wait_limit_us = wait_limit_us
     c.coord_scale[:] = [float(x) for x in coord_scale]
+    c.origin[:] = [int(x) for x in origin]
     return c
 
 
@@ -154,7 +159,8 @@ def config_from_shape(s, flags: int = 0, wait_limit_us: int = 0) -> Config:
     return make_config(s.Z, s.H, s.W, Hq=s.Hq, Hkv=s.Hkv, d_h=s.d_h, m=(s.m_z, s.m_y, s.m_x),
                        rope_base=s.rope_base, block=(s.bz, s.by, s.bx), radius=(s.rz, s.ry, s.rx),
                        softmax_scale=s.softmax_scale, dtype=s.dtype, flags=flags,
-                       coord_scale=getattr(s, "coord_scale", (1.0, 1.0, 1.0)), wait_limit_us=wait_limit_us)
+                       coord_scale=getattr(s, "coord_scale", (1.0, 1.0, 1.0)), wait_limit_us=wait_limit_us,
+                       origin=getattr(s, "origin", (0, 0, 0)))
 
 
 def validate(cfg: Config) -> int:
@@ -283,6 +289,31 @@ def summary_attn(cfg, q_rot, k_sum, v_sum, o_loc, gate, out, err=None, stream=No
     _check_err("summary_attn", err)
     _check(lib.pack3d_summary_attn(ctypes.byref(cfg), _ptr(q_rot), _ptr(k_sum), _ptr(v_sum), _ptr(o_loc),
                                    _ptr(gate), _ptr(out), _ptr(err), _stream(stream)), "pack3d_summary_attn")
+
+
+def summary_attn_rows(cfg, tokens: int, summaries: int, q_rot, k_sum, v_sum, o_loc, gate, out, err=None,
+                      stream=None):
+    """Stages 4+5 for `tokens` query tokens against `summaries` summaries (pack3d_summary_attn_rows):
+    q_rot / out [tokens, Hq, d_h], o_loc [tokens, Hq, d_h] float, gate [tokens, Hq, 2] float,
+    k_sum / v_sum [summaries, Hkv, d_h]; the config supplies heads, scale, dtype and flags."""
+    import torch
+    if validate(cfg) == 0:
+        tdt = torch.bfloat16 if cfg.dtype == BF16 else torch.float32
+        want = {"q_rot": (tdt, tokens * cfg.Hq * cfg.d_h), "out": (tdt, tokens * cfg.Hq * cfg.d_h),
+                "k_sum": (tdt, summaries * cfg.Hkv * cfg.d_h), "v_sum": (tdt, summaries * cfg.Hkv * cfg.d_h),
+                "o_loc": (torch.float32, tokens * cfg.Hq * cfg.d_h), "gate": (torch.float32, tokens * cfg.Hq * 2)}
+        for name, t in (("q_rot", q_rot), ("out", out), ("k_sum", k_sum), ("v_sum", v_sum), ("o_loc", o_loc),
+                        ("gate", gate)):
+            if t is None or isinstance(t, int):
+                continue
+            dt, count = want[name]
+            if t.dtype != dt or t.numel() != count:
+                raise ValueError(f"summary_attn_rows: {name} must be {dt} with {count} elements, "
+                                 f"got {t.dtype} with {t.numel()}")
+    _check_err("summary_attn_rows", err)
+    _check(lib.pack3d_summary_attn_rows(ctypes.byref(cfg), int(tokens), int(summaries), _ptr(q_rot), _ptr(k_sum),
+                                        _ptr(v_sum), _ptr(o_loc), _ptr(gate), _ptr(out), _ptr(err),
+                                        _stream(stream)), "pack3d_summary_attn_rows")
 
 
 def _check_forward_args(what, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err):

@@ -32,6 +32,7 @@ Shape make_shape(const pack3d_config& c) {
   s.wait_ns = c.wait_limit_us > 0 ? (unsigned long long)c.wait_limit_us * 1000ull : 2000000000ull;
   s.stall = (c.flags & PACK3D_FLAG_DIAG_STALL) ? 1 : 0;
   s.sa_build = (c.flags & PACK3D_FLAG_SUMMARY_ONE_TILE) ? 1 : ((c.flags & PACK3D_FLAG_SUMMARY_TWO_TILE) ? 2 : 0);
+  for (int a = 0; a < 3; ++a) s.origin[a] = c.origin[a];
   const int m[3] = {c.m_z, c.m_y, c.m_x};
   const int ext[3] = {c.Z, c.H, c.W};
   int p = 0, off = 0;
@@ -170,7 +171,7 @@ void pack3d_default_config(pack3d_config* cfg, int32_t Z, int32_t H, int32_t W) 
 
 pack3d_status pack3d_validate_config(const pack3d_config* c) {
   if (!c) return PACK3D_ERR_INVALID_ARG;
-  if (c->reserved0 != 0 || c->wait_limit_us < 0) return PACK3D_ERR_INVALID_ARG;
+  if (c->reserved0 != 0 || c->reserved2 != 0 || c->wait_limit_us < 0) return PACK3D_ERR_INVALID_ARG;
   if (c->dtype != PACK3D_F32 && c->dtype != PACK3D_BF16) return PACK3D_ERR_DTYPE;
   if (c->Z < 0 || c->H < 0 || c->W < 0) return PACK3D_ERR_SHAPE;   // a zero extent is an empty volume
   const long long N = (long long)c->Z * c->H * c->W;
@@ -278,6 +279,30 @@ pack3d_status pack3d_summary_attn(const pack3d_config* cfg, const void* q_rot, c
       (o_loc && !aligned16(o_loc)))
     return PACK3D_ERR_ALIGNMENT;
   const Shape s = make_shape(*cfg);
+  cudaError_t e;
+  if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
+    e = launch_summary_attn_tc(s, q_rot, k_sum, v_sum, o_loc, gate, out, err_word, (cudaStream_t)stream);
+  else
+    e = launch_summary_attn_simt(s, cfg->dtype, q_rot, k_sum, v_sum, o_loc, gate, out, (cudaStream_t)stream);
+  return cuda_status(e);
+}
+
+pack3d_status pack3d_summary_attn_rows(const pack3d_config* cfg, int64_t tokens, int64_t summaries, const void* q_rot,
+                                       const void* k_sum, const void* v_sum, const float* o_loc, const float* gate,
+                                       void* out, int32_t* err_word, void* stream) {
+  pack3d_status st = pack3d_validate_config(cfg);
+  if (st != PACK3D_OK) return st;
+  if (tokens < 0 || summaries < 0) return PACK3D_ERR_INVALID_ARG;
+  if (tokens == 0 || summaries == 0) return PACK3D_OK;
+  // The same 32-bit element-index bound as a lattice (tokens x Hq x 64 and summaries x Hkv x 64).
+  if (tokens >= (1LL << 31) / 128 || summaries >= (1LL << 31) / 128) return PACK3D_ERR_SHAPE;
+  if (!q_rot || !k_sum || !v_sum || !out || (gate && !o_loc)) return PACK3D_ERR_INVALID_ARG;
+  if (!aligned16(q_rot) || !aligned16(k_sum) || !aligned16(v_sum) || !aligned16(out) ||
+      (o_loc && !aligned16(o_loc)))
+    return PACK3D_ERR_ALIGNMENT;
+  Shape s = make_shape(*cfg);
+  s.N = (int)tokens;
+  s.M = (int)summaries;
   cudaError_t e;
   if (cfg->dtype == PACK3D_BF16 && !(cfg->flags & PACK3D_FLAG_SIMT_SUMMARY))
     e = launch_summary_attn_tc(s, q_rot, k_sum, v_sum, o_loc, gate, out, err_word, (cudaStream_t)stream);

@@ -35,6 +35,7 @@ struct Shape {
   unsigned long long wait_ns;     // limit of every bounded pipeline wait
   int stall;                      // diagnostic: withhold one pipeline step (PACK3D_FLAG_DIAG_STALL)
   int sa_build;                   // query x summary build: 0 by size, 1 one-tile, 2 two-tile
+  int origin[3];                  // lattice origin: rotation angles use origin[a] + c_a
 };
 
 Shape make_shape(const pack3d_config& c);
@@ -82,7 +83,8 @@ __device__ __forceinline__ void stg16(void* p, const uint4& v) {
 
 // ---- axial RoPE tables -----------------------------------------------------
 // Table layout (float2 = cos, sin): plane p owns the contiguous entries
-// [pair_off[p], pair_off[p] + extent of its axis), one per coordinate value.
+// [pair_off[p], pair_off[p] + extent of its axis), one per local coordinate
+// value c; the entry holds the angle of the coordinate origin[axis] + c.
 // The angle omega * c is formed in double and reduced modulo 2*pi in double
 // (a two-part 2*pi, Cody-Waite style), so the float sincos sees an argument in
 // [-pi, pi].
@@ -110,7 +112,7 @@ __device__ __forceinline__ void build_rope_table(float2* tab, const Shape& s) {
 #pragma unroll
     for (int step = kMaxPairs / 2; step > 0; step >>= 1)
       if (p + step < s.npairs && s.pair_off[p + step] <= e) p += step;
-    tab[e] = rope_cos_sin(s.omega[p] * (double)(e - s.pair_off[p]));
+    tab[e] = rope_cos_sin(s.omega[p] * (double)(e - s.pair_off[p] + s.origin[s.pair_axis[p]]));
   }
 }
 
@@ -144,7 +146,8 @@ struct PlaneLut {
 
 // Rotates the 2*NP values f (planes p0 .. p0+NP-1) by R at the coordinate
 // (z, y, x), which may be fractional (a block centre): the angles are formed
-// directly, without the integer-coordinate tables.
+// directly, without the integer-coordinate tables.  The coordinate is the
+// rotation frame's (callers add the lattice origin).
 template <int NP>
 __device__ __forceinline__ void rotate_at(float* f, const Shape& s, int p0, double z, double y, double x) {
 #pragma unroll

@@ -421,8 +421,8 @@ __global__ void __launch_bounds__(kSbThreads) summaries_bwd_kernel(
     float f[2] = {dk.x, dk.y};
     const int jx = j % s.nbx, jy = (j / s.nbx) % s.nby, jz = j / (s.nbx * s.nby);
     if (lane < s.npairs)
-      rotate_at<1>(f, s, lane, -(jz * s.bz + 0.5 * (s.bz - 1)), -(jy * s.by + 0.5 * (s.by - 1)),
-                   -(jx * s.bx + 0.5 * (s.bx - 1)));
+      rotate_at<1>(f, s, lane, -(s.origin[0] + jz * s.bz + 0.5 * (s.bz - 1)),
+                   -(s.origin[1] + jy * s.by + 0.5 * (s.by - 1)), -(s.origin[2] + jx * s.bx + 0.5 * (s.bx - 1)));
     dk = make_float2(f[0], f[1]);
   }
   const int32_t* mem = members + (size_t)j * s.v;

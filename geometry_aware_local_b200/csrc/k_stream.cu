@@ -231,8 +231,8 @@ __global__ void __launch_bounds__(kSumThreads) summaries_kernel(
       }
     }
     if (!is_v && s.center)
-      rotate_at<NP>(acc, s, part * NP, jz * s.bz + 0.5 * (s.bz - 1), jy * s.by + 0.5 * (s.by - 1),
-                    jx * s.bx + 0.5 * (s.bx - 1));
+      rotate_at<NP>(acc, s, part * NP, s.origin[0] + jz * s.bz + 0.5 * (s.bz - 1),
+                    s.origin[1] + jy * s.by + 0.5 * (s.by - 1), s.origin[2] + jx * s.bx + 0.5 * (s.bx - 1));
     T* dst = is_v ? vs : ks;
     stg16(dst + ((size_t)j * s.Hkv + g) * kDh + part * NE, float_to_chunk(acc, T()));
   }
@@ -299,8 +299,8 @@ __global__ void __launch_bounds__(kSumThreads) summaries_generic_kernel(
       for (int k = 0; k < NE; ++k) acc[k] = fmaf(a, f[k], acc[k]);
     }
     if (!is_v && s.center)
-      rotate_at<NE / 2>(acc, s, part * (NE / 2), jz * s.bz + 0.5 * (s.bz - 1), jy * s.by + 0.5 * (s.by - 1),
-                        jx * s.bx + 0.5 * (s.bx - 1));
+      rotate_at<NE / 2>(acc, s, part * (NE / 2), s.origin[0] + jz * s.bz + 0.5 * (s.bz - 1),
+                        s.origin[1] + jy * s.by + 0.5 * (s.by - 1), s.origin[2] + jx * s.bx + 0.5 * (s.bx - 1));
     T* dst = is_v ? vs : ks;
     stg16(dst + ((size_t)j * s.Hkv + g) * kDh + part * NE, float_to_chunk(acc, T()));
   }
@@ -467,8 +467,9 @@ __global__ void __launch_bounds__(kSumWarpThreads) summaries_warp_kernel(
     // lane takes the pairs of its own planes by shuffle.
     // (Summary-centre variant: at the block's geometric centre instead.)
     const double half = s.center ? 0.5 : 0.0;
-    const double cpos = my_axis == 0 ? jz * s.bz + half * (s.bz - 1)
-                                     : (my_axis == 1 ? jy * s.by + half * (s.by - 1) : jx * s.bx + half * (s.bx - 1));
+    const double cpos = (my_axis < 3 ? s.origin[my_axis] : 0) +
+                        (my_axis == 0 ? jz * s.bz + half * (s.bz - 1)
+                                      : (my_axis == 1 ? jy * s.by + half * (s.by - 1) : jx * s.bx + half * (s.bx - 1)));
     const float2 cb = my_axis < 3 ? rope_cos_sin(my_omega * cpos) : make_float2(1.f, 0.f);
 #pragma unroll
     for (int i = 0; i < SPL; ++i)

@@ -140,6 +140,16 @@ typedef struct {
                                  [0, 1] and coord_scale[0] != 1 rescales z (the
                                  rotary-configuration sweep of the summary page,
                                  "Main Findings")                                */
+    int32_t origin[3];        /* lattice origin (z, y, x) in the frame the rotation
+                                 uses, 0 by default: the lattice covers sites
+                                 origin + [0,Z) x [0,H) x [0,W), coords stay local
+                                 (from 0), and every rotation angle is
+                                 omega_{a,r} * coord_scale[a] * (origin[a] + c_a).
+                                 A sub-volume (a z-slab of a larger lattice) then
+                                 rotates by its sites' true coordinates, as Key
+                                 design 1 requires; the local branch does not
+                                 depend on it (relative positions only)           */
+    int32_t reserved2;        /* must be 0                                       */
 } pack3d_config;
 
 /* Fills cfg with the pages' defaults for a Z x H x W lattice: Hq=8, Hkv=2,
@@ -221,6 +231,23 @@ pack3d_status pack3d_summary_attn(const pack3d_config *cfg, const void *q_rot,
                                   const void *k_sum, const void *v_sum, const float *o_loc,
                                   const float *gate, void *out, int32_t *err_word,
                                   void *stream);
+
+/* Stages 4+5 for an explicit number of query rows and summaries: as
+ * pack3d_summary_attn, but q_rot, o_loc, gate and out hold `tokens` tokens
+ * (T [tokens,Hq,d_h], float [tokens,Hq,d_h], float [tokens,Hq,2]) and k_sum,
+ * v_sum hold `summaries` summaries (T [summaries,Hkv,d_h]), instead of the N and
+ * M = N / |B| of the config's lattice (the config supplies the heads, the
+ * scale, the dtype and the flags).  This is the form a part of a volume uses
+ * when it attends to the summaries of the whole volume, e.g. one z-slab of a
+ * volume split over several GPUs, against the all-gathered summaries (every
+ * query still sees all M summaries, Key design 3).  tokens, summaries >= 0;
+ * tokens == 0 or summaries == 0 returns PACK3D_OK at once (no summary: out is
+ * not written).  Errors as pack3d_summary_attn; a count that is too large for
+ * 32-bit element indices -> PACK3D_ERR_SHAPE. */
+pack3d_status pack3d_summary_attn_rows(const pack3d_config *cfg, int64_t tokens, int64_t summaries,
+                                       const void *q_rot, const void *k_sum, const void *v_sum,
+                                       const float *o_loc, const float *gate, void *out,
+                                       int32_t *err_word, void *stream);
 
 /* The whole forward pass: index map, summaries, RoPE on Q and K_loc, local
  * branch, query-summary branch with the gate, all stream-ordered on `stream`.

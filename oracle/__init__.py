@@ -43,7 +43,8 @@ class _Cfg(ctypes.Structure):
                 ("base", ctypes.c_double),
                 ("bz", ctypes.c_int32), ("by", ctypes.c_int32), ("bx", ctypes.c_int32),
                 ("rz", ctypes.c_int32), ("ry", ctypes.c_int32), ("rx", ctypes.c_int32),
-                ("scale", ctypes.c_double), ("cscale", ctypes.c_double * 3)]
+                ("scale", ctypes.c_double), ("cscale", ctypes.c_double * 3),
+                ("origin", ctypes.c_double * 3)]
 
 
 _lib = None
@@ -85,7 +86,8 @@ def _cfg(s, scale: Optional[float] = None) -> _Cfg:
     return _Cfg(s.Z, s.H, s.W, s.Hq, s.Hkv, s.d_h, s.m_z, s.m_y, s.m_x, float(s.rope_base),
                 s.bz, s.by, s.bx, s.rz, s.ry, s.rx,
                 float(s.softmax_scale if scale is None else scale),
-                (ctypes.c_double * 3)(*[float(x) for x in s.coord_scale]))
+                (ctypes.c_double * 3)(*[float(x) for x in s.coord_scale]),
+                (ctypes.c_double * 3)(*[float(x) for x in getattr(s, "origin", (0, 0, 0))]))
 
 
 def as_f64(x) -> np.ndarray:

@@ -56,6 +56,7 @@ typedef struct {
     int32_t rz, ry, rx;
     double scale;
     double cscale[3];   /* coordinate scale per axis: angle = omega * cscale[a] * c_a */
+    double origin[3];   /* lattice origin: the true coordinate of local site c is origin + c */
 } orc_cfg;
 
 /* ---- lattice and index map ------------------------------------------- */
@@ -92,7 +93,9 @@ int orc_build_index(const orc_cfg *c, const int32_t *coords, int32_t *g2p, int32
 
 /* Angle of rotary pair p for coordinate (z,y,x) (a lattice site, or the
  * fractional centre of a block); returns 0 for untouched dims through
- * *active = 0. */
+ * *active = 0.  R(c) is driven by the site's true coordinate (Key design 1):
+ * for a lattice that is part of a larger volume, its origin plus the local
+ * coordinate. */
 static double pair_angle(const orc_cfg *c, int p, double z, double y, double x, int *active)
 {
     int axis_pairs[3] = {c->mz, c->my, c->mx};
@@ -103,7 +106,7 @@ static double pair_angle(const orc_cfg *c, int p, double z, double y, double x, 
             int r = p - first;
             double omega = pow(c->base, -(double)r / (double)axis_pairs[a]);
             *active = 1;
-            return omega * (c->cscale[a] * coord[a]);
+            return omega * (c->cscale[a] * (c->origin[a] + coord[a]));
         }
         first += axis_pairs[a];
     }

@@ -69,6 +69,7 @@ class Pack3DShape:
     value_scale: float = 0.125   # multiplier on the Q/K/V draws
     packing: str = "raster"
     coord_scale: tuple = (1.0, 1.0, 1.0)   # per-axis RoPE coordinate scale (z, y, x)
+    origin: tuple = (0, 0, 0)              # lattice origin in the rotation's frame (a sub-volume's offset)
 
     @property
     def N(self) -> int:

@@ -142,6 +142,19 @@ def test_rope_coordinate_scale_and_allocation_match_complex_form(scale, m):
     assert np.abs(oracle.rotate(s, coords, x) - expect).max() < 1e-12
 
 
+@pytest.mark.parametrize("origin", [(7, 0, 0), (3, -5, 11)])
+def test_rope_origin_is_rotation_at_true_coordinate(origin):
+    # A lattice that is one part of a larger volume (a z-slab) rotates its local site c by
+    # R(origin + c): the rotation is driven by true coordinates (Key design 1).
+    s = TINY.replace(origin=origin)
+    rng = np.random.default_rng(9)
+    coords = np.stack([rng.integers(0, n, 40) for n in (s.Z, s.H, s.W)], axis=1).astype(np.int32)
+    x = rng.standard_normal((40, 2, 64))
+    expect = rope_complex(s, coords + np.asarray(origin), x)
+    assert np.abs(oracle.rotate(s, coords, x) - expect).max() < 1e-12
+    assert np.abs(oracle.rotate(s, coords, x) - oracle.rotate(TINY, coords, x)).max() > 1e-3
+
+
 # ------------------------------------------------------------ index map -----
 
 @pytest.mark.parametrize("packing", synth.PACKINGS)
@@ -294,6 +307,28 @@ def test_summary_center_is_pooled_key_rotated_at_block_centre(blocks):
     expect = rope_complex(s, _block_centres(s), pooled)
     got, _ = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"], center=True)
     assert np.abs(got - expect).max() < 1e-12
+
+
+@pytest.mark.parametrize("center", [False, True], ids=["token", "centre"])
+def test_summaries_with_origin_use_true_coordinates(center):
+    # Both summary forms of a sub-volume whose first plane is true plane 9: the rotation
+    # before pooling (Key design 2) and the centre variant both see origin + local coordinate.
+    origin = (9, 0, 0)
+    s = small(Z=4, origin=origin)
+    inp, g2p, mem = _summary_case(s, seed=8)
+    coords = inp["coords"].numpy()
+    kc, sc = oracle.as_f64(inp["k_cmp"]), oracle.as_f64(inp["scores"])
+    a = scipy.special.softmax(sc[mem], axis=1)                               # [M, v, Hkv]
+    if center:
+        expect = rope_complex(s, _block_centres(s) + np.asarray(origin), np.einsum("jug,jugd->jgd", a, kc[mem]))
+    else:
+        kr = rope_complex(s, coords + np.asarray(origin), kc)
+        expect = np.einsum("jug,jugd->jgd", a, kr[mem])
+    got, vs = oracle.summaries(s, coords, mem, inp["k_cmp"], inp["v_cmp"], inp["scores"], center=center)
+    assert np.abs(got - expect).max() < 1e-12
+    _, vs0 = oracle.summaries(s.replace(origin=(0, 0, 0)), coords, mem, inp["k_cmp"], inp["v_cmp"],
+                              inp["scores"], center=center)
+    assert np.abs(vs - vs0).max() == 0                                          # values carry no rotation
 
 
 def test_summary_center_error_within_rotation_bound():
