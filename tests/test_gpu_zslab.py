@@ -138,3 +138,33 @@ def test_summary_attn_rows_on_a_subset_of_rows(p3):
     p3.summary_attn_rows(cfg, 0, k_all.shape[0], whole["q_rot"][:0], k_all, v_all, whole["o_loc"][:0],
                          d["gate"][:0], out[:0], err)
     assert p3.check_status(err) == 0 and torch.equal(out, before)
+
+
+def test_forward_on_a_one_rank_nccl_group(p3):
+    """zslab.forward as a rank calls it, through NCCL: one rank (every call here has one GPU),
+    so no halo and a one-part all-gather; the result must be the whole-volume forward's."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+
+    from geometry_aware_local_b200 import zslab
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda:0"))
+    try:
+        s = synth.Pack3DShape(Z=5, H=12, W=20, Hq=8, Hkv=2, rz=1, ry=3, rx=3, dtype="bf16", value_scale=0.125,
+                              packing="random")
+        inp = synth.make_inputs(s, seed=53)
+        d = {k: v.cuda() for k, v in inp.items() if k != "sites"}
+        cfg = p3.config_from_shape(s)
+        out = zslab.forward(cfg, d, 0, 1)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    whole = whole_volume(p3, cfg, s, d)
+    assert rel_err(out.float().cpu(), whole["out"].float().cpu()) <= 1e-2
+    ref = oracle.forward(s, inp)["out"]
+    assert rel_err(out.float().cpu().numpy(), ref) <= TOL["bf16"]

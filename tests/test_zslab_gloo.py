@@ -7,9 +7,11 @@ Here the stages are the oracle's (float64, CPU), the exchanges are gloo's, and
 the arrangement of tensors (which rows are sent, how the extended lattice is
 laid out, which summaries are a rank's own, how the gathered summaries are
 ordered) is the library's own z-slab module.  Every rank's outputs must equal
-the whole-volume oracle's for the same tokens: the local window of a boundary
+the whole-volume oracle's for the same tokens (the local window of a boundary
 query, the summaries of every block and the rotation of every token depend on
-all of it being right.
+all of it being right), and the index map and block membership of its own
+planes, mapped to whole-volume token ids, must equal the whole volume's bit
+for bit.
 """
 import datetime
 import os
@@ -59,12 +61,23 @@ def _rank(rank, world, port, shape_kw, center, q):
         st, g2p, mem = oracle.build_index(se, ext["coords"])
         assert st == 0
         coords = ext["coords"].numpy()
+        # The index map and block membership of the rank's own planes, mapped to whole-volume
+        # token ids (own tokens through take_slab's indices, halo tokens through their true
+        # coordinates), must be the whole volume's, bit for bit.
+        st_w, g2p_w, mem_w = oracle.build_index(s, inp["coords"])
+        true_z = coords[:, 0] + (p.z0 - p.lo)
+        ext2glob = g2p_w[(true_z * s.H + coords[:, 1]) * s.W + coords[:, 2]].astype(np.int64)
+        ext2glob[:p.tokens] = idx.numpy()
+        hw, bpp = s.H * s.W, (s.H // s.by) * (s.W // s.bx)
+        index_exact = bool(np.array_equal(ext2glob[g2p[p.lo * hw:(p.lo + p.planes) * hw]],
+                                          g2p_w[p.z0 * hw:p.z1 * hw]) and
+                           np.array_equal(ext2glob[mem[p.lo * bpp:(p.lo + p.planes) * bpp]],
+                                          mem_w[p.z0 * bpp:p.z1 * bpp]))
         rows = np.arange(p.tokens)
         qr = oracle.rotate(se, coords[:p.tokens], ext["q"][:p.tokens])
         kr = oracle.rotate(se, coords, ext["k_loc"])
         ks, vs = oracle.summaries(se, coords, mem, ext["k_cmp"], ext["v_cmp"], ext["scores"], center=center)
         ol = oracle.local_attn(se, coords, g2p, qr, kr, ext["v_loc"].numpy(), rows)
-        bpp = (s.H // s.by) * (s.W // s.bx)
         k_own, v_own = zslab.own_summaries(torch.from_numpy(ks), torch.from_numpy(vs), p, bpp)
         k_all, v_all = zslab.gather_summaries(k_own, v_own, p, bpp)
         oc = oracle.summary_attn(se, qr, k_all.numpy(), v_all.numpy())
@@ -73,9 +86,9 @@ def _rank(rank, world, port, shape_kw, center, q):
         q.put((rank, float(np.abs(out - ref).max() / np.abs(ref).max()),
                float(np.abs(ol - whole["o_loc"][idx.numpy()]).max()),
                float(max(np.abs(k_all.numpy() - whole["k_sum"]).max(), np.abs(v_all.numpy() - whole["v_sum"]).max())),
-               p.lo, p.hi, None))
+               p.lo, p.hi, index_exact, None))
     except Exception as e:                       # report instead of hanging the parent
-        q.put((rank, None, None, None, None, None, repr(e)))
+        q.put((rank, None, None, None, None, None, None, repr(e)))
         raise
     finally:
         dist.destroy_process_group()
@@ -100,8 +113,9 @@ def _run(world, shape_kw=None, center=False):
 @pytest.mark.parametrize("world", [2, 3])
 def test_zslab_ranks_equal_whole_volume(world):
     got = _run(world)
-    for rank, out_err, loc_err, sum_err, lo, hi, _ in got:
+    for rank, out_err, loc_err, sum_err, lo, hi, index_exact, _ in got:
         assert lo == (0 if rank == 0 else 2) and hi == (0 if rank == world - 1 else 2)
+        assert index_exact, rank
         assert out_err < 1e-12, (rank, out_err)
         assert loc_err < 1e-12, (rank, loc_err)
         assert sum_err < 1e-12, (rank, sum_err)
@@ -110,8 +124,8 @@ def test_zslab_ranks_equal_whole_volume(world):
 def test_zslab_centre_variant_and_shifted_volume():
     # The summary-centre variant, and a volume that itself starts at a nonzero origin.
     got = _run(2, dict(origin=(5, 2, 0), rz=1), center=True)
-    for rank, out_err, loc_err, sum_err, *_ in got:
-        assert out_err < 1e-12 and loc_err < 1e-12 and sum_err < 1e-12, rank
+    for rank, out_err, loc_err, sum_err, lo, hi, index_exact, _ in got:
+        assert out_err < 1e-12 and loc_err < 1e-12 and sum_err < 1e-12 and index_exact, rank
 
 
 # ------------------------------------------------------------- host plan -----
