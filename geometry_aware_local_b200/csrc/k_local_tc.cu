@@ -10,7 +10,7 @@
 // taken one key unit at a time: half of a lattice z-plane of the halo, i.e.
 // (2 + ry) rows of (4 + 2rx) sites (at most 5 x 10 = 50 keys), padded to
 // NU <= 64 keys.  Per unit:
-//   S = Q K^T  (M=128, N=NU, K=64; A, B from shared memory) into one of two
+//   S = Q K^T  (M=128, N=NU, K=64; A, B from shared memory) into one of three
 //   S / P buffers of tensor memory;
 //   softmax on the rows whose z window contains the unit's plane (the other
 //   layer's warps write P = 0): the lattice-box mask is a per-row bit mask of
@@ -22,10 +22,12 @@
 // The kernel is persistent: CTA c takes items c, c + grid, c + 2 grid, ...,
 // and the units of its items form one stream, so the gathers and MMAs of the
 // next item start while the current one's last units and epilogue run.  The
-// query tile is triple-buffered and the O accumulator double-buffered by item.
+// query tile is triple-buffered.  One O accumulator suffices: the softmax warps
+// read an item's O out (and signal o_free) before they write the next item's
+// first P, which its first O += P V needs anyway.
 // Warp roles (224 threads, two CTAs per SM):
 //   * warps 0-3, softmax: thread = row = tensor-memory lane;
-//   * warp 4, S: issues S of unit t+2 once O += P V of unit t has freed its
+//   * warp 4, S: issues S of unit t+3 once O += P V of unit t has freed its
 //     S / P buffer and the unit's keys (and, at an item's first unit, its query
 //     tile) have landed;
 //   * warp 5, P V: issues O += P V of unit t once P(t) is written, never held
@@ -38,8 +40,9 @@
 // An item's output rows leave through its own query tile (no longer read by
 // then): each softmax warp stages its 32 rows there, half a row at a time, and
 // writes them back as whole 128-byte segments, instead of every thread
-// storing its own 256-byte row (32 cache lines per warp instruction).
-// Tensor memory: S / P buffers at columns 0 and 64, O buffers at 128 and 192.
+// storing its own 256-byte row (32 cache lines per warp instruction); the
+// gather warp refills a query tile once q_out says its output has left.
+// Tensor memory: S / P buffers at columns 0, 64 and 128, O at 192.
 // Supported: bf16, G = 4, rz = 1, ry <= 3, rx <= 3 (the SIMT kernel covers the
 // rest).  Every mbarrier wait is bounded; a CTA that gives up lets its issued
 // copies and MMAs complete before it frees tensor memory.
@@ -62,14 +65,15 @@ constexpr int kQBufs = 3;                         // query tiles
 constexpr int kQBytes = kRows * kDh * 2;          // 16 KiB query tile
 constexpr int kSlotOff = kQBufs * kQBytes;        // slot s: K at kSlotOff + 2 s kTileBytes, V after it
 constexpr int kBarOff = kSlotOff + kSlots * 2 * kTileBytes;
-// barriers: q_full[3], q_free[3], kv_full[kSlots], slot_free[kSlots], s_full[2], p_full[2],
-// pv_done[2], o_free[2], drain[2]
-constexpr int kNumBars = 2 * kQBufs + 2 * kSlots + 2 + 2 + 2 + 2 + 2;
+constexpr int kSP = 3;                            // S / P buffers in tensor memory
+// barriers: q_full[3], q_free[3], kv_full[kSlots], slot_free[kSlots], s_full[kSP], p_full[kSP],
+// pv_done[kSP], o_free, q_out[kQBufs], drain[2]
+constexpr int kNumBars = 2 * kQBufs + 2 * kSlots + 3 * kSP + 1 + kQBufs + 2;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;   // + barriers, wait control, alignment slack
 constexpr int kCtasPerSm = 2;
 static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
-constexpr int kTmemCols = 256;                    // S / P buffer b at 64 b, O buffer c at 128 + 64 c
-constexpr int kColO = 128;
+constexpr int kTmemCols = 256;                    // S / P buffer b at 64 b, O at 192
+constexpr int kColO = 64 * kSP;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct LocalArgs {
@@ -138,11 +142,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
   auto q_free = [&](int c) { return bar0 + 8 * (kQBufs + c); };        // S MMAs done reading tile c
   auto kv_full = [&](int s) { return bar0 + 8 * (2 * kQBufs + s); };   // slot s holds K and V
   auto slot_free = [&](int s) { return bar0 + 8 * (2 * kQBufs + kSlots + s); };  // O += P V read slot s
-  auto s_full = [&](int b) { return bar0 + 8 * (kB + b); };            // S in buffer b
-  auto p_full = [&](int b) { return bar0 + 8 * (kB + 2 + b); };        // P in buffer b, O rescaled
-  auto pv_done = [&](int b) { return bar0 + 8 * (kB + 4 + b); };       // O += P V from buffer b done
-  auto o_free = [&](int c) { return bar0 + 8 * (kB + 6 + c); };        // O buffer c read out
-  auto drain = [&](int w) { return bar0 + 8 * (kB + 8 + w); };         // abort path: warp w's MMAs completed
+  auto s_full = [&](int b) { return bar0 + 8 * (kB + b); };                 // S in buffer b
+  auto p_full = [&](int b) { return bar0 + 8 * (kB + kSP + b); };           // P in buffer b, O rescaled
+  auto pv_done = [&](int b) { return bar0 + 8 * (kB + 2 * kSP + b); };      // O += P V from buffer b done
+  auto o_free = [&]() { return bar0 + 8 * (kB + 3 * kSP); };                // the item's O read out
+  auto q_out = [&](int c) { return bar0 + 8 * (kB + 3 * kSP + 1 + c); };    // query tile c's output stored
+  auto drain = [&](int w) { return bar0 + 8 * (kB + 3 * kSP + 1 + kQBufs + w); };  // abort path: warp w's MMAs completed
   volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + 8 * kNumBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + 8 * kNumBars + sizeof(ptx::WaitCtl));
   auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
@@ -153,12 +158,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
       ptx::mbar_init(q_full(c), 32);           // one cp.async arrival per gather thread
       ptx::mbar_init(q_free(c), 1);
     }
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < kSP; ++c) {
       ptx::mbar_init(s_full(c), 1);
       ptx::mbar_init(p_full(c), 4);            // one arrival per softmax warp
       ptx::mbar_init(pv_done(c), 1);
-      ptx::mbar_init(o_free(c), 4);
     }
+    ptx::mbar_init(o_free(), 4);
+    for (int c = 0; c < kQBufs; ++c) ptx::mbar_init(q_out(c), 4);
     for (int s = 0; s < kSlots; ++s) {
       ptx::mbar_init(kv_full(s), 32);
       ptx::mbar_init(slot_free(s), 1);
@@ -202,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
     auto load_query = [&](int k, int i) {
       // The tile's previous item: its S MMAs are done and its output has left the tile.
       if (k >= kQBufs && !(wait(q_free(k % kQBufs), ((k / kQBufs) - 1) & 1) &&
-                           wait(o_free((k - kQBufs) & 1), ((k - kQBufs) >> 1) & 1)))
+                           wait(q_out(k % kQBufs), ((k / kQBufs) - 1) & 1)))
         return false;
       const Item it = decode_item(a, i);
       int qi[4];
@@ -259,36 +265,38 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
       for (int ii = blockIdx.x; ii < a.nitems; ii += gridDim.x) total += decode_item(a, ii).nunits;
       bool ok = true;
       if (warp == kSWarp) {
-        // S(t) into buffer t % 2 once K(t) (and, at an item's first unit, its query tile) has
-        // landed and O += P V(t-2) has read that buffer's P.  (PACK3D_FLAG_DIAG_STALL
+        // S(t) into buffer t % 3 once K(t) (and, at an item's first unit, its query tile) has
+        // landed and O += P V(t-3) has read that buffer's P.  (PACK3D_FLAG_DIAG_STALL
         // withholds the S of the CTA's last unit.)
         const int s_units = a.stall ? total - 1 : total;
         for (; ok && t < s_units; next()) {
           if (!(ok = wait(kv_full(t % kSlots), (t / kSlots) & 1))) break;
           if (u == 0 && !(ok = wait(q_full(k % kQBufs), (k / kQBufs) & 1))) break;
-          if (t >= 2 && !(ok = wait(pv_done(t & 1), ((t >> 1) - 1) & 1))) break;
+          if (t >= kSP && !(ok = wait(pv_done(t % kSP), ((t / kSP) - 1) & 1))) break;
           ptx::tc_fence_after();
+          ptx::fence_proxy_async_smem();   // the gathered tiles were written by cp.async
           const uint32_t kt = k_tile(t), qt = q_tile(k);
 #pragma unroll
           for (int kk = 0; kk < kDh / 16; ++kk)
-            ptx::mma_ss(tmem + 64 * (t & 1), ptx::smem_desc_sw128(qt + kk * 32, 16, 1024),
+            ptx::mma_ss(tmem + 64 * (t % kSP), ptx::smem_desc_sw128(qt + kk * 32, 16, 1024),
                         ptx::smem_desc_sw128(kt + kk * 32, 16, 1024), idescS, kk > 0);
-          ptx::tc_commit(s_full(t & 1));
+          ptx::tc_commit(s_full(t % kSP));
           if (u == n - 1) ptx::tc_commit(q_free(k % kQBufs));   // the item's last read of its query tile
         }
       } else {
         // O(item) += P(t) V(t) once the softmax warps have written P(t); an item's first unit
-        // starts its O buffer afresh once the softmax warps have read out the item two back.
+        // starts O afresh once the softmax warps have read out the previous item's.
         for (; ok && t < total; next()) {
-          if (!(ok = wait(p_full(t & 1), (t >> 1) & 1))) break;
-          if (u == 0 && k >= 2 && !(ok = wait(o_free(k & 1), ((k >> 1) - 1) & 1))) break;
+          if (!(ok = wait(p_full(t % kSP), (t / kSP) & 1))) break;
+          if (u == 0 && k >= 1 && !(ok = wait(o_free(), (k - 1) & 1))) break;
           ptx::tc_fence_after();
+          ptx::fence_proxy_async_smem();   // the gathered V tile was written by cp.async
           const uint32_t vt = k_tile(t) + kTileBytes;
-          const uint32_t tO = tmem + kColO + 64 * (k & 1);
+          const uint32_t tO = tmem + kColO;
           for (int kk = 0; kk < a.NU / 16; ++kk)
-            ptx::mma_ts(tO, tmem + 64 * (t & 1) + kk * 8, ptx::smem_desc_sw128(vt + kk * 2048, 8192, 1024),
+            ptx::mma_ts(tO, tmem + 64 * (t % kSP) + kk * 8, ptx::smem_desc_sw128(vt + kk * 2048, 8192, 1024),
                         idescPV, (u > 0 || kk > 0) ? 1u : 0u);
-          ptx::tc_commit(pv_done(t & 1));
+          ptx::tc_commit(pv_done(t % kSP));
           ptx::tc_commit(slot_free(t % kSlots));
         }
       }
@@ -301,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     const float c = a.scale_log2;
     bool ok = true;
-    int t = 0;
+    int t = 0, sb = 0, sph = 0;   // unit count, its S / P buffer and that buffer's phase
     for (int k = 0, i = blockIdx.x; ok && i < a.nitems; ++k, i += gridDim.x) {
       const Item it = decode_item(a, i);
       const int qi = query_index(a, it, tid);   // where this row's output goes (read at the item's end)
@@ -329,13 +337,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
           (half ? mask1 : mask0)[1] = (uint32_t)(m >> 32);
         }
       }
-      const uint32_t tO = trow + kColO + 64 * (k & 1);
+      const uint32_t tO = trow + kColO;
       float m_used = -INFINITY, l = 0.f;
       for (int u = 0; u < it.nunits; ++u, ++t) {
         const int zp = it.zlo + (u >> 1);
         const bool uses = zp >= it.z0 + lz - 1 && zp <= it.z0 + lz + 1;  // warp-uniform (layer = warp / 2)
-        const uint32_t tS = trow + 64 * (t & 1);
-        if (!(ok = __all_sync(0xffffffffu, wait(s_full(t & 1), (t >> 1) & 1)))) break;
+        const uint32_t tS = trow + 64 * sb;
+        if (!(ok = __all_sync(0xffffffffu, wait(s_full(sb), sph)))) break;
         ptx::tc_fence_after();
         if (uses) {
           uint32_t sv[kUnitKeys];
@@ -385,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
           if (__any_sync(0xffffffffu, f != 1.f)) {
             // O is rescaled once O += P V of the item's previous unit has completed,
             // before this unit's O += P V is issued.
-            if (!(ok = __all_sync(0xffffffffu, wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1)))) break;
+            if (!(ok = __all_sync(0xffffffffu, wait(pv_done(sb == 0 ? kSP - 1 : sb - 1), sb == 0 ? sph ^ 1 : sph)))) break;
             ptx::tc_fence_after();
             uint32_t o[32];
 #pragma unroll
@@ -405,14 +413,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(p_full(t & 1));
+        if (lane == 0) ptx::mbar_arrive(p_full(sb));
+        if (++sb == kSP) {   // the S / P buffer and its phase of the next unit
+          sb = 0;
+          sph ^= 1;
+        }
       }
       if (!ok) break;
       // The item's output: its last O += P V has completed.
-      if (!(ok = __all_sync(0xffffffffu, wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1)))) break;
+      if (!(ok = __all_sync(0xffffffffu, wait(pv_done(sb == 0 ? kSP - 1 : sb - 1), sb == 0 ? sph ^ 1 : sph)))) break;
       ptx::tc_fence_after();
       uint32_t o[2][32];
       ptx::tmem_ld64_sync(tO, &o[0][0]);
+      // O is in registers: the next item's first O += P V may overwrite it.
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(o_free());
       const float inv = 1.f / l;
       if (a.stats && qi >= 0) a.stats[4 * ((size_t)qi * a.Hq + it.g * 4 + hh)] = m_used + log2f(l);
       // Rows 32 warp .. 32 warp + 31 of the item's query tile hold this warp's
@@ -440,8 +456,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) local_attn_tc_kernel(con
         }
         __syncwarp();
       }
-      ptx::tc_fence_before();
-      if (lane == 0) ptx::mbar_arrive(o_free(k & 1));
+      if (lane == 0) ptx::mbar_arrive(q_out(k % kQBufs));   // the query tile may be refilled
     }
   }
 
