@@ -423,3 +423,22 @@ def test_forward_large_sampled_rows(p3, name):
     ref = oracle.forward(s, inp, rows)["out"]
     assert rel_err(out[rows].double().numpy(), ref) <= TOL["bf16"]
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("name", ["4m", "8m"])
+def test_forward_query_tiled_sizes_sampled_rows(p3, name):
+    """4M and 8M tokens (M = 262,144 and 524,288 summaries): element offsets of q, out and
+    o_loc pass 2^31 (4M x 8 heads x 64 = 2^31, 8M twice that), and the query x summary
+    kernel walks 2,048 and 4,096 summary tiles.  Values are drawn on the device (the host
+    recipe's float32 draws would not fit); the sampled rows include the first and the last
+    32 packed rows, and the oracle gets the same values copied back."""
+    s = synth.CONFIGS[name]
+    d = synth.make_inputs_on_device(s, s.packing, seed=0)
+    out = run_forward(p3, s, d)
+    rows = np.unique(np.concatenate([synth.sample_rows(s.N, 96, seed=5), np.arange(s.N - 32, s.N)]))
+    inp = {k: v.cpu() for k, v in d.items()}
+    del d
+    torch.cuda.empty_cache()
+    ref = oracle.forward(s, inp, rows)
+    assert rel_err(out[rows].double().numpy(), ref["out"]) <= TOL["bf16"]
+    assert rel_err(out[-32:].double().numpy(), ref["out"][-32:]) <= TOL["bf16"]
