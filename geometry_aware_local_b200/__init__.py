@@ -46,7 +46,8 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: 
 
 ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
                 "pack3d_build_index", "pack3d_rope", "pack3d_rope_qk", "pack3d_build_summaries", "pack3d_local_attn",
-                "pack3d_summary_attn", "pack3d_summary_attn_rows", "pack3d_forward", "pack3d_forward_noalloc",
+                "pack3d_summary_attn", "pack3d_summary_attn_rows", "pack3d_gather_rows", "pack3d_forward",
+                "pack3d_forward_noalloc",
                 "pack3d_pipeline_create",
                 "pack3d_pipeline_destroy", "pack3d_host_workspace_bytes", "pack3d_forward_host",
                 "pack3d_train_workspace_bytes", "pack3d_forward_backward", "pack3d_check_status",
@@ -102,6 +103,7 @@ def _load():
         "pack3d_local_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P]),
         "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "pack3d_summary_attn_rows": (ctypes.c_int, [C, ctypes.c_int64, ctypes.c_int64] + [P] * 8),
+        "pack3d_gather_rows": (ctypes.c_int, [P, ctypes.c_int64, P, P, ctypes.c_int64, P]),
         "pack3d_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
         "pack3d_forward_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
         "pack3d_pipeline_create": (ctypes.c_int, [ctypes.POINTER(P)]),
@@ -314,6 +316,19 @@ def summary_attn_rows(cfg, tokens: int, summaries: int, q_rot, k_sum, v_sum, o_l
     _check(lib.pack3d_summary_attn_rows(ctypes.byref(cfg), int(tokens), int(summaries), _ptr(q_rot), _ptr(k_sum),
                                         _ptr(v_sum), _ptr(o_loc), _ptr(gate), _ptr(out), _ptr(err),
                                         _stream(stream)), "pack3d_summary_attn_rows")
+
+
+def gather_rows(idx, src, dst, stream=None):
+    """dst[i] = src[idx[i]] row by row (pack3d_gather_rows); idx int32 [n], src [rows, ...] and dst [n, ...]
+    contiguous with the same row shape and dtype; a negative index gives a zero row."""
+    import torch
+    n = idx.numel()
+    same_rows = src.dtype == dst.dtype and tuple(src.shape[1:]) == tuple(dst.shape[1:]) and dst.shape[0] == n
+    if idx.dtype != torch.int32 or not same_rows or not all(t.is_contiguous() for t in (idx, src, dst)):
+        raise ValueError("gather_rows: idx must be int32 [n], src and dst contiguous rows of one shape and dtype")
+    row_bytes = dst[0].numel() * dst.element_size() if n else 16
+    _check(lib.pack3d_gather_rows(_ptr(idx), int(n), _ptr(src), _ptr(dst), int(row_bytes), _stream(stream)),
+           "pack3d_gather_rows")
 
 
 def _check_forward_args(what, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err):

@@ -311,6 +311,15 @@ pack3d_status pack3d_summary_attn_rows(const pack3d_config* cfg, int64_t tokens,
   return cuda_status(e);
 }
 
+pack3d_status pack3d_gather_rows(const int32_t* idx, int64_t n, const void* src, void* dst, int64_t row_bytes,
+                                 void* stream) {
+  if (n < 0 || row_bytes <= 0 || row_bytes % 16 != 0) return PACK3D_ERR_INVALID_ARG;
+  if (n == 0) return PACK3D_OK;
+  if (!idx || !src || !dst) return PACK3D_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return PACK3D_ERR_ALIGNMENT;
+  return cuda_status(launch_gather_rows(idx, n, src, dst, row_bytes, (cudaStream_t)stream));
+}
+
 pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, const void* q, const void* k_loc,
                              const void* v_loc, const void* k_cmp, const void* v_cmp, const float* scores,
                              const float* gate, void* out, void* workspace, size_t workspace_bytes,

@@ -44,6 +44,8 @@ struct Train {
   float* dgate;        // [N, Hq, 2]
 };
 
+cudaError_t launch_gather_rows(const int32_t* idx, long long n, const void* src, void* dst, long long row_bytes,
+                               cudaStream_t st);
 cudaError_t launch_build_index(const Shape& s, const int32_t* coords, int32_t* g2p,
                                int32_t* members, int32_t* err, cudaStream_t st);
 

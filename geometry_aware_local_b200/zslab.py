@@ -5,29 +5,31 @@ with summary blocks one plane thick (b_z = 1) no block straddles two slabs,
 a query's local window reaches only r_z planes past its slab (Key design 3),
 and the compressed branch needs every summary of the volume (Key design 3:
 every token attends to all M summaries).  Rank r of `world` owns the planes
-[z0, z1) of the lattice and
+[z0, z1) of the lattice and runs, per step:
 
-1. sends the K_loc / V_loc rows of its first and last r_z planes to the ranks
-   below and above and receives theirs (point-to-point: the halo);
-2. runs the index map, summaries, RoPE and local attention on its slab
-   extended by the received halo planes, as a lattice whose `origin` is the
-   true z of its first plane, so every rotation uses true coordinates (Key
-   design 1);
-3. all-gathers the summaries of its own blocks; slabs are contiguous and in
-   rank order, so the concatenation is the whole volume's summary array in
-   its raster block order;
-4. runs the query x summary stage with the gate for its own tokens against
-   all M summaries (`pack3d_summary_attn_rows`).
+1. the local keys and values of its first and last r_z planes, gathered in
+   raster order through its index map (`pack3d_gather_rows`), go to the ranks
+   below and above, and theirs arrive straight into its halo rows (NCCL
+   point-to-point);
+2. summaries, RoPE and local attention run on its slab extended by the halo
+   planes, a lattice whose config `origin` is the true z of its first plane,
+   so every rotation uses true coordinates (Key design 1);
+3. the summaries of its own blocks (one contiguous range: blocks are planes of
+   b_z = 1) are all-gathered; slabs are contiguous and in rank order, so the
+   result is the whole volume's summary array in raster block order;
+4. the query x summary stage and the gate run for its own tokens against all
+   M summaries (`pack3d_summary_attn_rows`).
 
-A rank passes its own tokens (any packing; coordinates local to its slab, z
-from 0) and gets their outputs in the same order.  The exchanges use
-torch.distributed (NCCL between GPUs; any backend for the host logic).  This
-module only moves and arranges tensors; every stage runs in the library's
-kernels.  Halo tokens carry zero queries and gate logits (their outputs are
-dropped) and zero compressed keys, values and scores (their summaries are
-dropped).  `forward` composes the phases; `prepare`, `local_stage`,
-`own_summaries`, `gather_summaries` and `global_stage` are the phases
-themselves.
+`Plan` sets a rank up once for its fixed coordinates: the extended lattice's
+coordinates and index map (built once; the geometry does not change between
+steps), and every buffer.  The caller writes its own tokens' inputs into
+`Plan.inputs()` (views of the extended arrays, any order within the slab) and
+calls `Plan.forward()`.  Halo tokens carry zero queries, gate logits,
+compressed keys, values and scores; their outputs and summaries are dropped.
+Every per-step data movement is a library kernel or a NCCL call; PyTorch only
+holds the buffers and runs the collectives.  The phases are also callable one
+by one (`pack_halo`, `halo_views`, `local`, `summary_part`, `attend`), which
+is how a single process can run every rank's work in turn.
 """
 from __future__ import annotations
 
@@ -54,7 +56,9 @@ def slab_bounds(Z: int, world: int) -> List[Tuple[int, int]]:
 class SlabPlan:
     """Rank `rank`'s part of a Z x H x W volume: its planes [z0, z1), the halo
     planes it receives from below (`lo`) and from above (`hi`), and the
-    extended lattice of Z_ext planes that starts at true plane z0 - lo."""
+    extended lattice of Z_ext planes that starts at true plane z0 - lo.  Rows of
+    the extended arrays: the rank's own tokens first, then the `lo` planes below
+    and the `hi` planes above, each in raster order."""
     Z: int
     H: int
     W: int
@@ -82,6 +86,33 @@ class SlabPlan:
     def tokens(self) -> int:
         return self.planes * self.plane_sites
 
+    @property
+    def halo_below(self) -> Tuple[int, int]:
+        """Rows of the extended arrays that hold the planes received from below."""
+        return self.tokens, self.tokens + self.lo * self.plane_sites
+
+    @property
+    def halo_above(self) -> Tuple[int, int]:
+        """Rows of the extended arrays that hold the planes received from above."""
+        a = self.tokens + self.lo * self.plane_sites
+        return a, a + self.hi * self.plane_sites
+
+    @property
+    def send_below(self) -> Tuple[int, int]:
+        """Sites (raster over the extended lattice) of the own planes the rank below receives."""
+        a = self.lo * self.plane_sites
+        return a, a + min(self.rz, self.planes) * self.plane_sites
+
+    @property
+    def send_above(self) -> Tuple[int, int]:
+        """Sites (raster over the extended lattice) of the own planes the rank above receives."""
+        b = (self.lo + self.planes) * self.plane_sites
+        return b - min(self.rz, self.planes) * self.plane_sites, b
+
+    def own_blocks(self, blocks_per_plane: int) -> Tuple[int, int]:
+        """The extended lattice's blocks that are the rank's own (raster block order)."""
+        return self.lo * blocks_per_plane, (self.lo + self.planes) * blocks_per_plane
+
 
 def make_plan(cfg, rank: int, world: int) -> SlabPlan:
     """Rank `rank`'s slab of the volume `cfg` describes (whose origin the slabs inherit)."""
@@ -95,17 +126,6 @@ def make_plan(cfg, rank: int, world: int) -> SlabPlan:
     return SlabPlan(Z, H, W, rz, rank, world, z0, z1, min(rz, z0), min(rz, Z - z1))
 
 
-def take_slab(inp: Dict, p: SlabPlan):
-    """Rank p.rank's tokens of a whole volume's inputs, in their input order, with z made local
-    to the slab.  Returns (their indices in `inp`, their inputs)."""
-    import torch
-    z = inp["coords"][:, 0]
-    idx = torch.nonzero((z >= p.z0) & (z < p.z1)).flatten()
-    own = {k: inp[k].index_select(0, idx).contiguous() for k in NAMES}
-    own["coords"][:, 0] -= p.z0
-    return idx, own
-
-
 def ext_config(cfg, p: SlabPlan):
     """Config of the extended lattice: Z_ext planes whose first one is true plane z0 - lo."""
     c = type(cfg).from_buffer_copy(cfg)
@@ -114,143 +134,200 @@ def ext_config(cfg, p: SlabPlan):
     return c
 
 
-def boundary_rows(coords, p: SlabPlan):
-    """Indices of this rank's tokens on its first r_z planes and on its last r_z planes, each in raster
-    order over (z, y, x): what the ranks below and above receive as their halo."""
+def ext_coords(coords, p: SlabPlan):
+    """Coordinates of the extended lattice's rows: the own tokens' (z local to the slab, shifted
+    by lo), then the halo planes below and above in raster order."""
     import torch
-    c = coords.long()
-    order = torch.argsort((c[:, 0] * p.H + c[:, 1]) * p.W + c[:, 2])   # the slab's sites in raster order
-    n = min(p.rz, p.planes) * p.plane_sites
-    return order[:n], order[p.tokens - n:]
-
-
-def exchange_halo(k_loc, v_loc, coords, p: SlabPlan, group=None):
-    """Sends the K_loc / V_loc rows of this rank's first r_z planes to the rank below and of its last
-    r_z planes to the rank above, and receives theirs.  Returns (below, above), tensors
-    [lo * H * W, 2, Hkv, d_h] and [hi * H * W, 2, Hkv, d_h] (K then V) in raster order."""
-    import torch
-    import torch.distributed as dist
-    first, last = boundary_rows(coords, p)
-    kv = torch.stack([k_loc, v_loc], dim=1)
-    below = kv.new_empty((p.lo * p.plane_sites,) + tuple(kv.shape[1:]))
-    above = kv.new_empty((p.hi * p.plane_sites,) + tuple(kv.shape[1:]))
-    ops = []
-    if p.lo:
-        ops.append(dist.P2POp(dist.isend, kv.index_select(0, first).contiguous(), p.rank - 1, group))
-        ops.append(dist.P2POp(dist.irecv, below, p.rank - 1, group))
-    if p.hi:
-        ops.append(dist.P2POp(dist.isend, kv.index_select(0, last).contiguous(), p.rank + 1, group))
-        ops.append(dist.P2POp(dist.irecv, above, p.rank + 1, group))
-    if ops:
-        for req in dist.batch_isend_irecv(ops):
-            req.wait()
-    return below, above
-
-
-def prepare(inp: Dict, below, above, p: SlabPlan) -> Dict:
-    """The extended lattice's inputs: this rank's tokens first (z shifted by lo), then the halo planes
-    received from below (z = 0 .. lo-1) and from above (the last hi planes), each in raster order.
-    Halo tokens get their K_loc / V_loc rows and zeros elsewhere."""
-    import torch
-    own = {k: inp[k] for k in NAMES}
-    dev = own["q"].device
-    n_lo, n_hi = p.lo * p.plane_sites, p.hi * p.plane_sites
+    dev = coords.device
 
     def plane_coords(z_from: int, count: int):
         idx = torch.arange(count, device=dev, dtype=torch.int64)
         return torch.stack([z_from + idx // p.plane_sites, (idx // p.W) % p.H, idx % p.W], dim=1).to(torch.int32)
 
     shift = torch.tensor([p.lo, 0, 0], dtype=torch.int32, device=dev)
-    ext = {"coords": torch.cat([own["coords"] + shift, plane_coords(0, n_lo),
-                                plane_coords(p.lo + p.planes, n_hi)])}
-
-    def pad(t, halo_rows=None):
-        zeros = t.new_zeros((n_lo + n_hi,) + tuple(t.shape[1:]))
-        if halo_rows is not None:
-            zeros = halo_rows
-        return torch.cat([t, zeros])
-
-    ext["k_loc"] = pad(own["k_loc"], torch.cat([below[:, 0], above[:, 0]]))
-    ext["v_loc"] = pad(own["v_loc"], torch.cat([below[:, 1], above[:, 1]]))
-    for k in ("q", "k_cmp", "v_cmp", "scores", "gate"):
-        ext[k] = pad(own[k])
-    return {k: v.contiguous() for k, v in ext.items()}
+    return torch.cat([coords.to(torch.int32) + shift, plane_coords(0, p.lo * p.plane_sites),
+                      plane_coords(p.lo + p.planes, p.hi * p.plane_sites)]).contiguous()
 
 
-def own_summaries(k_sum, v_sum, p: SlabPlan, blocks_per_plane: int):
-    """The summaries of this rank's own blocks (planes lo .. lo + planes - 1 of the extended lattice)."""
-    a = p.lo * blocks_per_plane
-    b = a + p.planes * blocks_per_plane
-    return k_sum[a:b], v_sum[a:b]
-
-
-def gather_summaries(k_own, v_own, p: SlabPlan, blocks_per_plane: int, group=None):
-    """All ranks' own summaries, concatenated in rank order (= the volume's raster block order)."""
-    import torch
-    import torch.distributed as dist
-    bounds = slab_bounds(p.Z, p.world)
-    most = max(b - a for a, b in bounds) * blocks_per_plane
-    kv = torch.stack([k_own, v_own], dim=1)
-    padded = kv.new_zeros((most,) + tuple(kv.shape[1:]))
-    padded[:kv.shape[0]] = kv
-    parts = [torch.empty_like(padded) for _ in range(p.world)]
-    dist.all_gather(parts, padded, group=group)
-    allkv = torch.cat([parts[r][:(b - a) * blocks_per_plane] for r, (a, b) in enumerate(bounds)])
-    return allkv[:, 0].contiguous(), allkv[:, 1].contiguous()
-
-
-def local_stage(cfg_e, ext: Dict, err, stream=None):
-    """Index map, summaries, RoPE and local attention on the extended lattice (library kernels).
-    Returns q_rot, o_loc (every extended token) and k_sum, v_sum (every extended block)."""
-    import torch
-
-    from . import build_index, build_summaries, local_attn, rope_qk
-    dev = ext["q"].device
-    N, M, v = cfg_e.N, cfg_e.M, cfg_e.v
-    g2p = torch.empty(N, dtype=torch.int32, device=dev)
-    mem = torch.empty(M, v, dtype=torch.int32, device=dev)
-    build_index(cfg_e, ext["coords"], g2p, mem, err, stream)
-    k_sum = torch.empty(M, cfg_e.Hkv, cfg_e.d_h, dtype=ext["q"].dtype, device=dev)
-    v_sum = torch.empty_like(k_sum)
-    build_summaries(cfg_e, mem, ext["k_cmp"], ext["v_cmp"], ext["scores"], k_sum, v_sum, stream)
-    q_rot, k_rot = torch.empty_like(ext["q"]), torch.empty_like(ext["k_loc"])
-    rope_qk(cfg_e, ext["coords"], ext["q"], q_rot, ext["k_loc"], k_rot, stream)
-    o_loc = torch.empty(N, cfg_e.Hq, cfg_e.d_h, dtype=torch.float32, device=dev)
-    local_attn(cfg_e, g2p, q_rot, k_rot, ext["v_loc"], o_loc, err, stream)
-    return q_rot, o_loc, k_sum, v_sum
-
-
-def global_stage(cfg_e, tokens: int, q_rot, k_all, v_all, o_loc, gate, err, stream=None):
-    """The query x summary stage and the gate for the first `tokens` extended rows (this rank's own)."""
-    import torch
-
-    from . import summary_attn_rows
-    out = torch.empty_like(q_rot[:tokens])
-    summary_attn_rows(cfg_e, tokens, k_all.shape[0], q_rot[:tokens], k_all, v_all, o_loc[:tokens],
-                      gate[:tokens], out, err, stream)
+def summary_parts(cfg, world: int) -> List[Tuple[int, int, int]]:
+    """How the ranks' summaries are all-gathered: a part of `most` summaries per rank (the
+    largest rank's count), taken from its extended summary array at `start`, whose own blocks
+    begin `offset` summaries into it.  Returns [(start, offset, count)] in rank order; with
+    even slabs every offset is 0 and every count equals most.  A smaller rank's part extends
+    into its halo blocks (above it, or below it for the last rank), which are dropped."""
+    bpp = (cfg.H // cfg.by) * (cfg.W // cfg.bx)
+    plans = [make_plan(cfg, r, world) for r in range(world)]
+    most = max(p.planes for p in plans) * bpp
+    out = []
+    for p in plans:
+        a, b = p.own_blocks(bpp)
+        start = a if a + most <= p.Z_ext * bpp else b - most
+        out.append((start, a - start, b - a))
     return out
+
+
+def take_slab(inp: Dict, p: SlabPlan):
+    """Rank p.rank's tokens of a whole volume's inputs, in their input order, with z made local
+    to the slab.  Returns (their indices in `inp`, their inputs).  (For tests and examples that
+    hold a whole volume in one process.)"""
+    import torch
+    z = inp["coords"][:, 0]
+    idx = torch.nonzero((z >= p.z0) & (z < p.z1)).flatten()
+    own = {k: inp[k].index_select(0, idx).contiguous() for k in NAMES}
+    own["coords"][:, 0] -= p.z0
+    return idx, own
+
+
+class Plan:
+    """One rank's z-slab forward, set up once for the rank's fixed token coordinates.
+
+    `coords` (int32 [tokens, 3], on the rank's CUDA device) are the rank's own
+    tokens' lattice coordinates with z local to its slab (0 .. planes-1); their
+    order is the order of `inputs()` and of the output."""
+
+    def __init__(self, cfg, coords, rank: int, world: int, group=None, stream=None):
+        import torch
+
+        from . import BF16, Pack3DError, build_index, check_status, validate
+        st = validate(cfg)
+        if st != 0:
+            raise Pack3DError(st, "z-slab config")
+        self.cfg, self.group, self.stream = cfg, group, stream
+        self.p = p = make_plan(cfg, rank, world)
+        if coords.shape[0] != p.tokens:
+            raise ValueError(f"rank {rank} owns {p.tokens} tokens, got {coords.shape[0]}")
+        self.cfg_e = ce = ext_config(cfg, p)
+        dev = coords.device
+        dt = torch.bfloat16 if cfg.dtype == BF16 else torch.float32
+        N, M, Hq, Hkv, d = ce.N, ce.M, cfg.Hq, cfg.Hkv, cfg.d_h
+
+        def zeros(*shape, dtype=dt):
+            return torch.zeros(shape, dtype=dtype, device=dev)
+
+        # Extended inputs; the halo rows stay zero except K_loc / V_loc, received every step.
+        self.ext = {"coords": ext_coords(coords, p), "q": zeros(N, Hq, d), "k_loc": zeros(N, Hkv, d),
+                    "v_loc": zeros(N, Hkv, d), "k_cmp": zeros(N, Hkv, d), "v_cmp": zeros(N, Hkv, d),
+                    "scores": zeros(N, Hkv, dtype=torch.float32), "gate": zeros(N, Hq, 2, dtype=torch.float32)}
+        self.err = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.g2p = torch.empty(N, dtype=torch.int32, device=dev)
+        self.members = torch.empty(M, ce.v, dtype=torch.int32, device=dev)
+        build_index(ce, self.ext["coords"], self.g2p, self.members, self.err, stream)
+        st = check_status(self.err, stream)
+        if st != 0:
+            raise Pack3DError(st, "z-slab index map (the coordinates must cover the slab once each)")
+        self.q_rot, self.k_rot = torch.empty_like(self.ext["q"]), torch.empty_like(self.ext["k_loc"])
+        self.o_loc = zeros(N, Hq, d, dtype=torch.float32)
+        self.k_sum, self.v_sum = zeros(M, Hkv, d), zeros(M, Hkv, d)
+        self.out = zeros(p.tokens, Hq, d)
+        # Halo send buffers and the rows of the extended arrays they are gathered from (a slice
+        # of the index map: the boundary planes' sites in raster order).
+        self.send = {}
+        for side, (a, b), n in (("below", p.send_below, p.lo), ("above", p.send_above, p.hi)):
+            if n:
+                self.send[side] = (self.g2p[a:b], zeros(b - a, Hkv, d), zeros(b - a, Hkv, d))
+        # The whole volume's summaries: gathered straight into k_all / v_all with even slabs, else
+        # into padded parts and compacted by a row gather.
+        parts = summary_parts(cfg, world)
+        self.part = parts[rank]
+        self.most = max(c for _, _, c in parts)
+        M_all = sum(c for _, _, c in parts)
+        self.k_all, self.v_all = zeros(M_all, Hkv, d), zeros(M_all, Hkv, d)
+        self.uneven = any(o != 0 or c != self.most for _, o, c in parts)
+        if self.uneven:
+            self.k_pad, self.v_pad = zeros(self.most * world, Hkv, d), zeros(self.most * world, Hkv, d)
+            self.compact = torch.cat([torch.arange(r * self.most + o, r * self.most + o + c, dtype=torch.int32)
+                                      for r, (_, o, c) in enumerate(parts)]).to(dev)
+
+    def inputs(self) -> Dict:
+        """Views of the extended arrays' own rows, to be written before `forward` (in the order
+        of the coordinates the plan was made with)."""
+        t = self.p.tokens
+        return {k: v[:t] for k, v in self.ext.items() if k != "coords"}
+
+    # ---- the phases ----------------------------------------------------------------------------
+    def pack_halo(self):
+        """Gathers the boundary planes' K_loc / V_loc rows into the send buffers (raster order)."""
+        from . import gather_rows
+        for idx, ks, vs in self.send.values():
+            gather_rows(idx, self.ext["k_loc"], ks, self.stream)
+            gather_rows(idx, self.ext["v_loc"], vs, self.stream)
+
+    def halo_views(self):
+        """(below, above): None, or the (K_loc, V_loc) row views the neighbour's planes go to."""
+        out = []
+        for a, b in (self.p.halo_below, self.p.halo_above):
+            out.append((self.ext["k_loc"][a:b], self.ext["v_loc"][a:b]) if b > a else None)
+        return tuple(out)
+
+    def local(self):
+        """Summaries, RoPE and local attention on the extended lattice."""
+        from . import build_summaries, local_attn, rope_qk
+        e, ce = self.ext, self.cfg_e
+        build_summaries(ce, self.members, e["k_cmp"], e["v_cmp"], e["scores"], self.k_sum, self.v_sum, self.stream)
+        rope_qk(ce, e["coords"], e["q"], self.q_rot, e["k_loc"], self.k_rot, self.stream)
+        local_attn(ce, self.g2p, self.q_rot, self.k_rot, e["v_loc"], self.o_loc, self.err, self.stream)
+
+    def summary_part(self):
+        """The rows of k_sum / v_sum this rank contributes to the all-gather (its own blocks, plus
+        halo blocks up to the common part size when slabs are uneven)."""
+        start = self.part[0]
+        return self.k_sum[start:start + self.most], self.v_sum[start:start + self.most]
+
+    def attend(self):
+        """The query x summary stage and the gate for the own tokens against k_all / v_all."""
+        from . import summary_attn_rows
+        t = self.p.tokens
+        summary_attn_rows(self.cfg_e, t, self.k_all.shape[0], self.q_rot[:t], self.k_all, self.v_all,
+                          self.o_loc[:t], self.ext["gate"][:t], self.out, self.err, self.stream)
+        return self.out
+
+    # ---- the exchanges (NCCL between GPUs) ------------------------------------------------------
+    def exchange_halo(self):
+        import torch.distributed as dist
+        p, ops = self.p, []
+        below, above = self.halo_views()
+        for side, peer, recv in (("below", p.rank - 1, below), ("above", p.rank + 1, above)):
+            if side in self.send:
+                _, ks, vs = self.send[side]
+                ops += [dist.P2POp(dist.isend, ks, peer, self.group), dist.P2POp(dist.isend, vs, peer, self.group),
+                        dist.P2POp(dist.irecv, recv[0], peer, self.group),
+                        dist.P2POp(dist.irecv, recv[1], peer, self.group)]
+        if ops:
+            for req in dist.batch_isend_irecv(ops):
+                req.wait()
+
+    def gather_summaries(self):
+        import torch.distributed as dist
+
+        from . import gather_rows
+        k_part, v_part = self.summary_part()
+        if not self.uneven:
+            dist.all_gather_into_tensor(self.k_all, k_part, group=self.group)
+            dist.all_gather_into_tensor(self.v_all, v_part, group=self.group)
+            return
+        dist.all_gather_into_tensor(self.k_pad, k_part, group=self.group)
+        dist.all_gather_into_tensor(self.v_pad, v_part, group=self.group)
+        gather_rows(self.compact, self.k_pad, self.k_all, self.stream)
+        gather_rows(self.compact, self.v_pad, self.v_all, self.stream)
+
+    def forward(self):
+        """One step of the rank's forward pass; returns its tokens' outputs [tokens, Hq, d_h]."""
+        from . import Pack3DError, check_status
+        self.pack_halo()
+        self.exchange_halo()
+        self.local()
+        self.gather_summaries()
+        out = self.attend()
+        st = check_status(self.err, self.stream)
+        if st != 0:
+            raise Pack3DError(st, "z-slab forward")
+        return out
 
 
 def forward(cfg, inp: Dict, rank: int, world: int, group=None, stream=None):
-    """This rank's part of the forward pass of the volume `cfg` split over `world` ranks: `inp` holds
-    its own tokens (CUDA tensors, coordinates local to its slab); returns their outputs."""
-    import torch
-
-    from . import check_status
-    p = make_plan(cfg, rank, world)
-    if inp["q"].shape[0] != p.tokens:
-        raise ValueError(f"rank {rank} owns {p.tokens} tokens, got {inp['q'].shape[0]}")
-    cfg_e = ext_config(cfg, p)
-    blocks_per_plane = (cfg.H // cfg.by) * (cfg.W // cfg.bx)
-    err = torch.zeros(4, dtype=torch.int32, device=inp["q"].device)
-    below, above = exchange_halo(inp["k_loc"], inp["v_loc"], inp["coords"], p, group)
-    ext = prepare(inp, below, above, p)
-    q_rot, o_loc, k_sum, v_sum = local_stage(cfg_e, ext, err, stream)
-    k_own, v_own = own_summaries(k_sum, v_sum, p, blocks_per_plane)
-    k_all, v_all = gather_summaries(k_own, v_own, p, blocks_per_plane, group)
-    out = global_stage(cfg_e, p.tokens, q_rot, k_all, v_all, o_loc, ext["gate"], err, stream)
-    st = check_status(err, stream)
-    if st != 0:
-        from . import Pack3DError
-        raise Pack3DError(st, "z-slab forward")
-    return out
+    """One rank's forward pass of the volume `cfg` split over `world` ranks, set up for this call
+    only: `inp` holds its own tokens (CUDA tensors, coordinates local to its slab)."""
+    plan = Plan(cfg, inp["coords"], rank, world, group, stream)
+    for k, v in plan.inputs().items():
+        v.copy_(inp[k])
+    return plan.forward()

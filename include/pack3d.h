@@ -249,6 +249,21 @@ pack3d_status pack3d_summary_attn_rows(const pack3d_config *cfg, int64_t tokens,
                                        const float *o_loc, const float *gate, void *out,
                                        int32_t *err_word, void *stream);
 
+/* Row gather for the z-slab split of one volume over several ranks (the
+ * summary page and papernotes.org Key design 3: a query's local window reaches
+ * r_z planes into the neighbouring slab, so each rank sends the local keys and
+ * values of its boundary planes, found through its grid-to-packed map):
+ *   dst row i = src row idx[i]   for 0 <= i < n,
+ * rows of row_bytes bytes (a positive multiple of 16), idx[i] < 0 giving a
+ * zero row.  idx (int32, n entries), src and dst are device pointers owned by
+ * the caller; src and dst 16-byte aligned; every idx[i] must be a row of src
+ * (not checked on the device).  n == 0 returns PACK3D_OK with nothing
+ * launched.  Errors: null pointer, n < 0 or row_bytes not a positive multiple
+ * of 16 -> PACK3D_ERR_INVALID_ARG; misaligned src or dst ->
+ * PACK3D_ERR_ALIGNMENT; a failed launch -> PACK3D_ERR_CUDA. */
+pack3d_status pack3d_gather_rows(const int32_t *idx, int64_t n, const void *src, void *dst,
+                                 int64_t row_bytes, void *stream);
+
 /* The whole forward pass: index map, summaries, RoPE on Q and K_loc, local
  * branch, query-summary branch with the gate, all stream-ordered on `stream`.
  * workspace: device buffer of at least pack3d_workspace_bytes(cfg) bytes,

@@ -126,6 +126,17 @@ def test_host_errors_return_before_launch(p3):
     assert lib.pack3d_forward(cfgp, *args, fake + 16, ws, fake, None) == 6
     assert lib.pack3d_forward(cfgp, *args, fake, ws, None, None) == 1
     assert lib.pack3d_check_status(None, None) == 1
+    # the z-slab entry points: an explicit row count, and the row gather
+    assert lib.pack3d_summary_attn_rows(cfgp, -1, 4, fake, fake, fake, None, None, fake, None, None) == 1
+    assert lib.pack3d_summary_attn_rows(cfgp, 0, 4, None, None, None, None, None, None, None, None) == 0
+    assert lib.pack3d_summary_attn_rows(cfgp, 8, 4, None, fake, fake, None, None, fake, None, None) == 1
+    assert lib.pack3d_summary_attn_rows(cfgp, 8, 4, bad, fake, fake, None, None, fake, None, None) == 3
+    assert lib.pack3d_summary_attn_rows(cfgp, 1 << 24, 4, fake, fake, fake, None, None, fake, None, None) == 2
+    assert lib.pack3d_gather_rows(None, 0, None, None, 16, None) == 0
+    assert lib.pack3d_gather_rows(fake, -1, fake, fake, 16, None) == 1
+    assert lib.pack3d_gather_rows(fake, 4, fake, fake, 24, None) == 1
+    assert lib.pack3d_gather_rows(None, 4, fake, fake, 16, None) == 1
+    assert lib.pack3d_gather_rows(fake, 4, bad, fake, 16, None) == 3
     # the host-buffer pipeline: no pipeline handle, then a workspace too small for the staging copies
     hws = p3.host_workspace_bytes(c)
     assert hws > ws + 50 * 1024 * 1024

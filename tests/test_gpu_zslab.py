@@ -1,10 +1,10 @@
 """The z-slab split of one volume on one GPU: every rank's steps, in turn, in one process.
 
-No rank waits on another here: the halo planes and the gathered summaries are
-handed from one rank's tensors to the next by indexing, where the
-distributed path sends them (the gloo tests cover that host logic).  Each rank
-runs the library's kernels on its extended lattice, whose origin is the true z
-of its first plane; the concatenation of all ranks' outputs must match the
+No rank waits on another here: every rank's zslab.Plan runs its phases in
+turn (the boundary rows gathered by pack3d_gather_rows, summaries, RoPE and
+local attention, the summary compaction, the query x summary stage), and the
+two NCCL steps are replaced by copies between the plans' buffers.  Each rank
+works on its extended lattice, whose origin is the true z of its first plane; the concatenation of all ranks' outputs must match the
 whole-volume call: summaries and rotated queries bit for bit (the same
 arithmetic at the same true coordinates), the local branch and the output
 within the parity tolerance of the float64 oracle, and against the
@@ -53,33 +53,49 @@ def whole_volume(p3, cfg, s, d):
 
 
 def emulate(p3, cfg, s, d, world):
-    """Every rank's phases on this GPU; returns the whole-volume arrays assembled from the ranks."""
+    """Every rank's zslab.Plan phases on this GPU, the NCCL steps replaced by copies between the
+    plans' buffers; returns the whole-volume arrays assembled from the ranks."""
     from geometry_aware_local_b200 import zslab
-    plans = [zslab.make_plan(cfg, r, world) for r in range(world)]
-    takes = [zslab.take_slab(d, p) for p in plans]
-    edges = [zslab.boundary_rows(own["coords"], p) for p, (_, own) in zip(plans, takes)]
-    kv = [torch.stack([own["k_loc"], own["v_loc"]], dim=1) for _, own in takes]
-    none = kv[0][:0]
-    bpp = (cfg.H // cfg.by) * (cfg.W // cfg.bx)
-    err = torch.zeros(4, dtype=torch.int32, device="cuda")
-    ranks = []
-    for r, p in enumerate(plans):
-        below = kv[r - 1][edges[r - 1][1]] if p.lo else none      # the last rz planes of the rank below
-        above = kv[r + 1][edges[r + 1][0]] if p.hi else none      # the first rz planes of the rank above
-        ext = zslab.prepare(takes[r][1], below, above, p)
-        cfg_e = zslab.ext_config(cfg, p)
-        q_rot, o_loc, k_sum, v_sum = zslab.local_stage(cfg_e, ext, err)
-        ranks.append((cfg_e, ext, q_rot, o_loc) + tuple(zslab.own_summaries(k_sum, v_sum, p, bpp)))
-    k_all = torch.cat([rk[4] for rk in ranks])
-    v_all = torch.cat([rk[5] for rk in ranks])
-    res = dict(k_sum=k_all, v_sum=v_all, q_rot=torch.empty_like(d["q"]), out=torch.empty_like(d["q"]),
-               o_loc=torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device="cuda"))
-    for p, (idx, _), (cfg_e, ext, q_rot, o_loc, _, _) in zip(plans, takes, ranks):
-        out = zslab.global_stage(cfg_e, p.tokens, q_rot, k_all, v_all, o_loc, ext["gate"], err)
-        res["out"][idx] = out
-        res["q_rot"][idx] = q_rot[:p.tokens]
-        res["o_loc"][idx] = o_loc[:p.tokens]
-    assert p3.check_status(err) == 0
+    plans, takes = [], []
+    for r in range(world):
+        idx, own = zslab.take_slab(d, zslab.make_plan(cfg, r, world))
+        plan = zslab.Plan(cfg, own["coords"], r, world)
+        for k, v in plan.inputs().items():
+            v.copy_(own[k])
+        plans.append(plan)
+        takes.append(idx)
+    for plan in plans:
+        plan.pack_halo()
+    for r, plan in enumerate(plans):
+        below, above = plan.halo_views()
+        if below is not None:                      # the rank below sent its last planes
+            _, ks, vs = plans[r - 1].send["above"]
+            below[0].copy_(ks)
+            below[1].copy_(vs)
+        if above is not None:                      # the rank above sent its first planes
+            _, ks, vs = plans[r + 1].send["below"]
+            above[0].copy_(ks)
+            above[1].copy_(vs)
+    for plan in plans:
+        plan.local()
+    parts = [plan.summary_part() for plan in plans]
+    for plan in plans:                             # the all-gather, then the compaction
+        if plan.uneven:
+            plan.k_pad.copy_(torch.cat([k for k, _ in parts]))
+            plan.v_pad.copy_(torch.cat([v for _, v in parts]))
+            p3.gather_rows(plan.compact, plan.k_pad, plan.k_all)
+            p3.gather_rows(plan.compact, plan.v_pad, plan.v_all)
+        else:
+            plan.k_all.copy_(torch.cat([k for k, _ in parts]))
+            plan.v_all.copy_(torch.cat([v for _, v in parts]))
+    res = dict(k_sum=plans[0].k_all, v_sum=plans[0].v_all, q_rot=torch.empty_like(d["q"]),
+               out=torch.empty_like(d["q"]), o_loc=torch.empty(s.N, s.Hq, s.d_h, dtype=torch.float32, device="cuda"))
+    for plan, idx in zip(plans, takes):
+        t = plan.p.tokens
+        res["out"][idx] = plan.attend()
+        res["q_rot"][idx] = plan.q_rot[:t]
+        res["o_loc"][idx] = plan.o_loc[:t]
+        assert p3.check_status(plan.err) == 0
     return res
 
 
@@ -168,3 +184,18 @@ def test_forward_on_a_one_rank_nccl_group(p3):
     assert rel_err(out.float().cpu(), whole["out"].float().cpu()) <= 1e-2
     ref = oracle.forward(s, inp)["out"]
     assert rel_err(out.float().cpu().numpy(), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("n,row_shape,dtype", [(1, (2, 64), torch.bfloat16), (1000, (2, 64), torch.bfloat16),
+                                               (777, (8, 64), torch.float32), (5, (4,), torch.float32)])
+def test_gather_rows_bit_exact(p3, n, row_shape, dtype):
+    """pack3d_gather_rows: dst row i is src row idx[i], a negative index a zero row (byte moves only)."""
+    gen = torch.Generator(device="cuda").manual_seed(n)
+    src = torch.randn((3000,) + row_shape, generator=gen, device="cuda").to(dtype)
+    idx = torch.randint(-1, 3000, (n,), generator=gen, device="cuda", dtype=torch.int32)
+    dst = torch.full((n,) + row_shape, 7.0, device="cuda", dtype=dtype)
+    p3.gather_rows(idx, src, dst)
+    torch.cuda.synchronize()
+    want = src.index_select(0, idx.clamp(min=0).long())
+    want[idx < 0] = 0
+    assert torch.equal(dst, want)

@@ -4,9 +4,11 @@ Each rank takes the tokens of its planes, exchanges its boundary planes' local
 keys and values with its neighbours, and runs the stages on its slab extended
 by the received halo, a lattice whose origin is the true z of its first plane.
 Here the stages are the oracle's (float64, CPU), the exchanges are gloo's, and
-the arrangement of tensors (which rows are sent, how the extended lattice is
-laid out, which summaries are a rank's own, how the gathered summaries are
-ordered) is the library's own z-slab module.  Every rank's outputs must equal
+the layout is the library's z-slab module's (the extended lattice's
+coordinates and rows, which index-map slice is sent and where the halo lands,
+which summaries each rank contributes to the all-gather and which of them are
+kept); the row movement itself, done on the GPU by pack3d_gather_rows and
+NCCL, is done here by CPU indexing.  Every rank's outputs must equal
 the whole-volume oracle's for the same tokens (the local window of a boundary
 query, the summaries of every block and the rotation of every token depend on
 all of it being right), and the index map and block membership of its own
@@ -22,6 +24,8 @@ import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
+
+NAMES = ("coords", "q", "k_loc", "v_loc", "k_cmp", "v_cmp", "scores", "gate")
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -53,18 +57,21 @@ def _rank(rank, world, port, shape_kw, center, q):
         s = _shape(**shape_kw)
         inp = synth.make_inputs(s, seed=41)
         whole = oracle.forward(s, inp, center=center)
+        st_w, g2p_w, mem_w = oracle.build_index(s, inp["coords"])
         p = zslab.make_plan(s, rank, world)
         idx, own = zslab.take_slab(inp, p)
-        below, above = zslab.exchange_halo(own["k_loc"], own["v_loc"], own["coords"], p)
-        ext = zslab.prepare(own, below, above, p)
+        # The extended lattice as zslab.Plan lays it out: own rows, then the halo planes.
+        coords = zslab.ext_coords(own["coords"], p).numpy()
         se = s.replace(Z=p.Z_ext, origin=(s.origin[0] + p.z0 - p.lo, s.origin[1], s.origin[2]))
-        st, g2p, mem = oracle.build_index(se, ext["coords"])
+        st, g2p, mem = oracle.build_index(se, coords)
         assert st == 0
-        coords = ext["coords"].numpy()
+        N_e = p.Z_ext * s.H * s.W
+        ext = {k: torch.zeros((N_e,) + tuple(own[k].shape[1:]), dtype=own[k].dtype) for k in NAMES if k != "coords"}
+        for k in ext:
+            ext[k][:p.tokens] = own[k]
         # The index map and block membership of the rank's own planes, mapped to whole-volume
         # token ids (own tokens through take_slab's indices, halo tokens through their true
         # coordinates), must be the whole volume's, bit for bit.
-        st_w, g2p_w, mem_w = oracle.build_index(s, inp["coords"])
         true_z = coords[:, 0] + (p.z0 - p.lo)
         ext2glob = g2p_w[(true_z * s.H + coords[:, 1]) * s.W + coords[:, 2]].astype(np.int64)
         ext2glob[:p.tokens] = idx.numpy()
@@ -73,19 +80,41 @@ def _rank(rank, world, port, shape_kw, center, q):
                                           g2p_w[p.z0 * hw:p.z1 * hw]) and
                            np.array_equal(ext2glob[mem[p.lo * bpp:(p.lo + p.planes) * bpp]],
                                           mem_w[p.z0 * bpp:p.z1 * bpp]))
+        # Halo: the boundary planes' rows (index-map slices, raster order) to the neighbours,
+        # theirs into the halo rows.
+        ops = []
+        for peer, (a, b), (ra, rb), n in ((rank - 1, p.send_below, p.halo_below, p.lo),
+                                          (rank + 1, p.send_above, p.halo_above, p.hi)):
+            if n:
+                rows = torch.from_numpy(g2p[a:b].astype(np.int64))
+                for name in ("k_loc", "v_loc"):
+                    ops.append(dist.P2POp(dist.isend, ext[name].index_select(0, rows).contiguous(), peer))
+                    ops.append(dist.P2POp(dist.irecv, ext[name][ra:rb], peer))
+        if ops:
+            for req in dist.batch_isend_irecv(ops):
+                req.wait()
         rows = np.arange(p.tokens)
         qr = oracle.rotate(se, coords[:p.tokens], ext["q"][:p.tokens])
         kr = oracle.rotate(se, coords, ext["k_loc"])
         ks, vs = oracle.summaries(se, coords, mem, ext["k_cmp"], ext["v_cmp"], ext["scores"], center=center)
         ol = oracle.local_attn(se, coords, g2p, qr, kr, ext["v_loc"].numpy(), rows)
-        k_own, v_own = zslab.own_summaries(torch.from_numpy(ks), torch.from_numpy(vs), p, bpp)
-        k_all, v_all = zslab.gather_summaries(k_own, v_own, p, bpp)
-        oc = oracle.summary_attn(se, qr, k_all.numpy(), v_all.numpy())
+        # Summaries: every rank's part (summary_parts), all-gathered, then the own blocks kept.
+        parts = zslab.summary_parts(s, world)
+        start, _, _ = parts[rank]
+        most = max(c for _, _, c in parts)
+        got = []
+        for arr in (ks, vs):
+            part = torch.from_numpy(np.ascontiguousarray(arr[start:start + most]))
+            bufs = [torch.empty_like(part) for _ in range(world)]
+            dist.all_gather(bufs, part)
+            got.append(np.concatenate([bufs[r].numpy()[o:o + c] for r, (_, o, c) in enumerate(parts)]))
+        k_all, v_all = got
+        oc = oracle.summary_attn(se, qr, k_all, v_all)
         out = oracle.gate_mix(se, ext["gate"].numpy(), ol, oc, rows)
         ref = whole["out"][idx.numpy()]
         q.put((rank, float(np.abs(out - ref).max() / np.abs(ref).max()),
                float(np.abs(ol - whole["o_loc"][idx.numpy()]).max()),
-               float(max(np.abs(k_all.numpy() - whole["k_sum"]).max(), np.abs(v_all.numpy() - whole["v_sum"]).max())),
+               float(max(np.abs(k_all - whole["k_sum"]).max(), np.abs(v_all - whole["v_sum"]).max())),
                p.lo, p.hi, index_exact, None))
     except Exception as e:                       # report instead of hanging the parent
         q.put((rank, None, None, None, None, None, None, repr(e)))
@@ -147,18 +176,28 @@ def test_slab_bounds_and_plan():
         zslab.slab_bounds(3, 4)
 
 
-def test_boundary_rows_are_raster_planes():
-    import synth
+def test_layout_ranges_and_summary_parts():
     from geometry_aware_local_b200 import zslab
-    s = _shape(Z=4)
-    inp = synth.make_inputs(s, seed=3)
-    p = zslab.make_plan(s, 0, 1)
-    first, last = zslab.boundary_rows(inp["coords"], p)
-    c = inp["coords"][first]
-    n = s.rz * s.H * s.W
-    want = np.stack(np.meshgrid(np.arange(s.rz), np.arange(s.H), np.arange(s.W), indexing="ij"), -1).reshape(n, 3)
-    assert np.array_equal(c.numpy(), want)
-    assert np.array_equal(inp["coords"][last].numpy(), want + np.array([s.Z - s.rz, 0, 0]))
+    s = _shape(Z=7)                       # 4 + 3 planes over two ranks, 8 x 12 sites per plane, rz = 2
+    p0, p1 = zslab.make_plan(s, 0, 2), zslab.make_plan(s, 1, 2)
+    hw = s.H * s.W
+    # rank 0: own planes 0-3 (rows 0 .. 4hw), halo above = true planes 4-5 after them
+    assert (p0.lo, p0.hi, p0.Z_ext) == (0, 2, 6)
+    assert p0.halo_below == (4 * hw, 4 * hw) and p0.halo_above == (4 * hw, 6 * hw)
+    assert p0.send_above == (2 * hw, 4 * hw)           # its last two planes, extended-lattice sites
+    # rank 1: halo below = true planes 2-3 (extended planes 0-1), own planes 4-6 (extended 2-4)
+    assert (p1.lo, p1.hi, p1.Z_ext) == (2, 0, 5)
+    assert p1.halo_below == (3 * hw, 5 * hw) and p1.halo_above == (5 * hw, 5 * hw)
+    assert p1.send_below == (2 * hw, 4 * hw)
+    # summaries: 4 and 3 planes of 4 x 3 blocks; rank 1's part reaches back into its halo blocks
+    bpp = (s.H // s.by) * (s.W // s.bx)
+    assert zslab.summary_parts(s, 2) == [(0, 0, 4 * bpp), (1 * bpp, 1 * bpp, 3 * bpp)]
+    even = zslab.summary_parts(_shape(Z=8), 2)
+    assert all(o == 0 and c == 4 * bpp for _, o, c in even)
+    ext = zslab.ext_coords(torch.zeros((p1.tokens, 3), dtype=torch.int32), p1)
+    assert ext.shape == (p1.Z_ext * hw, 3)
+    assert ext[:p1.tokens, 0].eq(2).all()                 # own z shifted by lo
+    assert ext[p1.tokens:, 0].tolist() == [z for z in (0, 1) for _ in range(hw)]
 
 
 def test_ext_config_shifts_origin_and_keeps_everything_else():
