@@ -4,9 +4,9 @@
 // memory allocation, the first loads, the gate epilogue) is a large share of
 // its time, and one-tile CTAs two per SM hide it behind each other; with many
 // summary tiles the two-tile CTA, which reads every k~ / v~ tile once for both
-// query tiles, is faster.  Measured on B200: 65k tokens (32 summary tiles)
-// 0.78-0.80 ms one-tile vs 0.81 ms two-tile; 262k tokens (128 summary tiles)
-// 11.46 ms vs 10.8-10.9 ms.
+// query tiles, is faster.  Measured on B200: 65k tokens (M = 4,096) 0.78-0.80
+// ms one-tile vs 0.81 ms two-tile; 262k tokens (M = 16,384) 11.46 ms vs
+// 10.8-10.9 ms.  The threshold is in summaries (48 tiles of 128).
 #include "common.cuh"
 #include "internal.h"
 

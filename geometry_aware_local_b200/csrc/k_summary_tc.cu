@@ -7,7 +7,8 @@
 //
 // One CTA = kGroups 128-row query tiles of one kv head sharing every summary
 // tile (rows are (token, q head) pairs of the kv group: 128/G tokens x G
-// heads); the default is two tiles and 128-summary tiles.
+// heads); the default is two tiles and 128-summary tiles (the one-tile build,
+// k_summary_tc_one.cu, uses 96-summary tiles and two P buffers).
 //   * the last warp streams k~ / v~ tiles (kBN summaries x 64 dims, bf16,
 //     128-byte swizzle) through a TMA ring; the Q tiles are loaded once.
 //   * one warp per group issues that group's tcgen05.mma: S = Q k~^T (M=128,
@@ -21,8 +22,8 @@
 // At d_h = 64 each exponential pairs with only 256 MMA flops, so the softmax
 // sets the pace: packed f32x2 FMA/add, a three-input max and MUFU.ex2.  O is
 // rescaled lazily (only when a row maximum grows by more than
-// 2^8).  Tensor memory (512 columns), group w at w*kGroupCols: S, P (packed
-// bf16), O.
+// 2^8).  Tensor memory, group w at w*kGroupCols: S, P (packed bf16; one or two
+// buffers), O.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -42,12 +43,19 @@ namespace {
 
 // Compile-time shape of the pipeline: query tiles (softmax warpgroups) per
 // CTA and summaries per tile.  Tensor memory per group: S (kBN columns), P
-// (kBN/2), O (64), i.e. 256 columns for (2, 128) and 160 for (3, 64).
+// (kBN/2 per buffer), O (64), i.e. 256 columns for (2, 128) with one P buffer
+// and for (1, 96) with two.
 #ifndef PACK3D_SA_GROUPS
 #define PACK3D_SA_GROUPS 2
 #endif
 #ifndef PACK3D_SA_BN
 #define PACK3D_SA_BN 128
+#endif
+// P buffers per group: with two, the exponentials of tile j are written while
+// O += P v~ of tile j-1 still reads the other buffer (tensor memory per group:
+// S kBN + 2 x kBN/2 + O 64, i.e. 256 columns at kBN = 96).
+#ifndef PACK3D_SA_PBUFS
+#define PACK3D_SA_PBUFS 1
 #endif
 constexpr int kBM = 128;                      // rows per query tile
 constexpr int kBN = PACK3D_SA_BN;             // summaries per tile
@@ -55,7 +63,8 @@ constexpr int kGroups = PACK3D_SA_GROUPS;     // query tiles (softmax warpgroups
 constexpr int kMmaWarp = 4 * kGroups;          // first MMA warp; one per group
 constexpr int kTmaWarp = kMmaWarp + kGroups;
 constexpr int kThreads = 32 * (kTmaWarp + 1);
-constexpr int kColS = 0, kColP = kBN, kColO = kBN + kBN / 2;
+constexpr int kPBufs = PACK3D_SA_PBUFS;
+constexpr int kColS = 0, kColP = kBN, kColO = kBN + kPBufs * (kBN / 2);
 constexpr int kGroupCols = kColO + kDh;       // tensor-memory columns per group
 constexpr int kQBytes = kBM * kDh * 2;        // 16 KiB
 constexpr int kKVBytes = kBN * kDh * 2;
@@ -84,8 +93,11 @@ constexpr int kPairsPerChunk = kBN / 2 / kPChunks;   // packed P columns per chu
 constexpr int kMmasPerChunk = kBN / 16 / kPChunks;   // K = 16 steps of O += P v~ per chunk
 static_assert(kPairsPerChunk % 16 == 0, "P chunks are stored 16 columns at a time");
 // barriers: full[S], empty[S], qfull, then per group: s_full, s_free, o_final,
-// p_full[kPChunks], p_free[kPChunks], drain (the abort path's MMA drain)
-constexpr int kGroupBars = 4 + 2 * kPChunks;
+// p_full[kPSlots], p_free[kPSlots] (per P chunk, or per P buffer), drain (the
+// abort path's MMA drain)
+static_assert(kPBufs == 1 || kPChunks == 1, "P buffers or P chunks, not both");
+constexpr int kPSlots = kPChunks * kPBufs;           // p_full / p_free barriers per group
+constexpr int kGroupBars = 4 + 2 * kPSlots;
 constexpr int kNumBars = 2 * kStages + 1 + kGroups * kGroupBars;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
@@ -141,8 +153,8 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
   auto s_free = [&](int w) { return gbar(w, 1); };
   auto o_final = [&](int w) { return gbar(w, 2); };
   auto p_full = [&](int w, int c) { return gbar(w, 3 + c); };
-  auto p_free = [&](int w, int c) { return gbar(w, 3 + kPChunks + c); };
-  auto drain = [&](int w) { return gbar(w, 3 + 2 * kPChunks); };
+  auto p_free = [&](int w, int c) { return gbar(w, 3 + kPSlots + c); };
+  auto drain = [&](int w) { return gbar(w, 3 + 2 * kPSlots); };
   volatile ptx::WaitCtl* ctl = reinterpret_cast<volatile ptx::WaitCtl*>(smem + kBarOff + kNumBars * 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8 + sizeof(ptx::WaitCtl));
   auto wait = [&](uint32_t bar, uint32_t parity) { return ptx::mbar_wait(bar, parity, ctl); };
@@ -158,7 +170,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       ptx::mbar_init(s_free(w), 4);       // one arrival per softmax warp
       ptx::mbar_init(o_final(w), 1);
       ptx::mbar_init(drain(w), 1);
-      for (int c = 0; c < kPChunks; ++c) {
+      for (int c = 0; c < kPSlots; ++c) {
         ptx::mbar_init(p_full(w, c), 4);
         ptx::mbar_init(p_free(w, c), 1);
       }
@@ -224,13 +236,14 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
       };
       auto issue_pv = [&](int j, int c) {
         const uint32_t vaddr = sbase + kStageOff + (j % kStages) * kStageBytes + kKVBytes;
+        const int pb = j % kPBufs;                       // this tile's P buffer
 #pragma unroll
         for (int i = 0; i < kMmasPerChunk; ++i) {
           const int kk = c * kMmasPerChunk + i;
-          ptx::mma_ts(tO, tP + kk * 8, ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024), kIdescPV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_ts(tO, tP + pb * (kBN / 2) + kk * 8, ptx::smem_desc_sw128(vaddr + kk * 2048, 8192, 1024),
+                      kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::tc_commit(p_free(w, c));
+        ptx::tc_commit(p_free(w, c + pb));
         if (c == kPChunks - 1) {
           ptx::tc_commit(empty(j % kStages));
           if (j == T - 1) ptx::tc_commit(o_final(w));
@@ -249,7 +262,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           issue_s(j + 1);
         }
         for (int c = 0; ok && c < kPChunks; ++c) {
-          if (!(ok = wait(p_full(w, c), j & 1))) break;
+          if (!(ok = wait(p_full(w, c + j % kPBufs), (j / kPBufs) & 1))) break;
           ptx::tc_fence_after();
           issue_pv(j, c);
         }
@@ -279,6 +292,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     auto load_s = [&](uint32_t* sv, int j) {
 #pragma unroll
       for (int q = 0; q < kBN / 64; ++q) ptx::tmem_ld64_sync(trow + kColS + 64 * q, sv + 64 * q);
+      if constexpr (kBN % 64 == 32) ptx::tmem_ld32_sync(trow + kColS + kBN - 32, sv + kBN - 32);
       if ((j + 1) * kBN > a.M) {
         const int lim = a.M - j * kBN;
 #pragma unroll
@@ -302,7 +316,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     };
     // Exponentials of chunk cc of one S row, written to the P buffer 16 packed
     // columns at a time; the (unrounded) values are added to rs.
-    auto exps_chunk = [&](const uint32_t* sv, int cc, float2* rs) {
+    auto exps_chunk = [&](const uint32_t* sv, int cc, float2* rs, uint32_t tPb) {
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_used, -m_used);
 #pragma unroll
       for (int q = 0; q < kPairsPerChunk / 16; ++q) {
@@ -316,7 +330,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           rs[k & 1] = __fadd2_rn(rs[k & 1], p);
           pk[k] = pack_bf16x2(p.x, p.y);
         }
-        ptx::tmem_st16(tP + cc * kPairsPerChunk + 16 * q, pk);
+        ptx::tmem_st16(tPb + cc * kPairsPerChunk + 16 * q, pk);
       }
     };
     // One arrival per warp: every lane's tensor-memory accesses are complete
@@ -343,18 +357,21 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           m_used = mxs;
         }
         const bool rescale = j > 0 && __any_sync(0xffffffffu, f != 1.f);
+        const int pb = j % kPBufs;                       // this tile's P buffer
 #pragma unroll
         for (int cc = 0; cc < kPChunks; ++cc) {
-          if (j > 0) {
-            if (!(ok = __all_sync(0xffffffffu, wait(p_free(w, cc), (j - 1) & 1)))) break;
+          if (j >= kPBufs) {
+            // The buffer's previous tile (j - kPBufs) has been read by its O += P v~.
+            if (!(ok = __all_sync(0xffffffffu, wait(p_free(w, cc + pb), ((j / kPBufs) - 1) & 1)))) break;
             ptx::tc_fence_after();
           }
-          exps_chunk(sv, cc, rs);
+          exps_chunk(sv, cc, rs, tP + pb * (kBN / 2));
           if (cc == 0 && rescale) {
             // O is rescaled before this tile's first O += P v~ is issued and
             // after the previous tile's last one has completed (its commit
             // covers all earlier MMAs of the group).
-            if (!(ok = __all_sync(0xffffffffu, wait(p_free(w, kPChunks - 1), (j - 1) & 1))))
+            const int pj = j - 1;
+            if (!(ok = __all_sync(0xffffffffu, wait(p_free(w, kPChunks - 1 + pj % kPBufs), (pj / kPBufs) & 1))))
               break;
             ptx::tc_fence_after();
             uint32_t r[16];
@@ -367,7 +384,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             }
           }
           ptx::tmem_wait_st();
-          warp_arrive(p_full(w, cc));
+          warp_arrive(p_full(w, cc + pb));
         }
         if (!ok) break;
       }

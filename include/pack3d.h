@@ -107,12 +107,13 @@ typedef enum { PACK3D_F32 = 0, PACK3D_BF16 = 1 } pack3d_dtype;
  * only (float, PACK3D_FLAG_SIMT_*): those have no pipeline waits. */
 #define PACK3D_FLAG_DIAG_STALL    0x8
 /* The tensor-core query x summary kernel comes in two builds: one 128-row query
- * tile per CTA with two CTAs per SM, and two tiles per CTA with one CTA per SM
- * (every summary tile read once for both).  By default the library picks the
- * one-tile build up to 48 summary tiles (M <= 6,144) and the two-tile build
- * above; these flags force one of them (setting both is an error).  Both
- * builds compute every row with the same sequence of operations, so their
- * outputs are identical bit for bit; the flags only move the cost. */
+ * tile per CTA with two CTAs per SM (summaries in tiles of 96, two P buffers),
+ * and two tiles per CTA with one CTA per SM (every tile of 128 summaries read
+ * once for both).  By default the library picks the one-tile build up to
+ * M <= 6,144 summaries and the two-tile build above; these flags force one of
+ * them (setting both is an error).  Both builds form the same products in the
+ * same order and group the softmax row sums differently, so their outputs
+ * agree to float rounding; the flags only move the cost. */
 #define PACK3D_FLAG_SUMMARY_ONE_TILE 0x10
 #define PACK3D_FLAG_SUMMARY_TWO_TILE 0x20
 

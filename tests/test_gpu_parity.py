@@ -141,13 +141,16 @@ def test_two_tile_build_matches_oracle(p3, name, s, packing):
 
 @pytest.mark.parametrize("s", [small(Z=4, H=32, W=40), small(Z=3, H=10, W=14, by=2, bx=2), small(Hq=8, Hkv=1)],
                          ids=["m-multi", "ragged-brick", "g8"])
-def test_one_and_two_tile_builds_are_bit_identical(p3, s):
-    """Both builds run every row through the same operations: o_cmp and the gated output agree bit for
-    bit, and so do the training forward's output and gate gradient."""
+def test_one_and_two_tile_builds_agree(p3, s):
+    """The one-tile build walks the summaries in tiles of 96, the two-tile build in tiles of 128: the
+    same products in the same order, with the row sums grouped differently, so o_cmp, the gated
+    output and the training forward's output and gradients agree to float rounding (within two bf16
+    ulps of the largest value); each build is checked against the oracle elsewhere."""
     d = to_dev(synth.make_inputs(s, "random", seed=14))
     a = run_stages(p3, s, d, flags=p3.FLAG_SUMMARY_ONE_TILE)
     b = run_stages(p3, s, d, flags=p3.FLAG_SUMMARY_TWO_TILE)
-    assert torch.equal(a["o_cmp"], b["o_cmp"]) and torch.equal(a["out"], b["out"])
+    for k in ("o_cmp", "out"):
+        assert rel_err(a[k].float().numpy(), b[k].float().numpy()) <= 8e-3, k
     dout = synth.make_dout(s, "random", seed=14).cuda()
     res = []
     for flags in (p3.FLAG_SUMMARY_ONE_TILE, p3.FLAG_SUMMARY_TWO_TILE):
@@ -159,9 +162,9 @@ def test_one_and_two_tile_builds_are_bit_identical(p3, s):
         p3.forward_backward(cfg, d["coords"], d["q"], d["k_loc"], d["v_loc"], d["k_cmp"], d["v_cmp"], d["scores"],
                             d["gate"], dout, out, grads, ws, err)
         assert p3.check_status(err) == 0
-        res.append((out.cpu(), grads["dgate"].cpu(), grads["dq"].cpu()))
-    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
-    assert torch.equal(res[0][2], res[1][2])
+        res.append((out.float().cpu(), grads["dgate"].float().cpu(), grads["dq"].float().cpu()))
+    for i, k in enumerate(("out", "dgate", "dq")):
+        assert rel_err(res[0][i].numpy(), res[1][i].numpy()) <= 8e-3, k
 
 
 def sharp_inputs(s, packing, seed):
