@@ -46,7 +46,8 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGNMENT", 4: "DTYPE", 5: 
 
 ENTRY_POINTS = ("pack3d_default_config", "pack3d_validate_config", "pack3d_workspace_bytes",
                 "pack3d_build_index", "pack3d_rope", "pack3d_rope_qk", "pack3d_build_summaries", "pack3d_local_attn",
-                "pack3d_summary_attn", "pack3d_summary_attn_rows", "pack3d_gather_rows", "pack3d_forward",
+                "pack3d_summary_attn", "pack3d_summary_attn_rows", "pack3d_gather_rows", "pack3d_exp2_fma_eval",
+                "pack3d_forward",
                 "pack3d_forward_noalloc",
                 "pack3d_pipeline_create",
                 "pack3d_pipeline_destroy", "pack3d_host_workspace_bytes", "pack3d_forward_host",
@@ -104,6 +105,7 @@ def _load():
         "pack3d_summary_attn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "pack3d_summary_attn_rows": (ctypes.c_int, [C, ctypes.c_int64, ctypes.c_int64] + [P] * 8),
         "pack3d_gather_rows": (ctypes.c_int, [P, ctypes.c_int64, P, P, ctypes.c_int64, P]),
+        "pack3d_exp2_fma_eval": (ctypes.c_int, [P, P, ctypes.c_int64, P]),
         "pack3d_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P, P]),
         "pack3d_forward_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
         "pack3d_pipeline_create": (ctypes.c_int, [ctypes.POINTER(P)]),
@@ -329,6 +331,16 @@ def gather_rows(idx, src, dst, stream=None):
     row_bytes = dst[0].numel() * dst.element_size() if n else 16
     _check(lib.pack3d_gather_rows(_ptr(idx), int(n), _ptr(src), _ptr(dst), int(row_bytes), _stream(stream)),
            "pack3d_gather_rows")
+
+
+def exp2_fma_eval(x, y, stream=None):
+    """y = 2^x by the FMA-pipe cubic the one-tile query x summary kernel uses (pack3d_exp2_fma_eval);
+    x and y float32 contiguous CUDA tensors of one size."""
+    import torch
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel() or \
+            not (x.is_contiguous() and y.is_contiguous()):
+        raise ValueError("exp2_fma_eval: x and y must be contiguous float32 tensors of one size")
+    _check(lib.pack3d_exp2_fma_eval(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)), "pack3d_exp2_fma_eval")
 
 
 def _check_forward_args(what, cfg, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out, err):

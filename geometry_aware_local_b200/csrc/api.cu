@@ -311,6 +311,13 @@ pack3d_status pack3d_summary_attn_rows(const pack3d_config* cfg, int64_t tokens,
   return cuda_status(e);
 }
 
+pack3d_status pack3d_exp2_fma_eval(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return PACK3D_ERR_INVALID_ARG;
+  if (n == 0) return PACK3D_OK;
+  if (!x || !y) return PACK3D_ERR_INVALID_ARG;
+  return cuda_status(launch_exp2_fma_eval(x, y, n, (cudaStream_t)stream));
+}
+
 pack3d_status pack3d_gather_rows(const int32_t* idx, int64_t n, const void* src, void* dst, int64_t row_bytes,
                                  void* stream) {
   if (n < 0 || row_bytes <= 0 || row_bytes % 16 != 0) return PACK3D_ERR_INVALID_ARG;

@@ -81,6 +81,28 @@ __device__ __forceinline__ void stg16(void* p, const uint4& v) {
   *reinterpret_cast<uint4*>(p) = v;
 }
 
+// ---- 2^x on the FMA pipe ----------------------------------------------------
+// For a pair: x = n + f with n = rint(x) (added to the float's exponent field)
+// and f in [-1/2, 1/2], 2^f from a cubic whose coefficients are the minimax
+// fit of the relative error by the Remez exchange (fit_exp2.py next to this
+// library reproduces them); the largest relative error of the float Horner
+// evaluation is 7.5e-5, far below bf16's 3.9e-3.  Inputs are clamped at -125
+// so the result stays a normal float (about 2.4e-38 in place of 0).
+__device__ __forceinline__ float2 exp2_fma(float2 x) {
+  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.055171669f;
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
+  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // ---- axial RoPE tables -----------------------------------------------------
 // Table layout (float2 = cos, sin): plane p owns the contiguous entries
 // [pair_off[p], pair_off[p] + extent of its axis), one per local coordinate

@@ -44,6 +44,7 @@ struct Train {
   float* dgate;        // [N, Hq, 2]
 };
 
+cudaError_t launch_exp2_fma_eval(const float* x, float* y, long long n, cudaStream_t st);
 cudaError_t launch_gather_rows(const int32_t* idx, long long n, const void* src, void* dst, long long row_bytes,
                                cudaStream_t st);
 cudaError_t launch_build_index(const Shape& s, const int32_t* coords, int32_t* g2p,

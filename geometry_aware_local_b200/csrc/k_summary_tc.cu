@@ -20,7 +20,9 @@
 //   * warps 0 .. 4*kGroups-1 are the softmax warpgroups, one per query tile,
 //     thread = row = TMEM lane.
 // At d_h = 64 each exponential pairs with only 256 MMA flops, so the softmax
-// sets the pace: packed f32x2 FMA/add, a three-input max and MUFU.ex2.  O is
+// sets the pace: packed f32x2 FMA/add, a three-input max and MUFU.ex2 (the
+// one-tile build evaluates 2 of every 16 exponential pairs on the FMA pipe
+// instead, which unloads MUFU).  O is
 // rescaled lazily (only when a row maximum grows by more than
 // 2^8).  Tensor memory, group w at w*kGroupCols: S, P (packed bf16; one or two
 // buffers), O.
@@ -56,6 +58,11 @@ namespace {
 // S kBN + 2 x kBN/2 + O 64, i.e. 256 columns at kBN = 96).
 #ifndef PACK3D_SA_PBUFS
 #define PACK3D_SA_PBUFS 1
+#endif
+// Of every 16 pairs of exponentials, this many are evaluated on the FMA pipe
+// (exp2_fma) instead of MUFU, spread evenly over the pairs.
+#ifndef PACK3D_SA_POLY
+#define PACK3D_SA_POLY 0
 #endif
 constexpr int kBM = 128;                      // rows per query tile
 constexpr int kBN = PACK3D_SA_BN;             // summaries per tile
@@ -101,6 +108,8 @@ constexpr int kGroupBars = 4 + 2 * kPSlots;
 constexpr int kNumBars = 2 * kStages + 1 + kGroups * kGroupBars;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+constexpr int kPoly = PACK3D_SA_POLY;
+__host__ __device__ constexpr bool poly_pair(int k) { return kPoly > 0 && ((k % 16) * kPoly) % 16 < kPoly; }
 static_assert(kGroups * kGroupCols <= kTmemCols, "tensor memory plan");
 
 constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kBM, kBN, false);      // S: N = kBN summaries
@@ -326,7 +335,7 @@ summary_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
           const int pair = cc * kPairsPerChunk + q * 16 + k;
           const float2 x =
               __ffma2_rn(make_float2(__uint_as_float(sv[2 * pair]), __uint_as_float(sv[2 * pair + 1])), c2, nm2);
-          const float2 p = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+          const float2 p = poly_pair(pair) ? exp2_fma(x) : make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
           rs[k & 1] = __fadd2_rn(rs[k & 1], p);
           pk[k] = pack_bf16x2(p.x, p.y);
         }

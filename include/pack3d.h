@@ -265,6 +265,17 @@ pack3d_status pack3d_summary_attn_rows(const pack3d_config *cfg, int64_t tokens,
 pack3d_status pack3d_gather_rows(const int32_t *idx, int64_t n, const void *src, void *dst,
                                  int64_t row_bytes, void *stream);
 
+/* Diagnostic: evaluates the FMA-pipe exponential that the one-tile build of
+ * the query x summary kernel uses for 2 of every 16 pairs of its softmax
+ * exponentials (Key design 3's softmax over the summaries): y[i] = 2^x[i]
+ * from x = n + f, n = rint(x) put into the float's exponent, 2^f by a cubic
+ * minimax fit (Remez exchange, relative error <= 7.5e-5 on [-1/2, 1/2]);
+ * x is clamped at -125, so the result of a very negative x is ~2.4e-38
+ * rather than 0.  x and y are device float arrays of n elements (caller
+ * owned).  n == 0 -> PACK3D_OK; n < 0 or a null pointer ->
+ * PACK3D_ERR_INVALID_ARG; a failed launch -> PACK3D_ERR_CUDA. */
+pack3d_status pack3d_exp2_fma_eval(const float *x, float *y, int64_t n, void *stream);
+
 /* The whole forward pass: index map, summaries, RoPE on Q and K_loc, local
  * branch, query-summary branch with the gate, all stream-ordered on `stream`.
  * workspace: device buffer of at least pack3d_workspace_bytes(cfg) bytes,

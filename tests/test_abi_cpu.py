@@ -137,6 +137,9 @@ def test_host_errors_return_before_launch(p3):
     assert lib.pack3d_gather_rows(fake, 4, fake, fake, 24, None) == 1
     assert lib.pack3d_gather_rows(None, 4, fake, fake, 16, None) == 1
     assert lib.pack3d_gather_rows(fake, 4, bad, fake, 16, None) == 3
+    assert lib.pack3d_exp2_fma_eval(None, None, 0, None) == 0
+    assert lib.pack3d_exp2_fma_eval(fake, fake, -1, None) == 1
+    assert lib.pack3d_exp2_fma_eval(None, fake, 4, None) == 1
     # the host-buffer pipeline: no pipeline handle, then a workspace too small for the staging copies
     hws = p3.host_workspace_bytes(c)
     assert hws > ws + 50 * 1024 * 1024

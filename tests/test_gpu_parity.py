@@ -445,3 +445,21 @@ def test_forward_query_tiled_sizes_sampled_rows(p3, name):
     ref = oracle.forward(s, inp, rows)
     assert rel_err(out[rows].double().numpy(), ref["out"]) <= TOL["bf16"]
     assert rel_err(out[-32:].double().numpy(), ref["out"][-32:]) <= TOL["bf16"]
+
+
+def test_exp2_fma_against_reference(p3):
+    """The FMA-pipe exponential of the one-tile query x summary build (pack3d_exp2_fma_eval) over the
+    inputs the kernel feeds it (x <= 8 after the lazy maximum; masked columns at -inf): relative error
+    within the fit's 7.5e-5 (plus float rounding) against a float64 2^x, and ~2.4e-38 for x <= -125."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 2_000_001), torch.arange(-125, 9, dtype=torch.float32),
+                   torch.arange(-125, 8, dtype=torch.float32) + 0.5,
+                   torch.tensor([-0.5, 0.5, 1e-7, -1e-7, 0.0])]).cuda()
+    y = torch.empty_like(x)
+    p3.exp2_fma_eval(x, y)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref) / ref).abs().max().item()
+    assert rel <= 8e-5, rel
+    low = torch.tensor([-125.0, -126.0, -200.0, -1e30, float("-inf")], device="cuda")
+    yl = torch.empty_like(low)
+    p3.exp2_fma_eval(low, yl)
+    assert (yl > 0).all() and (yl <= 2.4e-38).all() and torch.isfinite(yl).all()
