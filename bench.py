@@ -71,9 +71,9 @@ KERNELS_PER_STEP = 7   # 2 fills + index, rope (Q and K), summaries, local, summ
 # under profiles/.  Emptied whenever that kernel changes until it is captured
 # again (a workload without an entry reports null).
 SUMMARY_ATTN_TRAFFIC: Dict[str, tuple] = {
-    "65k": (212.879872e6 + 48.276480e6,
-            "ncu capture of summary_attn_tc_kernel<0> (one-tile build: 96-summary tiles, two P buffers) on the "
-            "65k volume (profiles/summary_attn_tc_65k.md)"),
+    "65k": (212.882176e6 + 48.153344e6,
+            "ncu capture of summary_attn_tc_kernel<0> (one-tile build: 96-summary tiles, two P buffers, 2 of 16 "
+            "exponential pairs on the FMA pipe) on the 65k volume (profiles/summary_attn_tc_65k.md)"),
 }
 # Nominal HBM bandwidth of the part (8 TB/s), reported beside the measured copy peak.
 HBM_NOMINAL_GBS = 8000.0
