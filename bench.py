@@ -551,6 +551,79 @@ def time_sizes(p3, flush, stream, dev, peaks) -> Dict:
     return res
 
 
+def time_zslab(p3, name: str, ranks: int, warmup: int, steps: int, flush, dev) -> Dict:
+    """The z-slab split of the volume over `ranks` ranks, every rank's kernels run in turn on this
+    GPU (zslab.Plan phases; the two NCCL exchanges are replaced by device copies outside the timed
+    regions).  Per rank and step: the boundary-row gather, summaries, RoPE and local attention on
+    its extended lattice, and the query x summary stage for its tokens, timed with CUDA events."""
+    import torch
+
+    from geometry_aware_local_b200 import zslab
+    s = synth.CONFIGS[name]
+    cfg = p3.config_from_shape(s)
+    d = synth.make_inputs_on_device(s, s.packing, seed=0, device=dev)
+    plans = []
+    for r in range(ranks):
+        _, own = zslab.take_slab(d, zslab.make_plan(cfg, r, ranks))
+        plan = zslab.Plan(cfg, own["coords"], r, ranks)
+        for k, v in plan.inputs().items():
+            v.copy_(own[k])
+        plans.append(plan)
+    del d
+    stream = torch.cuda.current_stream(dev)
+    per_rank = [[] for _ in plans]
+    for it in range(warmup + steps):
+        evs = []
+        for r, plan in enumerate(plans):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            plan.pack_halo()
+            plan.local()
+            e1.record(stream)
+            evs.append([e0, e1])
+        for r, plan in enumerate(plans):             # the halo exchange, as copies
+            below, above = plan.halo_views()
+            for view, side, peer in ((below, "above", r - 1), (above, "below", r + 1)):
+                if view is not None:
+                    _, ks, vs = plans[peer].send[side]
+                    view[0].copy_(ks)
+                    view[1].copy_(vs)
+        parts = [plan.summary_part() for plan in plans]
+        for plan in plans:                             # the summary all-gather, as copies
+            if plan.uneven:
+                plan.k_pad.copy_(torch.cat([k for k, _ in parts]))
+                plan.v_pad.copy_(torch.cat([v for _, v in parts]))
+                p3.gather_rows(plan.compact, plan.k_pad, plan.k_all)
+                p3.gather_rows(plan.compact, plan.v_pad, plan.v_all)
+            else:
+                plan.k_all.copy_(torch.cat([k for k, _ in parts]))
+                plan.v_all.copy_(torch.cat([v for _, v in parts]))
+        for r, plan in enumerate(plans):
+            flush()
+            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e2.record(stream)
+            plan.attend()
+            e3.record(stream)
+            evs[r] += [e2, e3]
+        torch.cuda.synchronize()
+        if it >= warmup:
+            for r, (e0, e1, e2, e3) in enumerate(evs):
+                per_rank[r].append(e0.elapsed_time(e1) + e2.elapsed_time(e3))
+    for plan in plans:
+        if p3.check_status(plan.err) != 0:
+            raise RuntimeError("device error in the z-slab ranks")
+    ms = [statistics.mean(v) for v in per_rank]
+    eb = 2 if s.dtype == "bf16" else 4
+    halo = [sum(2 * (b - a) * s.Hkv * s.d_h * eb for (a, b) in (pl.p.halo_below, pl.p.halo_above)) for pl in plans]
+    gathered = plans[0].k_all.shape[0] * s.Hkv * s.d_h * eb * 2
+    return {"ranks": ranks, "workload": WORKLOAD_TEXT[name], "per_rank_compute_ms": ms,
+            "max_rank_compute_ms": max(ms), "halo_bytes_received_per_rank": halo,
+            "summary_bytes_all_gathered": gathered, "steps": steps, "warmup": warmup,
+            "note": "every rank's kernels timed in turn on one GPU; the NCCL halo exchange and summary "
+                    "all-gather are not timed (device copies stand in for them)"}
+
+
 def run_ours(args, s):
     import torch
 
@@ -670,6 +743,8 @@ def run_ours(args, s):
             comp["dense_sdpa"]["speedup_of_pack3d"] = comp["dense_sdpa"]["ms"] / ms
     if comp:
         line["comparators"] = comp
+    if world == 1 and args.zslab_ranks > 1:
+        line["zslab_emulated"] = time_zslab(p3, args.config, args.zslab_ranks, args.warmup, args.steps, flush, dev)
     if world == 1 and args.config == "65k" and not args.no_sizes and not args.summary_center:
         del timer
         torch.cuda.empty_cache()
@@ -707,6 +782,9 @@ def main():
                     help="time only the training block (pack3d_forward_backward), inputs drawn on the device")
     ap.add_argument("--packing", choices=synth.PACKINGS, default=None,
                     help="override the workload's packing (the stress case times all of them)")
+    ap.add_argument("--zslab-ranks", type=int, default=0,
+                    help="also time the z-slab split of the volume over this many ranks, every rank's "
+                         "kernels in turn on this one GPU (the exchanges are not timed)")
     ap.add_argument("--summary-center", action="store_true",
                     help="time the summary-centre variant of the block summaries and report its error "
                          "against the exact rotate-before-compress form")
