@@ -4,9 +4,11 @@
 // memory allocation, the first loads, the gate epilogue) is a large share of
 // its time, and one-tile CTAs two per SM hide it behind each other; with many
 // summary tiles the two-tile CTA, which reads every k~ / v~ tile once for both
-// query tiles, is faster.  Measured on B200: 65k tokens (M = 4,096) 0.78-0.80
-// ms one-tile vs 0.81 ms two-tile; 262k tokens (M = 16,384) 11.46 ms vs
-// 10.8-10.9 ms.  The threshold is in summaries (48 tiles of 128).
+// query tiles, is faster.  Measured on B200 (summary attention alone, forced
+// builds, one process): M = 4,096 (65k tokens) 0.784 ms one-tile vs 0.831
+// two-tile; M = 16,384 (262k) 10.69 vs 10.87-10.99, but 11.13 against 10.8 in
+// a long run under the power cap; M = 32,768 44.71 vs 42.51; M = 65,536 (1M)
+// 180.1 vs 170.3.  So the one-tile build runs up to 48 tiles of 128 summaries.
 #include "common.cuh"
 #include "internal.h"
 
@@ -25,11 +27,11 @@ cudaError_t launch(const Shape& s, const void* qr, const void* ks, const void* v
 }  // namespace sa_one
 
 namespace {
-constexpr int kOneTileMaxSummaryTiles = 48;
+constexpr int kOneTileMaxSummaries = 6144;
 // s.sa_build forces a build (PACK3D_FLAG_SUMMARY_ONE_TILE / _TWO_TILE); 0 picks by size.
 bool one_tile(const Shape& s) {
   if (s.sa_build != 0) return s.sa_build == 1;
-  return (s.M + 127) / 128 <= kOneTileMaxSummaryTiles;
+  return s.M <= kOneTileMaxSummaries;
 }
 }  // namespace
 

@@ -107,18 +107,19 @@ def test_two_tile_training_forward_matches_oracle(p3, name, s, packing, flags):
         assert e <= TOL["bf16"], f"{name}: {key} rel err {e:.3e}"
 
 
-def test_forward_backward_large_m_sharp(p3):
-    """Above the one-tile limit by size: 28,672 tokens in 1x2x2 blocks, so M = 7,168 (56 summary tiles),
-    with Q x 8 and K_loc / 8 (exact in bf16) making the summary softmax sharp.  Every gradient against the
-    oracle's chain rule: dq, dgate and out on every row, the local key gradients on sampled keys, the
-    summary-side ones on sampled blocks."""
+@pytest.mark.parametrize("build", ["two-tile", "one-tile"])
+def test_forward_backward_large_m_sharp(p3, build):
+    """28,672 tokens in 1x2x2 blocks, so M = 7,168 (56 tiles of 128 summaries), each query x summary
+    build forced, with Q x 8 and K_loc / 8 (exact in bf16) making the summary softmax sharp.  Every
+    gradient against the oracle's chain rule: dq, dgate and out on every row, the local key gradients on
+    sampled keys, the summary-side ones on sampled blocks."""
     s = small(Z=4, H=64, W=112, by=2, bx=2, value_scale=1.0)
-    assert (s.M + 127) // 128 > 48
     inp = synth.make_inputs(s, "morton", seed=17)
     inp["q"] = (inp["q"].float() * 8.0).bfloat16()
     inp["k_loc"] = (inp["k_loc"].float() * 0.125).bfloat16()
     dout = synth.make_dout(s, "morton", seed=17)
-    gpu = run_fwd_bwd(p3, s, inp, dout)
+    flags = p3.FLAG_SUMMARY_TWO_TILE if build == "two-tile" else p3.FLAG_SUMMARY_ONE_TILE
+    gpu = run_fwd_bwd(p3, s, inp, dout, flags)
     rng = np.random.default_rng(23)
     keys = np.unique(np.concatenate([[0, s.N - 1], rng.choice(s.N, 254, replace=False)]))
     blocks = np.unique(np.concatenate([[0, s.M - 1], rng.choice(s.M, 62, replace=False)]))

@@ -178,14 +178,15 @@ def sharp_inputs(s, packing, seed):
     return inp
 
 
-def test_large_m_two_tile_build_sharp_logits(p3):
-    """131,072 tokens, M = 8,192 (64 summary tiles, the two-tile build by size) with a sharp summary
-    softmax: o_cmp and out on every row of the first, a middle and the last CTA's query tiles (two
-    128-row tiles per kv head each) and on 1,024 sampled tokens, element by element."""
+@pytest.mark.parametrize("build", ["two-tile", "one-tile"])
+def test_large_m_sharp_logits(p3, build):
+    """131,072 tokens, M = 8,192 (64 tiles of 128 summaries, 86 of 96) with a sharp summary softmax,
+    each build forced: o_cmp and out on every row of the first, a middle and the last two-tile CTA's
+    query tiles (two 128-row tiles per kv head each) and on 1,024 sampled tokens, element by element."""
     s = synth.Pack3DShape(Z=8, H=64, W=256, Hq=8, Hkv=2, value_scale=1.0)
-    assert (s.M + 127) // 128 > 48
     inp = sharp_inputs(s, "random", seed=7)
-    gpu = run_stages(p3, s, to_dev(inp))
+    flags = p3.FLAG_SUMMARY_TWO_TILE if build == "two-tile" else p3.FLAG_SUMMARY_ONE_TILE
+    gpu = run_stages(p3, s, to_dev(inp), flags=flags)
     per_cta = 2 * 128 // (s.Hq // s.Hkv)        # tokens of one two-tile CTA (both kv heads run it)
     mid = (s.N // 2) // per_cta * per_cta
     full_tiles = np.concatenate([np.arange(0, per_cta), np.arange(mid, mid + per_cta),
