@@ -452,6 +452,9 @@ def stage_fractions(s, st_ms, peaks) -> Dict:
         if "flops" in w:
             e["tflops"] = w["flops"] / t / 1e12
             e["tensor_frac"] = e["tflops"] / peaks["bf16_tflops"]
+            if peaks.get("bf16_tflops_sustained"):
+                # against the power-capped sustained GEMM rate, for launches long enough to run capped
+                e["tensor_frac_sustained"] = e["tflops"] / peaks["bf16_tflops_sustained"]
         stages[name] = e
     return stages
 
