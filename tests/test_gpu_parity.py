@@ -281,11 +281,12 @@ def test_rope_qk_equals_two_rope_calls(p3, dtype):
     assert torch.equal(qa, qb) and torch.equal(ka, kb)
 
 
-@pytest.mark.parametrize("name", ["tiny", "small", "65k"])
+@pytest.mark.parametrize("name", ["tiny", "small", "65k", "131k"])
 def test_forward_host_equals_forward(p3, name):
     """The host-buffer pipeline (copies overlapped, summary stage in token chunks) gives exactly the
-    device-buffer forward pass's output."""
-    s = {"tiny": synth.CONFIGS["tiny"], "small": small(Z=4, H=16, W=24), "65k": synth.CONFIGS["65k"]}[name]
+    device-buffer forward pass's output; 131k tokens (M = 8,192) chunks the two-tile build."""
+    s = {"tiny": synth.CONFIGS["tiny"], "small": small(Z=4, H=16, W=24), "65k": synth.CONFIGS["65k"],
+         "131k": synth.Pack3DShape(Z=8, H=64, W=256, Hq=8, Hkv=2, packing="block")}[name]
     inp = synth.make_inputs(s, s.packing, seed=5)
     d = to_dev(inp)
     ref = run_forward(p3, s, d)
