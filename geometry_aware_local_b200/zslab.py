@@ -183,7 +183,9 @@ class Plan:
 
     `coords` (int32 [tokens, 3], on the rank's CUDA device) are the rank's own
     tokens' lattice coordinates with z local to its slab (0 .. planes-1); their
-    order is the order of `inputs()` and of the output."""
+    order is the order of `inputs()` and of the output.  With world > 1 the
+    exchanges run on `group` (torch.distributed, NCCL between GPUs); a one-rank
+    plan needs no process group."""
 
     def __init__(self, cfg, coords, rank: int, world: int, group=None, stream=None):
         import torch
@@ -231,7 +233,10 @@ class Plan:
         self.part = parts[rank]
         self.most = max(c for _, _, c in parts)
         M_all = sum(c for _, _, c in parts)
-        self.k_all, self.v_all = zeros(M_all, Hkv, d), zeros(M_all, Hkv, d)
+        if world == 1:   # the rank's own summaries are the volume's: no gather, no copy
+            self.k_all, self.v_all = self.k_sum, self.v_sum
+        else:
+            self.k_all, self.v_all = zeros(M_all, Hkv, d), zeros(M_all, Hkv, d)
         self.uneven = any(o != 0 or c != self.most for _, o, c in parts)
         if self.uneven:
             self.k_pad, self.v_pad = zeros(self.most * world, Hkv, d), zeros(self.most * world, Hkv, d)
@@ -283,6 +288,8 @@ class Plan:
 
     # ---- the exchanges (NCCL between GPUs) ------------------------------------------------------
     def exchange_halo(self):
+        if self.p.world == 1:
+            return
         import torch.distributed as dist
         p, ops = self.p, []
         below, above = self.halo_views()
@@ -300,6 +307,8 @@ class Plan:
         import torch.distributed as dist
 
         from . import gather_rows
+        if self.p.world == 1:
+            return
         k_part, v_part = self.summary_part()
         if not self.uneven:
             dist.all_gather_into_tensor(self.k_all, k_part, group=self.group)

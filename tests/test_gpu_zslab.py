@@ -186,6 +186,21 @@ def test_forward_on_a_one_rank_nccl_group(p3):
     assert rel_err(out.float().cpu().numpy(), ref) <= TOL["bf16"]
 
 
+def test_single_rank_plan_needs_no_process_group(p3):
+    """A one-rank Plan runs without torch.distributed (no exchange, the summaries are the volume's)."""
+    from geometry_aware_local_b200 import zslab
+    s = synth.Pack3DShape(Z=3, H=12, W=20, Hq=8, Hkv=2, dtype="bf16", value_scale=0.125, packing="random")
+    inp = synth.make_inputs(s, seed=54)
+    d = {k: v.cuda() for k, v in inp.items() if k != "sites"}
+    cfg = p3.config_from_shape(s)
+    plan = zslab.Plan(cfg, d["coords"], 0, 1)
+    for k, v in plan.inputs().items():
+        v.copy_(d[k])
+    out = plan.forward()
+    whole = whole_volume(p3, cfg, s, d)
+    assert torch.equal(out, whole["out"])
+
+
 @pytest.mark.parametrize("n,row_shape,dtype", [(1, (2, 64), torch.bfloat16), (1000, (2, 64), torch.bfloat16),
                                                (777, (8, 64), torch.float32), (5, (4,), torch.float32)])
 def test_gather_rows_bit_exact(p3, n, row_shape, dtype):
