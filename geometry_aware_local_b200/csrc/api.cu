@@ -320,7 +320,7 @@ pack3d_status pack3d_exp2_fma_eval(const float* x, float* y, int64_t n, void* st
 
 pack3d_status pack3d_gather_rows(const int32_t* idx, int64_t n, const void* src, void* dst, int64_t row_bytes,
                                  void* stream) {
-  if (n < 0 || row_bytes <= 0 || row_bytes % 16 != 0) return PACK3D_ERR_INVALID_ARG;
+  if (n < 0 || row_bytes <= 0 || row_bytes % 16 != 0 || row_bytes / 16 > INT32_MAX) return PACK3D_ERR_INVALID_ARG;
   if (n == 0) return PACK3D_OK;
   if (!idx || !src || !dst) return PACK3D_ERR_INVALID_ARG;
   if (!aligned16(src) || !aligned16(dst)) return PACK3D_ERR_ALIGNMENT;

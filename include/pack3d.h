@@ -259,8 +259,8 @@ pack3d_status pack3d_summary_attn_rows(const pack3d_config *cfg, int64_t tokens,
  * zero row.  idx (int32, n entries), src and dst are device pointers owned by
  * the caller; src and dst 16-byte aligned; every idx[i] must be a row of src
  * (not checked on the device).  n == 0 returns PACK3D_OK with nothing
- * launched.  Errors: null pointer, n < 0 or row_bytes not a positive multiple
- * of 16 -> PACK3D_ERR_INVALID_ARG; misaligned src or dst ->
+ * launched.  Errors: null pointer, n < 0, or row_bytes not a positive multiple
+ * of 16 or above 16 x (2^31 - 1) -> PACK3D_ERR_INVALID_ARG; misaligned src or dst ->
  * PACK3D_ERR_ALIGNMENT; a failed launch -> PACK3D_ERR_CUDA. */
 pack3d_status pack3d_gather_rows(const int32_t *idx, int64_t n, const void *src, void *dst,
                                  int64_t row_bytes, void *stream);

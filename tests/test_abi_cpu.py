@@ -135,6 +135,7 @@ def test_host_errors_return_before_launch(p3):
     assert lib.pack3d_gather_rows(None, 0, None, None, 16, None) == 0
     assert lib.pack3d_gather_rows(fake, -1, fake, fake, 16, None) == 1
     assert lib.pack3d_gather_rows(fake, 4, fake, fake, 24, None) == 1
+    assert lib.pack3d_gather_rows(fake, 4, fake, fake, 16 * (2**31), None) == 1
     assert lib.pack3d_gather_rows(None, 4, fake, fake, 16, None) == 1
     assert lib.pack3d_gather_rows(fake, 4, bad, fake, 16, None) == 3
     assert lib.pack3d_exp2_fma_eval(None, None, 0, None) == 0
