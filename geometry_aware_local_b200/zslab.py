@@ -185,7 +185,10 @@ class Plan:
     tokens' lattice coordinates with z local to its slab (0 .. planes-1); their
     order is the order of `inputs()` and of the output.  With world > 1 the
     exchanges run on `group` (torch.distributed, NCCL between GPUs); a one-rank
-    plan needs no process group."""
+    plan needs no process group.  `stream` (None: torch's current stream; a
+    torch.cuda.Stream or a raw cudaStream_t) carries every phase and, through
+    torch's current-stream context, the exchanges; with an explicit stream the
+    caller orders its writes of `inputs()` before `forward` on that stream."""
 
     def __init__(self, cfg, coords, rank: int, world: int, group=None, stream=None):
         import torch
@@ -242,6 +245,20 @@ class Plan:
             self.k_pad, self.v_pad = zeros(self.most * world, Hkv, d), zeros(self.most * world, Hkv, d)
             self.compact = torch.cat([torch.arange(r * self.most + o, r * self.most + o + c, dtype=torch.int32)
                                       for r, (_, o, c) in enumerate(parts)]).to(dev)
+        # The buffers above were filled on torch's current stream; the phases run on `stream`.
+        if stream is not None:
+            torch.cuda.synchronize(dev)
+
+    def _on_stream(self):
+        """Context in which torch.distributed calls order themselves after the phases' kernels:
+        NCCL waits for torch's current stream, so that must be the plan's stream."""
+        import contextlib
+
+        import torch
+        if self.stream is None:
+            return contextlib.nullcontext()
+        s = self.stream
+        return torch.cuda.stream(torch.cuda.ExternalStream(s) if isinstance(s, int) else s)
 
     def inputs(self) -> Dict:
         """Views of the extended arrays' own rows, to be written before `forward` (in the order
@@ -300,8 +317,9 @@ class Plan:
                         dist.P2POp(dist.irecv, recv[0], peer, self.group),
                         dist.P2POp(dist.irecv, recv[1], peer, self.group)]
         if ops:
-            for req in dist.batch_isend_irecv(ops):
-                req.wait()
+            with self._on_stream():
+                for req in dist.batch_isend_irecv(ops):
+                    req.wait()
 
     def gather_summaries(self):
         import torch.distributed as dist
@@ -310,12 +328,13 @@ class Plan:
         if self.p.world == 1:
             return
         k_part, v_part = self.summary_part()
-        if not self.uneven:
-            dist.all_gather_into_tensor(self.k_all, k_part, group=self.group)
-            dist.all_gather_into_tensor(self.v_all, v_part, group=self.group)
-            return
-        dist.all_gather_into_tensor(self.k_pad, k_part, group=self.group)
-        dist.all_gather_into_tensor(self.v_pad, v_part, group=self.group)
+        with self._on_stream():
+            if not self.uneven:
+                dist.all_gather_into_tensor(self.k_all, k_part, group=self.group)
+                dist.all_gather_into_tensor(self.v_all, v_part, group=self.group)
+                return
+            dist.all_gather_into_tensor(self.k_pad, k_part, group=self.group)
+            dist.all_gather_into_tensor(self.v_pad, v_part, group=self.group)
         gather_rows(self.compact, self.k_pad, self.k_all, self.stream)
         gather_rows(self.compact, self.v_pad, self.v_all, self.stream)
 

@@ -201,6 +201,28 @@ def test_single_rank_plan_needs_no_process_group(p3):
     assert torch.equal(out, whole["out"])
 
 
+@pytest.mark.parametrize("raw", [False, True])
+def test_single_rank_plan_on_a_side_stream(p3, raw):
+    """A Plan given its own stream (a torch stream, or the raw handle) runs every phase there, and
+    its exchanges would run with that stream as torch's current one (the stream NCCL orders after)."""
+    from geometry_aware_local_b200 import zslab
+    s = synth.Pack3DShape(Z=4, H=12, W=20, Hq=8, Hkv=2, dtype="bf16", value_scale=0.125, packing="morton")
+    inp = synth.make_inputs(s, seed=55)
+    d = {k: v.cuda() for k, v in inp.items() if k != "sites"}
+    cfg = p3.config_from_shape(s)
+    side = torch.cuda.Stream()
+    plan = zslab.Plan(cfg, d["coords"], 0, 1, stream=side.cuda_stream if raw else side)
+    with plan._on_stream():
+        assert torch.cuda.current_stream().cuda_stream == side.cuda_stream
+    for k, v in plan.inputs().items():
+        v.copy_(d[k])
+    side.wait_stream(torch.cuda.current_stream())
+    out = plan.forward()
+    torch.cuda.current_stream().wait_stream(side)
+    whole = whole_volume(p3, cfg, s, d)
+    assert torch.equal(out, whole["out"])
+
+
 @pytest.mark.parametrize("n,row_shape,dtype", [(1, (2, 64), torch.bfloat16), (1000, (2, 64), torch.bfloat16),
                                                (777, (8, 64), torch.float32), (5, (4,), torch.float32)])
 def test_gather_rows_bit_exact(p3, n, row_shape, dtype):
