@@ -1,10 +1,13 @@
 // C ABI of the PACK3D forward pass (see pack3d.h): host-side validation,
-// workspace carving and stream-ordered launches.  No entry point allocates,
-// frees or synchronises except pack3d_check_status.
+// workspace carving and stream-ordered launches.  No entry point allocates
+// device memory, frees or synchronises except pack3d_check_status;
+// pack3d_forward creates one side stream and two events per device on its
+// first call there (kept until the process exits).
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 
 #include "common.cuh"
@@ -70,17 +73,82 @@ ForwardWs carve_forward(const pack3d_config& c, uintptr_t base) {
   return w;
 }
 
+namespace {
+
+// The side stream RoPE runs on inside pack3d_forward: one non-blocking stream
+// and two events per device, made on the device's first uncaptured call.  The
+// mutex is held from the fork to the join, so calls from several host threads
+// never interleave their records and waits on the shared events (their side
+// work is serialised on the one side stream).
+constexpr int kMaxForkDevices = 64;
+struct Fork {
+  cudaStream_t side = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+};
+std::mutex g_fork_mutex;
+Fork g_fork[kMaxForkDevices];
+
+// Sets *out to the current device's side stream (made on first use), or to
+// nullptr when cs is being captured into a graph (every launch then stays on
+// cs) or the device number is out of the table's range.
+cudaError_t side_stream(cudaStream_t cs, std::unique_lock<std::mutex>& lock, Fork** out) {
+  *out = nullptr;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(cs, &cap);
+  if (e != cudaSuccess || cap != cudaStreamCaptureStatusNone) return e;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxForkDevices) return e;
+  lock = std::unique_lock<std::mutex>(g_fork_mutex);
+  Fork& f = g_fork[dev];
+  if (f.side == nullptr) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t a = nullptr, b = nullptr;
+    e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      if (b) cudaEventDestroy(b);
+      if (a) cudaEventDestroy(a);
+      if (st) cudaStreamDestroy(st);
+      return e;
+    }
+    f.side = st;
+    f.start = a;
+    f.done = b;
+  }
+  *out = &f;
+  return cudaSuccess;
+}
+
+}  // namespace
+
 cudaError_t enqueue_forward(const pack3d_config& c, const Shape& s, const ForwardWs& w, const int32_t* coords,
                             const void* q, const void* k_loc, const void* v_loc, const void* k_cmp,
                             const void* v_cmp, const float* scores, const float* gate, void* out, int32_t* err,
-                            cudaStream_t cs) {
-  // The summaries run before RoPE: both stream from HBM and are independent,
-  // and the summaries write 1/16 of what they read, so RoPE starts with few
-  // dirty L2 lines to evict; in the other order the summaries stage would
-  // pay for writing back RoPE's output (about 10 % of its time at 262k tokens).
-  cudaError_t e = launch_build_index(s, coords, w.g2p, w.members, err, cs);
+                            cudaStream_t cs, bool fork) {
+  // RoPE reads only the coordinates and the inputs: with `fork` it runs on
+  // the side stream, started after everything already on cs, while the index
+  // map and the summaries run on cs; local attention waits for both.  On one
+  // stream the summaries run before RoPE: both stream from HBM and are
+  // independent, and the summaries write 1/16 of what they read, so RoPE
+  // starts with few dirty L2 lines to evict; in the other order the summaries
+  // stage would pay for writing back RoPE's output (about 10 % of its time at
+  // 262k tokens).
+  std::unique_lock<std::mutex> lock;
+  Fork* f = nullptr;
+  cudaError_t e = fork ? side_stream(cs, lock, &f) : cudaSuccess;
+  if (e == cudaSuccess && f) {
+    e = cudaEventRecord(f->start, cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(f->side, f->start, 0);
+    if (e == cudaSuccess) e = launch_rope(s, c.dtype, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, f->side);
+    if (e == cudaSuccess) e = cudaEventRecord(f->done, f->side);
+  }
+  if (e == cudaSuccess) e = launch_build_index(s, coords, w.g2p, w.members, err, cs);
   if (e == cudaSuccess) e = launch_summaries(s, c.dtype, w.members, k_cmp, v_cmp, scores, w.k_sum, w.v_sum, cs);
-  if (e == cudaSuccess) e = launch_rope(s, c.dtype, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, cs);
+  if (e == cudaSuccess)
+    e = f ? cudaStreamWaitEvent(cs, f->done, 0)
+          : launch_rope(s, c.dtype, coords, q, w.q_rot, s.Hq, k_loc, w.k_rot, s.Hkv, cs);
   if (e == cudaSuccess)
     e = launch_local(s, c.dtype, c.flags, w.g2p, w.q_rot, w.k_rot, v_loc, w.o_loc, err, cs);
   if (e == cudaSuccess) {
@@ -344,7 +412,7 @@ pack3d_status pack3d_forward(const pack3d_config* cfg, const int32_t* coords, co
     return PACK3D_ERR_ALIGNMENT;
   const Shape s = make_shape(*cfg);
   return cuda_status(enqueue_forward(*cfg, s, w, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out,
-                                     err_word, (cudaStream_t)stream));
+                                     err_word, (cudaStream_t)stream, true));
 }
 
 size_t pack3d_train_workspace_bytes(const pack3d_config* cfg) {

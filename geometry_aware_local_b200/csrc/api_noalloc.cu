@@ -88,7 +88,7 @@ extern "C" pack3d_status pack3d_forward_noalloc(const pack3d_config* cfg, const 
   const ForwardWs w = carve_forward(*cfg, (uintptr_t)base);
   const Shape s = make_shape(*cfg);
   const cudaError_t e = enqueue_forward(*cfg, s, w, coords, q, k_loc, v_loc, k_cmp, v_cmp, scores, gate, out,
-                                        err_word, (cudaStream_t)stream);
+                                        err_word, (cudaStream_t)stream, false);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return PACK3D_ERR_CUDA;

@@ -28,11 +28,14 @@ struct ForwardWs {
 ForwardWs carve_forward(const pack3d_config& c, uintptr_t base);
 
 // The forward pass's launches, stream-ordered on st, on a carved workspace
-// (pack3d_forward and pack3d_forward_noalloc both run exactly this).
+// (pack3d_forward and pack3d_forward_noalloc both run exactly this).  With
+// `fork`, RoPE runs on a per-device side stream (made on first use) that
+// starts after st's earlier work and that st waits for before local
+// attention; inside a stream capture, or without `fork`, all launches stay on st.
 cudaError_t enqueue_forward(const pack3d_config& c, const Shape& s, const ForwardWs& w, const int32_t* coords,
                             const void* q, const void* k_loc, const void* v_loc, const void* k_cmp,
                             const void* v_cmp, const float* scores, const float* gate, void* out, int32_t* err,
-                            cudaStream_t st);
+                            cudaStream_t st, bool fork);
 
 // Extra outputs of the forward pass when it runs as the first half of the
 // training block (pack3d_forward_backward): per (token, q head) row four

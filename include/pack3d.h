@@ -277,7 +277,13 @@ pack3d_status pack3d_gather_rows(const int32_t *idx, int64_t n, const void *src,
 pack3d_status pack3d_exp2_fma_eval(const float *x, float *y, int64_t n, void *stream);
 
 /* The whole forward pass: index map, summaries, RoPE on Q and K_loc, local
- * branch, query-summary branch with the gate, all stream-ordered on `stream`.
+ * branch, query-summary branch with the gate, all stream-ordered on `stream`:
+ * the pass starts after the work already on `stream` and later work on it
+ * sees every output.  Inside, RoPE runs on a library-owned side stream
+ * concurrently with the index map and the summaries (one non-blocking stream
+ * and two events per device, made on the device's first call and kept until
+ * the process exits; calls from several host threads take turns on them).
+ * While `stream` is being captured into a graph, every launch stays on it.
  * workspace: device buffer of at least pack3d_workspace_bytes(cfg) bytes,
  * 256-byte aligned; its contents on entry do not matter.  err_word: device int32
  * the caller zeroed before its first use (required). */
