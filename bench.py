@@ -5,9 +5,12 @@
 
 One step = one pass of the whole hot path over one synthetic volume: index
 map, block summaries, axial RoPE on Q and K_loc, local attention, query x
-summary attention with the gate.  The timed step calls the C ABI stage entry
-points in the order pack3d_forward runs them, with CUDA events between stages
-on the launching stream, so each kernel's live duration is known.  L2 is
+summary attention with the gate.  The timed step is one pack3d_forward call
+on device buffers, CUDA events around it on the launching stream (the
+library runs RoPE on its side stream next to the index map and the
+summaries).  A second, staged pass calls the C ABI stage entry points in
+turn on one stream with CUDA events between them, so each kernel's live
+duration is known (``stages``, ``staged_ms_per_step``).  L2 is
 flushed between steps, outside the timed events: a 256 MiB write, then a
 256 MiB read of another buffer, so that no input is left in L2 and none of
 the flush's dirty lines is written back inside a timed kernel (``--flush
