@@ -1,5 +1,7 @@
 """The z-slab split of one volume over several ranks, host logic on CPU gloo ranks.
 
+(The last group of tests below runs zslab.Plan's own exchange code on gloo ranks.)
+
 Each rank takes the tokens of its planes, exchanges its boundary planes' local
 keys and values with its neighbours, and runs the stages on its slab extended
 by the received halo, a lattice whose origin is the true z of its first plane.
@@ -155,6 +157,130 @@ def test_zslab_centre_variant_and_shifted_volume():
     got = _run(2, dict(origin=(5, 2, 0), rz=1), center=True)
     for rank, out_err, loc_err, sum_err, lo, hi, index_exact, _ in got:
         assert out_err < 1e-12 and loc_err < 1e-12 and sum_err < 1e-12 and index_exact, rank
+
+
+# ------------------------------------------------- zslab.Plan on gloo ranks -----
+#
+# zslab.Plan itself on CPU gloo ranks: its buffers, its index-map slices, its halo
+# exchange (batch_isend_irecv) and its summary all-gather (all_gather_into_tensor,
+# then the compaction for uneven slabs) run as written; only the library's kernel
+# calls are replaced, for this test, by the oracle's stages on the extended
+# lattice (and the row gather by CPU indexing).  The outputs must equal the
+# whole-volume oracle's, the halo rows the neighbours' boundary planes bit for
+# bit, and the gathered summaries the whole volume's.
+
+def _install_oracle_stand_ins(p3, se, state):
+    """Replaces the binding's kernel calls the Plan makes by the oracle's stages on the extended
+    lattice `se` (test infrastructure; the product path never calls the oracle)."""
+    import oracle
+
+    def build_index(cfg, coords, g2p, members, err, stream=None):
+        assert (cfg.Z, tuple(cfg.origin)) == (se.Z, tuple(se.origin))   # the Plan's extended config
+        st, g, m = oracle.build_index(se, coords.numpy())
+        assert st == 0
+        g2p.copy_(torch.from_numpy(g))
+        members.copy_(torch.from_numpy(m))
+        state["coords"] = coords.numpy().copy()
+
+    def build_summaries(cfg, members, k_cmp, v_cmp, scores, k_sum, v_sum, stream=None):
+        ks, vs = oracle.summaries(se, state["coords"], members, k_cmp, v_cmp, scores)
+        k_sum.copy_(torch.from_numpy(ks))
+        v_sum.copy_(torch.from_numpy(vs))
+
+    def rope_qk(cfg, coords, q, q_rot, k, k_rot, stream=None):
+        q_rot.copy_(torch.from_numpy(oracle.rotate(se, coords, q)))
+        k_rot.copy_(torch.from_numpy(oracle.rotate(se, coords, k)))
+
+    def local_attn(cfg, g2p, q_rot, k_rot, v_loc, o_loc, err=None, stream=None):
+        t = state["tokens"]   # the own rows come first in the extended layout
+        o = oracle.local_attn(se, state["coords"], g2p, q_rot[:t], k_rot, v_loc, np.arange(t))
+        o_loc[:t].copy_(torch.from_numpy(o))
+
+    def summary_attn_rows(cfg, tokens, summaries, q_rot, k_sum, v_sum, o_loc, gate, out, err=None, stream=None):
+        assert k_sum.shape[0] == summaries and q_rot.shape[0] == tokens
+        oc = oracle.summary_attn(se, q_rot, k_sum, v_sum)
+        out.copy_(torch.from_numpy(oracle.gate_mix(se, gate, o_loc, oc, np.arange(tokens))))
+
+    def gather_rows(idx, src, dst, stream=None):
+        i = idx.long()
+        rows = src.index_select(0, i.clamp(min=0))
+        rows[i < 0] = 0
+        dst.copy_(rows)
+
+    def check_status(err, stream=None):
+        return int(err.abs().sum())
+
+    for name, fn in (("build_index", build_index), ("build_summaries", build_summaries), ("rope_qk", rope_qk),
+                     ("local_attn", local_attn), ("summary_attn_rows", summary_attn_rows),
+                     ("gather_rows", gather_rows), ("check_status", check_status)):
+        setattr(p3, name, fn)
+
+
+def _plan_rank(rank, world, port, shape_kw, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    import geometry_aware_local_b200 as p3
+    import oracle
+    import synth
+    from geometry_aware_local_b200 import zslab
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        s = _shape(**shape_kw)
+        inp = synth.make_inputs(s, seed=43)
+        whole = oracle.forward(s, inp)
+        _, g2p_w, _ = oracle.build_index(s, inp["coords"])
+        cfg = p3.config_from_shape(s)
+        p = zslab.make_plan(cfg, rank, world)
+        se = s.replace(Z=p.Z_ext, origin=(s.origin[0] + p.z0 - p.lo, s.origin[1], s.origin[2]))
+        _install_oracle_stand_ins(p3, se, {"tokens": p.tokens})
+        idx, own = zslab.take_slab(inp, p)
+        plan = zslab.Plan(cfg, own["coords"], rank, world)
+        for k, v in plan.inputs().items():
+            v.copy_(own[k])
+        out = plan.forward().double().numpy()
+        ref = whole["out"][idx.numpy()]
+        out_err = float(np.abs(out - ref).max() / np.abs(ref).max())
+        # The halo rows: the neighbours' boundary planes in raster order, bit for bit.
+        hw = s.H * s.W
+        halo_exact = True
+        for (a, b), z_from in ((p.halo_below, p.z0 - p.lo), (p.halo_above, p.z1)):
+            if b > a:
+                tok = torch.from_numpy(g2p_w[z_from * hw:z_from * hw + (b - a)].astype(np.int64))
+                for name in ("k_loc", "v_loc"):
+                    halo_exact = halo_exact and torch.equal(plan.ext[name][a:b], inp[name].index_select(0, tok))
+        k_err = max(float(np.abs(plan.k_all.double().numpy() - whole["k_sum"]).max() / np.abs(whole["k_sum"]).max()),
+                    float(np.abs(plan.v_all.double().numpy() - whole["v_sum"]).max() / np.abs(whole["v_sum"]).max()))
+        q.put((rank, out_err, k_err, halo_exact, plan.uneven, p.lo, p.hi, None))
+    except Exception as e:                       # report instead of hanging the parent
+        q.put((rank, None, None, None, None, None, None, repr(e)))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,Z,uneven", [(2, 8, False), (2, 7, True), (3, 7, True)])
+def test_plan_exchanges_on_gloo_ranks(world, Z, uneven):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_plan_rank, args=(r, world, port, dict(Z=Z), q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted((q.get(timeout=240) for _ in procs), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+    for rank, *_, err in got:
+        assert err is None, f"rank {rank}: {err}"
+    assert all(p.exitcode == 0 for p in procs)
+    for rank, out_err, k_err, halo_exact, was_uneven, lo, hi, _ in got:
+        assert (lo > 0) == (rank > 0) and (hi > 0) == (rank < world - 1), rank
+        assert was_uneven == uneven, rank
+        assert halo_exact, rank
+        # float32 buffers between the oracle's float64 stages
+        assert out_err < 1e-5, (rank, out_err)
+        assert k_err < 1e-6, (rank, k_err)
 
 
 # ------------------------------------------------------------- host plan -----
